@@ -1,0 +1,554 @@
+/*
+ * dq_oracle.c -- plain fp64 CPU reference of the DualQuant dual-scale
+ * block-coordinate-descent (BCD) weight-quantization solver.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the oracle that the CUDA path is
+ * checked against.  Only the tests, the smoke check and the CPU-baseline leg of
+ * the benchmark load it; the product path never does.  It shares no code, header
+ * or table with the CUDA library.
+ *
+ * Sources (web pages on the method; cited by title and section):
+ *  [R5] "DualQuant: Calibration-Free Dual-Scale Weight and Activation
+ *       Quantization" reproduction README (daiwk.github.io): "Original paper"
+ *       flowchart, "Core equations", "Local reproduction".
+ *  [P2] "DualQuant: Dual-scale Calibration-free Weight-and-Activation
+ *       Quantization for LLMs" (arXiv 2610.13767) summary (paperlayer.ai):
+ *       §3 Quantization preliminaries, §4.3 MSE optimization via BCD,
+ *       App. A.1 variable splitting, App. B closed-form solutions.
+ *  [L1] SQuant lesson, "Chapter 2: Quantization from Scratch" (uniform
+ *       quantizer, worked int8 example).
+ *  [T4] "Round-to-Nearest & basic weight quantization" tutorial, sections
+ *       "Round-to-Nearest (RTN)" and "Absmax (Symmetric) Quantization".
+ *
+ * Everything here is written as the plain definition: loops in natural order
+ * (j ascending inside a block, i ascending inside a column), fp64 arithmetic,
+ * no blocking or fusion.  Readings of points the pages leave open:
+ *  - Q rounds to the nearest grid value, ties to the "even" neighbour (even
+ *    integer for INT4; even mantissa bit for E2M1), values past the ends clip.
+ *    The decision compares W with boundary*(a*b), which is exact in fp64
+ *    because a*b and boundary*(a*b) have few significant bits.
+ *  - Projection onto admissible inverse scales = nearest admissible value in
+ *    linear distance (the minimiser of the 1-D quadratic); fp16/bf16/E4M3 ties
+ *    go to the even mantissa, E8M0 ties go to the larger power of two.
+ *  - NVFP4: one fp32 tensor scale s_T = fp32(amax / (6*448)) fixed at init;
+ *    block inverse scale a = s_T * e with e a positive finite E4M3 value.
+ *  - "Scale 1 for an all-zero code slice": a = 1 (INT4, MXINT4), e = 1 (NVFP4),
+ *    b = 1.
+ *  - Init: b = 1 and a = Proj(absmax(block) / qmax), qmax = 7 (INT4 grid
+ *    [-8,7]) or 6 (E2M1); an all-zero block gets scale 1.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define DQO_OK 0
+#define DQO_EINVAL 1
+#define DQO_ENONFINITE 4
+#define DQO_ENOMEM 6
+
+/* formats (numbering mirrors the library's public enum by value only) */
+#define DQO_INT4 0
+#define DQO_MXINT4 1
+#define DQO_NVFP4 2
+/* element dtypes */
+#define DQO_F32 0
+#define DQO_BF16 1
+#define DQO_F16 2
+/* projection kinds for dqo_project() */
+#define DQO_PROJ_F16 0
+#define DQO_PROJ_BF16 1
+#define DQO_PROJ_E4M3 2
+#define DQO_PROJ_E8M0 3
+
+/* ------------------------------------------------------------------------ */
+/* Format grids Q ([P2] §3; [R5] "Local reproduction": INT4 codebook [-8,7]). */
+
+static const double INT4_GRID[16] = {-8, -7, -6, -5, -4, -3, -2, -1, 0, 1, 2, 3, 4, 5, 6, 7};
+static const unsigned char INT4_EVEN[16] = {1, 0, 1, 0, 1, 0, 1, 0, 1, 0, 1, 0, 1, 0, 1, 0};
+/* E2M1 values and, per value, whether its mantissa bit is 0 ("even").
+ * magnitudes 0,0.5,1,1.5,2,3,4,6 have encodings 000,001,010,011,100,101,110,111 */
+static const double E2M1_GRID[15] = {-6, -4, -3, -2, -1.5, -1, -0.5, 0, 0.5, 1, 1.5, 2, 3, 4, 6};
+static const unsigned char E2M1_EVEN[15] = {0, 1, 0, 1, 0, 1, 0, 1, 0, 1, 0, 1, 0, 1, 0};
+
+/*
+ * Nearest grid value to w/scale ([L1] Ch. 2 round-to-nearest then clip;
+ * [P2] §3 "nearest representable value").  grid[] is sorted ascending; the
+ * boundary between grid[k] and grid[k+1] is their midpoint h_k.  For scale > 0,
+ * w/scale > h_k exactly when w > h_k*scale, so the decision is a scan of
+ * comparisons.  An exact tie (w == h_k*scale) picks the neighbour flagged even.
+ * Values below the first / above the last boundary land on the end values
+ * (clip).  Returns the grid index.
+ */
+int dqo_quant_index(double w, double scale, const double* grid, const unsigned char* even, int n) {
+  int idx = 0;
+  for (int k = 0; k + 1 < n; ++k) {
+    double h = 0.5 * (grid[k] + grid[k + 1]);
+    double t = h * scale;
+    if (w > t) {
+      idx = k + 1;
+    } else if (w == t) {
+      idx = even[k] ? k : k + 1;
+      break;
+    } else {
+      break;
+    }
+  }
+  return idx;
+}
+
+/* Symmetric absmax scale max|w|/qmax ([T4] "Absmax (Symmetric) Quantization";
+ * [P2] §3 "Δ = max(|W|)/qmax"). */
+double dqo_absmax_scale(const double* w, int64_t n, double qmax) {
+  double m = 0.0;
+  for (int64_t i = 0; i < n; ++i) {
+    double v = fabs(w[i]);
+    if (v > m) m = v;
+  }
+  return m / qmax;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Projection onto admissible (hardware-legal) positive inverse scales
+ * ([R5] "Core equations": "Projection is on inverse scales"; [P2] App. B
+ * "projecting to the nearest representable value").                       */
+
+/*
+ * Nearest positive finite value of a binary float format with `mbits`
+ * explicit mantissa bits, smallest normal exponent `emin` (subnormals below
+ * it) and largest finite value `vmax`.  Ties go to the value whose last
+ * mantissa bit is 0.  Anything at or below the smallest positive value maps to
+ * it (zero is not admissible); anything at or above vmax maps to vmax.
+ */
+static double project_float(double v, int mbits, int emin, double vmax) {
+  double minsub = ldexp(1.0, emin - mbits);
+  if (!(v > minsub)) return minsub;
+  if (v >= vmax) return vmax;
+  int e;
+  frexp(v, &e);           /* v = f * 2^e, f in [0.5, 1) -> binade exponent e-1 */
+  int E = e - 1;
+  if (E < emin) E = emin; /* subnormal range: fixed spacing */
+  double ulp = ldexp(1.0, E - mbits);
+  double k = floor(v / ulp); /* v/ulp is an exact power-of-two scaling */
+  double lo = k * ulp, hi = (k + 1.0) * ulp, mid = (k + 0.5) * ulp;
+  double r;
+  if (v < mid)
+    r = lo;
+  else if (v > mid)
+    r = hi;
+  else
+    r = (fmod(k, 2.0) == 0.0) ? lo : hi;
+  if (r < minsub) r = minsub;
+  if (r > vmax) r = vmax;
+  return r;
+}
+
+/* E8M0 power-of-two scales with exponent in [-126, 126] ([R5] "Local
+ * reproduction"); nearest in linear distance, a tie (1.5 * 2^k) goes up. */
+static double project_pow2(double v) {
+  if (!(v > ldexp(1.0, -126))) return ldexp(1.0, -126);
+  if (v >= ldexp(1.0, 126)) return ldexp(1.0, 126);
+  int e;
+  frexp(v, &e);
+  double lo = ldexp(1.0, e - 1), hi = ldexp(1.0, e);
+  double mid = 1.5 * lo;
+  double r = (v < mid) ? lo : hi;
+  if (r > ldexp(1.0, 126)) r = ldexp(1.0, 126);
+  return r;
+}
+
+double dqo_project(int kind, double v) {
+  switch (kind) {
+    case DQO_PROJ_F16: return project_float(v, 10, -14, 65504.0);
+    case DQO_PROJ_BF16: return project_float(v, 7, -126, ldexp(255.0, 120)); /* (2-2^-7)*2^127 */
+    case DQO_PROJ_E4M3: return project_float(v, 3, -6, 448.0);
+    case DQO_PROJ_E8M0: return project_pow2(v);
+  }
+  return NAN;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Storage encodings of admissible values (all inputs are exactly
+ * representable; these only rewrite them as bit patterns).                 */
+
+static uint16_t encode_float_bits(double v, int mbits, int emin, int ebits) {
+  /* v > 0 and exactly representable */
+  int e;
+  frexp(v, &e);
+  int E = e - 1;
+  int bias = 1 - emin;
+  uint32_t expfield, mant;
+  if (E < emin) {
+    expfield = 0;
+    mant = (uint32_t)ldexp(v, mbits - emin);
+  } else {
+    expfield = (uint32_t)(E + bias);
+    mant = (uint32_t)(ldexp(v, mbits - E) - ldexp(1.0, mbits));
+  }
+  (void)ebits;
+  return (uint16_t)((expfield << mbits) | mant);
+}
+
+static uint8_t e2m1_nibble(double q) {
+  double m = fabs(q);
+  uint8_t code;
+  if (m == 0.0) return 0; /* zero is always the +0 encoding */
+  if (m == 0.5) code = 1;
+  else if (m == 1.0) code = 2;
+  else if (m == 1.5) code = 3;
+  else if (m == 2.0) code = 4;
+  else if (m == 3.0) code = 5;
+  else if (m == 4.0) code = 6;
+  else code = 7; /* 6.0 */
+  return (uint8_t)((q < 0 ? 8 : 0) | code);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Solver state and steps                                                    */
+
+typedef struct {
+  int64_t M, N;
+  int fmt, G, nb;
+  int col_kind;  /* projection kind for b */
+  double sT;     /* NVFP4 tensor scale (1 otherwise) */
+  const double* W;
+} problem;
+
+static double qmax_of(int fmt) { return fmt == DQO_NVFP4 ? 6.0 : 7.0; }
+
+/* block inverse scale value a from its stored factor (NVFP4 stores e, a = s_T*e) */
+static double a_value(const problem* p, double stored) { return p->fmt == DQO_NVFP4 ? p->sT * stored : stored; }
+
+/* projection of an LS inverse-scale value onto F_a; returns the stored factor */
+static double project_a(const problem* p, double v) {
+  if (p->fmt == DQO_INT4) return dqo_project(DQO_PROJ_F16, v);
+  if (p->fmt == DQO_MXINT4) return dqo_project(DQO_PROJ_E8M0, v);
+  return dqo_project(DQO_PROJ_E4M3, v / p->sT); /* nearest s_T*e to v */
+}
+
+/* Q(W/(a b)) -> grid value ([R5] flowchart "Black-box format grid Q") */
+static double quant_value(const problem* p, double w, double a, double b) {
+  double ab = a * b;
+  if (p->fmt == DQO_NVFP4) return E2M1_GRID[dqo_quant_index(w, ab, E2M1_GRID, E2M1_EVEN, 15)];
+  return INT4_GRID[dqo_quant_index(w, ab, INT4_GRID, INT4_EVEN, 16)];
+}
+
+/* requantize every element with the current (a, b)  ([R5] "Core equations":
+ * requantize after each update).  q is [M][N]. */
+void dqo_requant_impl(const problem* p, const double* astored, const double* b, double* q) {
+  int64_t M = p->M, N = p->N;
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < M; ++i)
+    for (int64_t j = 0; j < N; ++j) {
+      double a = a_value(p, astored[i * p->nb + j / p->G]);
+      q[i * N + j] = quant_value(p, p->W[i * N + j], a, b[j]);
+    }
+}
+
+/*
+ * Row/block update with codes fixed ([R5] "Core equations": with R = Q̂ D_b,
+ * a_i <- Proj_Fa( sum_j W_ij R_ij / sum_j R_ij^2 ), scale 1 for an all-zero
+ * code slice).  `raw` (optional) receives the unprojected least-squares value
+ * (NaN for an all-zero slice).
+ */
+void dqo_row_update_impl(const problem* p, const double* q, const double* b, double* astored, double* raw) {
+  int64_t M = p->M, N = p->N;
+  int G = p->G, nb = p->nb;
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < M; ++i)
+    for (int g = 0; g < nb; ++g) {
+      double num = 0.0, den = 0.0;
+      for (int jj = 0; jj < G; ++jj) {
+        int64_t j = (int64_t)g * G + jj;
+        double R = q[i * N + j] * b[j];
+        num += p->W[i * N + j] * R;
+        den += R * R;
+      }
+      double v = (den == 0.0) ? NAN : num / den;
+      if (raw) raw[i * nb + g] = v;
+      astored[i * nb + g] = (den == 0.0) ? 1.0 : project_a(p, v);
+    }
+}
+
+/*
+ * Column update with codes fixed ([R5] "Core equations": with S = D_a Q̂,
+ * b_j <- Proj_Fb( sum_i W_ij S_ij / sum_i S_ij^2 ), scale 1 for an all-zero
+ * code slice).  Column sums run over i ascending; the loop nest walks rows in
+ * the outer loop so memory is read row by row, which does not change the
+ * per-column summation order.
+ */
+void dqo_col_update_impl(const problem* p, const double* q, const double* astored, double* b, double* raw) {
+  int64_t M = p->M, N = p->N;
+  const int64_t CH = 256;
+  int64_t nch = (N + CH - 1) / CH;
+#pragma omp parallel for schedule(static)
+  for (int64_t c = 0; c < nch; ++c) {
+    double num[256], den[256];
+    int64_t j0 = c * CH, j1 = j0 + CH < N ? j0 + CH : N;
+    for (int64_t j = j0; j < j1; ++j) num[j - j0] = den[j - j0] = 0.0;
+    for (int64_t i = 0; i < M; ++i)
+      for (int64_t j = j0; j < j1; ++j) {
+        double S = a_value(p, astored[i * p->nb + j / p->G]) * q[i * N + j];
+        num[j - j0] += p->W[i * N + j] * S;
+        den[j - j0] += S * S;
+      }
+    for (int64_t j = j0; j < j1; ++j) {
+      double d = den[j - j0];
+      double v = (d == 0.0) ? NAN : num[j - j0] / d;
+      if (raw) raw[j] = v;
+      b[j] = (d == 0.0) ? 1.0 : dqo_project(p->col_kind, v);
+    }
+  }
+}
+
+/* reconstruction MSE (1/MN) sum (W - a q b)^2: rows summed in order, each row
+ * summed over j ascending. */
+double dqo_mse_impl(const problem* p, const double* q, const double* astored, const double* b) {
+  int64_t M = p->M, N = p->N;
+  double* rows = (double*)malloc(sizeof(double) * (size_t)M);
+  if (!rows) return NAN;
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < M; ++i) {
+    double s = 0.0;
+    for (int64_t j = 0; j < N; ++j) {
+      double r = p->W[i * N + j] - a_value(p, astored[i * p->nb + j / p->G]) * q[i * N + j] * b[j];
+      s += r * r;
+    }
+    rows[i] = s;
+  }
+  double tot = 0.0;
+  for (int64_t i = 0; i < M; ++i) tot += rows[i];
+  free(rows);
+  return tot / ((double)M * (double)N);
+}
+
+/* Absmax RTN init ([T4] absmax; [P2] §3 symmetric scale; spec config:
+ * beta = 1).  NVFP4 first fixes s_T = fp32(amax / (6*448)). */
+static void init_scales(problem* p, double* astored, double* b) {
+  int64_t M = p->M, N = p->N;
+  if (p->fmt == DQO_NVFP4) {
+    double amax = 0.0;
+    for (int64_t k = 0; k < M * N; ++k)
+      if (fabs(p->W[k]) > amax) amax = fabs(p->W[k]);
+    if (amax == 0.0) {
+      p->sT = 1.0;
+    } else {
+      float s = (float)(amax / 2688.0);
+      if (s == 0.0f) s = ldexpf(1.0f, -149); /* nearest positive fp32 */
+      p->sT = (double)s;
+    }
+  } else {
+    p->sT = 1.0;
+  }
+  double qmax = qmax_of(p->fmt);
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < M; ++i)
+    for (int g = 0; g < p->nb; ++g) {
+      double m = dqo_absmax_scale(p->W + i * N + (int64_t)g * p->G, p->G, 1.0);
+      astored[i * p->nb + g] = (m == 0.0) ? 1.0 : project_a(p, m / qmax);
+    }
+  for (int64_t j = 0; j < N; ++j) b[j] = 1.0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Public oracle entry points                                                */
+
+static int load_problem(problem* p, const void* W, int wdt, int64_t M, int64_t N, int fmt, int G, int col_dt,
+                        double** Wd_out) {
+  if (!W || M <= 0 || N <= 0 || G <= 0 || N % G != 0 || N % 2 != 0) return DQO_EINVAL;
+  if (fmt < 0 || fmt > 2 || (col_dt != DQO_F16 && col_dt != DQO_BF16)) return DQO_EINVAL;
+  double* Wd = (double*)malloc(sizeof(double) * (size_t)(M * N));
+  if (!Wd) return DQO_ENOMEM;
+  int bad = 0;
+  for (int64_t k = 0; k < M * N; ++k) {
+    double v;
+    if (wdt == DQO_F32) {
+      v = ((const float*)W)[k];
+    } else if (wdt == DQO_BF16) {
+      uint32_t u = (uint32_t)((const uint16_t*)W)[k] << 16;
+      float f;
+      memcpy(&f, &u, 4);
+      v = f;
+    } else {
+      uint16_t h = ((const uint16_t*)W)[k];
+      int s = h >> 15, e = (h >> 10) & 31, m = h & 1023;
+      if (e == 31) v = m ? NAN : INFINITY;
+      else if (e == 0) v = ldexp((double)m, -24);
+      else v = ldexp((double)(m + 1024), e - 25);
+      if (s) v = -v;
+    }
+    if (!isfinite(v)) bad = 1;
+    Wd[k] = v;
+  }
+  if (bad) {
+    free(Wd);
+    return DQO_ENONFINITE;
+  }
+  p->M = M;
+  p->N = N;
+  p->fmt = fmt;
+  p->G = G;
+  p->nb = (int)(N / G);
+  p->col_kind = (col_dt == DQO_F16) ? DQO_PROJ_F16 : DQO_PROJ_BF16;
+  p->sT = 1.0;
+  p->W = Wd;
+  *Wd_out = Wd;
+  return DQO_OK;
+}
+
+static void pack_codes(const problem* p, const double* q, uint8_t* codes) {
+  int64_t M = p->M, N = p->N;
+  for (int64_t i = 0; i < M; ++i)
+    for (int64_t j = 0; j < N; j += 2) {
+      uint8_t lo, hi;
+      if (p->fmt == DQO_NVFP4) {
+        lo = e2m1_nibble(q[i * N + j]);
+        hi = e2m1_nibble(q[i * N + j + 1]);
+      } else {
+        lo = (uint8_t)((int)q[i * N + j] & 0xF);
+        hi = (uint8_t)((int)q[i * N + j + 1] & 0xF);
+      }
+      codes[(i * N + j) / 2] = (uint8_t)(lo | (hi << 4));
+    }
+}
+
+/*
+ * The whole solver ([R5] flowchart and "Core equations"; [P2] §4.3, §5.3):
+ *   init (absmax RTN, b = 1); q = Q(W/(a b)); mse[0]
+ *   for t = 1..iters:
+ *     row update (codes fixed) -> project -> requantize
+ *     column update (codes fixed) -> project -> requantize; mse[t]
+ * Outputs (any may be NULL except mse when iters >= 0 is wanted):
+ *   codes      [M][N/2] packed nibbles, even column in the low nibble
+ *   a_out      [M][N/G] stored block scale values (fp16 value / 2^k / E4M3 e)
+ *   b_out      [N] column inverse scales
+ *   sT_out     NVFP4 tensor scale (1 for the other formats)
+ *   mse        [iters+1]
+ *   q_out      [M][N] final grid values
+ *   trace_a    [(iters+1)][M][N/G] block scales after init and each iteration
+ *   trace_b    [(iters+1)][N]
+ */
+int dqo_solve(const void* W, int wdt, int64_t M, int64_t N, int fmt, int G, int iters, int col_dt, uint8_t* codes,
+              double* a_out, double* b_out, double* sT_out, double* mse, double* q_out, double* trace_a,
+              double* trace_b) {
+  if (iters < 0) return DQO_EINVAL;
+  problem p;
+  double* Wd = NULL;
+  int st = load_problem(&p, W, wdt, M, N, fmt, G, col_dt, &Wd);
+  if (st != DQO_OK) return st;
+  int64_t nA = M * p.nb;
+  double* a = (double*)malloc(sizeof(double) * (size_t)nA);
+  double* b = (double*)malloc(sizeof(double) * (size_t)N);
+  double* q = (double*)malloc(sizeof(double) * (size_t)(M * N));
+  if (!a || !b || !q) {
+    free(a);
+    free(b);
+    free(q);
+    free(Wd);
+    return DQO_ENOMEM;
+  }
+  init_scales(&p, a, b);
+  dqo_requant_impl(&p, a, b, q);
+  if (mse) mse[0] = dqo_mse_impl(&p, q, a, b);
+  if (trace_a) memcpy(trace_a, a, sizeof(double) * (size_t)nA);
+  if (trace_b) memcpy(trace_b, b, sizeof(double) * (size_t)N);
+  for (int t = 1; t <= iters; ++t) {
+    dqo_row_update_impl(&p, q, b, a, NULL);
+    dqo_requant_impl(&p, a, b, q);
+    dqo_col_update_impl(&p, q, a, b, NULL);
+    dqo_requant_impl(&p, a, b, q);
+    if (mse) mse[t] = dqo_mse_impl(&p, q, a, b);
+    if (trace_a) memcpy(trace_a + (size_t)t * nA, a, sizeof(double) * (size_t)nA);
+    if (trace_b) memcpy(trace_b + (size_t)t * N, b, sizeof(double) * (size_t)N);
+  }
+  if (codes) pack_codes(&p, q, codes);
+  if (a_out) memcpy(a_out, a, sizeof(double) * (size_t)nA);
+  if (b_out) memcpy(b_out, b, sizeof(double) * (size_t)N);
+  if (sT_out) *sT_out = p.sT;
+  if (q_out) memcpy(q_out, q, sizeof(double) * (size_t)(M * N));
+  free(a);
+  free(b);
+  free(q);
+  free(Wd);
+  return DQO_OK;
+}
+
+/* RTN = the solver's initial iterate ([R5]: RTN with beta = 1 is the start). */
+int dqo_rtn(const void* W, int wdt, int64_t M, int64_t N, int fmt, int G, int col_dt, uint8_t* codes, double* a_out,
+            double* b_out, double* sT_out, double* mse0) {
+  return dqo_solve(W, wdt, M, N, fmt, G, 0, col_dt, codes, a_out, b_out, sT_out, mse0, NULL, NULL, NULL);
+}
+
+/*
+ * Single steps from a given state, for pinning each step on its own and for
+ * checking a GPU iterate against one oracle iteration.  astored holds stored
+ * block-scale values (E4M3 e for NVFP4), sT the NVFP4 tensor scale.
+ * mode: 0 = requantize -> q_out
+ *       1 = row update from q_in  -> astored (in place), raw_out
+ *       2 = column update from q_in -> b (in place), raw_out
+ *       3 = one full BCD iteration from (astored, b): row update, requantize,
+ *           column update, requantize -> astored, b, q_out (the codes q is
+ *           recomputed from the given state first)
+ *       4 = reconstruction MSE of (q_in, astored, b) -> *mse_out
+ */
+int dqo_step(const void* W, int wdt, int64_t M, int64_t N, int fmt, int G, int col_dt, double sT, int mode,
+             double* astored, double* b, const double* q_in, double* q_out, double* raw_out, double* mse_out) {
+  problem p;
+  double* Wd = NULL;
+  int st = load_problem(&p, W, wdt, M, N, fmt, G, col_dt, &Wd);
+  if (st != DQO_OK) return st;
+  p.sT = (fmt == DQO_NVFP4) ? sT : 1.0;
+  st = DQO_OK;
+  if (mode == 0) {
+    dqo_requant_impl(&p, astored, b, q_out);
+  } else if (mode == 1) {
+    dqo_row_update_impl(&p, q_in, b, astored, raw_out);
+  } else if (mode == 2) {
+    dqo_col_update_impl(&p, q_in, astored, b, raw_out);
+  } else if (mode == 3) {
+    double* q = (double*)malloc(sizeof(double) * (size_t)(M * N));
+    if (!q) {
+      free(Wd);
+      return DQO_ENOMEM;
+    }
+    dqo_requant_impl(&p, astored, b, q);
+    dqo_row_update_impl(&p, q, b, astored, NULL);
+    dqo_requant_impl(&p, astored, b, q);
+    dqo_col_update_impl(&p, q, astored, b, NULL);
+    dqo_requant_impl(&p, astored, b, q);
+    if (q_out) memcpy(q_out, q, sizeof(double) * (size_t)(M * N));
+    free(q);
+  } else if (mode == 4) {
+    *mse_out = dqo_mse_impl(&p, q_in, astored, b);
+  } else {
+    st = DQO_EINVAL;
+  }
+  free(Wd);
+  return st;
+}
+
+/* Storage bit patterns of admissible values: fp16 / bf16 (16-bit), E4M3 and
+ * E8M0 (8-bit).  v must be admissible (checked by the caller). */
+uint32_t dqo_encode(int kind, double v) {
+  if (kind == DQO_PROJ_F16) return encode_float_bits(v, 10, -14, 5);
+  if (kind == DQO_PROJ_BF16) return encode_float_bits(v, 7, -126, 8);
+  if (kind == DQO_PROJ_E4M3) return encode_float_bits(v, 3, -6, 4);
+  int e;
+  frexp(v, &e);
+  return (uint32_t)(e - 1 + 127);
+}
+
+/* grid quantizer of a format on one value (for pins) -> grid value */
+double dqo_quant_value(int fmt, double w, double ab) {
+  if (fmt == DQO_NVFP4) return E2M1_GRID[dqo_quant_index(w, ab, E2M1_GRID, E2M1_EVEN, 15)];
+  return INT4_GRID[dqo_quant_index(w, ab, INT4_GRID, INT4_EVEN, 16)];
+}
+
+int dqo_num_threads(void) {
+#ifdef _OPENMP
+  extern int omp_get_max_threads(void);
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
