@@ -1,0 +1,335 @@
+"""Benchmark of the DualQuant BCD solver on B200: weight-elements x BCD-iterations per second.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl dq|reference]
+
+A step is one full solve (RTN init, all BCD iterations, final codes and MSE) of
+the workload's synthetic matrix, already resident in HBM.  L2 is flushed
+(a 512 MB write) before every step, outside the timed events.  With N > 1
+(torchrun) every rank solves its own replica of the workload (no data-path
+collective: the solver does not shard) and the value is the sum over ranks
+divided by the slowest rank's time.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from calibration_free_weight_dualquant_b200 import binding, synth  # noqa: E402
+
+DEFAULT_WORKLOAD = "nvfp4_g16_gateup_14336x4096"
+METRIC = "weight-elems x BCD-iters/sec"
+UNIT = "elem*iter/s"
+L2_FLUSH_BYTES = 512 << 20
+KERNEL_SOURCES = ["calibration_free_weight_dualquant_b200/csrc/dq_solver.cu",
+                  "calibration_free_weight_dualquant_b200/csrc/dq_device.cuh"]
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def profile_traffic(workload: str):
+    """dram bytes per k_iter launch from the committed ncu summary, if it matches the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "k_iter_%s.json" % workload)
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    if d.get("kernel_hash") != kernel_hash():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: torch.device):
+        try:
+            self.dev = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+        except Exception:
+            self.dev = "0"
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.dev, "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self) -> dict:
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in getattr(self, "lines", []):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+        return rank, world, local, dist
+    return 0, 1, 0, None
+
+
+def max_over_ranks(x: float, dist) -> float:
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(dist):
+    if dist is not None:
+        dist.barrier()
+
+
+def cpu_baseline(wl, budget_s: float = 12.0) -> dict:
+    """The oracle, as it stands, on a bounded row sample of the workload on the host cores."""
+    import oracle
+    W = synth.make_weight(wl)
+    cores = oracle.num_threads()
+    rows = max(8, min(wl.rows, 64))
+    while True:
+        Win, wdt = synth.to_oracle_input(W[:rows].contiguous())
+        t0 = time.perf_counter()
+        oracle.solve(Win, wdt, wl.fmt, wl.group, wl.iters, wl.col_dtype)
+        dt = time.perf_counter() - t0
+        if dt > budget_s / 4 or rows >= wl.rows:
+            break
+        rows = min(wl.rows, int(rows * max(2.0, (budget_s / 4) / max(dt, 1e-3))))
+    return {"value": rows * wl.cols * wl.iters / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": "first %d of %d rows x %d cols, all %d iterations, %.2f s" % (rows, wl.rows, wl.cols, wl.iters,
+                                                                                  dt)}
+
+
+def run_reference(args, wl, rank, world, dist):
+    """Reference arm: the CPU oracle on the host cores, one bounded row sample per step."""
+    if rank != 0:
+        return
+    import oracle
+    W = synth.make_weight(wl)
+    rows = max(8, min(wl.rows, args.ref_rows))
+    Win, wdt = synth.to_oracle_input(W[:rows].contiguous())
+    for _ in range(args.warmup):
+        oracle.solve(Win, wdt, wl.fmt, wl.group, wl.iters, wl.col_dtype)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.solve(Win, wdt, wl.fmt, wl.group, wl.iters, wl.col_dtype)
+        times.append(time.perf_counter() - t0)
+    tot = sum(times)
+    value = rows * wl.cols * wl.iters * args.steps / tot
+    cores = oracle.num_threads()
+    sample = "first %d of %d rows x %d cols, all %d iterations per step" % (rows, wl.rows, wl.cols, wl.iters)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(wl, world), "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores,
+                                                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_of(wl, world) -> dict:
+    return {"workload": wl.name, "rows": wl.rows, "cols": wl.cols, "format": wl.fmt, "group": wl.group,
+            "iters": wl.iters, "w_dtype": wl.wdtype, "col_dtype": wl.col_dtype,
+            "l2": "flushed before each step (512 MB write, untimed)", "parallelism": "replicas x%d" % world}
+
+
+def algorithmic_bytes_per_iter(wl) -> int:
+    wsz = 4 if wl.wdtype == "f32" else 2
+    asz = 2 if wl.fmt == "int4" else 1
+    nb = wl.cols // wl.group
+    return wl.rows * wl.cols * wsz + 2 * wl.rows * nb * asz + 2 * wl.cols * 2
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="dq", choices=["dq", "reference"])
+    ap.add_argument("--ref-rows", type=int, default=256)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    wl = synth.WORKLOADS[args.workload]
+    rank, world, local, dist = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            run_reference(args, wl, rank, world, dist)
+            return
+        run_dq(args, wl, rank, world, local, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+def run_dq(args, wl, rank, world, local, dist):
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    binding.load_library()
+    W = synth.make_weight(wl, seed=wl.seed + 7919 * rank)
+    Wd = W.to(dev)
+    T = wl.iters
+    out = binding.alloc_outputs(wl.rows, wl.cols, wl.fmt, wl.group, wl.col_dtype, T, dev)
+    ws = torch.empty(binding.workspace_bytes(wl.rows, wl.cols, wl.fmt, wl.group), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def solve(iters, o=out):
+        binding.dq_solve(Wd, wl.fmt, wl.group, iters, wl.col_dtype, out=o, workspace=ws, stream=stream, check=False)
+
+    def timed(iters, steps, o=out):
+        ts = []
+        for _ in range(steps):
+            flush.fill_(1)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            solve(iters, o)
+            e1.record(stream)
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return ts
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        solve(T)
+    torch.cuda.synchronize()
+    st = binding.load_library().dq_sync_status(ws.data_ptr(), stream.cuda_stream)
+    if st != 0:
+        raise binding.DQError(st, "bench warm-up")
+
+    barrier(dist)
+    torch.cuda.synchronize()
+    with ClockSampler(dev) as clk:
+        step_ms = timed(T, args.steps)
+    torch.cuda.synchronize()
+    barrier(dist)
+    total_ms = max_over_ranks(sum(step_ms), dist)
+
+    # steady-state iteration time of the dominant kernel (k_iter): (t(T) - t(0)) / T, median of runs
+    out0 = binding.alloc_outputs(wl.rows, wl.cols, wl.fmt, wl.group, wl.col_dtype, 0, dev)
+    t0s = timed(0, max(3, args.steps), out0)
+    tTs = step_ms
+    iter_ms = (statistics.median(tTs) - statistics.median(t0s)) / T
+    iter_ms = max_over_ranks(iter_ms, dist)
+
+    # end to end through the public API with host buffers (pinned), copies inside the timed region
+    Wh = W.pin_memory()
+    host_out = binding.alloc_outputs(wl.rows, wl.cols, wl.fmt, wl.group, wl.col_dtype, T, "cpu")
+    for k in host_out:
+        host_out[k] = host_out[k].pin_memory()
+    dws = torch.empty(binding.host_workspace_bytes(wl.rows, wl.cols, W.dtype, wl.fmt, wl.group, T),
+                      dtype=torch.uint8, device=dev)
+    binding.solve(Wh, wl.fmt, wl.group, T, wl.col_dtype, out=host_out, device_workspace=dws)
+    e2e_ms = []
+    for _ in range(max(3, args.steps // 2)):
+        flush.fill_(1)
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        binding.solve(Wh, wl.fmt, wl.group, T, wl.col_dtype, out=host_out, device_workspace=dws)
+        e1.record(stream)
+        e1.synchronize()
+        e2e_ms.append(e0.elapsed_time(e1))
+    e2e_total = max_over_ranks(sum(e2e_ms), dist)
+    nb = binding.output_nbytes(wl.rows, wl.cols, wl.fmt, wl.group, wl.col_dtype)
+    h2d = W.numel() * W.element_size()
+    d2h = nb["codes"] + nb["block_scales"] + nb["col_scales"] + nb["tensor_scale"] + 8 * (T + 1)
+
+    if rank != 0:
+        return
+    elems = wl.rows * wl.cols
+    value = world * elems * T * args.steps / (total_ms * 1e-3)
+    e2e_value = world * elems * T * len(e2e_ms) / (e2e_total * 1e-3)
+    peaks = measured_peaks()
+    alg = algorithmic_bytes_per_iter(wl)
+    achieved = alg / (iter_ms * 1e-3) / 1e9
+    traffic = profile_traffic(wl.name)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32+f64", "data": "synthetic",
+        "config": config_of(wl, world),
+        "final_mse": float(out["mse"][-1].item()),
+        "ms_per_iter": iter_ms,
+        "roofline": {"bound": "hbm", "kernel": "k_iter", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                     "algorithmic_bytes_per_launch": alg, "peak_source": peaks["source"]},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps * (T + 3),
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,218 @@
+"""Thin ctypes binding of ``libdq.so`` (C ABI in ``include/dq.h``).
+
+Argument marshalling only: torch supplies device memory and the current
+stream; every step of the solver runs in the library's CUDA kernels.  There is
+no CPU fallback -- without the built library or a CUDA device every call
+raises :class:`DQError`.
+"""
+from __future__ import annotations
+
+import ctypes
+import enum
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "lib", "libdq.so")
+
+STATUS = {0: "DQ_OK", 1: "DQ_EINVAL", 2: "DQ_EUNSUPPORTED", 3: "DQ_EWORKSPACE", 4: "DQ_ENONFINITE", 5: "DQ_ECUDA"}
+
+
+class Format(enum.IntEnum):
+    INT4 = 0
+    MXINT4 = 1
+    NVFP4 = 2
+
+
+_FMT_NAMES = {"int4": Format.INT4, "mxint4": Format.MXINT4, "nvfp4": Format.NVFP4}
+_DTYPES = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
+_COL_DTYPES = {"f16": torch.float16, "bf16": torch.bfloat16}
+DEFAULT_GROUP = {Format.INT4: 64, Format.MXINT4: 32, Format.NVFP4: 16}
+DEFAULT_COL_DTYPE = {Format.INT4: "f16", Format.MXINT4: "bf16", Format.NVFP4: "bf16"}
+
+
+class DQError(RuntimeError):
+    def __init__(self, status: int, where: str = ""):
+        self.status = status
+        super().__init__("%s%s" % (STATUS.get(status, "status %d" % status), (" in " + where) if where else ""))
+
+
+class _Outputs(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("block_scales", ctypes.c_void_p), ("tensor_scale", ctypes.c_void_p),
+                ("col_scales", ctypes.c_void_p), ("mse", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def load_library():
+    """Load libdq.so (built in-tree by ``build.py``); raise if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise DQError(5, "load_library: %s is not built (run __graft_entry__.build())" % LIB_PATH)
+    lib = ctypes.CDLL(LIB_PATH)
+    I64, I, SZ, P = ctypes.c_int64, ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
+    lib.dq_workspace_bytes.argtypes = [I64, I64, I, I]
+    lib.dq_workspace_bytes.restype = SZ
+    lib.dq_rtn.argtypes = [P, I, I64, I64, I, I, I, ctypes.POINTER(_Outputs), P, SZ, P]
+    lib.dq_rtn.restype = I
+    lib.dq_solve.argtypes = [P, I, I64, I64, I, I, I, I, ctypes.POINTER(_Outputs), P, SZ, P]
+    lib.dq_solve.restype = I
+    lib.dq_sync_status.argtypes = [P, P]
+    lib.dq_sync_status.restype = I
+    lib.dq_host_workspace_bytes.argtypes = [I64, I64, I, I, I, I]
+    lib.dq_host_workspace_bytes.restype = SZ
+    lib.dq_solve_host.argtypes = [P, I, I64, I64, I, I, I, I, ctypes.POINTER(_Outputs), P, SZ, P]
+    lib.dq_solve_host.restype = I
+    lib.dq_status_str.argtypes = [I]
+    lib.dq_status_str.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def _fmt(fmt) -> Format:
+    return _FMT_NAMES[fmt] if isinstance(fmt, str) else Format(fmt)
+
+
+def output_nbytes(rows: int, cols: int, fmt, group: Optional[int] = None, col_dtype: Optional[str] = None) -> dict:
+    """Bytes of each output: packed codes, block scales, column scales (host-side size arithmetic)."""
+    f = _fmt(fmt)
+    g = DEFAULT_GROUP[f] if group is None else group
+    cd = DEFAULT_COL_DTYPE[f] if col_dtype is None else col_dtype
+    return {"codes": rows * cols // 2, "block_scales": rows * (cols // g) * (2 if f == Format.INT4 else 1),
+            "col_scales": cols * 2, "tensor_scale": 4 if f == Format.NVFP4 else 0}
+
+
+def workspace_bytes(rows: int, cols: int, fmt, group: Optional[int] = None) -> int:
+    f = _fmt(fmt)
+    g = DEFAULT_GROUP[f] if group is None else group
+    return int(load_library().dq_workspace_bytes(rows, cols, int(f), g))
+
+
+def alloc_outputs(rows: int, cols: int, fmt, group: int, col_dtype: str, iters: int, device) -> dict:
+    f = _fmt(fmt)
+    nb = cols // group
+    return {
+        "codes": torch.empty((rows, cols // 2), dtype=torch.uint8, device=device),
+        "block_scales": torch.empty((rows, nb), dtype=torch.float16 if f == Format.INT4 else torch.uint8,
+                                    device=device),
+        "tensor_scale": torch.empty(1, dtype=torch.float32, device=device),
+        "col_scales": torch.empty(cols, dtype=_COL_DTYPES[col_dtype], device=device),
+        "mse": torch.empty(iters + 1, dtype=torch.float64, device=device),
+    }
+
+
+def _outputs_struct(out: dict) -> _Outputs:
+    return _Outputs(out["codes"].data_ptr(), out["block_scales"].data_ptr(), out["tensor_scale"].data_ptr(),
+                    out["col_scales"].data_ptr(), out["mse"].data_ptr())
+
+
+def _stream_ptr(stream) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def dq_solve(W: torch.Tensor, fmt, group: Optional[int] = None, iters: int = 0, col_dtype: Optional[str] = None,
+             out: Optional[dict] = None, workspace: Optional[torch.Tensor] = None, stream=None,
+             check: bool = True) -> dict:
+    """Enqueue dq_solve on a CUDA tensor W [rows, cols]; returns the output tensors.
+
+    ``check`` waits for the stream and raises on a device-reported status
+    (non-finite W).  Pass preallocated ``out`` / ``workspace`` to avoid
+    allocations (e.g. when timing)."""
+    lib = load_library()
+    if not W.is_cuda:
+        raise DQError(1, "dq_solve: W must be a CUDA tensor (use solve() for host tensors)")
+    f = _fmt(fmt)
+    g = DEFAULT_GROUP[f] if group is None else group
+    cd = DEFAULT_COL_DTYPE[f] if col_dtype is None else col_dtype
+    rows, cols = W.shape
+    if W.dtype not in _DTYPES or not W.is_contiguous():
+        raise DQError(1, "dq_solve: W must be contiguous f32/bf16/f16")
+    if out is None:
+        out = alloc_outputs(rows, cols, f, g, cd, iters, W.device)
+    if workspace is None:
+        nbytes = lib.dq_workspace_bytes(rows, cols, int(f), g)
+        if nbytes == 0:
+            raise DQError(1, "dq_workspace_bytes")
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
+    o = _outputs_struct(out)
+    st = lib.dq_solve(W.data_ptr(), _DTYPES[W.dtype], rows, cols, int(f), g, iters, 0 if cd == "f32" else
+                      (2 if cd == "f16" else 1), ctypes.byref(o), workspace.data_ptr(), workspace.numel(),
+                      _stream_ptr(stream))
+    if st != 0:
+        raise DQError(st, "dq_solve")
+    if check:
+        st = lib.dq_sync_status(workspace.data_ptr(), _stream_ptr(stream))
+        if st != 0:
+            raise DQError(st, "dq_solve (device)")
+    out["workspace"] = workspace
+    return out
+
+
+def dq_rtn(W: torch.Tensor, fmt, group: Optional[int] = None, col_dtype: Optional[str] = None, **kw) -> dict:
+    """Absmax RTN (beta = 1) through the library's dq_rtn entry point."""
+    lib = load_library()
+    f = _fmt(fmt)
+    g = DEFAULT_GROUP[f] if group is None else group
+    cd = DEFAULT_COL_DTYPE[f] if col_dtype is None else col_dtype
+    rows, cols = W.shape
+    out = kw.get("out") or alloc_outputs(rows, cols, f, g, cd, 0, W.device)
+    ws = kw.get("workspace")
+    if ws is None:
+        ws = torch.empty(lib.dq_workspace_bytes(rows, cols, int(f), g), dtype=torch.uint8, device=W.device)
+    o = _outputs_struct(out)
+    stream = kw.get("stream")
+    st = lib.dq_rtn(W.data_ptr(), _DTYPES[W.dtype], rows, cols, int(f), g, 2 if cd == "f16" else 1, ctypes.byref(o),
+                    ws.data_ptr(), ws.numel(), _stream_ptr(stream))
+    if st != 0:
+        raise DQError(st, "dq_rtn")
+    st = lib.dq_sync_status(ws.data_ptr(), _stream_ptr(stream))
+    if st != 0:
+        raise DQError(st, "dq_rtn (device)")
+    return out
+
+
+def host_workspace_bytes(rows: int, cols: int, w_dtype: torch.dtype, fmt, group: int, iters: int) -> int:
+    return int(load_library().dq_host_workspace_bytes(rows, cols, _DTYPES[w_dtype], int(_fmt(fmt)), group, iters))
+
+
+def solve(W: torch.Tensor, fmt="nvfp4", group: Optional[int] = None, iters: int = 15,
+          col_dtype: Optional[str] = None, out: Optional[dict] = None, device_workspace: Optional[torch.Tensor] = None,
+          stream=None) -> dict:
+    """User-level solve.  A host (CPU) W goes through ``dq_solve_host``: the copy
+    to the device, the solve and the copy of the outputs back all happen inside
+    the library call, and host output tensors are returned.  A CUDA W goes
+    through ``dq_solve``."""
+    f = _fmt(fmt)
+    g = DEFAULT_GROUP[f] if group is None else group
+    cd = DEFAULT_COL_DTYPE[f] if col_dtype is None else col_dtype
+    if W.is_cuda:
+        return dq_solve(W, f, g, iters, cd, out=out, stream=stream)
+    lib = load_library()
+    rows, cols = W.shape
+    if W.dtype not in _DTYPES or not W.is_contiguous():
+        raise DQError(1, "solve: W must be contiguous f32/bf16/f16")
+    if out is None:
+        out = alloc_outputs(rows, cols, f, g, cd, iters, "cpu")
+    if device_workspace is None:
+        nbytes = lib.dq_host_workspace_bytes(rows, cols, _DTYPES[W.dtype], int(f), g, iters)
+        if nbytes == 0:
+            raise DQError(1, "dq_host_workspace_bytes")
+        device_workspace = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    o = _outputs_struct(out)
+    st = lib.dq_solve_host(W.data_ptr(), _DTYPES[W.dtype], rows, cols, int(f), g, iters, 2 if cd == "f16" else 1,
+                           ctypes.byref(o), device_workspace.data_ptr(), device_workspace.numel(),
+                           _stream_ptr(stream))
+    if st != 0:
+        raise DQError(st, "dq_solve_host")
+    return out
+
+
+def rtn(W: torch.Tensor, fmt="nvfp4", group: Optional[int] = None, col_dtype: Optional[str] = None) -> dict:
+    """User-level absmax RTN (the 0-iteration solve)."""
+    return solve(W, fmt, group, 0, col_dtype)

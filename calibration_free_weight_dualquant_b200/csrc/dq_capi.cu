@@ -1,0 +1,240 @@
+// dq_capi.cu -- the C ABI of libdq.so (declared in include/dq.h): host-side
+// validation, workspace layout and the stream-ordered launch of the solver.
+#include "dq.h"
+#include "dq_internal.h"
+
+#include <cstring>
+
+namespace {
+
+using dq::Problem;
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct Plan {
+  int TS, n_strips, P, segmax, nb;
+  int64_t L;
+  size_t off_counters, off_col_part, off_cta_part, total;
+};
+
+// Argument checks that do not touch memory.  Returns DQ_OK or an error code.
+int check_shape(int64_t rows, int64_t cols, int format, int group) {
+  if (rows <= 0 || cols <= 0 || (cols & 1) || group <= 0) return DQ_EINVAL;
+  if (format < DQ_INT4 || format > DQ_NVFP4) return DQ_EINVAL;
+  if (cols % group != 0) return DQ_EINVAL;
+  if (format == DQ_MXINT4 && group != 32) return DQ_EUNSUPPORTED;
+  if (format == DQ_NVFP4 && group != 16) return DQ_EUNSUPPORTED;
+  // a block spans group/8 lanes of a warp: a power of two from 1 to 32
+  if (group < 8 || group > dq::kStripMax || (group & (group - 1)) != 0) return DQ_EUNSUPPORTED;
+  if (rows > ((int64_t)1 << 40) / cols) return DQ_EUNSUPPORTED;  // keeps all index products in int64 range
+  if (cols / group > INT32_MAX) return DQ_EUNSUPPORTED;
+  return DQ_OK;
+}
+
+int device_sms(int* sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DQ_ECUDA;
+  if (cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return DQ_ECUDA;
+  return DQ_OK;
+}
+
+// Schedule and workspace layout for the current device.
+int make_plan(int64_t M, int64_t N, int group, Plan* pl) {
+  int sms = 0;
+  int st = device_sms(&sms);
+  if (st != DQ_OK) return st;
+  pl->nb = (int)(N / group);
+  pl->TS = (dq::kStripMax / group) * group;
+  pl->n_strips = (int)((N + pl->TS - 1) / pl->TS);
+  pl->L = (int64_t)pl->n_strips * M;
+  int64_t P = (int64_t)sms * dq::kCtasPerSm;
+  int64_t byrows = pl->L / dq::kMinRowsPerCta;
+  if (byrows < P) P = byrows < 1 ? 1 : byrows;
+  pl->P = (int)P;
+  const int64_t len = (pl->L + P - 1) / P;
+  pl->segmax = (int)((len + M - 1) / M + 1);
+  size_t off = align_up(sizeof(dq::WsHeader));
+  pl->off_counters = off;
+  off += align_up(sizeof(unsigned) * (size_t)pl->n_strips);
+  pl->off_col_part = off;
+  off += align_up(sizeof(double2) * (size_t)pl->P * (size_t)pl->segmax * (size_t)pl->TS);
+  pl->off_cta_part = off;
+  off += align_up(sizeof(double) * (size_t)pl->P);
+  pl->total = off;
+  return DQ_OK;
+}
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+int check_outputs(const dq_outputs* out, int format, int col_dtype) {
+  if (!out || !out->codes || !out->block_scales || !out->col_scales || !out->mse) return DQ_EINVAL;
+  if (format == DQ_NVFP4 && !out->tensor_scale) return DQ_EINVAL;
+  if (!aligned(out->codes, 4) || !aligned(out->block_scales, 2) || !aligned(out->col_scales, 2) ||
+      !aligned(out->mse, 8) || (out->tensor_scale && !aligned(out->tensor_scale, 4)))
+    return DQ_EINVAL;
+  (void)col_dtype;
+  return DQ_OK;
+}
+
+int solve_impl(const void* W, int w_dtype, int64_t rows, int64_t cols, int format, int group, int iters,
+               int col_dtype, const dq_outputs* out, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  int st = check_shape(rows, cols, format, group);
+  if (st != DQ_OK) return st;
+  if (w_dtype < DQ_F32 || w_dtype > DQ_F16) return DQ_EINVAL;
+  if (col_dtype != DQ_F16 && col_dtype != DQ_BF16) return DQ_EUNSUPPORTED;
+  if (iters < 0) return DQ_EINVAL;
+  if (!W || !aligned(W, 16)) return DQ_EINVAL;
+  st = check_outputs(out, format, col_dtype);
+  if (st != DQ_OK) return st;
+  if (!workspace || !aligned(workspace, kAlign)) return DQ_EINVAL;
+  Plan pl;
+  st = make_plan(rows, cols, group, &pl);
+  if (st != DQ_OK) return st;
+  if (workspace_bytes < pl.total) return DQ_EWORKSPACE;
+
+  char* ws = static_cast<char*>(workspace);
+  Problem p;
+  std::memset(&p, 0, sizeof(p));
+  p.W = W;
+  p.wdt = w_dtype;
+  p.fmt = format;
+  p.G = group;
+  p.col_dt = col_dtype;
+  p.M = rows;
+  p.N = cols;
+  p.nb = pl.nb;
+  p.TS = pl.TS;
+  p.n_strips = pl.n_strips;
+  p.P = pl.P;
+  p.segmax = pl.segmax;
+  p.L = pl.L;
+  p.codes = out->codes;
+  p.a_store = out->block_scales;
+  p.b_store = out->col_scales;
+  p.sT_out = out->tensor_scale;
+  p.mse = out->mse;
+  p.hdr = reinterpret_cast<dq::WsHeader*>(ws);
+  p.strip_counter = reinterpret_cast<unsigned*>(ws + pl.off_counters);
+  p.col_part = reinterpret_cast<double2*>(ws + pl.off_col_part);
+  p.cta_part = reinterpret_cast<double*>(ws + pl.off_cta_part);
+
+  // header and arrival counters start at zero; the partial buffers need no init
+  if (cudaMemsetAsync(ws, 0, pl.off_col_part, stream) != cudaSuccess) return DQ_ECUDA;
+  if (dq::launch_solve(p, iters, pl.P, stream) != cudaSuccess) return DQ_ECUDA;
+  return DQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t dq_workspace_bytes(int64_t rows, int64_t cols, int format, int group) {
+  if (check_shape(rows, cols, format, group) != DQ_OK) return 0;
+  Plan pl;
+  if (make_plan(rows, cols, group, &pl) != DQ_OK) return 0;
+  return pl.total;
+}
+
+int dq_solve(const void* W, int w_dtype, int64_t rows, int64_t cols, int format, int group, int iters, int col_dtype,
+             const dq_outputs* out, void* workspace, size_t workspace_bytes, void* stream) {
+  return solve_impl(W, w_dtype, rows, cols, format, group, iters, col_dtype, out, workspace, workspace_bytes,
+                    static_cast<cudaStream_t>(stream));
+}
+
+int dq_rtn(const void* W, int w_dtype, int64_t rows, int64_t cols, int format, int group, int col_dtype,
+           const dq_outputs* out, void* workspace, size_t workspace_bytes, void* stream) {
+  return solve_impl(W, w_dtype, rows, cols, format, group, 0, col_dtype, out, workspace, workspace_bytes,
+                    static_cast<cudaStream_t>(stream));
+}
+
+int dq_sync_status(const void* workspace, void* stream) {
+  if (!workspace) return DQ_EINVAL;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DQ_ECUDA;
+  unsigned flags = 0;
+  if (cudaMemcpy(&flags, workspace, sizeof(flags), cudaMemcpyDeviceToHost) != cudaSuccess) return DQ_ECUDA;
+  return (flags & dq::kFlagNonFinite) ? DQ_ENONFINITE : DQ_OK;
+}
+
+static size_t wsize(int dt) { return dt == DQ_F32 ? 4 : 2; }
+
+size_t dq_host_workspace_bytes(int64_t rows, int64_t cols, int w_dtype, int format, int group, int iters) {
+  if (w_dtype < DQ_F32 || w_dtype > DQ_F16 || iters < 0) return 0;
+  size_t solver = dq_workspace_bytes(rows, cols, format, group);
+  if (solver == 0) return 0;
+  const size_t nb = (size_t)(cols / group);
+  size_t tot = align_up((size_t)rows * cols * wsize(w_dtype));
+  tot += align_up((size_t)rows * cols / 2);
+  tot += align_up((size_t)rows * nb * (format == DQ_INT4 ? 2 : 1));
+  tot += kAlign;  // tensor scale
+  tot += align_up((size_t)cols * 2);
+  tot += align_up((size_t)(iters + 1) * sizeof(double));
+  return tot + solver;
+}
+
+int dq_solve_host(const void* W_host, int w_dtype, int64_t rows, int64_t cols, int format, int group, int iters,
+                  int col_dtype, const dq_outputs* out_host, void* device_workspace, size_t device_workspace_bytes,
+                  void* stream) {
+  int st = check_shape(rows, cols, format, group);
+  if (st != DQ_OK) return st;
+  if (!W_host || w_dtype < DQ_F32 || w_dtype > DQ_F16 || iters < 0) return DQ_EINVAL;
+  if (!out_host || !device_workspace || !aligned(device_workspace, kAlign)) return DQ_EINVAL;
+  const size_t need = dq_host_workspace_bytes(rows, cols, w_dtype, format, group, iters);
+  if (need == 0) return DQ_ECUDA;
+  if (device_workspace_bytes < need) return DQ_EWORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* base = static_cast<char*>(device_workspace);
+  const size_t nb = (size_t)(cols / group);
+  const size_t bytes_w = (size_t)rows * cols * wsize(w_dtype);
+  const size_t bytes_codes = (size_t)rows * cols / 2;
+  const size_t bytes_a = (size_t)rows * nb * (format == DQ_INT4 ? 2 : 1);
+  const size_t bytes_b = (size_t)cols * 2;
+  const size_t bytes_mse = (size_t)(iters + 1) * sizeof(double);
+  char* dW = base;
+  base += align_up(bytes_w);
+  dq_outputs dout;
+  dout.codes = base;
+  base += align_up(bytes_codes);
+  dout.block_scales = base;
+  base += align_up(bytes_a);
+  dout.tensor_scale = reinterpret_cast<float*>(base);
+  base += kAlign;
+  dout.col_scales = base;
+  base += align_up(bytes_b);
+  dout.mse = reinterpret_cast<double*>(base);
+  base += align_up(bytes_mse);
+  void* ws = base;
+  const size_t ws_bytes = device_workspace_bytes - (size_t)(base - static_cast<char*>(device_workspace));
+
+  if (cudaMemcpyAsync(dW, W_host, bytes_w, cudaMemcpyHostToDevice, s) != cudaSuccess) return DQ_ECUDA;
+  st = solve_impl(dW, w_dtype, rows, cols, format, group, iters, col_dtype, &dout, ws, ws_bytes, s);
+  if (st != DQ_OK) return st;
+  if (out_host->codes && cudaMemcpyAsync(out_host->codes, dout.codes, bytes_codes, cudaMemcpyDeviceToHost, s))
+    return DQ_ECUDA;
+  if (out_host->block_scales &&
+      cudaMemcpyAsync(out_host->block_scales, dout.block_scales, bytes_a, cudaMemcpyDeviceToHost, s))
+    return DQ_ECUDA;
+  if (out_host->tensor_scale &&
+      cudaMemcpyAsync(out_host->tensor_scale, dout.tensor_scale, sizeof(float), cudaMemcpyDeviceToHost, s))
+    return DQ_ECUDA;
+  if (out_host->col_scales &&
+      cudaMemcpyAsync(out_host->col_scales, dout.col_scales, bytes_b, cudaMemcpyDeviceToHost, s))
+    return DQ_ECUDA;
+  if (out_host->mse && cudaMemcpyAsync(out_host->mse, dout.mse, bytes_mse, cudaMemcpyDeviceToHost, s))
+    return DQ_ECUDA;
+  return dq_sync_status(ws, stream);
+}
+
+const char* dq_status_str(int status) {
+  switch (status) {
+    case DQ_OK: return "DQ_OK";
+    case DQ_EINVAL: return "DQ_EINVAL: invalid argument";
+    case DQ_EUNSUPPORTED: return "DQ_EUNSUPPORTED: unsupported format/group/dtype combination";
+    case DQ_EWORKSPACE: return "DQ_EWORKSPACE: workspace too small";
+    case DQ_ENONFINITE: return "DQ_ENONFINITE: W holds Inf or NaN";
+    case DQ_ECUDA: return "DQ_ECUDA: CUDA runtime error";
+  }
+  return "unknown dq_status";
+}
+
+}  // extern "C"

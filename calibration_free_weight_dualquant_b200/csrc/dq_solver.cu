@@ -1,0 +1,385 @@
+// dq_solver.cu -- CUDA kernels (sm_100a) of the DualQuant dual-scale BCD solver.
+//
+// Method (DualQuant reproduction README, flowchart and "Core equations";
+// DualQuant arXiv 2610.13767 summary, §4.3 and App. B):
+//   init  : b = 1, a = Proj_Fa(absmax(block)/qmax)  (absmax round-to-nearest)
+//   iterate t = 1..T:
+//     q  = Q(W/(a b))                 codes of the current iterate
+//     a <- Proj_Fa(sum W q b / sum (q b)^2)   per block, codes fixed
+//     q' = Q(W/(a b))                 requantize after the block update
+//     b <- Proj_Fb(sum W a q' / sum (a q')^2) per column, codes fixed
+//   scale 1 for an all-zero code slice; codes are a function of (W, a, b).
+//
+// HBM layout and schedule.  One pass over W per iteration: kernel k_iter
+// fuses, for every element, the requantization of the current iterate, the
+// block sums (reduced over the G/8 lanes of a block with xor shuffles, which
+// give every lane the bit-identical total), the block update, the
+// requantization with the new block scale and the column sums.  Columns are
+// cut into strips of TS <= 256 columns; the (strip, row) pairs are laid out
+// strip-major and split evenly into P contiguous ranges, one per CTA
+// (P = 2 CTAs per SM), so every CTA streams the same number of rows.  A CTA
+// keeps its columns' sums in registers, reduces them over its 8 warps in
+// shared memory and writes one fp64 partial per (CTA, strip) it touched; the
+// last CTA to finish a strip (atomic ticket, no waiting) sums the partials of
+// that strip in CTA order -- a fixed order, so the result is deterministic --
+// and writes the new column scales.  The reconstruction MSE of the iterate
+// entering iteration t is accumulated from the block sums,
+// sum (W - a q b)^2 = sum W^2 - sum_blocks (2 a num - a^2 den),
+// per CTA, then summed in CTA order by the last CTA.
+#include "dq_device.cuh"
+#include "dq_internal.h"
+
+namespace dq {
+
+__device__ __forceinline__ int64_t cta_of(int64_t u, int64_t P, int64_t L) { return ((u + 1) * P - 1) / L; }
+__device__ __forceinline__ int64_t range_begin(int64_t k, int64_t P, int64_t L) { return k * L / P; }
+
+// Fast-path scale factors are trusted when they stay inside [2^-100, 2^100]:
+// then every product that lands near a rounding boundary is a normal fp32
+// number and the relative error bound behind kGuard holds.
+__device__ __forceinline__ bool in_range(float x) { return x >= 0x1p-100f && x <= 0x1p100f; }
+
+// Last-arriving CTA election for a counter: every thread has already issued its
+// writes; returns true in all threads of the CTA that arrived last.
+__device__ __forceinline__ bool arrive_last(unsigned* counter, unsigned expected, int* s_flag) {
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const unsigned prev = atomicAdd(counter, 1u);
+    *s_flag = (prev == expected - 1u) ? 1 : 0;
+  }
+  __syncthreads();
+  const bool last = *s_flag != 0;
+  if (last) __threadfence();
+  return last;
+}
+
+// ---------------------------------------------------------------------------
+// Statistics pass: non-finite check, max |W|, sum W^2.
+template <int WDT>
+__global__ void __launch_bounds__(kThreads) k_stats(Problem p) {
+  __shared__ double red[kThreads];
+  __shared__ int s_last;
+  const int64_t nchunks = p.M * p.N / 8;
+  float amax = 0.f;
+  double s2 = 0.0;
+  bool bad = false;
+  for (int64_t c = (int64_t)blockIdx.x * kThreads + threadIdx.x; c < nchunks; c += (int64_t)gridDim.x * kThreads) {
+    float w[8];
+    load8<WDT>(p.W, c * 8, w);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      bad |= !isfinite(w[k]);
+      amax = fmaxf(amax, fabsf(w[k]));
+      s2 = fma((double)w[k], (double)w[k], s2);
+    }
+  }
+  if (bad) atomicOr(&p.hdr->flags, kFlagNonFinite);
+  // max of non-negative floats = max of their bit patterns (order independent)
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((threadIdx.x & 31) == 0 && isfinite(amax)) atomicMax(&p.hdr->amax_bits, __float_as_uint(amax));
+  red[threadIdx.x] = s2;
+  __syncthreads();
+  for (int o = kThreads / 2; o > 0; o >>= 1) {
+    if (threadIdx.x < o) red[threadIdx.x] += red[threadIdx.x + o];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) p.cta_part[blockIdx.x] = red[0];
+  if (arrive_last(&p.hdr->cta_counter, gridDim.x, &s_last)) {
+    if (threadIdx.x == 0) {
+      double tot = 0.0;
+      for (unsigned k = 0; k < gridDim.x; ++k) tot += __ldcg(&p.cta_part[k]);
+      p.hdr->sumW2 = tot;
+      p.hdr->cta_counter = 0u;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Init: s_T (NVFP4), a = Proj(absmax/qmax) per block (1 for an all-zero
+// block), b = 1.
+template <int FMT, int WDT>
+__global__ void __launch_bounds__(kThreads) k_init(Problem p) {
+  if (p.hdr->flags & kFlagNonFinite) return;
+  double sTd = 1.0;
+  if (FMT == FMT_NVFP4) {
+    const float amax = __uint_as_float(p.hdr->amax_bits);
+    float s = amax == 0.f ? 1.f : __double2float_rn((double)amax / 2688.0);
+    if (s == 0.f) s = 0x1p-149f;
+    sTd = (double)s;
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+      p.hdr->sT = s;
+      if (p.sT_out) *p.sT_out = s;
+    }
+  } else if (blockIdx.x == 0 && threadIdx.x == 0) {
+    p.hdr->sT = 1.f;
+    if (p.sT_out) *p.sT_out = 1.f;
+  }
+  const double qmax = FMT == FMT_NVFP4 ? 6.0 : 7.0;
+  const int64_t nblocks = p.M * p.nb;
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  for (int64_t blk = (int64_t)blockIdx.x * kThreads + threadIdx.x; blk < nblocks; blk += stride) {
+    const int64_t i = blk / p.nb, g = blk % p.nb;
+    const int64_t off = i * p.N + g * p.G;
+    float m = 0.f;
+    for (int c = 0; c < p.G; c += 8) {
+      float w[8];
+      load8<WDT>(p.W, off + c, w);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) m = fmaxf(m, fabsf(w[k]));
+    }
+    const double a = (m == 0.f) ? 1.0 : a_project<FMT>((double)m / qmax, sTd);
+    a_encode<FMT>(p.a_store, blk, a);
+  }
+  for (int64_t j = (int64_t)blockIdx.x * kThreads + threadIdx.x; j < p.N; j += stride) b_encode(p.b_store, p.col_dt, j, 1.0);
+}
+
+// ---------------------------------------------------------------------------
+// One BCD iteration (see the file header).  Writes mse[t-1].
+template <int FMT, int WDT>
+__global__ void __launch_bounds__(kThreads, 2) k_iter(Problem p, int t) {
+  if (p.hdr->flags & kFlagNonFinite) return;
+  __shared__ double2 red[kWarps][kStripMax];
+  __shared__ double mred[kThreads];
+  __shared__ int s_last;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int lpb = p.G / 8;  // lanes per block
+  const float sT = p.hdr->sT;
+  const double sTd = (double)sT;
+  const float isT = FMT == FMT_NVFP4 ? 1.f / sT : 1.f;
+  const bool sT_ok = FMT != FMT_NVFP4 || in_range(isT);
+  const int64_t k = blockIdx.x;
+  const int64_t u_begin = range_begin(k, p.P, p.L), u_end = range_begin(k + 1, p.P, p.L);
+  const int64_t s_first = u_begin / p.M;
+  double mse_acc = 0.0;
+
+  for (int64_t u = u_begin; u < u_end;) {
+    const int64_t s = u / p.M;
+    const int64_t r0 = u - s * p.M;
+    const int64_t r1 = min(p.M, r0 + (u_end - u));
+    const int64_t c0 = s * p.TS;
+    const int width = (int)min((int64_t)p.TS, p.N - c0);
+    const bool active = lane * 8 < width;
+    const int64_t col = c0 + lane * 8;
+
+    float bj[8], cb[8];
+    bool col_ok = sT_ok;
+    double cn[8], cd[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      cn[c] = 0.0;
+      cd[c] = 0.0;
+      bj[c] = 1.f;
+      cb[c] = 1.f;
+    }
+    if (active) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        bj[c] = b_decode(p.b_store, p.col_dt, col + c);
+        cb[c] = __frcp_rn(bj[c]) * isT;
+        col_ok = col_ok && in_range(cb[c]);
+      }
+    }
+
+    for (int64_t r = r0 + warp; r < r1; r += kWarps) {
+      float w[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      float aold = 1.f;
+      const int64_t bidx = r * p.nb + col / p.G;
+      double num = 0.0, den = 0.0;
+      float u8[8];
+      if (active) {
+        load8<WDT>(p.W, r * p.N + col, w);
+        aold = a_decode<FMT>(p.a_store, bidx);
+        const float ia = __frcp_rn(aold);
+        const bool ok = col_ok && in_range(ia);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          u8[c] = w[c] * cb[c];
+          const float q = quant<FMT>(w[c], u8[c], ia, ok, aold, bj[c], sTd);
+          const float qb = q * bj[c];  // exact: <= 15 significant bits
+          const double qbd = (double)qb;
+          num = fma((double)w[c], qbd, num);
+          den = fma(qbd, qbd, den);
+        }
+      }
+      for (int o = 1; o < lpb; o <<= 1) {
+        num += __shfl_xor_sync(0xffffffffu, num, o);
+        den += __shfl_xor_sync(0xffffffffu, den, o);
+      }
+      if (active) {
+        // MSE contribution of this block at the incoming iterate
+        const double aval = FMT == FMT_NVFP4 ? sTd * (double)aold : (double)aold;
+        if ((lane & (lpb - 1)) == 0) mse_acc += aval * (aval * den - 2.0 * num);
+        const double anew_d = den == 0.0 ? 1.0 : a_project<FMT>(num / den, sTd);
+        const float anew = (float)anew_d;  // exact
+        if ((lane & (lpb - 1)) == 0) a_encode<FMT>(p.a_store, bidx, anew_d);
+        const float ia = __frcp_rn(anew);
+        const bool ok = col_ok && in_range(ia);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const float q = quant<FMT>(w[c], u8[c], ia, ok, anew, bj[c], sTd);
+          const double sa = (double)(q * anew);  // exact; NVFP4 leaves s_T out
+          cn[c] = fma((double)w[c], sa, cn[c]);
+          cd[c] = fma(sa, sa, cd[c]);
+        }
+      }
+    }
+
+    // CTA reduction of the column sums over the 8 warps, fixed order
+    if (active) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) red[warp][lane * 8 + c] = make_double2(cn[c], cd[c]);
+    }
+    __syncthreads();
+    const int64_t slot = k * p.segmax + (s - s_first);
+    if (threadIdx.x < width) {
+      double2 acc = red[0][threadIdx.x];
+      for (int wi = 1; wi < kWarps; ++wi) {
+        acc.x += red[wi][threadIdx.x].x;
+        acc.y += red[wi][threadIdx.x].y;
+      }
+      p.col_part[slot * p.TS + threadIdx.x] = acc;
+    }
+    const int64_t k_first = cta_of(s * p.M, p.P, p.L);
+    const int64_t k_last = cta_of((s + 1) * p.M - 1, p.P, p.L);
+    if (arrive_last(&p.strip_counter[s], (unsigned)(k_last - k_first + 1), &s_last)) {
+      if (threadIdx.x < width) {
+        double2 acc = make_double2(0.0, 0.0);
+        for (int64_t kk = k_first; kk <= k_last; ++kk) {
+          const int64_t sl = kk * p.segmax + (s - range_begin(kk, p.P, p.L) / p.M);
+          const double2 v = __ldcg(&p.col_part[sl * p.TS + threadIdx.x]);
+          acc.x += v.x;
+          acc.y += v.y;
+        }
+        double bnew;
+        if (acc.y == 0.0) {
+          bnew = 1.0;
+        } else {
+          const double v = FMT == FMT_NVFP4 ? (acc.x / acc.y) / sTd : acc.x / acc.y;
+          bnew = b_project(v, p.col_dt);
+        }
+        b_encode(p.b_store, p.col_dt, c0 + threadIdx.x, bnew);
+      }
+      if (threadIdx.x == 0) p.strip_counter[s] = 0u;
+    }
+    __syncthreads();
+    u = (s + 1) * p.M;
+  }
+
+  // MSE of the incoming iterate: CTA sum, then CTA-ordered total
+  mred[threadIdx.x] = mse_acc;
+  __syncthreads();
+  for (int o = kThreads / 2; o > 0; o >>= 1) {
+    if (threadIdx.x < o) mred[threadIdx.x] += mred[threadIdx.x + o];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) p.cta_part[k] = mred[0];
+  if (arrive_last(&p.hdr->cta_counter, (unsigned)p.P, &s_last)) {
+    if (threadIdx.x == 0) {
+      double tot = p.hdr->sumW2;
+      for (int64_t kk = 0; kk < p.P; ++kk) tot += __ldcg(&p.cta_part[kk]);
+      p.mse[t - 1] = tot / ((double)p.M * (double)p.N);
+      p.hdr->cta_counter = 0u;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Final pass: codes of the final iterate, nibble packing, direct MSE.
+template <int FMT, int WDT>
+__global__ void __launch_bounds__(kThreads) k_final(Problem p, int T) {
+  if (p.hdr->flags & kFlagNonFinite) return;
+  __shared__ double mred[kThreads];
+  __shared__ int s_last;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const float sT = p.hdr->sT;
+  const double sTd = (double)sT;
+  const float isT = FMT == FMT_NVFP4 ? 1.f / sT : 1.f;
+  const bool sT_ok = FMT != FMT_NVFP4 || in_range(isT);
+  const int64_t k = blockIdx.x;
+  const int64_t u_begin = range_begin(k, p.P, p.L), u_end = range_begin(k + 1, p.P, p.L);
+  double acc = 0.0;
+  for (int64_t u = u_begin; u < u_end;) {
+    const int64_t s = u / p.M;
+    const int64_t r0 = u - s * p.M;
+    const int64_t r1 = min(p.M, r0 + (u_end - u));
+    const int64_t c0 = s * p.TS;
+    const int width = (int)min((int64_t)p.TS, p.N - c0);
+    const bool active = lane * 8 < width;
+    const int64_t col = c0 + lane * 8;
+    if (active) {
+      float bj[8], cb[8];
+      bool col_ok = sT_ok;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        bj[c] = b_decode(p.b_store, p.col_dt, col + c);
+        cb[c] = __frcp_rn(bj[c]) * isT;
+        col_ok = col_ok && in_range(cb[c]);
+      }
+      for (int64_t r = r0 + warp; r < r1; r += kWarps) {
+        float w[8];
+        load8<WDT>(p.W, r * p.N + col, w);
+        const float a = a_decode<FMT>(p.a_store, r * p.nb + col / p.G);
+        const float ia = __frcp_rn(a);
+        const bool ok = col_ok && in_range(ia);
+        const double aval = FMT == FMT_NVFP4 ? sTd * (double)a : (double)a;
+        uint32_t packed = 0;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const float q = quant<FMT>(w[c], w[c] * cb[c], ia, ok, a, bj[c], sTd);
+          packed |= nibble<FMT>(q) << (4 * c);
+          const double res = (double)w[c] - aval * (double)q * (double)bj[c];
+          acc = fma(res, res, acc);
+        }
+        reinterpret_cast<uint32_t*>(p.codes)[(r * p.N + col) / 8] = packed;
+      }
+    }
+    u = (s + 1) * p.M;
+  }
+  mred[threadIdx.x] = acc;
+  __syncthreads();
+  for (int o = kThreads / 2; o > 0; o >>= 1) {
+    if (threadIdx.x < o) mred[threadIdx.x] += mred[threadIdx.x + o];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) p.cta_part[k] = mred[0];
+  if (arrive_last(&p.hdr->cta_counter, (unsigned)p.P, &s_last)) {
+    if (threadIdx.x == 0) {
+      double tot = 0.0;
+      for (int64_t kk = 0; kk < p.P; ++kk) tot += __ldcg(&p.cta_part[kk]);
+      p.mse[T] = tot / ((double)p.M * (double)p.N);
+      p.hdr->cta_counter = 0u;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host-side launch of the whole solve on one stream.
+
+template <int FMT, int WDT>
+static cudaError_t run_typed(const Problem& p, int iters, int stats_ctas, cudaStream_t st) {
+  k_stats<WDT><<<stats_ctas, kThreads, 0, st>>>(p);
+  k_init<FMT, WDT><<<stats_ctas, kThreads, 0, st>>>(p);
+  for (int t = 1; t <= iters; ++t) k_iter<FMT, WDT><<<(unsigned)p.P, kThreads, 0, st>>>(p, t);
+  k_final<FMT, WDT><<<(unsigned)p.P, kThreads, 0, st>>>(p, iters);
+  return cudaGetLastError();
+}
+
+template <int FMT>
+static cudaError_t run_fmt(const Problem& p, int iters, int stats_ctas, cudaStream_t st) {
+  switch (p.wdt) {
+    case DT_F32: return run_typed<FMT, DT_F32>(p, iters, stats_ctas, st);
+    case DT_BF16: return run_typed<FMT, DT_BF16>(p, iters, stats_ctas, st);
+    default: return run_typed<FMT, DT_F16>(p, iters, stats_ctas, st);
+  }
+}
+
+cudaError_t launch_solve(const Problem& p, int iters, int stats_ctas, cudaStream_t st) {
+  switch (p.fmt) {
+    case FMT_INT4: return run_fmt<FMT_INT4>(p, iters, stats_ctas, st);
+    case FMT_MXINT4: return run_fmt<FMT_MXINT4>(p, iters, stats_ctas, st);
+    default: return run_fmt<FMT_NVFP4>(p, iters, stats_ctas, st);
+  }
+}
+
+}  // namespace dq

@@ -1,0 +1,133 @@
+/*
+ * dq.h -- C ABI of the B200 DualQuant solver library (libdq.so).
+ *
+ * The library computes the DualQuant dual-scale block-coordinate-descent (BCD)
+ * weight quantization of one matrix on one GPU:
+ *
+ *     W  ~  D_a . Q( W / (a b) ) . D_b           (a: block inverse scales,
+ *                                                 b: column inverse scales)
+ *
+ * as defined by the DualQuant reproduction README ("Core equations": the
+ * dual-scale model, the closed-form row and column inverse-scale updates with
+ * codes fixed, projection onto representable inverse scales, requantization
+ * after each update, scale 1 for an all-zero code slice) and by the DualQuant
+ * (arXiv 2610.13767) summary (§3 formats, §4.3 BCD, App. B closed forms).
+ *
+ * Conventions shared by every entry point
+ *  - All tensor pointers are DEVICE pointers unless the name says host; the
+ *    caller owns every buffer.  The library allocates no memory and keeps no
+ *    global state between calls; calls on different streams with different
+ *    workspaces are independent.
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and is asynchronous: a DQ_OK return means the arguments were
+ *    valid and the kernels were enqueued.  Conditions detected on the device
+ *    (non-finite W) are reported by dq_sync_status().
+ *  - Matrices are row-major, `rows` x `cols`, densely packed.
+ *  - W is never modified.
+ *  - Errors found on the host (bad sizes, NULL pointers, short workspace) are
+ *    returned before anything is enqueued; nothing is written then.
+ */
+#ifndef DQ_H
+#define DQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DQ_OK = 0,
+  DQ_EINVAL = 1,        /* NULL pointer, non-positive size, cols not a multiple of group, ... */
+  DQ_EUNSUPPORTED = 2,  /* valid but unsupported combination (e.g. group size for the format) */
+  DQ_EWORKSPACE = 3,    /* workspace smaller than dq_workspace_bytes() */
+  DQ_ENONFINITE = 4,    /* W holds Inf or NaN (reported by dq_sync_status / dq_solve_host) */
+  DQ_ECUDA = 5          /* a CUDA runtime call failed */
+} dq_status;
+
+/* Formats (DualQuant §3; reproduction README "Local reproduction"):
+ *  DQ_INT4   grid [-8,7], block inverse scales fp16, group 8, 16, 32, 64, 128
+ *            or 256; column inverse scales fp16 or bf16.
+ *  DQ_MXINT4 grid [-8,7], group 32, block inverse scales 2^k with k in
+ *            [-126,126] stored as E8M0 bytes (k+127).
+ *  DQ_NVFP4  E2M1 grid {0,+-0.5,+-1,+-1.5,+-2,+-3,+-4,+-6}, group 16, block
+ *            inverse scale a = s_T * e with e an FP8 E4M3 value (stored as the
+ *            E4M3 byte) and one fp32 tensor scale s_T = fp32(amax|W| / 2688). */
+typedef enum { DQ_INT4 = 0, DQ_MXINT4 = 1, DQ_NVFP4 = 2 } dq_format;
+
+typedef enum { DQ_F32 = 0, DQ_BF16 = 1, DQ_F16 = 2 } dq_dtype;
+
+/* Outputs (device pointers, caller-owned).
+ *  codes         uint8 [rows][cols/2]: two 4-bit codes per byte, the even
+ *                column in the low nibble.  INT4/MXINT4: two's-complement
+ *                nibble of q in [-8,7].  NVFP4: E2M1 nibble s|ee|m; a zero
+ *                code is always 0x0.
+ *  block_scales  [rows][cols/group]: fp16 (INT4), E8M0 byte (MXINT4), E4M3
+ *                byte (NVFP4).
+ *  tensor_scale  one float: s_T for NVFP4, 1.0 for the other formats (which
+ *                accept NULL here).
+ *  col_scales    [cols] inverse column scales, fp16 or bf16 (col_dtype).
+ *  mse           double [iters+1]: mse[0] is the RTN reconstruction MSE,
+ *                mse[t] the MSE after BCD iteration t, each
+ *                (1/(rows*cols)) * sum (W - a*q*b)^2.
+ * The solver uses block_scales and col_scales as its working state, so they
+ * must not alias W or the workspace. */
+typedef struct {
+  void* codes;
+  void* block_scales;
+  float* tensor_scale;
+  void* col_scales;
+  double* mse;
+} dq_outputs;
+
+/* Device workspace bytes dq_rtn / dq_solve need for this shape (0 on invalid
+ * arguments).  The workspace is scratch: its contents on entry do not matter,
+ * and it must stay untouched by the caller until the enqueued work finishes
+ * (or until dq_sync_status returns).  Alignment: 256 bytes. */
+size_t dq_workspace_bytes(int64_t rows, int64_t cols, int format, int group);
+
+/* Absmax round-to-nearest with column scales 1: the solver's initial iterate
+ * and its comparison point (DualQuant §3 "symmetric scale max|W|/qmax", qmax 7
+ * for INT4/MXINT4 and 6 for E2M1, projected onto the admissible set; an
+ * all-zero block gets scale 1).  Bit-identical to dq_solve(..., iters = 0).
+ * Writes codes, block_scales, tensor_scale, col_scales (all 1) and mse[0]. */
+int dq_rtn(const void* W, int w_dtype, int64_t rows, int64_t cols, int format, int group, int col_dtype,
+           const dq_outputs* out, void* workspace, size_t workspace_bytes, void* stream);
+
+/* The BCD solver (reproduction README flowchart and "Core equations"):
+ * RTN init, then `iters` iterations of
+ *   block update with codes fixed   a <- Proj_Fa( sum W q b / sum (q b)^2 )
+ *   requantize                      q <- Q( W / (a b) )
+ *   column update with codes fixed  b <- Proj_Fb( sum W a q / sum (a q)^2 )
+ *   requantize
+ * with scale 1 for an all-zero code slice.  iters >= 0; mse has iters+1
+ * entries. */
+int dq_solve(const void* W, int w_dtype, int64_t rows, int64_t cols, int format, int group, int iters, int col_dtype,
+             const dq_outputs* out, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Waits for `stream`, then reports what the device recorded in `workspace`
+ * during the last dq_rtn / dq_solve that used it: DQ_OK, DQ_ENONFINITE, or
+ * DQ_ECUDA if the wait itself failed. */
+int dq_sync_status(const void* workspace, void* stream);
+
+/* Device bytes dq_solve_host needs: room for a device copy of W, the outputs
+ * and the solver workspace (0 on invalid arguments). */
+size_t dq_host_workspace_bytes(int64_t rows, int64_t cols, int w_dtype, int format, int group, int iters);
+
+/* dq_solve with HOST input and outputs: copies W (host, ideally pinned) into
+ * `device_workspace`, solves there, copies the outputs back into the host
+ * buffers of `out_host`, and waits for the stream.  Returns the final status
+ * (including DQ_ENONFINITE).  Same argument rules as dq_solve. */
+int dq_solve_host(const void* W_host, int w_dtype, int64_t rows, int64_t cols, int format, int group, int iters,
+                  int col_dtype, const dq_outputs* out_host, void* device_workspace, size_t device_workspace_bytes,
+                  void* stream);
+
+/* Static string for a status code. */
+const char* dq_status_str(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DQ_H */

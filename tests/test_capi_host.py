@@ -1,0 +1,67 @@
+"""CPU-side checks of the C ABI library and the host logic of the binding (no GPU)."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from calibration_free_weight_dualquant_b200 import binding, build, synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "dq.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dq_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib_path():
+    return build.build()
+
+
+def test_library_exports_every_declared_symbol(lib_path):
+    names = declared_symbols()
+    assert {"dq_rtn", "dq_solve", "dq_workspace_bytes", "dq_sync_status", "dq_status_str"} <= set(names)
+    out = subprocess.run(["nm", "-D", "--defined-only", lib_path], capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (dq_\w+)", out))
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    lib = ctypes.CDLL(lib_path)
+    for n in names:
+        assert hasattr(lib, n)
+
+
+def test_status_strings(lib_path):
+    lib = ctypes.CDLL(lib_path)
+    lib.dq_status_str.restype = ctypes.c_char_p
+    for code, name in binding.STATUS.items():
+        assert lib.dq_status_str(code).decode().startswith(name)
+    assert b"unknown" in lib.dq_status_str(99)
+
+
+def test_output_sizes_storage_pin():
+    """DualQuant App. I / Table 12: 224 linears at INT4-G64 -> 3.49 GB codes + 0.22 GB fp16 scales."""
+    tot_codes = tot_scales = 0
+    for _ in range(synth.LLAMA31_8B_LAYERS):
+        for _, r, c in synth.LLAMA31_8B_LAYER:
+            n = binding.output_nbytes(r, c, "int4", 64, "f16")
+            tot_codes += n["codes"]
+            tot_scales += n["block_scales"]
+    assert "%.2f" % (tot_codes / 1e9) == "3.49"
+    assert "%.2f" % (tot_scales / 1e9) == "0.22"
+    n = binding.output_nbytes(4096, 4096, "nvfp4")
+    assert n["block_scales"] == 4096 * 256 and n["tensor_scale"] == 4
+    n = binding.output_nbytes(4096, 14336, "mxint4")
+    assert n["block_scales"] == 4096 * 448 and n["col_scales"] == 14336 * 2
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(binding, "_lib", None)
+    with pytest.raises(binding.DQError):
+        binding.load_library()

@@ -1,0 +1,221 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle on the same seeded inputs.
+
+Bar (spec tolerances): codes, block scales, column scales and the NVFP4
+tensor scale bit-exact; every per-iteration MSE within 1e-4 relative.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from calibration_free_weight_dualquant_b200 import binding, synth
+from gpu_helpers import block_scale_values, col_scale_values, compare_with_oracle
+
+pytestmark = pytest.mark.gpu
+
+MSE_RTOL = 1e-4
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.fail("CUDA device required for -m gpu tests")
+    binding.load_library()
+
+
+def run_both(Wcpu: torch.Tensor, fmt, group, iters, col_dtype, label=""):
+    gpu = binding.dq_solve(Wcpu.cuda(), fmt, group, iters, col_dtype)
+    Win, wdt = synth.to_oracle_input(Wcpu)
+    orc = oracle.solve(Win, wdt, fmt, group, iters, col_dtype)
+    compare_with_oracle(fmt, gpu, orc, MSE_RTOL, label)
+    return gpu, orc
+
+
+# small shapes spanning several column strips, several CTAs per strip and a ragged tail
+SMALL = {
+    "int4_g64_256x512_f32": (333, 704),
+    "int4_g64_qproj_4096x4096": (333, 704),
+    "mxint4_g32_downproj_4096x14336": (301, 608),
+    "nvfp4_g16_gateup_14336x4096": (339, 528),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_parity_small_workload_recipe(name):
+    wl = synth.WORKLOADS[name]
+    M, N = SMALL[name]
+    W = synth.make_weight(wl, M, N, seed=wl.seed + 7)
+    gpu, orc = run_both(W, wl.fmt, wl.group, wl.iters, wl.col_dtype, name)
+    mse = gpu["mse"].cpu().numpy()
+    assert np.all(mse[1:] <= mse[:-1] * (1 + 1e-9))
+
+
+@pytest.mark.parametrize("fmt,group,col_dtype,M,N,iters", [
+    ("int4", 64, "f16", 1000, 1344, 6),
+    ("mxint4", 32, "bf16", 777, 1056, 6),
+    ("nvfp4", 16, "bf16", 1203, 800, 6),
+])
+def test_parity_many_ctas(fmt, group, col_dtype, M, N, iters):
+    wl = synth.WORKLOADS["nvfp4_g16_gateup_14336x4096"]
+    W = synth.make_weight(wl, M, N, seed=77)
+    run_both(W, fmt, group, iters, col_dtype, "many_ctas")
+
+
+@pytest.mark.parametrize("fmt,group,col_dtype,M,N,wdtype", [
+    ("int4", 8, "f16", 1, 8, torch.float32),
+    ("int4", 256, "bf16", 5, 512, torch.bfloat16),
+    ("int4", 128, "f16", 7, 384, torch.float16),
+    ("mxint4", 32, "bf16", 2, 32, torch.float32),
+    ("nvfp4", 16, "bf16", 3, 16, torch.bfloat16),
+    ("nvfp4", 16, "f16", 65, 272, torch.float16),
+])
+def test_parity_edge_shapes_and_dtypes(fmt, group, col_dtype, M, N, wdtype):
+    g = torch.Generator().manual_seed(M * 1000 + N)
+    W = (torch.randn(M, N, generator=g) * 0.05).to(wdtype)
+    run_both(W, fmt, group, 5, col_dtype, "edge")
+
+
+@pytest.mark.parametrize("fmt,group,col_dtype", [("int4", 64, "f16"), ("mxint4", 32, "bf16"), ("nvfp4", 16, "bf16")])
+def test_parity_zero_slices(fmt, group, col_dtype):
+    g = torch.Generator().manual_seed(5)
+    W = torch.randn(40, 4 * group, generator=g) * 0.02
+    W[3, group:2 * group] = 0
+    W[:, 5] = 0
+    W[17] = 0
+    run_both(W.to(torch.bfloat16), fmt, group, 6, col_dtype, "zero_slices")
+    run_both(torch.zeros(9, 2 * group, dtype=torch.bfloat16), fmt, group, 3, col_dtype, "all_zero")
+
+
+@pytest.mark.parametrize("fmt,group,col_dtype", [("int4", 64, "f16"), ("mxint4", 32, "bf16"), ("nvfp4", 16, "bf16")])
+def test_parity_exact_ties(fmt, group, col_dtype):
+    """Weights on a coarse dyadic lattice make exact rounding ties frequent."""
+    g = torch.Generator().manual_seed(9)
+    W = torch.randint(-24, 25, (64, 8 * group), generator=g).float() * 2.0 ** -7
+    W[:, 3] *= 8
+    run_both(W.to(torch.bfloat16), fmt, group, 8, col_dtype, "ties")
+
+
+@pytest.mark.parametrize("fmt,group,col_dtype", [("int4", 64, "f16"), ("mxint4", 32, "bf16"), ("nvfp4", 16, "bf16")])
+@pytest.mark.parametrize("mag", [1e-33, 1e-12, 1e4, 1e30])
+def test_parity_extreme_magnitudes(fmt, group, col_dtype, mag):
+    """Scales at the ends of the admissible sets (saturation, smallest values, fp64 fallback of the candidate)."""
+    g = torch.Generator().manual_seed(11)
+    W = torch.randn(16, 2 * group, generator=g) * mag
+    W[:, 1] *= 1e3 if mag < 1 else 1.0
+    run_both(W.float(), fmt, group, 4, col_dtype, "mag%g" % mag)
+
+
+@pytest.mark.parametrize("fmt", ["int4", "mxint4", "nvfp4"])
+def test_zero_iterations_is_rtn_and_deterministic(fmt):
+    wl = synth.WORKLOADS["nvfp4_g16_gateup_14336x4096"]
+    W = synth.make_weight(wl, 250, 1024, seed=3).cuda()
+    r = binding.dq_rtn(W, fmt)
+    s = binding.dq_solve(W, fmt, iters=0)
+    for k in ("codes", "block_scales", "col_scales", "mse"):
+        assert torch.equal(r[k], s[k]), k
+    s1 = binding.dq_solve(W, fmt, iters=7)
+    s2 = binding.dq_solve(W, fmt, iters=7)
+    for k in ("codes", "block_scales", "col_scales", "mse", "tensor_scale"):
+        assert torch.equal(s1[k], s2[k]), k
+    assert float(s1["mse"][0]) == pytest.approx(float(r["mse"][0]), rel=1e-12)
+
+
+def test_host_entry_point_matches_device():
+    wl = synth.WORKLOADS["mxint4_g32_downproj_4096x14336"]
+    W = synth.make_weight(wl, 96, 640, seed=4)
+    host = binding.solve(W.pin_memory(), "mxint4", 32, 5, "bf16")
+    dev = binding.dq_solve(W.cuda(), "mxint4", 32, 5, "bf16")
+    for k in ("codes", "block_scales", "col_scales", "mse"):
+        assert torch.equal(host[k], dev[k].cpu()), k
+
+
+def test_nonfinite_input_reported():
+    W = torch.zeros(8, 64, dtype=torch.bfloat16)
+    W[2, 3] = float("nan")
+    with pytest.raises(binding.DQError) as e:
+        binding.dq_solve(W.cuda(), "int4", 64, 2, "f16")
+    assert e.value.status == 4
+    W[2, 3] = float("inf")
+    with pytest.raises(binding.DQError) as e:
+        binding.solve(W, "nvfp4", 16, 2)
+    assert e.value.status == 4
+
+
+def test_invalid_arguments_rejected_on_host():
+    lib = binding.load_library()
+    W = torch.zeros(4, 64, dtype=torch.bfloat16, device="cuda")
+    out = binding.alloc_outputs(4, 64, "int4", 64, "f16", 2, "cuda")
+    o = binding._outputs_struct(out)
+    ws = torch.empty(lib.dq_workspace_bytes(4, 64, 0, 64), dtype=torch.uint8, device="cuda")
+    import ctypes
+    s = torch.cuda.current_stream().cuda_stream
+
+    def call(**kw):
+        args = dict(W=W.data_ptr(), wdt=1, M=4, N=64, fmt=0, G=64, iters=2, cdt=2, ws=ws.data_ptr(),
+                    wsb=ws.numel())
+        args.update(kw)
+        return lib.dq_solve(args["W"], args["wdt"], args["M"], args["N"], args["fmt"], args["G"], args["iters"],
+                            args["cdt"], ctypes.byref(o), args["ws"], args["wsb"], s)
+
+    assert call() == 0
+    assert call(G=48) == 1            # cols not a multiple of group
+    assert call(fmt=1, G=64) == 2     # MXINT4 needs group 32
+    assert call(fmt=2, G=32) == 2     # NVFP4 needs group 16
+    assert call(M=0) == 1
+    assert call(N=63, G=7) == 1
+    assert call(iters=-1) == 1
+    assert call(wsb=ws.numel() - 1) == 3
+    assert call(W=W.data_ptr() + 2) == 1   # W must be 16-byte aligned
+    assert call(cdt=0) == 2
+    assert call(G=24, N=72) == 2      # group must be a power of two in [8, 256]
+    assert call(W=0) == 1
+    assert lib.dq_workspace_bytes(4, 64, 1, 64) == 0
+    torch.cuda.synchronize()
+
+
+# ---------------------------------------------------------------------------
+# Full sizes, in the launch configuration the benchmark times
+
+
+def full_weight(name):
+    wl = synth.WORKLOADS[name]
+    return wl, synth.make_weight(wl)
+
+
+def test_full_size_qproj_int4_against_full_oracle():
+    """4096x4096 bf16 INT4-G64, 20 iterations: the whole solve against the oracle."""
+    wl, W = full_weight("int4_g64_qproj_4096x4096")
+    run_both(W, wl.fmt, wl.group, wl.iters, wl.col_dtype, wl.name)
+
+
+@pytest.mark.parametrize("name", ["mxint4_g32_downproj_4096x14336", "nvfp4_g16_gateup_14336x4096",
+                                  "int4_g64_256x512_f32"])
+def test_full_size_last_iteration_and_final_state(name):
+    """Full-size solve: the last GPU iteration equals one oracle iteration from the GPU's previous
+    iterate (every block and column scale, bit-exact); the codes equal Q(W/(a b)) of the final
+    scales; the final MSE equals the oracle's MSE of that state; MSE is monotone."""
+    wl, W = full_weight(name)
+    Wd = W.cuda()
+    T = wl.iters
+    prev = binding.dq_solve(Wd, wl.fmt, wl.group, T - 1, wl.col_dtype)
+    last = binding.dq_solve(Wd, wl.fmt, wl.group, T, wl.col_dtype)
+    sT = float(last["tensor_scale"].cpu()[0]) if wl.fmt == "nvfp4" else 1.0
+    a_prev = block_scale_values(wl.fmt, prev["block_scales"])
+    b_prev = col_scale_values(prev["col_scales"])
+    Win, wdt = synth.to_oracle_input(W)
+    a_o, b_o = oracle.iterate(Win, wdt, wl.fmt, wl.group, wl.col_dtype, sT, a_prev, b_prev)
+    a_last = block_scale_values(wl.fmt, last["block_scales"])
+    b_last = col_scale_values(last["col_scales"])
+    assert np.array_equal(a_last, a_o), int((a_last != a_o).sum())
+    assert np.array_equal(b_last, b_o), int((b_last != b_o).sum())
+    # codes of the final state and its MSE
+    q = oracle.requant(Win, wdt, wl.fmt, wl.group, wl.col_dtype, sT, a_last, b_last)
+    import bruteforce as bf
+    assert np.array_equal(bf.decode_codes(wl.fmt, last["codes"].cpu().numpy()), q)
+    mse_o = oracle.mse(Win, wdt, wl.fmt, wl.group, wl.col_dtype, sT, q, a_last, b_last)
+    mse = last["mse"].cpu().numpy()
+    assert mse[-1] == pytest.approx(mse_o, rel=MSE_RTOL)
+    assert np.all(mse[1:] <= mse[:-1] * (1 + 1e-9))
+    np.testing.assert_allclose(mse[:-1], prev["mse"].cpu().numpy(), rtol=1e-12)
