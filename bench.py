@@ -33,7 +33,9 @@ METRIC = "weight-elems x BCD-iters/sec"
 UNIT = "elem*iter/s"
 L2_FLUSH_BYTES = 512 << 20
 KERNEL_SOURCES = ["calibration_free_weight_dualquant_b200/csrc/dq_solver.cu",
-                  "calibration_free_weight_dualquant_b200/csrc/dq_device.cuh"]
+                  "calibration_free_weight_dualquant_b200/csrc/dq_device.cuh",
+                  "calibration_free_weight_dualquant_b200/csrc/dq_fast.cuh",
+                  "calibration_free_weight_dualquant_b200/csrc/dq_iter.cuh"]
 
 
 def kernel_hash() -> str:
@@ -215,8 +217,19 @@ def main():
     ap.add_argument("--impl", default="dq", choices=["dq", "reference"])
     ap.add_argument("--ref-rows", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end timing")
+    ap.add_argument("--rows", type=int, help="override the workload's rows (profiling cases)")
+    ap.add_argument("--cols", type=int, help="override the workload's cols (profiling cases)")
+    ap.add_argument("--iters", type=int, help="override the workload's BCD iterations")
     args = ap.parse_args()
     wl = synth.WORKLOADS[args.workload]
+    if args.rows or args.cols or args.iters:
+        import dataclasses
+        rows = args.rows or wl.rows
+        cols = args.cols or wl.cols
+        iters = args.iters or wl.iters
+        wl = dataclasses.replace(wl, name="%s@%dx%d_T%d" % (wl.name, rows, cols, iters), rows=rows, cols=cols,
+                                 iters=iters)
     rank, world, local, dist = dist_setup(args.gpus)
     try:
         if args.impl == "reference":
@@ -271,6 +284,7 @@ def run_dq(args, wl, rank, world, local, dist):
     torch.cuda.synchronize()
     barrier(dist)
     total_ms = max_over_ranks(sum(step_ms), dist)
+    exact_paths = binding.diagnostics(ws, stream)
 
     # steady-state iteration time of the dominant kernel (k_iter): (t(T) - t(0)) / T, median of runs
     out0 = binding.alloc_outputs(wl.rows, wl.cols, wl.fmt, wl.group, wl.col_dtype, 0, dev)
@@ -279,7 +293,39 @@ def run_dq(args, wl, rank, world, local, dist):
     iter_ms = (statistics.median(tTs) - statistics.median(t0s)) / T
     iter_ms = max_over_ranks(iter_ms, dist)
 
-    # end to end through the public API with host buffers (pinned), copies inside the timed region
+    e2e_line = None
+    if not args.no_e2e:
+        e2e_line = run_e2e(args, wl, W, T, dev, stream, flush, dist, world)
+    if rank != 0:
+        return
+    elems = wl.rows * wl.cols
+    value = world * elems * T * args.steps / (total_ms * 1e-3)
+    peaks = measured_peaks()
+    alg = algorithmic_bytes_per_iter(wl)
+    achieved = alg / (iter_ms * 1e-3) / 1e9
+    traffic = profile_traffic(wl.name)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32+f64", "data": "synthetic",
+        "config": config_of(wl, world),
+        "final_mse": float(out["mse"][-1].item()),
+        "ms_per_iter": iter_ms,
+        "roofline": {"bound": "hbm", "kernel": "k_iter", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                     "algorithmic_bytes_per_launch": alg, "peak_source": peaks["source"]},
+        "e2e": e2e_line,
+        "gpu_launches": args.steps * (T + 3),
+        "exact_paths_last_step": exact_paths,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, wl, W, T, dev, stream, flush, dist, world):
+    """Same metric through the public host-buffer API: pinned W in, outputs back, copies timed."""
     Wh = W.pin_memory()
     host_out = binding.alloc_outputs(wl.rows, wl.cols, wl.fmt, wl.group, wl.col_dtype, T, "cpu")
     for k in host_out:
@@ -302,33 +348,8 @@ def run_dq(args, wl, rank, world, local, dist):
     nb = binding.output_nbytes(wl.rows, wl.cols, wl.fmt, wl.group, wl.col_dtype)
     h2d = W.numel() * W.element_size()
     d2h = nb["codes"] + nb["block_scales"] + nb["col_scales"] + nb["tensor_scale"] + 8 * (T + 1)
-
-    if rank != 0:
-        return
-    elems = wl.rows * wl.cols
-    value = world * elems * T * args.steps / (total_ms * 1e-3)
-    e2e_value = world * elems * T * len(e2e_ms) / (e2e_total * 1e-3)
-    peaks = measured_peaks()
-    alg = algorithmic_bytes_per_iter(wl)
-    achieved = alg / (iter_ms * 1e-3) / 1e9
-    traffic = profile_traffic(wl.name)
-    line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32+f64", "data": "synthetic",
-        "config": config_of(wl, world),
-        "final_mse": float(out["mse"][-1].item()),
-        "ms_per_iter": iter_ms,
-        "roofline": {"bound": "hbm", "kernel": "k_iter", "achieved": achieved, "peak": peaks["hbm_gbs"],
-                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
-                     "algorithmic_bytes_per_launch": alg, "peak_source": peaks["source"]},
-        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": args.steps * (T + 3),
-        "clocks": clk.summary(),
-    }
-    if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(wl)
-    print(json.dumps(line), flush=True)
+    e2e_value = world * wl.rows * wl.cols * T * len(e2e_ms) / (e2e_total * 1e-3)
+    return {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
 
 if __name__ == "__main__":

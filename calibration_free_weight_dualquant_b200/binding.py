@@ -68,6 +68,8 @@ def load_library():
     lib.dq_host_workspace_bytes.restype = SZ
     lib.dq_solve_host.argtypes = [P, I, I64, I64, I, I, I, I, ctypes.POINTER(_Outputs), P, SZ, P]
     lib.dq_solve_host.restype = I
+    lib.dq_diagnostics.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint64)]
+    lib.dq_diagnostics.restype = I
     lib.dq_status_str.argtypes = [I]
     lib.dq_status_str.restype = ctypes.c_char_p
     _lib = lib
@@ -216,3 +218,13 @@ def solve(W: torch.Tensor, fmt="nvfp4", group: Optional[int] = None, iters: int 
 def rtn(W: torch.Tensor, fmt="nvfp4", group: Optional[int] = None, col_dtype: Optional[str] = None) -> dict:
     """User-level absmax RTN (the 0-iteration solve)."""
     return solve(W, fmt, group, 0, col_dtype)
+
+
+def diagnostics(workspace: torch.Tensor, stream=None) -> dict:
+    """Exact-path counters of the last solve that used this workspace."""
+    lib = load_library()
+    arr = (ctypes.c_uint64 * 3)()
+    st = lib.dq_diagnostics(workspace.data_ptr(), _stream_ptr(stream), arr)
+    if st != 0:
+        raise DQError(st, "dq_diagnostics")
+    return {"quant_exact_lane_rows": int(arr[0]), "block_exact": int(arr[1]), "col_exact": int(arr[2])}

@@ -13,7 +13,7 @@ constexpr size_t kAlign = 256;
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 struct Plan {
-  int TS, n_strips, P, segmax, nb;
+  int TS, n_strips, P, segmax, P_final, segmax_final, nb;
   int64_t L;
   size_t off_counters, off_col_part, off_cta_part, total;
 };
@@ -48,19 +48,21 @@ int make_plan(int64_t M, int64_t N, int group, Plan* pl) {
   pl->TS = (dq::kStripMax / group) * group;
   pl->n_strips = (int)((N + pl->TS - 1) / pl->TS);
   pl->L = (int64_t)pl->n_strips * M;
-  int64_t P = (int64_t)sms * dq::kCtasPerSm;
-  int64_t byrows = pl->L / dq::kMinRowsPerCta;
-  if (byrows < P) P = byrows < 1 ? 1 : byrows;
-  pl->P = (int)P;
-  const int64_t len = (pl->L + P - 1) / P;
-  pl->segmax = (int)((len + M - 1) / M + 1);
+  const int64_t byrows = pl->L / dq::kMinRowsPerCta;
+  auto ctas = [&](int64_t want) { return (int)(byrows < want ? (byrows < 1 ? 1 : byrows) : want); };
+  // a CTA's contiguous range of len rows touches at most ceil(len/M) + 1 strips
+  auto segs = [&](int64_t P) { return (int)(((pl->L + P - 1) / P + M - 1) / M + 1); };
+  pl->P = ctas((int64_t)sms * dq::kCtasPerSm);
+  pl->segmax = segs(pl->P);
+  pl->P_final = ctas((int64_t)sms * dq::kFinalCtasPerSm);
+  pl->segmax_final = segs(pl->P_final);
   size_t off = align_up(sizeof(dq::WsHeader));
   pl->off_counters = off;
   off += align_up(sizeof(unsigned) * (size_t)pl->n_strips);
   pl->off_col_part = off;
   off += align_up(sizeof(double2) * (size_t)pl->P * (size_t)pl->segmax * (size_t)pl->TS);
   pl->off_cta_part = off;
-  off += align_up(sizeof(double) * (size_t)pl->P);
+  off += align_up(sizeof(double) * (size_t)(pl->P > pl->P_final ? pl->P : pl->P_final));
   pl->total = off;
   return DQ_OK;
 }
@@ -108,6 +110,8 @@ int solve_impl(const void* W, int w_dtype, int64_t rows, int64_t cols, int forma
   p.n_strips = pl.n_strips;
   p.P = pl.P;
   p.segmax = pl.segmax;
+  p.P_final = pl.P_final;
+  p.segmax_final = pl.segmax_final;
   p.L = pl.L;
   p.codes = out->codes;
   p.a_store = out->block_scales;
@@ -121,7 +125,7 @@ int solve_impl(const void* W, int w_dtype, int64_t rows, int64_t cols, int forma
 
   // header and arrival counters start at zero; the partial buffers need no init
   if (cudaMemsetAsync(ws, 0, pl.off_col_part, stream) != cudaSuccess) return DQ_ECUDA;
-  if (dq::launch_solve(p, iters, pl.P, stream) != cudaSuccess) return DQ_ECUDA;
+  if (dq::launch_solve(p, iters, pl.P_final, stream) != cudaSuccess) return DQ_ECUDA;
   return DQ_OK;
 }
 
@@ -153,7 +157,19 @@ int dq_sync_status(const void* workspace, void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DQ_ECUDA;
   unsigned flags = 0;
   if (cudaMemcpy(&flags, workspace, sizeof(flags), cudaMemcpyDeviceToHost) != cudaSuccess) return DQ_ECUDA;
-  return (flags & dq::kFlagNonFinite) ? DQ_ENONFINITE : DQ_OK;
+  if (flags & dq::kFlagNonFinite) return DQ_ENONFINITE;
+  return (flags & dq::kFlagTimeout) ? DQ_ECUDA : DQ_OK;
+}
+
+int dq_diagnostics(const void* workspace, void* stream, uint64_t out[3]) {
+  if (!workspace || !out) return DQ_EINVAL;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DQ_ECUDA;
+  dq::WsHeader h;
+  if (cudaMemcpy(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return DQ_ECUDA;
+  out[0] = h.n_quant_exact;
+  out[1] = h.n_block_exact;
+  out[2] = h.n_col_exact;
+  return DQ_OK;
 }
 
 static size_t wsize(int dt) { return dt == DQ_F32 ? 4 : 2; }

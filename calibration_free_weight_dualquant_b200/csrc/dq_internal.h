@@ -9,9 +9,11 @@ namespace dq {
 constexpr int kThreads = 256;   // 8 warps per CTA
 constexpr int kWarps = kThreads / 32;
 constexpr int kStripMax = 256;  // columns per strip (8 per lane, 32 lanes)
-constexpr int kCtasPerSm = 2;
+constexpr int kCtasPerSm = 1;        // per-iteration pass: one 544-thread CTA per SM
+constexpr int kFinalCtasPerSm = 4;   // one-time passes
 constexpr int64_t kMinRowsPerCta = 64;
 constexpr unsigned kFlagNonFinite = 1u;
+constexpr unsigned kFlagTimeout = 2u;  // a bounded pipeline wait gave up (results invalid)
 
 // Device workspace header (first 256 bytes of the workspace).
 struct WsHeader {
@@ -20,6 +22,10 @@ struct WsHeader {
   unsigned cta_counter;  // arrival ticket for CTA-ordered totals
   float sT;              // NVFP4 tensor scale (1 otherwise)
   double sumW2;          // sum of W^2 (fp64)
+  // diagnostics: how often the exact paths ran in the per-iteration passes
+  unsigned long long n_quant_exact;  // lane-rows (8 elements) decided on the exact path
+  unsigned long long n_block_exact;  // block updates taken in fp64
+  unsigned long long n_col_exact;    // column updates recomputed exactly over all rows
 };
 
 // Everything a kernel needs, passed by value.
@@ -30,8 +36,10 @@ struct Problem {
   int nb;        // blocks per row = N / G
   int TS;        // strip width (columns), multiple of G and of 8, <= kStripMax
   int n_strips;  // ceil(N / TS)
-  int P;         // CTAs of the persistent passes
-  int segmax;    // max (CTA, strip) segments per CTA
+  int P;         // CTAs of the per-iteration pass
+  int segmax;    // max (CTA, strip) segments per CTA of that pass
+  int P_final;   // CTAs of the one-time passes (stats, init, final)
+  int segmax_final;
   int64_t L;     // n_strips * M (strip-major row units)
   void* codes;
   void* a_store;
@@ -41,7 +49,7 @@ struct Problem {
   WsHeader* hdr;
   unsigned* strip_counter;  // [n_strips]
   double2* col_part;        // [P * segmax][TS] (sum W a q, sum (a q)^2)
-  double* cta_part;         // [P]
+  double* cta_part;         // [max(P, P_final)]
 };
 
 cudaError_t launch_solve(const Problem& p, int iters, int stats_ctas, cudaStream_t st);

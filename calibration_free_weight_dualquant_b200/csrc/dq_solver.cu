@@ -27,17 +27,12 @@
 // sum (W - a q b)^2 = sum W^2 - sum_blocks (2 a num - a^2 den),
 // per CTA, then summed in CTA order by the last CTA.
 #include "dq_device.cuh"
+#include "dq_fast.cuh"
 #include "dq_internal.h"
+#include "dq_iter.cuh"
 
 namespace dq {
 
-__device__ __forceinline__ int64_t cta_of(int64_t u, int64_t P, int64_t L) { return ((u + 1) * P - 1) / L; }
-__device__ __forceinline__ int64_t range_begin(int64_t k, int64_t P, int64_t L) { return k * L / P; }
-
-// Fast-path scale factors are trusted when they stay inside [2^-100, 2^100]:
-// then every product that lands near a rounding boundary is a normal fp32
-// number and the relative error bound behind kGuard holds.
-__device__ __forceinline__ bool in_range(float x) { return x >= 0x1p-100f && x <= 0x1p100f; }
 
 // Last-arriving CTA election for a counter: every thread has already issued its
 // writes; returns true in all threads of the CTA that arrived last.
@@ -135,156 +130,6 @@ __global__ void __launch_bounds__(kThreads) k_init(Problem p) {
 }
 
 // ---------------------------------------------------------------------------
-// One BCD iteration (see the file header).  Writes mse[t-1].
-template <int FMT, int WDT>
-__global__ void __launch_bounds__(kThreads, 2) k_iter(Problem p, int t) {
-  if (p.hdr->flags & kFlagNonFinite) return;
-  __shared__ double2 red[kWarps][kStripMax];
-  __shared__ double mred[kThreads];
-  __shared__ int s_last;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int lpb = p.G / 8;  // lanes per block
-  const float sT = p.hdr->sT;
-  const double sTd = (double)sT;
-  const float isT = FMT == FMT_NVFP4 ? 1.f / sT : 1.f;
-  const bool sT_ok = FMT != FMT_NVFP4 || in_range(isT);
-  const int64_t k = blockIdx.x;
-  const int64_t u_begin = range_begin(k, p.P, p.L), u_end = range_begin(k + 1, p.P, p.L);
-  const int64_t s_first = u_begin / p.M;
-  double mse_acc = 0.0;
-
-  for (int64_t u = u_begin; u < u_end;) {
-    const int64_t s = u / p.M;
-    const int64_t r0 = u - s * p.M;
-    const int64_t r1 = min(p.M, r0 + (u_end - u));
-    const int64_t c0 = s * p.TS;
-    const int width = (int)min((int64_t)p.TS, p.N - c0);
-    const bool active = lane * 8 < width;
-    const int64_t col = c0 + lane * 8;
-
-    float bj[8], cb[8];
-    bool col_ok = sT_ok;
-    double cn[8], cd[8];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      cn[c] = 0.0;
-      cd[c] = 0.0;
-      bj[c] = 1.f;
-      cb[c] = 1.f;
-    }
-    if (active) {
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        bj[c] = b_decode(p.b_store, p.col_dt, col + c);
-        cb[c] = __frcp_rn(bj[c]) * isT;
-        col_ok = col_ok && in_range(cb[c]);
-      }
-    }
-
-    for (int64_t r = r0 + warp; r < r1; r += kWarps) {
-      float w[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      float aold = 1.f;
-      const int64_t bidx = r * p.nb + col / p.G;
-      double num = 0.0, den = 0.0;
-      float u8[8];
-      if (active) {
-        load8<WDT>(p.W, r * p.N + col, w);
-        aold = a_decode<FMT>(p.a_store, bidx);
-        const float ia = __frcp_rn(aold);
-        const bool ok = col_ok && in_range(ia);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          u8[c] = w[c] * cb[c];
-          const float q = quant<FMT>(w[c], u8[c], ia, ok, aold, bj[c], sTd);
-          const float qb = q * bj[c];  // exact: <= 15 significant bits
-          const double qbd = (double)qb;
-          num = fma((double)w[c], qbd, num);
-          den = fma(qbd, qbd, den);
-        }
-      }
-      for (int o = 1; o < lpb; o <<= 1) {
-        num += __shfl_xor_sync(0xffffffffu, num, o);
-        den += __shfl_xor_sync(0xffffffffu, den, o);
-      }
-      if (active) {
-        // MSE contribution of this block at the incoming iterate
-        const double aval = FMT == FMT_NVFP4 ? sTd * (double)aold : (double)aold;
-        if ((lane & (lpb - 1)) == 0) mse_acc += aval * (aval * den - 2.0 * num);
-        const double anew_d = den == 0.0 ? 1.0 : a_project<FMT>(num / den, sTd);
-        const float anew = (float)anew_d;  // exact
-        if ((lane & (lpb - 1)) == 0) a_encode<FMT>(p.a_store, bidx, anew_d);
-        const float ia = __frcp_rn(anew);
-        const bool ok = col_ok && in_range(ia);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const float q = quant<FMT>(w[c], u8[c], ia, ok, anew, bj[c], sTd);
-          const double sa = (double)(q * anew);  // exact; NVFP4 leaves s_T out
-          cn[c] = fma((double)w[c], sa, cn[c]);
-          cd[c] = fma(sa, sa, cd[c]);
-        }
-      }
-    }
-
-    // CTA reduction of the column sums over the 8 warps, fixed order
-    if (active) {
-#pragma unroll
-      for (int c = 0; c < 8; ++c) red[warp][lane * 8 + c] = make_double2(cn[c], cd[c]);
-    }
-    __syncthreads();
-    const int64_t slot = k * p.segmax + (s - s_first);
-    if (threadIdx.x < width) {
-      double2 acc = red[0][threadIdx.x];
-      for (int wi = 1; wi < kWarps; ++wi) {
-        acc.x += red[wi][threadIdx.x].x;
-        acc.y += red[wi][threadIdx.x].y;
-      }
-      p.col_part[slot * p.TS + threadIdx.x] = acc;
-    }
-    const int64_t k_first = cta_of(s * p.M, p.P, p.L);
-    const int64_t k_last = cta_of((s + 1) * p.M - 1, p.P, p.L);
-    if (arrive_last(&p.strip_counter[s], (unsigned)(k_last - k_first + 1), &s_last)) {
-      if (threadIdx.x < width) {
-        double2 acc = make_double2(0.0, 0.0);
-        for (int64_t kk = k_first; kk <= k_last; ++kk) {
-          const int64_t sl = kk * p.segmax + (s - range_begin(kk, p.P, p.L) / p.M);
-          const double2 v = __ldcg(&p.col_part[sl * p.TS + threadIdx.x]);
-          acc.x += v.x;
-          acc.y += v.y;
-        }
-        double bnew;
-        if (acc.y == 0.0) {
-          bnew = 1.0;
-        } else {
-          const double v = FMT == FMT_NVFP4 ? (acc.x / acc.y) / sTd : acc.x / acc.y;
-          bnew = b_project(v, p.col_dt);
-        }
-        b_encode(p.b_store, p.col_dt, c0 + threadIdx.x, bnew);
-      }
-      if (threadIdx.x == 0) p.strip_counter[s] = 0u;
-    }
-    __syncthreads();
-    u = (s + 1) * p.M;
-  }
-
-  // MSE of the incoming iterate: CTA sum, then CTA-ordered total
-  mred[threadIdx.x] = mse_acc;
-  __syncthreads();
-  for (int o = kThreads / 2; o > 0; o >>= 1) {
-    if (threadIdx.x < o) mred[threadIdx.x] += mred[threadIdx.x + o];
-    __syncthreads();
-  }
-  if (threadIdx.x == 0) p.cta_part[k] = mred[0];
-  if (arrive_last(&p.hdr->cta_counter, (unsigned)p.P, &s_last)) {
-    if (threadIdx.x == 0) {
-      double tot = p.hdr->sumW2;
-      for (int64_t kk = 0; kk < p.P; ++kk) tot += __ldcg(&p.cta_part[kk]);
-      p.mse[t - 1] = tot / ((double)p.M * (double)p.N);
-      p.hdr->cta_counter = 0u;
-    }
-  }
-}
-
-// ---------------------------------------------------------------------------
 // Final pass: codes of the final iterate, nibble packing, direct MSE.
 template <int FMT, int WDT>
 __global__ void __launch_bounds__(kThreads) k_final(Problem p, int T) {
@@ -358,10 +203,17 @@ __global__ void __launch_bounds__(kThreads) k_final(Problem p, int T) {
 
 template <int FMT, int WDT>
 static cudaError_t run_typed(const Problem& p, int iters, int stats_ctas, cudaStream_t st) {
-  k_stats<WDT><<<stats_ctas, kThreads, 0, st>>>(p);
-  k_init<FMT, WDT><<<stats_ctas, kThreads, 0, st>>>(p);
-  for (int t = 1; t <= iters; ++t) k_iter<FMT, WDT><<<(unsigned)p.P, kThreads, 0, st>>>(p, t);
-  k_final<FMT, WDT><<<(unsigned)p.P, kThreads, 0, st>>>(p, iters);
+  constexpr int ES = WDT == DT_F32 ? 4 : 2;
+  const size_t smem = iter_smem_bytes(ES);
+  cudaError_t e = cudaFuncSetAttribute(k_iter<FMT, WDT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  Problem pf = p;
+  pf.P = p.P_final;
+  pf.segmax = p.segmax_final;
+  k_stats<WDT><<<stats_ctas, kThreads, 0, st>>>(pf);
+  k_init<FMT, WDT><<<stats_ctas, kThreads, 0, st>>>(pf);
+  for (int t = 1; t <= iters; ++t) k_iter<FMT, WDT><<<(unsigned)p.P, kIterThreads, smem, st>>>(p, t);
+  k_final<FMT, WDT><<<(unsigned)pf.P, kThreads, 0, st>>>(pf, iters);
   return cudaGetLastError();
 }
 

@@ -123,6 +123,16 @@ int dq_solve_host(const void* W_host, int w_dtype, int64_t rows, int64_t cols, i
                   int col_dtype, const dq_outputs* out_host, void* device_workspace, size_t device_workspace_bytes,
                   void* stream);
 
+/* Diagnostics of the last solve that used `workspace` (waits for `stream`):
+ *   out[0]  lane-rows (8 consecutive elements) whose grid decisions took the
+ *           exact path (an fp32 candidate within the guard band of a rounding
+ *           boundary, or a scale outside the fast path's range),
+ *   out[1]  block inverse-scale updates taken in fp64 (fp32 value too close to
+ *           a projection midpoint, a zero or out-of-range sum),
+ *   out[2]  column inverse-scale updates recomputed exactly over all rows.
+ * Counts cover the BCD iterations only (not init or the final pass). */
+int dq_diagnostics(const void* workspace, void* stream, uint64_t out[3]);
+
 /* Static string for a status code. */
 const char* dq_status_str(int status);
 
