@@ -21,7 +21,7 @@ struct WsHeader {
   unsigned amax_bits;    // max |W| as fp32 bits
   unsigned cta_counter;  // arrival ticket for CTA-ordered totals
   float sT;              // NVFP4 tensor scale (1 otherwise)
-  double sumW2;          // sum of W^2 (fp64)
+  double reserved;
   // diagnostics: how often the exact paths ran in the per-iteration passes
   unsigned long long n_quant_exact;  // lane-rows (8 elements) decided on the exact path
   unsigned long long n_block_exact;  // block updates taken in fp64

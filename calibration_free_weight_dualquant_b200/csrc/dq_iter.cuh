@@ -6,10 +6,11 @@
 // of the current column strip, one row per bulk (TMA) copy, into a ring of
 // shared-memory tiles of kRowsPerTile rows, guarded by full/empty mbarriers.
 // Consumer warp w takes rows w and w + 15 of every tile; lane l takes the 8
-// consecutive columns 8l..8l+7 of the strip.  Per element the consumers run the
-// fp32 fast paths and fall back to the exact definitions where those flag.
-// Column sums run in fp32 for kRun rows of a lane and are then added into fp64
-// accumulators kept in shared memory.
+// consecutive columns 8l..8l+7 of the strip as 4 pairs, and the arithmetic on
+// pairs runs as packed f32x2 instructions.  Per element the consumers run the
+// fp32 fast paths and settle flagged elements exactly.  Column sums and the
+// reconstruction residuals run in fp32 for kRun rows of a lane and are then
+// added into fp64 accumulators kept in shared memory.
 #pragma once
 
 #include "dq_device.cuh"
@@ -35,48 +36,87 @@ constexpr double kColErr = 2.0 * kRun * 0x1p-24 + 1e-11;
 constexpr float kRelGuard = 0x1p-20f;
 
 __host__ __device__ constexpr int ring_stages(int es) { return kRingBytes / (kRowsPerTile * kStripMax * es); }
-__host__ __device__ constexpr size_t iter_col_acc_bytes() {
-  return (size_t)kConsumerWarps * kStripMax * sizeof(double2);
+// fp64 accumulators per consumer warp: 8 column pairs (sum W a q, sum (a q)^2) x 32 lanes + 32 residual sums
+__host__ __device__ constexpr size_t iter_acc_bytes() {
+  return (size_t)kConsumerWarps * (kStripMax * sizeof(double2) + 32 * sizeof(double));
 }
 __host__ __device__ constexpr size_t iter_smem_bytes(int es) {
-  return (size_t)kRingBytes + iter_col_acc_bytes() + 2 * sizeof(uint64_t) * ring_stages(es) +
+  return (size_t)kRingBytes + iter_acc_bytes() + 2 * sizeof(uint64_t) * ring_stages(es) +
          (2 + kStripMax + 4) * sizeof(int);
 }
 
 // ---------------------------------------------------------------------------
-// E2M1 fast path with the hardware conversion: both ends of the bracket
-// [x~ (1 - g), x~ (1 + g)] are converted (round to nearest even, saturating);
-// equal codes prove the exact quotient has that code too (rounding is
-// monotone), different codes flag the pair for the exact path.
+// Packed f32x2 arithmetic (one instruction for a pair of elements).
+typedef unsigned long long f2;
+__device__ __forceinline__ f2 pk(float lo, float hi) {
+  f2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float lo_of(f2 v) {
+  float a, b;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+  return a;
+}
+__device__ __forceinline__ float hi_of(f2 v) {
+  float a, b;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+  return b;
+}
+__device__ __forceinline__ f2 mul2(f2 a, f2 b) {
+  f2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
+  f2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ f2 add2(f2 a, f2 b) {
+  f2 d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f2 splat(float v) { return pk(v, v); }
+
+// ---------------------------------------------------------------------------
+// E2M1 conversions (round to nearest even, saturating) and decode.
 __device__ __forceinline__ uint32_t cvt_e2m1x2(float hi, float lo) {
   uint32_t r;
   asm("{\n.reg .b8 t;\ncvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\ncvt.u32.u8 %0, t;\n}" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
-__device__ __forceinline__ float2 dec_e2m1x2(uint32_t code) {  // low nibble -> .x, high nibble -> .y
+__device__ __forceinline__ f2 dec_e2m1x2(uint32_t code) {  // low nibble -> low float, high nibble -> high float
   uint32_t h;
   asm("{\n.reg .b8 t;\ncvt.u8.u32 t, %1;\ncvt.rn.f16x2.e2m1x2 %0, t;\n}" : "=r"(h) : "r"(code));
-  return __half22float2(*reinterpret_cast<const __half2*>(&h));
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
+  return pk(f.x, f.y);
 }
 
-__device__ __forceinline__ void req8_e2m1(const float uw[8], float ia, float q[8], bool& near) {
-  const float ilo = ia * (1.f - kRelGuard), ihi = ia * (1.f + kRelGuard);
-#pragma unroll
-  for (int c = 0; c < 8; c += 2) {
-    const uint32_t lo = cvt_e2m1x2(uw[c + 1] * ilo, uw[c] * ilo);
-    const uint32_t hi = cvt_e2m1x2(uw[c + 1] * ihi, uw[c] * ihi);
-    near |= lo != hi;
-    const float2 d = dec_e2m1x2(lo);
-    q[c] = d.x;
-    q[c + 1] = d.y;
+// Block-scale factor from storage, decoded with the hardware where it can.
+template <int FMT>
+__device__ __forceinline__ float a_load(const void* store, int64_t idx) {
+  if (FMT == FMT_INT4) {
+    return __half2float(__ldg(reinterpret_cast<const __half*>(store) + idx));
+  } else if (FMT == FMT_MXINT4) {
+    return __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned char*>(store) + idx) << 23);
+  } else {
+    const unsigned short v = __ldg(reinterpret_cast<const unsigned char*>(store) + idx);
+    uint32_t h;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(v));
+    return __half2float(__ushort_as_half((unsigned short)(h & 0xFFFFu)));
   }
 }
 
-// Per-lane state of a column strip segment: b, the candidate factor cb = 1/b
-// (times 1/s_T for NVFP4), the guard threshold per column (MXINT4 columns with a
-// power-of-two b have an exact candidate and need no guard), fp32 column runs.
+// Per-lane state of a column strip segment, as 4 column pairs: b, the
+// candidate factor cb = 1/b (times 1/s_T for NVFP4), fp32 column runs, and the
+// guard threshold per column (MXINT4 columns with a power-of-two b have an exact
+// candidate and need no guard).
 struct ColState {
-  float bj[8], cb[8], thr[8], cn[8], cd[8];
+  f2 b2[4], cb2[4], cn2[4], cd2[4];
+  float thr[8];
+  f2 res2;  // fp32 run of squared reconstruction residuals
   bool ok;
 };
 
@@ -89,43 +129,128 @@ __device__ __noinline__ float qexact64(float w, float a, float b, double sTd) {
   return q_int4<FMT>(xt, w, a, b, sTd);
 }
 
-// Requantize the 8 elements of a lane with block factor a (stored value).
-// Fast path for all lanes; a lane with a flagged element re-derives which
-// elements are close to a boundary and settles only those exactly.
+// Fast requantization of the 8 elements (4 pairs u2 = W * cb) of a lane with
+// block factor a; `near` is raised for a lane with an element too close to a
+// rounding boundary (or factors outside the fast range).
 template <int FMT>
-__device__ __forceinline__ void requant8(const float w[8], const float uw[8], float a, const ColState& cs, float sT,
-                                         double sTd, bool active, float q[8], unsigned* s_cnt) {
-  const float ia = rcp_approx(a);
-  const bool ok = cs.ok && in_range(ia);
-  bool near = !ok;
+__device__ __forceinline__ void req_fast(const f2 u2[4], float a, const ColState& cs, float& ia, bool& ok, f2 q2[4],
+                                         bool& near) {
+  ia = rcp_approx(a);
+  ok = cs.ok && in_range(ia);
+  near = !ok;
   if (FMT == FMT_NVFP4) {
-    req8_e2m1(uw, ia, q, near);
+    const f2 ilo = splat(ia * (1.f - kRelGuard)), ihi = splat(ia * (1.f + kRelGuard));
+    f2 lo[4], hi[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      lo[i] = mul2(u2[i], ilo);
+      hi[i] = mul2(u2[i], ihi);
+    }
+    uint32_t clo, chi, h0, h1, h2, h3;
+    asm("{\n.reg .b8 l0, l1, l2, l3, g0, g1, g2, g3;\n"
+        "cvt.rn.satfinite.e2m1x2.f32 l0, %7, %6;\n"
+        "cvt.rn.satfinite.e2m1x2.f32 l1, %9, %8;\n"
+        "cvt.rn.satfinite.e2m1x2.f32 l2, %11, %10;\n"
+        "cvt.rn.satfinite.e2m1x2.f32 l3, %13, %12;\n"
+        "cvt.rn.satfinite.e2m1x2.f32 g0, %15, %14;\n"
+        "cvt.rn.satfinite.e2m1x2.f32 g1, %17, %16;\n"
+        "cvt.rn.satfinite.e2m1x2.f32 g2, %19, %18;\n"
+        "cvt.rn.satfinite.e2m1x2.f32 g3, %21, %20;\n"
+        "mov.b32 %0, {l0, l1, l2, l3};\n"
+        "mov.b32 %1, {g0, g1, g2, g3};\n"
+        "cvt.rn.f16x2.e2m1x2 %2, l0;\n"
+        "cvt.rn.f16x2.e2m1x2 %3, l1;\n"
+        "cvt.rn.f16x2.e2m1x2 %4, l2;\n"
+        "cvt.rn.f16x2.e2m1x2 %5, l3;\n}"
+        : "=r"(clo), "=r"(chi), "=r"(h0), "=r"(h1), "=r"(h2), "=r"(h3)
+        : "f"(lo_of(lo[0])), "f"(hi_of(lo[0])), "f"(lo_of(lo[1])), "f"(hi_of(lo[1])), "f"(lo_of(lo[2])),
+          "f"(hi_of(lo[2])), "f"(lo_of(lo[3])), "f"(hi_of(lo[3])), "f"(lo_of(hi[0])), "f"(hi_of(hi[0])),
+          "f"(lo_of(hi[1])), "f"(hi_of(hi[1])), "f"(lo_of(hi[2])), "f"(hi_of(hi[2])), "f"(lo_of(hi[3])),
+          "f"(hi_of(hi[3])));
+    near |= clo != chi;
+    const uint32_t hh[4] = {h0, h1, h2, h3};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hh[i]));
+      q2[i] = pk(f.x, f.y);
+    }
+  } else {
+    const f2 ia2 = splat(ia), nia2 = splat(-ia), m2 = splat(12582912.f), nm2 = splat(-12582912.f);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const f2 qu = add2(fma2(u2[i], ia2, m2), nm2);  // round half even
+      const f2 r = fma2(u2[i], nia2, qu);             // qu - x~
+      const float t0 = FMT == FMT_MXINT4 ? cs.thr[2 * i] : 0.5f - kGuard;
+      const float t1 = FMT == FMT_MXINT4 ? cs.thr[2 * i + 1] : 0.5f - kGuard;
+      near |= fabsf(lo_of(r)) > t0;
+      near |= fabsf(hi_of(r)) > t1;
+      q2[i] = pk(fminf(fmaxf(lo_of(qu), -8.f), 7.f), fminf(fmaxf(hi_of(qu), -8.f), 7.f));
+    }
+  }
+}
+
+// Exact settling of a flagged lane: re-derive which elements are close to a
+// boundary and decide only those exactly (all 8 in fp64 when the factors are
+// outside the fast range).
+template <int FMT>
+__device__ __forceinline__ void req_slow(const f2 w2[4], const f2 u2[4], float a, float ia, bool ok, const ColState& cs,
+                                         float sT, double sTd, f2 q2[4]) {
+  float q[8], w[8], u[8], b[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    q[2 * i] = lo_of(q2[i]);
+    q[2 * i + 1] = hi_of(q2[i]);
+    w[2 * i] = lo_of(w2[i]);
+    w[2 * i + 1] = hi_of(w2[i]);
+    u[2 * i] = lo_of(u2[i]);
+    u[2 * i + 1] = hi_of(u2[i]);
+    b[2 * i] = lo_of(cs.b2[i]);
+    b[2 * i + 1] = hi_of(cs.b2[i]);
+  }
+  if (!ok) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) q[c] = qexact64<FMT>(w[c], a, b[c], sTd);
+  } else if (FMT == FMT_NVFP4) {
+    const float ilo = ia * (1.f - kRelGuard), ihi = ia * (1.f + kRelGuard);
+#pragma unroll
+    for (int c = 0; c < 8; c += 2) {
+      const uint32_t lo = cvt_e2m1x2(u[c + 1] * ilo, u[c] * ilo);
+      const uint32_t hi = cvt_e2m1x2(u[c + 1] * ihi, u[c] * ihi);
+      const uint32_t diff = lo ^ hi;
+      if (diff & 0x0Fu) q[c] = qexact32_e2m1(w[c], u[c], ia, a * b[c], sT);
+      if (diff & 0xF0u) q[c + 1] = qexact32_e2m1(w[c + 1], u[c + 1], ia, a * b[c + 1], sT);
+    }
   } else {
 #pragma unroll
-    for (int c = 0; c < 8; ++c) q[c] = qfast_int4(uw[c], ia, FMT == FMT_MXINT4 ? cs.thr[c] : 0.5f - kGuard, near);
+    for (int c = 0; c < 8; ++c) {
+      const float qu = fmaf(u[c], ia, 12582912.f) - 12582912.f;
+      const float thr = FMT == FMT_MXINT4 ? cs.thr[c] : 0.5f - kGuard;
+      if (fabsf(fmaf(u[c], ia, -qu)) > thr) q[c] = qexact32_int4(w[c], u[c], ia, a * b[c]);
+    }
   }
-  if (near && active) {
-    atomicAdd(&s_cnt[0], 1u);
-    if (!ok) {
 #pragma unroll
-      for (int c = 0; c < 8; ++c) q[c] = qexact64<FMT>(w[c], a, cs.bj[c], sTd);
-    } else if (FMT == FMT_NVFP4) {
-      const float ilo = ia * (1.f - kRelGuard), ihi = ia * (1.f + kRelGuard);
-#pragma unroll
-      for (int c = 0; c < 8; c += 2) {
-        const uint32_t lo = cvt_e2m1x2(uw[c + 1] * ilo, uw[c] * ilo);
-        const uint32_t hi = cvt_e2m1x2(uw[c + 1] * ihi, uw[c] * ihi);
-        const uint32_t diff = lo ^ hi;
-        if (diff & 0x0Fu) q[c] = qexact32_e2m1(w[c], uw[c], ia, a * cs.bj[c], sT);
-        if (diff & 0xF0u) q[c + 1] = qexact32_e2m1(w[c + 1], uw[c + 1], ia, a * cs.bj[c + 1], sT);
-      }
-    } else {
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const float qu = fmaf(uw[c], ia, 12582912.f) - 12582912.f;
-        const float thr = FMT == FMT_MXINT4 ? cs.thr[c] : 0.5f - kGuard;
-        if (fabsf(fmaf(uw[c], ia, -qu)) > thr) q[c] = qexact32_int4(w[c], uw[c], ia, a * cs.bj[c]);
-      }
+  for (int i = 0; i < 4; ++i) q2[i] = pk(q[2 * i], q[2 * i + 1]);
+}
+
+// Requantize two rows of a lane (x = row a, y = row b) with block factors fa, fb.
+template <int FMT>
+__device__ __forceinline__ void req_pair(const f2 wx[4], const f2 ux[4], float fa, bool actx, const f2 wy[4],
+                                         const f2 uy[4], float fb, bool acty, const ColState& cs, float sT, double sTd,
+                                         f2 qx[4], f2 qy[4], unsigned* s_cnt) {
+  float iax, iay;
+  bool okx, oky, nx, ny;
+  req_fast<FMT>(ux, fa, cs, iax, okx, qx, nx);
+  req_fast<FMT>(uy, fb, cs, iay, oky, qy, ny);
+  nx = nx && actx;
+  ny = ny && acty;
+  if (nx || ny) {
+    if (nx) {
+      atomicAdd(&s_cnt[0], 1u);
+      req_slow<FMT>(wx, ux, fa, iax, okx, cs, sT, sTd, qx);
+    }
+    if (ny) {
+      atomicAdd(&s_cnt[0], 1u);
+      req_slow<FMT>(wy, uy, fb, iay, oky, cs, sT, sTd, qy);
     }
   }
 }
@@ -177,100 +302,158 @@ __device__ double2 column_exact(const Problem& p, int64_t j, float bj, double sT
   return r;
 }
 
-
+// ---------------------------------------------------------------------------
+// One row of W for one lane (8 elements as 4 pairs, exact fp32 values).
 template <int WDT>
-__device__ __forceinline__ void smem_row8(const unsigned char* src, float w[8]) {
+__device__ __forceinline__ void smem_row(const unsigned char* src, f2 w2[4]) {
   if (WDT == DT_F32) {
     const float4 x = *reinterpret_cast<const float4*>(src);
     const float4 y = *reinterpret_cast<const float4*>(src + 16);
-    w[0] = x.x; w[1] = x.y; w[2] = x.z; w[3] = x.w;
-    w[4] = y.x; w[5] = y.y; w[6] = y.z; w[7] = y.w;
+    w2[0] = pk(x.x, x.y);
+    w2[1] = pk(x.z, x.w);
+    w2[2] = pk(y.x, y.y);
+    w2[3] = pk(y.z, y.w);
   } else {
     const uint4 v = *reinterpret_cast<const uint4*>(src);
     const uint32_t uu[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       if (WDT == DT_BF16) {
-        w[2 * i] = __uint_as_float(uu[i] << 16);
-        w[2 * i + 1] = __uint_as_float(uu[i] & 0xFFFF0000u);
+        w2[i] = pk(__uint_as_float(uu[i] << 16), __uint_as_float(uu[i] & 0xFFFF0000u));
       } else {
         const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&uu[i]));
-        w[2 * i] = f.x;
-        w[2 * i + 1] = f.y;
+        w2[i] = pk(f.x, f.y);
       }
     }
   }
 }
 
-// One row of one lane: requantize the incoming iterate, block sums and update,
-// requantize, column sums.  Warp-collective (shuffles); `active` lanes hold
-// real columns.  Returns nothing; updates cs, mse_acc and the counters.
+// Block sums, residuals of the incoming iterate, for one row of one lane.
 template <int FMT>
-__device__ __forceinline__ void row_step(const Problem& p, const float w[8], float aold, int64_t bidx, bool active,
-                                         bool leader, int lpb, ColState& cs, float sT, float isT, double sTd,
-                                         double& mse_acc, unsigned* s_cnt) {
-  float uw[8], q[8];
+__device__ __forceinline__ void row_sums(const f2 w2[4], const f2 q2[4], float aold, const ColState& cs, float sT,
+                                         f2 rscale2, float& num, float& den, f2& res2) {
+  const f2 na2 = splat(FMT == FMT_NVFP4 ? -(aold * sT) : -aold);
+  f2 num2 = 0ull, den2 = 0ull;
 #pragma unroll
-  for (int c = 0; c < 8; ++c) uw[c] = w[c] * cs.cb[c];
-  requant8<FMT>(w, uw, aold, cs, sT, sTd, active, q, s_cnt);
-  float num = 0.f, den = 0.f;
+  for (int i = 0; i < 4; ++i) {
+    const f2 pq = mul2(q2[i], cs.b2[i]);
+    num2 = fma2(w2[i], pq, num2);
+    den2 = fma2(pq, pq, den2);
+    const f2 e = mul2(fma2(pq, na2, w2[i]), rscale2);  // residual times a power of two (range)
+    res2 = fma2(e, e, res2);
+  }
+  num = lo_of(num2) + hi_of(num2);
+  den = lo_of(den2) + hi_of(den2);
+}
+
+// Exact fp64 block sums of one row of one lane (warp-collective reduction).
+__device__ __forceinline__ void row_sums64(const f2 w2[4], const f2 q2[4], const ColState& cs, int lpb, double& n64,
+                                           double& d64) {
+  n64 = 0.0;
+  d64 = 0.0;
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    const float pq = q[c] * cs.bj[c];
-    num = fmaf(w[c], pq, num);
-    den = fmaf(pq, pq, den);
+  for (int i = 0; i < 4; ++i) {
+    const f2 pq = mul2(q2[i], cs.b2[i]);  // exact products
+    n64 = fma((double)lo_of(w2[i]), (double)lo_of(pq), n64);
+    d64 = fma((double)lo_of(pq), (double)lo_of(pq), d64);
+    n64 = fma((double)hi_of(w2[i]), (double)hi_of(pq), n64);
+    d64 = fma((double)hi_of(pq), (double)hi_of(pq), d64);
   }
   for (int o = 1; o < lpb; o <<= 1) {
-    num += __shfl_xor_sync(0xffffffffu, num, o);
-    den += __shfl_xor_sync(0xffffffffu, den, o);
-  }
-  bool amb = false;
-  float anew = a_fast<FMT>(num, den, isT, amb);
-  double nsum = (double)num, dsum = (double)den;
-  if (__any_sync(0xffffffffu, amb && active)) {
-    double n64 = 0.0, d64 = 0.0;
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const double pd = (double)(q[c] * cs.bj[c]);
-      n64 = fma((double)w[c], pd, n64);
-      d64 = fma(pd, pd, d64);
-    }
-    for (int o = 1; o < lpb; o <<= 1) {
-      n64 += __shfl_xor_sync(0xffffffffu, n64, o);
-      d64 += __shfl_xor_sync(0xffffffffu, d64, o);
-    }
-    if (amb) {
-      if (active && leader) atomicAdd(&s_cnt[1], 1u);
-      anew = d64 == 0.0 ? 1.f : (float)a_project<FMT>(n64 / d64, sTd);
-      nsum = n64;
-      dsum = d64;
-    }
-  }
-  if (active && leader) {
-    const double av = FMT == FMT_NVFP4 ? sTd * (double)aold : (double)aold;
-    mse_acc += av * (av * dsum - 2.0 * nsum);
-    a_store_f<FMT>(p.a_store, bidx, anew);
-  }
-  requant8<FMT>(w, uw, anew, cs, sT, sTd, active, q, s_cnt);
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    const float sv = q[c] * anew;  // exact; NVFP4 leaves s_T out
-    cs.cn[c] = fmaf(w[c], sv, cs.cn[c]);
-    cs.cd[c] = fmaf(sv, sv, cs.cd[c]);
+    n64 += __shfl_xor_sync(0xffffffffu, n64, o);
+    d64 += __shfl_xor_sync(0xffffffffu, d64, o);
   }
 }
 
-// fp32 column runs into the warp's fp64 accumulators (layout [warp][c][lane]).
-__device__ __forceinline__ void flush_runs(ColState& cs, double2* acc, int warp, int lane) {
+// Two rows of one lane (x = row a, y = row b; y may be absent, then its data
+// are zero and nothing of it is written): requantize the incoming iterate;
+// block sums, residuals and block updates; requantize with the new block
+// scales where they changed; column sums.  Warp-collective (shuffles and
+// votes); `active` lanes hold real columns and alone write results.
+template <int FMT>
+__device__ __forceinline__ void row_pair(const Problem& p, const f2 wx[4], float ax_old, int64_t bidx_x,
+                                         const f2 wy[4], float ay_old, int64_t bidx_y, bool has_y, bool active,
+                                         bool leader, int lpb, ColState& cs, float sT, float isT, double sTd,
+                                         f2 rscale2, unsigned* s_cnt) {
+  const bool actx = active, acty = active && has_y;
+  f2 ux[4], uy[4], qx[4], qy[4];
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    double2& a = acc[(warp * 8 + c) * 32 + lane];
-    double2 v = a;
-    v.x += (double)cs.cn[c];
-    v.y += (double)cs.cd[c];
-    a = v;
-    cs.cn[c] = cs.cd[c] = 0.f;
+  for (int i = 0; i < 4; ++i) {
+    ux[i] = mul2(wx[i], cs.cb2[i]);
+    uy[i] = mul2(wy[i], cs.cb2[i]);
   }
+  req_pair<FMT>(wx, ux, ax_old, actx, wy, uy, ay_old, acty, cs, sT, sTd, qx, qy, s_cnt);
+  float nx, dx, ny, dy;
+  row_sums<FMT>(wx, qx, ax_old, cs, sT, rscale2, nx, dx, cs.res2);
+  row_sums<FMT>(wy, qy, ay_old, cs, sT, rscale2, ny, dy, cs.res2);
+  for (int o = 1; o < lpb; o <<= 1) {
+    nx += __shfl_xor_sync(0xffffffffu, nx, o);
+    dx += __shfl_xor_sync(0xffffffffu, dx, o);
+    ny += __shfl_xor_sync(0xffffffffu, ny, o);
+    dy += __shfl_xor_sync(0xffffffffu, dy, o);
+  }
+  bool ambx = false, amby = false;
+  float anx = a_fast<FMT>(nx, dx, isT, ambx);
+  float any = a_fast<FMT>(ny, dy, isT, amby);
+  ambx = ambx && actx;
+  amby = amby && acty;
+  if (__any_sync(0xffffffffu, ambx || amby)) {
+    double n64, d64;
+    row_sums64(wx, qx, cs, lpb, n64, d64);
+    if (ambx) {
+      if (leader) atomicAdd(&s_cnt[1], 1u);
+      anx = d64 == 0.0 ? 1.f : (float)a_project<FMT>(n64 / d64, sTd);
+    }
+    row_sums64(wy, qy, cs, lpb, n64, d64);
+    if (amby) {
+      if (leader) atomicAdd(&s_cnt[1], 1u);
+      any = d64 == 0.0 ? 1.f : (float)a_project<FMT>(n64 / d64, sTd);
+    }
+  }
+  // the storage already holds the old factors; with a block scale unchanged the
+  // codes are unchanged too (same a, same b), so requantize only where it changed
+  const bool chx = anx != ax_old && actx, chy = any != ay_old && acty;
+  if (chx && leader) a_store_f<FMT>(p.a_store, bidx_x, anx);
+  if (chy && leader) a_store_f<FMT>(p.a_store, bidx_y, any);
+  if (__any_sync(0xffffffffu, chx || chy)) {
+    // recomputed rather than kept live across the block update (registers)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      ux[i] = mul2(wx[i], cs.cb2[i]);
+      uy[i] = mul2(wy[i], cs.cb2[i]);
+    }
+    req_pair<FMT>(wx, ux, anx, actx, wy, uy, any, acty, cs, sT, sTd, qx, qy, s_cnt);
+  }
+  const f2 anx2 = splat(anx), any2 = splat(any);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const f2 svx = mul2(qx[i], anx2);  // exact; NVFP4 leaves s_T out
+    const f2 svy = mul2(qy[i], any2);
+    cs.cn2[i] = fma2(wx[i], svx, cs.cn2[i]);
+    cs.cd2[i] = fma2(svx, svx, cs.cd2[i]);
+    cs.cn2[i] = fma2(wy[i], svy, cs.cn2[i]);
+    cs.cd2[i] = fma2(svy, svy, cs.cd2[i]);
+  }
+}
+
+// fp32 runs into the warp's fp64 accumulators (layout [warp][c][lane], then
+// [warp][lane] for the residuals).
+__device__ __forceinline__ void flush_runs(ColState& cs, double2* acc, double* racc, int warp, int lane,
+                                           bool active) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      double2& a = acc[(warp * 8 + 2 * i + h) * 32 + lane];
+      double2 v = a;
+      v.x += (double)(h ? hi_of(cs.cn2[i]) : lo_of(cs.cn2[i]));
+      v.y += (double)(h ? hi_of(cs.cd2[i]) : lo_of(cs.cd2[i]));
+      a = v;
+    }
+    cs.cn2[i] = cs.cd2[i] = 0ull;
+  }
+  if (active) racc[warp * 32 + lane] += (double)lo_of(cs.res2) + (double)hi_of(cs.res2);
+  cs.res2 = 0ull;
 }
 
 template <int FMT, int WDT>
@@ -281,7 +464,8 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t) {
   extern __shared__ __align__(128) unsigned char smem[];
   unsigned char* ring = smem;
   double2* acc = reinterpret_cast<double2*>(smem + kRingBytes);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kRingBytes + iter_col_acc_bytes());
+  double* racc = reinterpret_cast<double*>(acc + kConsumerWarps * kStripMax);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kRingBytes + iter_acc_bytes());
   uint64_t* empty = full + S;
   int* s_misc = reinterpret_cast<int*>(empty + S);  // [0] ticket result, [1] #ambiguous, [2..] columns
   unsigned* s_cnt = reinterpret_cast<unsigned*>(s_misc + 2 + kStripMax);  // exact-path counters
@@ -297,6 +481,7 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t) {
     mbar_fence_init();
     s_cnt[0] = s_cnt[1] = s_cnt[2] = 0u;
   }
+  if (threadIdx.x < kConsumers) racc[threadIdx.x] = 0.0;
   __syncthreads();
 
   const int64_t k = blockIdx.x;
@@ -304,7 +489,8 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t) {
 
   if (warp == kConsumerWarps) {
     // ---------------- producer warp ----------------
-    int64_t tile = 0;
+    int st = 0;
+    unsigned par = 1u;
     for (int64_t u = u_begin; u < u_end;) {
       const int64_t s = u / p.M;
       const int64_t r0 = u - s * p.M;
@@ -312,17 +498,17 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t) {
       const int64_t c0 = s * p.TS;
       const int width = (int)min((int64_t)p.TS, p.N - c0);
       const unsigned bytes = (unsigned)(width * ES);
-      for (int64_t tr = r0; tr < r1; tr += kRowsPerTile, ++tile) {
-        const int st = (int)(tile % S);
-        const unsigned par = (unsigned)((tile / S) & 1) ^ 1u;
+      const unsigned char* src = reinterpret_cast<const unsigned char*>(p.W) + ((r0 + lane) * p.N + c0) * (int64_t)ES;
+      const int64_t src_step = (int64_t)kRowsPerTile * p.N * ES;
+      for (int64_t tr = r0; tr < r1; tr += kRowsPerTile, src += src_step) {
         mbar_wait(&empty[st], par, &p.hdr->flags);
         const int nr = (int)min((int64_t)kRowsPerTile, r1 - tr);
         if (lane == 0) mbar_arrive_expect_tx(&full[st], (unsigned)nr * bytes);
         __syncwarp();
-        if (lane < nr) {
-          const unsigned char* src =
-              reinterpret_cast<const unsigned char*>(p.W) + ((tr + lane) * p.N + c0) * (int64_t)ES;
-          bulk_g2s(ring + st * stage_bytes + lane * row_bytes, src, bytes, &full[st]);
+        if (lane < nr) bulk_g2s(ring + st * stage_bytes + lane * row_bytes, src, bytes, &full[st]);
+        if (++st == S) {
+          st = 0;
+          par ^= 1u;
         }
       }
       u = (s + 1) * p.M;
@@ -333,13 +519,20 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t) {
   // ---------------- consumer warps ----------------
   const int lpb = p.G / 8;  // lanes per block
   const bool leader = (lane & (lpb - 1)) == 0;
+  // residuals are squared after scaling by rscale = 2^-floor(log2 amax), which
+  // keeps every square inside the fp32 range whatever the magnitude of W
+  const uint32_t amax_bits = p.hdr->amax_bits;
+  const int amax_exp = (amax_bits == 0u) ? 0 : (int)((amax_bits >> 23) & 0xFFu) - 127;
+  const float rscale = __uint_as_float((uint32_t)(127 - max(-126, min(126, amax_exp))) << 23);
+  const f2 rscale2 = splat(rscale);
+  const double rscale_d = (double)rscale;
   const float sT = p.hdr->sT;
   const double sTd = (double)sT;
   const float isT = FMT == FMT_NVFP4 ? __frcp_rn(sT) : 1.f;
   const bool sT_ok = FMT != FMT_NVFP4 || in_range(isT);
   const int64_t s_first = u_begin / p.M;
-  double mse_acc = 0.0;
-  int64_t tile = 0;
+  int st = 0;
+  unsigned par = 0u;
 
   for (int64_t u = u_begin; u < u_end;) {
     const int64_t s = u / p.M;
@@ -353,62 +546,67 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t) {
 
     ColState cs;
     cs.ok = sT_ok;
+    cs.res2 = 0ull;
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      cs.bj[c] = 1.f;
-      cs.cb[c] = 1.f;
-      cs.thr[c] = 0.5f - kGuard;
-      cs.cn[c] = cs.cd[c] = 0.f;
-      acc[(warp * 8 + c) * 32 + lane] = make_double2(0.0, 0.0);
-    }
-    if (active) {
+    for (int i = 0; i < 4; ++i) {
+      float bj[2] = {1.f, 1.f}, cb[2] = {1.f, 1.f};
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        cs.bj[c] = b_decode(p.b_store, p.col_dt, col + c);
-        cs.cb[c] = __frcp_rn(cs.bj[c]) * isT;
-        cs.ok = cs.ok && in_range(cs.cb[c]);
-        // MXINT4: a = 2^k, so a power-of-two b makes the candidate exact
-        if (FMT == FMT_MXINT4 && (__float_as_uint(cs.bj[c]) & 0x007FFFFFu) == 0u) cs.thr[c] = 2.f;
+      for (int h = 0; h < 2; ++h) {
+        const int c = 2 * i + h;
+        cs.thr[c] = 0.5f - kGuard;
+        if (active) {
+          bj[h] = b_decode(p.b_store, p.col_dt, col + c);
+          cb[h] = __frcp_rn(bj[h]) * isT;
+          cs.ok = cs.ok && in_range(cb[h]);
+          // MXINT4: a = 2^k, so a power-of-two b makes the candidate exact
+          if (FMT == FMT_MXINT4 && (__float_as_uint(bj[h]) & 0x007FFFFFu) == 0u) cs.thr[c] = 2.f;
+        }
+        acc[(warp * 8 + c) * 32 + lane] = make_double2(0.0, 0.0);
       }
+      cs.b2[i] = pk(bj[0], bj[1]);
+      cs.cb2[i] = pk(cb[0], cb[1]);
+      cs.cn2[i] = cs.cd2[i] = 0ull;
     }
     int run = 0;
     // block scales of this warp's rows, one tile ahead
+    const int64_t a_step = (int64_t)kRowsPerTile * p.nb;
+    int64_t aidx = (r0 + warp) * p.nb + blk_col;
     float an0 = 1.f, an1 = 1.f;
-    if (active && r0 + warp < r1) an0 = a_decode<FMT>(p.a_store, (r0 + warp) * p.nb + blk_col);
-    if (active && r0 + warp + kConsumerWarps < r1)
-      an1 = a_decode<FMT>(p.a_store, (r0 + warp + kConsumerWarps) * p.nb + blk_col);
+    if (active && r0 + warp < r1) an0 = a_load<FMT>(p.a_store, aidx);
+    if (active && r0 + warp + kConsumerWarps < r1) an1 = a_load<FMT>(p.a_store, aidx + kConsumerWarps * p.nb);
 
-    for (int64_t tr = r0; tr < r1; tr += kRowsPerTile, ++tile) {
-      const int st = (int)(tile % S);
-      const unsigned par = (unsigned)((tile / S) & 1);
+    for (int64_t tr = r0; tr < r1; tr += kRowsPerTile, aidx += a_step) {
       const int64_t ra = tr + warp, rb = ra + kConsumerWarps;
       const bool has_a = ra < r1, has_b = rb < r1;  // warp-uniform
       const float aa = an0, ab = an1;
-      if (active && ra + kRowsPerTile < r1) an0 = a_decode<FMT>(p.a_store, (ra + kRowsPerTile) * p.nb + blk_col);
-      if (active && rb + kRowsPerTile < r1) an1 = a_decode<FMT>(p.a_store, (rb + kRowsPerTile) * p.nb + blk_col);
+      if (active && ra + kRowsPerTile < r1) an0 = a_load<FMT>(p.a_store, aidx + a_step);
+      if (active && rb + kRowsPerTile < r1) an1 = a_load<FMT>(p.a_store, aidx + a_step + kConsumerWarps * p.nb);
       mbar_wait(&full[st], par, &p.hdr->flags);
-      float wa[8], wb[8];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) wa[c] = wb[c] = 0.f;
+      f2 wa[4], wb[4];
       const unsigned char* base = ring + st * stage_bytes + lane * 8 * ES;
-      if (active && has_a) smem_row8<WDT>(base + warp * row_bytes, wa);
-      if (active && has_b) smem_row8<WDT>(base + (warp + kConsumerWarps) * row_bytes, wb);
+      smem_row<WDT>(base + warp * row_bytes, wa);
+      smem_row<WDT>(base + (warp + kConsumerWarps) * row_bytes, wb);
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[st]);
-      if (has_a) {
-        row_step<FMT>(p, wa, aa, ra * p.nb + blk_col, active, leader, lpb, cs, sT, isT, sTd, mse_acc, s_cnt);
-        ++run;
+      if (++st == S) {
+        st = 0;
+        par ^= 1u;
       }
-      if (has_b) {
-        row_step<FMT>(p, wb, ab, rb * p.nb + blk_col, active, leader, lpb, cs, sT, isT, sTd, mse_acc, s_cnt);
-        ++run;
+      if (has_a) {
+        if (!has_b) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) wb[i] = 0ull;  // absent row: zeros contribute nothing
+        }
+        row_pair<FMT>(p, wa, aa, aidx, wb, ab, aidx + kConsumerWarps * p.nb, has_b, active, leader, lpb, cs, sT, isT,
+                      sTd, rscale2, s_cnt);
+        run += has_b ? 2 : 1;
       }
       if (run >= kRun) {
         run = 0;
-        flush_runs(cs, acc, warp, lane);
+        flush_runs(cs, acc, racc, warp, lane, active);
       }
     }
-    flush_runs(cs, acc, warp, lane);
+    flush_runs(cs, acc, racc, warp, lane, active);
 
     // CTA reduction of the column sums over the consumer warps, fixed order.
     // Thread t sums entry (c, l) = (t / 32, t % 32), i.e. column 8 (t % 32) + t / 32.
@@ -484,9 +682,10 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t) {
     u = (s + 1) * p.M;
   }
 
-  // MSE of the incoming iterate: CTA sum, then CTA-ordered total
+  // MSE of the incoming iterate: per-thread residual sums, CTA tree, then the
+  // CTA-ordered total (the residual accumulators are not reused above).
   double* mred = reinterpret_cast<double*>(acc);
-  mred[threadIdx.x] = mse_acc;
+  mred[threadIdx.x] = racc[threadIdx.x];
   consumer_sync(kConsumers);
   for (int o = kConsumerTreeTop; o > 0; o >>= 1) {
     if (threadIdx.x < o && threadIdx.x + o < kConsumers) mred[threadIdx.x] += mred[threadIdx.x + o];
@@ -501,9 +700,9 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t) {
     const unsigned prev = atomicAdd(&p.hdr->cta_counter, 1u);
     if (prev == (unsigned)p.P - 1u) {
       __threadfence();
-      double tot = p.hdr->sumW2;
+      double tot = 0.0;
       for (int64_t kk = 0; kk < p.P; ++kk) tot += __ldcg(&p.cta_part[kk]);
-      p.mse[t - 1] = tot / ((double)p.M * (double)p.N);
+      p.mse[t - 1] = tot / (rscale_d * rscale_d) / ((double)p.M * (double)p.N);
       p.hdr->cta_counter = 0u;
     }
   }

@@ -23,9 +23,9 @@
 // last CTA to finish a strip (atomic ticket, no waiting) sums the partials of
 // that strip in CTA order -- a fixed order, so the result is deterministic --
 // and writes the new column scales.  The reconstruction MSE of the iterate
-// entering iteration t is accumulated from the block sums,
-// sum (W - a q b)^2 = sum W^2 - sum_blocks (2 a num - a^2 den),
-// per CTA, then summed in CTA order by the last CTA.
+// entering iteration t is accumulated from the residuals W - a q b of the
+// requantized incoming iterate (fp32 runs into fp64), per CTA, then summed in
+// CTA order by the last CTA.
 #include "dq_device.cuh"
 #include "dq_fast.cuh"
 #include "dq_internal.h"
@@ -50,14 +50,11 @@ __device__ __forceinline__ bool arrive_last(unsigned* counter, unsigned expected
 }
 
 // ---------------------------------------------------------------------------
-// Statistics pass: non-finite check, max |W|, sum W^2.
+// Statistics pass: non-finite check and max |W| (for the NVFP4 tensor scale).
 template <int WDT>
 __global__ void __launch_bounds__(kThreads) k_stats(Problem p) {
-  __shared__ double red[kThreads];
-  __shared__ int s_last;
   const int64_t nchunks = p.M * p.N / 8;
   float amax = 0.f;
-  double s2 = 0.0;
   bool bad = false;
   for (int64_t c = (int64_t)blockIdx.x * kThreads + threadIdx.x; c < nchunks; c += (int64_t)gridDim.x * kThreads) {
     float w[8];
@@ -66,28 +63,12 @@ __global__ void __launch_bounds__(kThreads) k_stats(Problem p) {
     for (int k = 0; k < 8; ++k) {
       bad |= !isfinite(w[k]);
       amax = fmaxf(amax, fabsf(w[k]));
-      s2 = fma((double)w[k], (double)w[k], s2);
     }
   }
   if (bad) atomicOr(&p.hdr->flags, kFlagNonFinite);
   // max of non-negative floats = max of their bit patterns (order independent)
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   if ((threadIdx.x & 31) == 0 && isfinite(amax)) atomicMax(&p.hdr->amax_bits, __float_as_uint(amax));
-  red[threadIdx.x] = s2;
-  __syncthreads();
-  for (int o = kThreads / 2; o > 0; o >>= 1) {
-    if (threadIdx.x < o) red[threadIdx.x] += red[threadIdx.x + o];
-    __syncthreads();
-  }
-  if (threadIdx.x == 0) p.cta_part[blockIdx.x] = red[0];
-  if (arrive_last(&p.hdr->cta_counter, gridDim.x, &s_last)) {
-    if (threadIdx.x == 0) {
-      double tot = 0.0;
-      for (unsigned k = 0; k < gridDim.x; ++k) tot += __ldcg(&p.cta_part[k]);
-      p.hdr->sumW2 = tot;
-      p.hdr->cta_counter = 0u;
-    }
-  }
 }
 
 // ---------------------------------------------------------------------------
