@@ -70,6 +70,8 @@ def load_library():
     lib.dq_solve_host.restype = I
     lib.dq_diagnostics.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint64)]
     lib.dq_diagnostics.restype = I
+    lib.dq_solve_static.argtypes = [P, I, I64, I64, I, I, I, I, ctypes.POINTER(_Outputs), P, P]
+    lib.dq_solve_static.restype = I
     lib.dq_status_str.argtypes = [I]
     lib.dq_status_str.restype = ctypes.c_char_p
     _lib = lib
@@ -153,6 +155,43 @@ def dq_solve(W: torch.Tensor, fmt, group: Optional[int] = None, iters: int = 0, 
         if st != 0:
             raise DQError(st, "dq_solve (device)")
     out["workspace"] = workspace
+    return out
+
+
+def dq_solve_static(W: torch.Tensor, fmt, group: Optional[int] = None, iters: int = 0,
+                    col_dtype: Optional[str] = None, out: Optional[dict] = None, status: Optional[torch.Tensor] = None,
+                    stream=None, check: bool = True) -> dict:
+    """Enqueue dq_solve_static: dq_solve with its scratch in the library's own
+    fixed device array (no workspace).  ``status`` is an optional int32 CUDA
+    tensor of one element that receives the device-side status; with ``check``
+    the call waits for the stream and raises on a non-zero status.  Pass
+    preallocated ``out`` and ``status`` to keep the call free of allocations."""
+    lib = load_library()
+    if not W.is_cuda:
+        raise DQError(1, "dq_solve_static: W must be a CUDA tensor")
+    f = _fmt(fmt)
+    g = DEFAULT_GROUP[f] if group is None else group
+    cd = DEFAULT_COL_DTYPE[f] if col_dtype is None else col_dtype
+    rows, cols = W.shape
+    if W.dtype not in _DTYPES or not W.is_contiguous():
+        raise DQError(1, "dq_solve_static: W must be contiguous f32/bf16/f16")
+    if out is None:
+        out = alloc_outputs(rows, cols, f, g, cd, iters, W.device)
+    if status is None and check:
+        status = torch.full((1,), -1, dtype=torch.int32, device=W.device)
+    if status is not None and (status.dtype != torch.int32 or not status.is_cuda):
+        raise DQError(1, "dq_solve_static: status must be an int32 CUDA tensor")
+    o = _outputs_struct(out)
+    st = lib.dq_solve_static(W.data_ptr(), _DTYPES[W.dtype], rows, cols, int(f), g, iters, 2 if cd == "f16" else 1,
+                             ctypes.byref(o), None if status is None else status.data_ptr(), _stream_ptr(stream))
+    if st != 0:
+        raise DQError(st, "dq_solve_static")
+    if check:
+        (torch.cuda.current_stream() if stream is None else stream).synchronize()
+        dev_st = int(status.cpu()[0])
+        if dev_st != 0:
+            raise DQError(dev_st, "dq_solve_static (device)")
+    out["status"] = status
     return out
 
 

@@ -79,6 +79,10 @@ int check_outputs(const dq_outputs* out, int format, int col_dtype) {
   return DQ_OK;
 }
 
+}  // namespace
+
+namespace dq {
+
 int solve_impl(const void* W, int w_dtype, int64_t rows, int64_t cols, int format, int group, int iters,
                int col_dtype, const dq_outputs* out, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   int st = check_shape(rows, cols, format, group);
@@ -96,7 +100,7 @@ int solve_impl(const void* W, int w_dtype, int64_t rows, int64_t cols, int forma
   if (workspace_bytes < pl.total) return DQ_EWORKSPACE;
 
   char* ws = static_cast<char*>(workspace);
-  Problem p;
+  dq::Problem p;
   std::memset(&p, 0, sizeof(p));
   p.W = W;
   p.wdt = w_dtype;
@@ -129,7 +133,7 @@ int solve_impl(const void* W, int w_dtype, int64_t rows, int64_t cols, int forma
   return DQ_OK;
 }
 
-}  // namespace
+}  // namespace dq
 
 extern "C" {
 
@@ -142,13 +146,13 @@ size_t dq_workspace_bytes(int64_t rows, int64_t cols, int format, int group) {
 
 int dq_solve(const void* W, int w_dtype, int64_t rows, int64_t cols, int format, int group, int iters, int col_dtype,
              const dq_outputs* out, void* workspace, size_t workspace_bytes, void* stream) {
-  return solve_impl(W, w_dtype, rows, cols, format, group, iters, col_dtype, out, workspace, workspace_bytes,
+  return dq::solve_impl(W, w_dtype, rows, cols, format, group, iters, col_dtype, out, workspace, workspace_bytes,
                     static_cast<cudaStream_t>(stream));
 }
 
 int dq_rtn(const void* W, int w_dtype, int64_t rows, int64_t cols, int format, int group, int col_dtype,
            const dq_outputs* out, void* workspace, size_t workspace_bytes, void* stream) {
-  return solve_impl(W, w_dtype, rows, cols, format, group, 0, col_dtype, out, workspace, workspace_bytes,
+  return dq::solve_impl(W, w_dtype, rows, cols, format, group, 0, col_dtype, out, workspace, workspace_bytes,
                     static_cast<cudaStream_t>(stream));
 }
 
@@ -223,7 +227,7 @@ int dq_solve_host(const void* W_host, int w_dtype, int64_t rows, int64_t cols, i
   const size_t ws_bytes = device_workspace_bytes - (size_t)(base - static_cast<char*>(device_workspace));
 
   if (cudaMemcpyAsync(dW, W_host, bytes_w, cudaMemcpyHostToDevice, s) != cudaSuccess) return DQ_ECUDA;
-  st = solve_impl(dW, w_dtype, rows, cols, format, group, iters, col_dtype, &dout, ws, ws_bytes, s);
+  st = dq::solve_impl(dW, w_dtype, rows, cols, format, group, iters, col_dtype, &dout, ws, ws_bytes, s);
   if (st != DQ_OK) return st;
   if (out_host->codes && cudaMemcpyAsync(out_host->codes, dout.codes, bytes_codes, cudaMemcpyDeviceToHost, s))
     return DQ_ECUDA;

@@ -4,6 +4,8 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "dq.h"
+
 namespace dq {
 
 constexpr int kThreads = 256;   // 8 warps per CTA
@@ -53,5 +55,11 @@ struct Problem {
 };
 
 cudaError_t launch_solve(const Problem& p, int iters, int stats_ctas, cudaStream_t st);
+
+// Host-side validation, workspace layout and enqueue of a whole solve (the body
+// of dq_solve; `workspace` is a device address of at least the planned size).
+int solve_impl(const void* W, int w_dtype, int64_t rows, int64_t cols, int format, int group, int iters,
+               int col_dtype, const dq_outputs* out, void* workspace, size_t workspace_bytes,
+               cudaStream_t stream);
 
 }  // namespace dq

@@ -133,6 +133,40 @@ int dq_solve_host(const void* W_host, int w_dtype, int64_t rows, int64_t cols, i
  * Counts cover the BCD iterations only (not init or the final pass). */
 int dq_diagnostics(const void* workspace, void* stream, uint64_t out[3]);
 
+/* Size of the library-owned device scratch that dq_solve_static uses: 8 MiB.
+ * A shape fits when dq_workspace_bytes(rows, cols, format, group) is at most
+ * this; on a 148-SM B200 that holds every shape with cols <= 262144. */
+#define DQ_STATIC_SCRATCH_BYTES (8u << 20)
+
+/* dq_solve without a workspace argument, for callers that cannot allocate
+ * device memory.  The paper has no counterpart; this is a library-usage entry
+ * point.  It serves code that is not allowed to call cudaMalloc: a plugin or
+ * extension whose host application owns all device memory through its own
+ * pool, or a path on which an allocation would synchronise the device or
+ * could fail mid-run.  Such a caller still passes W and the outputs (its own
+ * buffers) but no workspace: the solver's scratch is a fixed array of
+ * DQ_STATIC_SCRATCH_BYTES defined in the library's device code, which every
+ * GPU that loads the library holds until the process exits.
+ *
+ * Arguments, layouts and results are those of dq_solve (bit-identical
+ * outputs); nothing is allocated: no cudaMalloc, cudaFree or allocating
+ * library routine.  Returns DQ_EWORKSPACE, before enqueueing anything, when
+ * the shape needs more scratch than DQ_STATIC_SCRATCH_BYTES.
+ *  status  optional (may be NULL) pointer the GPU can write, 4-byte aligned
+ *          (device memory or mapped host memory): after the solve, a stream-
+ *          ordered kernel stores DQ_OK, DQ_ENONFINITE or DQ_ECUDA there, the
+ *          device-side outcome that dq_sync_status reports for dq_solve.
+ * Set-up: the first call on each device, made with that device current, looks
+ * up the scratch array's device address (loading the module there); make
+ * that first call before any stream capture on the device.
+ * Sharing: all calls on one device share the same scratch, and each call
+ * clears the parts that must start at zero.  Calls whose work overlaps on the
+ * GPU (different streams, or several host threads, without ordering between
+ * them) race on that scratch and give wrong results; order them on one stream
+ * or wait between them. */
+int dq_solve_static(const void* W, int w_dtype, int64_t rows, int64_t cols, int format, int group, int iters,
+                    int col_dtype, const dq_outputs* out, int* status, void* stream);
+
 /* Static string for a status code. */
 const char* dq_status_str(int status);
 
