@@ -262,8 +262,9 @@ def rtn(W: torch.Tensor, fmt="nvfp4", group: Optional[int] = None, col_dtype: Op
 def diagnostics(workspace: torch.Tensor, stream=None) -> dict:
     """Exact-path counters of the last solve that used this workspace."""
     lib = load_library()
-    arr = (ctypes.c_uint64 * 3)()
+    arr = (ctypes.c_uint64 * 4)()
     st = lib.dq_diagnostics(workspace.data_ptr(), _stream_ptr(stream), arr)
     if st != 0:
         raise DQError(st, "dq_diagnostics")
-    return {"quant_exact_lane_rows": int(arr[0]), "block_exact": int(arr[1]), "col_exact": int(arr[2])}
+    return {"quant_exact_lane_rows": int(arr[0]), "block_exact": int(arr[1]), "col_exact": int(arr[2]),
+            "quant_tie_lane_rows": int(arr[3])}

@@ -165,7 +165,7 @@ int dq_sync_status(const void* workspace, void* stream) {
   return (flags & dq::kFlagTimeout) ? DQ_ECUDA : DQ_OK;
 }
 
-int dq_diagnostics(const void* workspace, void* stream, uint64_t out[3]) {
+int dq_diagnostics(const void* workspace, void* stream, uint64_t out[4]) {
   if (!workspace || !out) return DQ_EINVAL;
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DQ_ECUDA;
   dq::WsHeader h;
@@ -173,6 +173,7 @@ int dq_diagnostics(const void* workspace, void* stream, uint64_t out[3]) {
   out[0] = h.n_quant_exact;
   out[1] = h.n_block_exact;
   out[2] = h.n_col_exact;
+  out[3] = h.n_quant_tie;
   return DQ_OK;
 }
 

@@ -23,7 +23,7 @@ struct WsHeader {
   unsigned amax_bits;    // max |W| as fp32 bits
   unsigned cta_counter;  // arrival ticket for CTA-ordered totals
   float sT;              // NVFP4 tensor scale (1 otherwise)
-  double reserved;
+  unsigned long long n_quant_tie;    // lane-rows with a certified exact tie settled on the fast path
   // diagnostics: how often the exact paths ran in the per-iteration passes
   unsigned long long n_quant_exact;  // lane-rows (8 elements) decided on the exact path
   unsigned long long n_block_exact;  // block updates taken in fp64

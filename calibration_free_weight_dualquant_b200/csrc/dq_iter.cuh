@@ -56,11 +56,13 @@ __device__ __forceinline__ f2 pk(float lo, float hi) {
 __device__ __forceinline__ float lo_of(f2 v) {
   float a, b;
   asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+  (void)b;
   return a;
 }
 __device__ __forceinline__ float hi_of(f2 v) {
   float a, b;
   asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+  (void)a;
   return b;
 }
 __device__ __forceinline__ f2 mul2(f2 a, f2 b) {
@@ -118,7 +120,35 @@ struct ColState {
   float thr[8];
   f2 res2;  // fp32 run of squared reconstruction residuals
   bool ok;
+  bool tie_ok;  // a flagged element of this lane can only be an exact tie (see tie_certified)
 };
+
+// Significant bits of a positive normal float (1 + index of the lowest set
+// mantissa bit counted from the top): 1 for a power of two, 24 at most.
+__device__ __forceinline__ int sig_bits(float v) {
+  return 25 - __ffs((int)((__float_as_uint(v) & 0x007FFFFFu) | 0x00800000u));
+}
+
+// Tie certification.  Write W = w 2^g with w an odd integer below 2^11 (bf16 or
+// fp16 W), the element's scale product P = a b = p 2^h with p odd and at most k
+// bits long, and a rounding boundary B of the grid as an odd integer over a
+// power of two: at most 4 bits on the INT4 grid (the boundaries that matter
+// after clipping are +-1/2 .. +-15/2), 3 bits on E2M1 (1/4 .. 5).  Then
+// B P = n 2^f with n odd, and if W != B P, |W - B P| >= 2^min(g, f):
+//  * g >= f: |x - B| >= |B| / n >= 1 / (2 p) on the INT4 grid (absolute), and
+//    |x - B| / |B| >= 1 / n > 2^-(3 + k) on E2M1 (relative);
+//  * g < f:  |x - B| >= x / 2^11, i.e. 2^-13 absolute (|B| >= 1/2) or 2^-11
+//    relative.
+// The fast paths flag an element only when x lies within 2^-14 + 2^-19 of a
+// boundary (INT4 grid, absolute; candidate error included) or within
+// 1.5 * 2^-20 of it relative (E2M1 bracket plus candidate error).  So with
+// k <= 12 (INT4 grid) or k <= 15 (E2M1) every flagged element is an exact tie
+// x == B, whose answer is the even neighbour (round half to even).
+template <int FMT, int WDT>
+__device__ __forceinline__ bool tie_certified(int k_bits) {
+  if (WDT == DT_F32 || FMT == FMT_INT4) return false;  // INT4: fp16 a and b give k up to 22
+  return FMT == FMT_NVFP4 ? k_bits <= 15 : k_bits <= 12;
+}
 
 // Exact fp64 decision for one element (factors outside the fast range).
 template <int FMT>
@@ -134,10 +164,11 @@ __device__ __noinline__ float qexact64(float w, float a, float b, double sTd) {
 // rounding boundary (or factors outside the fast range).
 template <int FMT>
 __device__ __forceinline__ void req_fast(const f2 u2[4], float a, const ColState& cs, float& ia, bool& ok, f2 q2[4],
-                                         bool& near) {
+                                         bool& near, bool& tie) {
   ia = rcp_approx(a);
   ok = cs.ok && in_range(ia);
   near = !ok;
+  tie = false;
   if (FMT == FMT_NVFP4) {
     const f2 ilo = splat(ia * (1.f - kRelGuard)), ihi = splat(ia * (1.f + kRelGuard));
     f2 lo[4], hi[4];
@@ -148,26 +179,42 @@ __device__ __forceinline__ void req_fast(const f2 u2[4], float a, const ColState
     }
     uint32_t clo, chi, h0, h1, h2, h3;
     asm("{\n.reg .b8 l0, l1, l2, l3, g0, g1, g2, g3;\n"
-        "cvt.rn.satfinite.e2m1x2.f32 l0, %7, %6;\n"
-        "cvt.rn.satfinite.e2m1x2.f32 l1, %9, %8;\n"
-        "cvt.rn.satfinite.e2m1x2.f32 l2, %11, %10;\n"
-        "cvt.rn.satfinite.e2m1x2.f32 l3, %13, %12;\n"
-        "cvt.rn.satfinite.e2m1x2.f32 g0, %15, %14;\n"
-        "cvt.rn.satfinite.e2m1x2.f32 g1, %17, %16;\n"
-        "cvt.rn.satfinite.e2m1x2.f32 g2, %19, %18;\n"
-        "cvt.rn.satfinite.e2m1x2.f32 g3, %21, %20;\n"
+        "cvt.rn.satfinite.e2m1x2.f32 l0, %3, %2;\n"
+        "cvt.rn.satfinite.e2m1x2.f32 l1, %5, %4;\n"
+        "cvt.rn.satfinite.e2m1x2.f32 l2, %7, %6;\n"
+        "cvt.rn.satfinite.e2m1x2.f32 l3, %9, %8;\n"
+        "cvt.rn.satfinite.e2m1x2.f32 g0, %11, %10;\n"
+        "cvt.rn.satfinite.e2m1x2.f32 g1, %13, %12;\n"
+        "cvt.rn.satfinite.e2m1x2.f32 g2, %15, %14;\n"
+        "cvt.rn.satfinite.e2m1x2.f32 g3, %17, %16;\n"
         "mov.b32 %0, {l0, l1, l2, l3};\n"
-        "mov.b32 %1, {g0, g1, g2, g3};\n"
-        "cvt.rn.f16x2.e2m1x2 %2, l0;\n"
-        "cvt.rn.f16x2.e2m1x2 %3, l1;\n"
-        "cvt.rn.f16x2.e2m1x2 %4, l2;\n"
-        "cvt.rn.f16x2.e2m1x2 %5, l3;\n}"
-        : "=r"(clo), "=r"(chi), "=r"(h0), "=r"(h1), "=r"(h2), "=r"(h3)
+        "mov.b32 %1, {g0, g1, g2, g3};\n}"
+        : "=r"(clo), "=r"(chi)
         : "f"(lo_of(lo[0])), "f"(hi_of(lo[0])), "f"(lo_of(lo[1])), "f"(hi_of(lo[1])), "f"(lo_of(lo[2])),
           "f"(hi_of(lo[2])), "f"(lo_of(lo[3])), "f"(hi_of(lo[3])), "f"(lo_of(hi[0])), "f"(hi_of(hi[0])),
           "f"(lo_of(hi[1])), "f"(hi_of(hi[1])), "f"(lo_of(hi[2])), "f"(hi_of(hi[2])), "f"(lo_of(hi[3])),
           "f"(hi_of(hi[3])));
-    near |= clo != chi;
+    // The bracket codes differ only at elements within the bracket of a
+    // boundary, where they are the two neighbours (adjacent codes, one of them
+    // with an even mantissa bit).  On a tie-certified lane such an element is
+    // an exact tie: keep the neighbour whose low code bit is 0.
+    const uint32_t diff = clo ^ chi;
+    const uint32_t tmask = cs.tie_ok ? 0xFFFFFFFFu : 0u;
+    near |= (diff & ~tmask) != 0u;
+    const uint32_t code = clo ^ (diff & ((clo & 0x11111111u) * 15u) & tmask);
+    tie = (diff & tmask) != 0u;
+    // each byte is extracted explicitly (cvt.u8.u32) before its decode
+    asm("{\n.reg .b8 c0, c1, c2, c3;\n"
+        "cvt.u8.u32 c0, %4;\n"
+        "cvt.u8.u32 c1, %5;\n"
+        "cvt.u8.u32 c2, %6;\n"
+        "cvt.u8.u32 c3, %7;\n"
+        "cvt.rn.f16x2.e2m1x2 %0, c0;\n"
+        "cvt.rn.f16x2.e2m1x2 %1, c1;\n"
+        "cvt.rn.f16x2.e2m1x2 %2, c2;\n"
+        "cvt.rn.f16x2.e2m1x2 %3, c3;\n}"
+        : "=r"(h0), "=r"(h1), "=r"(h2), "=r"(h3)
+        : "r"(code & 0xFFu), "r"((code >> 8) & 0xFFu), "r"((code >> 16) & 0xFFu), "r"(code >> 24));
     const uint32_t hh[4] = {h0, h1, h2, h3};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -176,15 +223,35 @@ __device__ __forceinline__ void req_fast(const f2 u2[4], float a, const ColState
     }
   } else {
     const f2 ia2 = splat(ia), nia2 = splat(-ia), m2 = splat(12582912.f), nm2 = splat(-12582912.f);
+    bool flagged = false;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const f2 qu = add2(fma2(u2[i], ia2, m2), nm2);  // round half even
       const f2 r = fma2(u2[i], nia2, qu);             // qu - x~
       const float t0 = FMT == FMT_MXINT4 ? cs.thr[2 * i] : 0.5f - kGuard;
       const float t1 = FMT == FMT_MXINT4 ? cs.thr[2 * i + 1] : 0.5f - kGuard;
-      near |= fabsf(lo_of(r)) > t0;
-      near |= fabsf(hi_of(r)) > t1;
+      flagged |= fabsf(lo_of(r)) > t0;
+      flagged |= fabsf(hi_of(r)) > t1;
       q2[i] = pk(fminf(fmaxf(lo_of(qu), -8.f), 7.f), fminf(fmaxf(hi_of(qu), -8.f), 7.f));
+    }
+    if (flagged && cs.tie_ok) {
+      // certified exact ties x~ ~ n + 1/2: the even neighbour is 2 rint(x~ / 2)
+      tie = true;
+      const f2 hia2 = splat(0.5f * ia);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const f2 qu = add2(fma2(u2[i], ia2, m2), nm2);
+        const f2 r = fma2(u2[i], nia2, qu);
+        const f2 h = add2(fma2(u2[i], hia2, m2), nm2);
+        const f2 qe = add2(h, h);
+        const float t0 = FMT == FMT_MXINT4 ? cs.thr[2 * i] : 0.5f - kGuard;
+        const float t1 = FMT == FMT_MXINT4 ? cs.thr[2 * i + 1] : 0.5f - kGuard;
+        const float q0 = fabsf(lo_of(r)) > t0 ? lo_of(qe) : lo_of(qu);
+        const float q1 = fabsf(hi_of(r)) > t1 ? hi_of(qe) : hi_of(qu);
+        q2[i] = pk(fminf(fmaxf(q0, -8.f), 7.f), fminf(fmaxf(q1, -8.f), 7.f));
+      }
+    } else {
+      near |= flagged;
     }
   }
 }
@@ -238,11 +305,13 @@ __device__ __forceinline__ void req_pair(const f2 wx[4], const f2 ux[4], float f
                                          const f2 uy[4], float fb, bool acty, const ColState& cs, float sT, double sTd,
                                          f2 qx[4], f2 qy[4], unsigned* s_cnt) {
   float iax, iay;
-  bool okx, oky, nx, ny;
-  req_fast<FMT>(ux, fa, cs, iax, okx, qx, nx);
-  req_fast<FMT>(uy, fb, cs, iay, oky, qy, ny);
+  bool okx, oky, nx, ny, tx, ty;
+  req_fast<FMT>(ux, fa, cs, iax, okx, qx, nx, tx);
+  req_fast<FMT>(uy, fb, cs, iay, oky, qy, ny, ty);
   nx = nx && actx;
   ny = ny && acty;
+  const int ties = __popc(__ballot_sync(0xffffffffu, tx && actx)) + __popc(__ballot_sync(0xffffffffu, ty && acty));
+  if (ties && (threadIdx.x & 31) == 0) atomicAdd(&s_cnt[3], (unsigned)ties);
   if (nx || ny) {
     if (nx) {
       atomicAdd(&s_cnt[0], 1u);
@@ -479,7 +548,7 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t) {
       mbar_init(&empty[i], kConsumerWarps);
     }
     mbar_fence_init();
-    s_cnt[0] = s_cnt[1] = s_cnt[2] = 0u;
+    s_cnt[0] = s_cnt[1] = s_cnt[2] = s_cnt[3] = 0u;
   }
   if (threadIdx.x < kConsumers) racc[threadIdx.x] = 0.0;
   __syncthreads();
@@ -530,6 +599,7 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t) {
   const double sTd = (double)sT;
   const float isT = FMT == FMT_NVFP4 ? __frcp_rn(sT) : 1.f;
   const bool sT_ok = FMT != FMT_NVFP4 || in_range(isT);
+  const int sT_bits = sig_bits(sT);
   const int64_t s_first = u_begin / p.M;
   int st = 0;
   unsigned par = 0u;
@@ -547,6 +617,7 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t) {
     ColState cs;
     cs.ok = sT_ok;
     cs.res2 = 0ull;
+    int b_bits = 1;  // longest odd significand among the lane's column scales
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       float bj[2] = {1.f, 1.f}, cb[2] = {1.f, 1.f};
@@ -558,8 +629,10 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t) {
           bj[h] = b_decode(p.b_store, p.col_dt, col + c);
           cb[h] = __frcp_rn(bj[h]) * isT;
           cs.ok = cs.ok && in_range(cb[h]);
-          // MXINT4: a = 2^k, so a power-of-two b makes the candidate exact
-          if (FMT == FMT_MXINT4 && (__float_as_uint(bj[h]) & 0x007FFFFFu) == 0u) cs.thr[c] = 2.f;
+          b_bits = max(b_bits, sig_bits(bj[h]));
+          // MXINT4: a = 2^k, so a power-of-two b makes the candidate exact (for
+          // bf16/fp16 W the tie certificate covers these columns as well)
+          if (FMT == FMT_MXINT4 && WDT == DT_F32 && (__float_as_uint(bj[h]) & 0x007FFFFFu) == 0u) cs.thr[c] = 2.f;
         }
         acc[(warp * 8 + c) * 32 + lane] = make_double2(0.0, 0.0);
       }
@@ -567,6 +640,8 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t) {
       cs.cb2[i] = pk(cb[0], cb[1]);
       cs.cn2[i] = cs.cd2[i] = 0ull;
     }
+    // odd part of a b: E4M3 e has at most 4 significant bits, 2^k has 1
+    cs.tie_ok = tie_certified<FMT, WDT>(FMT == FMT_NVFP4 ? sT_bits + 4 + b_bits : b_bits);
     int run = 0;
     // block scales of this warp's rows, one tile ahead
     const int64_t a_step = (int64_t)kRowsPerTile * p.nb;
@@ -695,6 +770,7 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t) {
     if (s_cnt[0]) atomicAdd(&p.hdr->n_quant_exact, (unsigned long long)s_cnt[0]);
     if (s_cnt[1]) atomicAdd(&p.hdr->n_block_exact, (unsigned long long)s_cnt[1]);
     if (s_cnt[2]) atomicAdd(&p.hdr->n_col_exact, (unsigned long long)s_cnt[2]);
+    if (s_cnt[3]) atomicAdd(&p.hdr->n_quant_tie, (unsigned long long)s_cnt[3]);
     p.cta_part[k] = mred[0];
     __threadfence();
     const unsigned prev = atomicAdd(&p.hdr->cta_counter, 1u);

@@ -129,9 +129,13 @@ int dq_solve_host(const void* W_host, int w_dtype, int64_t rows, int64_t cols, i
  *           boundary, or a scale outside the fast path's range),
  *   out[1]  block inverse-scale updates taken in fp64 (fp32 value too close to
  *           a projection midpoint, a zero or out-of-range sum),
- *   out[2]  column inverse-scale updates recomputed exactly over all rows.
+ *   out[2]  column inverse-scale updates recomputed exactly over all rows,
+ *   out[3]  lane-rows holding an element that lies exactly on a rounding
+ *           boundary (a tie) and that the fast path settled as a certified tie
+ *           (the scale product has so few significant bits that a flagged
+ *           element can only be an exact tie).
  * Counts cover the BCD iterations only (not init or the final pass). */
-int dq_diagnostics(const void* workspace, void* stream, uint64_t out[3]);
+int dq_diagnostics(const void* workspace, void* stream, uint64_t out[4]);
 
 /* Size of the library-owned device scratch that dq_solve_static uses: 8 MiB.
  * A shape fits when dq_workspace_bytes(rows, cols, format, group) is at most

@@ -233,6 +233,53 @@ def test_exact_paths_exercised_and_bit_exact(fmt, group, col_dtype, name):
     W = synth.make_weight(wl, 1024, 2048, seed=5)
     gpu, _ = run_both(W, fmt, group, 20, col_dtype, "exact_paths")
     d = binding.diagnostics(gpu["workspace"])
-    assert d["quant_exact_lane_rows"] > 0, d
+    if fmt == "mxint4":  # bf16 W, 2^k a: every flagged element is a certified exact tie
+        assert d["quant_tie_lane_rows"] > 0, d
+    else:
+        assert d["quant_exact_lane_rows"] > 0, d
     if col_dtype == "f16":  # fp16 scales: near-midpoint LS values are common enough to be hit
         assert d["block_exact"] > 0 and d["col_exact"] > 0, d
+
+
+def short_tensor_scale_weight(M, N, wdtype, seed):
+    """Laplace weights whose max |W| is 2688 * 5 * 2^-13, so s_T = 5 * 2^-13 has 3 significant
+    bits: a b then has few bits and many elements land exactly on E2M1 rounding boundaries."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    W = np.clip(rng.laplace(0.0, 0.012, (M, N)), -1.5, 1.5).astype(np.float32)
+    W[M // 2, N // 3] = -2688.0 * 5.0 * 2.0 ** -13
+    return torch.from_numpy(W).to(wdtype)
+
+
+@pytest.mark.parametrize("wdtype,col_dtype,certified", [
+    (torch.bfloat16, "bf16", True),    # 3 + 4 + 8 bits: certified ties
+    (torch.float16, "bf16", True),
+    (torch.float16, "f16", None),      # fp16 b: certified only on lanes whose b have few bits
+    (torch.float32, "bf16", False),    # f32 W: never certified
+])
+def test_nvfp4_exact_ties(wdtype, col_dtype, certified):
+    """Exact ties W / (a b) == boundary: certified lanes settle them on the fast path (round half
+    to even in the code domain), the others on the exact path; both bit-exact."""
+    W = short_tensor_scale_weight(517, 1040, wdtype, 11)
+    gpu, orc = run_both(W, "nvfp4", 16, 6, col_dtype, "ties")
+    assert orc["sT"] == 5.0 * 2.0 ** -13
+    d = binding.diagnostics(gpu["workspace"])
+    if certified:
+        assert d["quant_tie_lane_rows"] > 0, d
+    elif certified is None:
+        assert d["quant_tie_lane_rows"] + d["quant_exact_lane_rows"] > 0, d
+    else:
+        assert d["quant_tie_lane_rows"] == 0 and d["quant_exact_lane_rows"] > 0, d
+
+
+@pytest.mark.parametrize("wdtype,col_dtype", [(torch.float16, "f16"), (torch.bfloat16, "bf16"),
+                                              (torch.float32, "bf16")])
+def test_mxint4_exact_ties(wdtype, col_dtype):
+    """MXINT4 with few-bit weights: W / (2^k b) hits half-integers exactly and often."""
+    g = torch.Generator().manual_seed(12)
+    W = (torch.randint(-40, 41, (389, 672), generator=g).float() * 2.0 ** -6).to(wdtype)
+    gpu, _ = run_both(W, "mxint4", 32, 6, col_dtype, "mx_ties")
+    d = binding.diagnostics(gpu["workspace"])
+    if wdtype != torch.float32:
+        assert d["quant_tie_lane_rows"] > 0, d
+    else:
+        assert d["quant_tie_lane_rows"] == 0, d
