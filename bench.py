@@ -68,7 +68,10 @@ def profile_traffic(workload: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+    """nvidia-smi clocks and throttle reasons sampled every 100 ms while running.
+
+    Entering starts the sampler and waits (up to 5 s) for its first sample, so
+    the samples cover the timed region that follows."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -80,31 +83,45 @@ class ClockSampler:
         except Exception:
             self.dev = "0"
         self.proc = None
+        self.lines = []
+        self.armed = 0
+
+    def _reader(self):
+        for line in self.proc.stdout:
+            if line.strip():
+                self.lines.append(line)
 
     def __enter__(self):
+        import threading
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", self.dev, "--query-gpu=" + self.FIELDS,
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+            return self
+        self.thread = threading.Thread(target=self._reader, daemon=True)
+        self.thread.start()
+        t0 = time.time()
+        while not self.lines and time.time() - t0 < 5.0 and self.proc.poll() is None:
+            time.sleep(0.01)
+        self.armed = len(self.lines)  # samples taken before the timed region are dropped
         return self
 
     def __exit__(self, *a):
-        self.lines = []
         if self.proc is not None:
             self.proc.terminate()
             try:
-                out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
+            self.thread.join(timeout=5)
+        self.lines = self.lines[self.armed:]
 
     def summary(self) -> dict:
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in getattr(self, "lines", []):
+        for line in self.lines:
             parts = [x.strip() for x in line.split(",")]
             if len(parts) < 9:
                 continue
@@ -175,6 +192,13 @@ def run_reference(args, wl, rank, world, dist):
     W = synth.make_weight(wl)
     rows = max(8, min(wl.rows, args.ref_rows))
     Win, wdt = synth.to_oracle_input(W[:rows].contiguous())
+    t0 = time.perf_counter()
+    oracle.solve(Win, wdt, wl.fmt, wl.group, wl.iters, wl.col_dtype)
+    t_one = time.perf_counter() - t0
+    budget_s = 90.0  # the whole timed run stays within a couple of minutes
+    if args.steps * t_one > budget_s:
+        rows = max(8, int(rows * budget_s / (args.steps * t_one)))
+        Win, wdt = synth.to_oracle_input(W[:rows].contiguous())
     for _ in range(args.warmup):
         oracle.solve(Win, wdt, wl.fmt, wl.group, wl.iters, wl.col_dtype)
     times = []
@@ -211,7 +235,7 @@ def algorithmic_bytes_per_iter(wl) -> int:
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="dq", choices=["dq", "reference"])
