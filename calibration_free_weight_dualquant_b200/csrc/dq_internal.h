@@ -52,6 +52,7 @@ struct Problem {
   unsigned* strip_counter;  // [n_strips]
   double2* col_part;        // [P * segmax][TS] (sum W a q, sum (a q)^2)
   double* cta_part;         // [max(P, P_final)]
+  int use_tmap;             // W streamed by 2-D tensor copies (else one bulk copy per row)
 };
 
 cudaError_t launch_solve(const Problem& p, int iters, int stats_ctas, cudaStream_t st);

@@ -3,8 +3,9 @@
 //
 // CTA = 15 consumer warps + 1 producer warp (16 warps, 4 per SM sub-partition,
 // so each thread may hold 128 registers).  The producer streams the CTA's rows
-// of the current column strip, one row per bulk (TMA) copy, into a ring of
-// shared-memory tiles of kRowsPerTile rows, guarded by full/empty mbarriers.
+// of the current column strip into a ring of shared-memory tiles of
+// kRowsPerTile rows, guarded by full/empty mbarriers: one 2-D tensor copy (TMA)
+// per tile, or one bulk copy per row when W admits no tensor map.
 // Consumer warp w takes rows w and w + 15 of every tile; lane l takes the 8
 // consecutive columns 8l..8l+7 of the strip as 4 pairs, and the arithmetic on
 // pairs runs as packed f32x2 instructions.  Per element the consumers run the
@@ -12,6 +13,8 @@
 // reconstruction residuals run in fp32 for kRun rows of a lane and are then
 // added into fp64 accumulators kept in shared memory.
 #pragma once
+
+#include <cuda.h>  // CUtensorMap
 
 #include "dq_device.cuh"
 #include "dq_fast.cuh"
@@ -526,7 +529,7 @@ __device__ __forceinline__ void flush_runs(ColState& cs, double2* acc, double* r
 }
 
 template <int FMT, int WDT>
-__global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t) {
+__global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t, const __grid_constant__ CUtensorMap wmap) {
   if (p.hdr->flags & kFlagNonFinite) return;
   constexpr int ES = WDT == DT_F32 ? 4 : 2;
   constexpr int S = ring_stages(ES);
@@ -569,6 +572,24 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t) {
       const unsigned bytes = (unsigned)(width * ES);
       const unsigned char* src = reinterpret_cast<const unsigned char*>(p.W) + ((r0 + lane) * p.N + c0) * (int64_t)ES;
       const int64_t src_step = (int64_t)kRowsPerTile * p.N * ES;
+      if (p.use_tmap) {
+        // one tensor copy per tile: kRowsPerTile rows x TS columns (zero-filled
+        // beyond the matrix), into the same row-major slot layout
+        for (int64_t tr = r0; tr < r1; tr += kRowsPerTile) {
+          mbar_wait(&empty[st], par, &p.hdr->flags);
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&full[st], (unsigned)stage_bytes);
+            tma_load_2d(ring + st * stage_bytes, &wmap, (int)c0, (int)tr, &full[st]);
+          }
+          __syncwarp();
+          if (++st == S) {
+            st = 0;
+            par ^= 1u;
+          }
+        }
+        u = (s + 1) * p.M;
+        continue;
+      }
       for (int64_t tr = r0; tr < r1; tr += kRowsPerTile, src += src_step) {
         mbar_wait(&empty[st], par, &p.hdr->flags);
         const int nr = (int)min((int64_t)kRowsPerTile, r1 - tr);

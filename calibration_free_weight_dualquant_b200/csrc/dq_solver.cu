@@ -26,6 +26,11 @@
 // entering iteration t is accumulated from the residuals W - a q b of the
 // requantized incoming iterate (fp32 runs into fp64), per CTA, then summed in
 // CTA order by the last CTA.
+#include <cudaTypedefs.h>  // PFN_cuTensorMapEncodeTiled
+
+#include <climits>
+#include <cstring>
+
 #include "dq_device.cuh"
 #include "dq_fast.cuh"
 #include "dq_internal.h"
@@ -182,18 +187,56 @@ __global__ void __launch_bounds__(kThreads) k_final(Problem p, int T) {
 // ---------------------------------------------------------------------------
 // Host-side launch of the whole solve on one stream.
 
+// The driver's tensor-map encoder, looked up once through the runtime.
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (PFN_cuTensorMapEncodeTiled_v12000) nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }();
+  return fn;
+}
+
+// 2-D tensor map of W (columns innermost) with a box of one ring tile:
+// kStripMax columns x kRowsPerTile rows.  Returns false when W cannot be
+// described (then k_iter copies one row at a time).
+template <int WDT>
+static bool encode_w_map(const Problem& p, CUtensorMap* map) {
+  constexpr int ES = WDT == DT_F32 ? 4 : 2;
+  std::memset(map, 0, sizeof(*map));
+  if (p.M > INT_MAX || p.TS != kStripMax || (p.N * ES) % 16 != 0) return false;
+  const PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)p.N, (cuuint64_t)p.M};
+  const cuuint64_t strides[1] = {(cuuint64_t)p.N * ES};
+  const cuuint32_t box[2] = {(cuuint32_t)kStripMax, (cuuint32_t)kRowsPerTile};
+  const cuuint32_t elem_strides[2] = {1, 1};
+  const CUtensorMapDataType dt = WDT == DT_F32    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                 : WDT == DT_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                  : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  return fn(map, dt, 2, const_cast<void*>(p.W), dims, strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int FMT, int WDT>
 static cudaError_t run_typed(const Problem& p, int iters, int stats_ctas, cudaStream_t st) {
   constexpr int ES = WDT == DT_F32 ? 4 : 2;
   const size_t smem = iter_smem_bytes(ES);
   cudaError_t e = cudaFuncSetAttribute(k_iter<FMT, WDT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  CUtensorMap wmap;
+  Problem pi = p;
+  pi.use_tmap = encode_w_map<WDT>(p, &wmap) ? 1 : 0;
   Problem pf = p;
   pf.P = p.P_final;
   pf.segmax = p.segmax_final;
   k_stats<WDT><<<stats_ctas, kThreads, 0, st>>>(pf);
   k_init<FMT, WDT><<<stats_ctas, kThreads, 0, st>>>(pf);
-  for (int t = 1; t <= iters; ++t) k_iter<FMT, WDT><<<(unsigned)p.P, kIterThreads, smem, st>>>(p, t);
+  for (int t = 1; t <= iters; ++t) k_iter<FMT, WDT><<<(unsigned)p.P, kIterThreads, smem, st>>>(pi, t, wmap);
   k_final<FMT, WDT><<<(unsigned)pf.P, kThreads, 0, st>>>(pf, iters);
   return cudaGetLastError();
 }
