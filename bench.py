@@ -165,10 +165,10 @@ def barrier(dist):
         dist.barrier()
 
 
-def cpu_baseline(wl, budget_s: float = 12.0) -> dict:
+def cpu_baseline(wl, budget_s: float = 12.0, W=None) -> dict:
     """The oracle, as it stands, on a bounded row sample of the workload on the host cores."""
     import oracle
-    W = synth.make_weight(wl)
+    W = synth.make_weight(wl) if W is None else W
     cores = oracle.num_threads()
     rows = max(8, min(wl.rows, 64))
     while True:
@@ -184,12 +184,13 @@ def cpu_baseline(wl, budget_s: float = 12.0) -> dict:
                                                                                   dt)}
 
 
-def run_reference(args, wl, rank, world, dist):
-    """Reference arm: the CPU oracle on the host cores, one bounded row sample per step."""
+def run_reference(args, wl, rank, world, dist, set_name=None):
+    """Reference arm: the CPU oracle on the host cores, one bounded row sample per step (for the
+    Llama set: rows of its layer-0 gate matrix, drawn with the set's generator)."""
     if rank != 0:
         return
     import oracle
-    W = synth.make_weight(wl)
+    W = synth.make_weight_device(wl, "cpu") if set_name else synth.make_weight(wl)
     rows = max(8, min(wl.rows, args.ref_rows))
     Win, wdt = synth.to_oracle_input(W[:rows].contiguous())
     t0 = time.perf_counter()
@@ -213,7 +214,8 @@ def run_reference(args, wl, rank, world, dist):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": config_of(wl, world), "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores,
+            "config": set_config(set_name, world) if set_name else config_of(wl, world),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores,
                                                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -223,6 +225,14 @@ def config_of(wl, world) -> dict:
     return {"workload": wl.name, "rows": wl.rows, "cols": wl.cols, "format": wl.fmt, "group": wl.group,
             "iters": wl.iters, "w_dtype": wl.wdtype, "col_dtype": wl.col_dtype,
             "l2": "flushed before each step (512 MB write, untimed)", "parallelism": "replicas x%d" % world}
+
+
+def set_config(name, world) -> dict:
+    fmt = synth.LLAMA_SETS[name]
+    wl = synth.llama_set(fmt)[0]
+    return {"workload": name, "matrices": len(synth.llama_set(fmt)), "elements": synth.llama_set_elements(),
+            "format": fmt, "group": wl.group, "iters": wl.iters, "w_dtype": wl.wdtype, "col_dtype": wl.col_dtype,
+            "l2": "inputs (14 GB) far larger than L2", "parallelism": "replicas x%d" % world}
 
 
 def algorithmic_bytes_per_iter(wl) -> int:
@@ -237,7 +247,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS) + sorted(synth.LLAMA_SETS))
     ap.add_argument("--impl", default="dq", choices=["dq", "reference"])
     ap.add_argument("--ref-rows", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -246,6 +256,18 @@ def main():
     ap.add_argument("--cols", type=int, help="override the workload's cols (profiling cases)")
     ap.add_argument("--iters", type=int, help="override the workload's BCD iterations")
     args = ap.parse_args()
+    if args.workload in synth.LLAMA_SETS:
+        rank, world, local, dist = dist_setup(args.gpus)
+        try:
+            if args.impl == "reference":
+                run_reference(args, synth.llama_set(synth.LLAMA_SETS[args.workload])[4], rank, world, dist,
+                              set_name=args.workload)
+            else:
+                run_dq_set(args, args.workload, rank, world, local, dist)
+        finally:
+            if dist is not None:
+                dist.destroy_process_group()
+        return
     wl = synth.WORKLOADS[args.workload]
     if args.rows or args.cols or args.iters:
         import dataclasses
@@ -345,6 +367,75 @@ def run_dq(args, wl, rank, world, local, dist):
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
+    print(json.dumps(line), flush=True)
+
+
+def run_dq_set(args, name, rank, world, local, dist):
+    """The whole 224-matrix Llama-3.1-8B linear set per step, queued on one stream by dq_solve_batched."""
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    binding.load_library()
+    fmt = synth.LLAMA_SETS[name]
+    wls = synth.llama_set(fmt)
+    T, g, cd = wls[0].iters, wls[0].group, wls[0].col_dtype
+    Ws = [synth.make_weight_device(wl, dev, seed=wl.seed + 7919 * rank) for wl in wls]
+    outs = [binding.alloc_outputs(wl.rows, wl.cols, fmt, g, cd, T, dev) for wl in wls]
+    outs0 = [binding.alloc_outputs(wl.rows, wl.cols, fmt, g, cd, 0, dev) for wl in wls]
+    ws = torch.empty(max(binding.workspace_bytes(wl.rows, wl.cols, fmt, g) for wl in wls), dtype=torch.uint8,
+                     device=dev)
+    status = torch.zeros(len(wls), dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(iters, steps, o):
+        ts = []
+        for _ in range(steps):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            binding.dq_solve_batched(Ws, fmt, g, iters, cd, outs=o, workspace=ws, status=status, stream=stream,
+                                     check=False)
+            e1.record(stream)
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return ts
+
+    timed(T, args.warmup, outs)
+    torch.cuda.synchronize()
+    if int(status.abs().sum()) != 0:
+        raise binding.DQError(int(status.max()), "bench warm-up (Llama set)")
+    barrier(dist)
+    torch.cuda.synchronize()
+    with ClockSampler(dev) as clk:
+        step_ms = timed(T, args.steps, outs)
+    torch.cuda.synchronize()
+    barrier(dist)
+    total_ms = max_over_ranks(sum(step_ms), dist)
+    t0s = timed(0, max(3, min(args.steps, 10)), outs0)
+    iter_ms = max_over_ranks((statistics.median(step_ms) - statistics.median(t0s)) / T, dist)
+    if rank != 0:
+        return
+    elems = synth.llama_set_elements()
+    value = world * elems * T * args.steps / (total_ms * 1e-3)
+    peaks = measured_peaks()
+    alg = sum(algorithmic_bytes_per_iter(wl) for wl in wls)
+    achieved = alg / (iter_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32+f64", "data": "synthetic",
+        "config": set_config(name, world),
+        "final_mse_layer0_q": float(outs[0]["mse"][-1].item()),
+        "ms_per_iter": iter_ms,
+        "roofline": {"bound": "hbm", "kernel": "k_iter", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "algorithmic_bytes_per_launch": alg, "peak_source": peaks["source"],
+                     "note": "per iteration of the whole set (224 launches of k_iter)"},
+        "e2e": None,
+        "gpu_launches": args.steps * len(wls) * (T + 3),
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wls[4], W=synth.make_weight_device(wls[4], "cpu"))
     print(json.dumps(line), flush=True)
 
 

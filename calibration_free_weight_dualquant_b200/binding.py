@@ -44,6 +44,11 @@ class _Outputs(ctypes.Structure):
                 ("col_scales", ctypes.c_void_p), ("mse", ctypes.c_void_p)]
 
 
+class _Matrix(ctypes.Structure):
+    _fields_ = [("W", ctypes.c_void_p), ("w_dtype", ctypes.c_int), ("rows", ctypes.c_int64),
+                ("cols", ctypes.c_int64), ("out", _Outputs)]
+
+
 _lib = None
 
 
@@ -72,6 +77,8 @@ def load_library():
     lib.dq_diagnostics.restype = I
     lib.dq_solve_static.argtypes = [P, I, I64, I64, I, I, I, I, ctypes.POINTER(_Outputs), P, P]
     lib.dq_solve_static.restype = I
+    lib.dq_solve_batched.argtypes = [ctypes.POINTER(_Matrix), I, I, I, I, I, P, P, SZ, ctypes.POINTER(I), P]
+    lib.dq_solve_batched.restype = I
     lib.dq_status_str.argtypes = [I]
     lib.dq_status_str.restype = ctypes.c_char_p
     _lib = lib
@@ -193,6 +200,54 @@ def dq_solve_static(W: torch.Tensor, fmt, group: Optional[int] = None, iters: in
             raise DQError(dev_st, "dq_solve_static (device)")
     out["status"] = status
     return out
+
+
+def dq_solve_batched(Ws, fmt, group: Optional[int] = None, iters: int = 0, col_dtype: Optional[str] = None,
+                     outs: Optional[list] = None, workspace: Optional[torch.Tensor] = None,
+                     status: Optional[torch.Tensor] = None, stream=None, check: bool = True) -> list:
+    """Enqueue dq_solve_batched: every CUDA matrix of ``Ws`` solved one after another on one stream with
+    one shared workspace.  Returns the list of output dicts; ``check`` waits and raises on the first
+    matrix whose device-side status is not DQ_OK."""
+    lib = load_library()
+    f = _fmt(fmt)
+    g = DEFAULT_GROUP[f] if group is None else group
+    cd = DEFAULT_COL_DTYPE[f] if col_dtype is None else col_dtype
+    n = len(Ws)
+    if n == 0:
+        return []
+    dev = Ws[0].device
+    for W in Ws:
+        if not W.is_cuda or W.dtype not in _DTYPES or not W.is_contiguous() or W.dim() != 2:
+            raise DQError(1, "dq_solve_batched: every W must be a contiguous 2-D CUDA f32/bf16/f16 tensor")
+    if outs is None:
+        outs = [alloc_outputs(W.shape[0], W.shape[1], f, g, cd, iters, dev) for W in Ws]
+    if workspace is None:
+        nbytes = max(int(lib.dq_workspace_bytes(W.shape[0], W.shape[1], int(f), g)) for W in Ws)
+        if nbytes == 0:
+            raise DQError(1, "dq_workspace_bytes")
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    if status is None:
+        status = torch.full((n,), -1, dtype=torch.int32, device=dev)
+    mats = (_Matrix * n)()
+    for i, (W, o) in enumerate(zip(Ws, outs)):
+        mats[i].W = W.data_ptr()
+        mats[i].w_dtype = _DTYPES[W.dtype]
+        mats[i].rows, mats[i].cols = W.shape
+        mats[i].out = _outputs_struct(o)
+    bad = ctypes.c_int(-1)
+    st = lib.dq_solve_batched(mats, n, int(f), g, iters, 2 if cd == "f16" else 1, status.data_ptr(),
+                              workspace.data_ptr(), workspace.numel(), ctypes.byref(bad), _stream_ptr(stream))
+    if st != 0:
+        raise DQError(st, "dq_solve_batched (matrix %d)" % bad.value)
+    if check:
+        (torch.cuda.current_stream() if stream is None else stream).synchronize()
+        sts = status.cpu().tolist()
+        for i, v in enumerate(sts):
+            if v != 0:
+                raise DQError(v, "dq_solve_batched (device, matrix %d)" % i)
+    for o in outs:
+        o["workspace"] = workspace
+    return outs
 
 
 def dq_rtn(W: torch.Tensor, fmt, group: Optional[int] = None, col_dtype: Optional[str] = None, **kw) -> dict:

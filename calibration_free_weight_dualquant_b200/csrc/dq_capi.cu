@@ -133,6 +133,12 @@ int solve_impl(const void* W, int w_dtype, int64_t rows, int64_t cols, int forma
   return DQ_OK;
 }
 
+// Device-side status of the solve that used `ws`, as a dq_status.
+__global__ void k_ws_status(const WsHeader* ws, int* status) {
+  const unsigned f = ws->flags;
+  *status = (f & kFlagNonFinite) ? DQ_ENONFINITE : ((f & kFlagTimeout) ? DQ_ECUDA : DQ_OK);
+}
+
 }  // namespace dq
 
 extern "C" {
@@ -244,6 +250,46 @@ int dq_solve_host(const void* W_host, int w_dtype, int64_t rows, int64_t cols, i
   if (out_host->mse && cudaMemcpyAsync(out_host->mse, dout.mse, bytes_mse, cudaMemcpyDeviceToHost, s))
     return DQ_ECUDA;
   return dq_sync_status(ws, stream);
+}
+
+int dq_solve_batched(const dq_matrix* mats, int count, int format, int group, int iters, int col_dtype, int* status,
+                     void* workspace, size_t workspace_bytes, int* bad_index, void* stream) {
+  if (count < 0 || (count > 0 && !mats)) return DQ_EINVAL;
+  if (status && !aligned(status, sizeof(int))) return DQ_EINVAL;
+  if (!workspace || !aligned(workspace, kAlign)) return DQ_EINVAL;
+  if (iters < 0) return DQ_EINVAL;
+  if (col_dtype != DQ_F16 && col_dtype != DQ_BF16) return DQ_EUNSUPPORTED;
+  // validate everything first: nothing is enqueued unless every matrix is valid
+  for (int i = 0; i < count; ++i) {
+    const dq_matrix& m = mats[i];
+    int st = check_shape(m.rows, m.cols, format, group);
+    if (st == DQ_OK && (m.w_dtype < DQ_F32 || m.w_dtype > DQ_F16 || !m.W || !aligned(m.W, 16))) st = DQ_EINVAL;
+    if (st == DQ_OK) st = check_outputs(&m.out, format, col_dtype);
+    if (st == DQ_OK) {
+      Plan pl;
+      st = make_plan(m.rows, m.cols, group, &pl);
+      if (st == DQ_OK && workspace_bytes < pl.total) st = DQ_EWORKSPACE;
+    }
+    if (st != DQ_OK) {
+      if (bad_index) *bad_index = i;
+      return st;
+    }
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  for (int i = 0; i < count; ++i) {
+    const dq_matrix& m = mats[i];
+    const int st = dq::solve_impl(m.W, m.w_dtype, m.rows, m.cols, format, group, iters, col_dtype, &m.out, workspace,
+                                  workspace_bytes, s);
+    if (st != DQ_OK) {
+      if (bad_index) *bad_index = i;
+      return st;
+    }
+    if (status) {
+      dq::k_ws_status<<<1, 1, 0, s>>>(static_cast<const dq::WsHeader*>(workspace), status + i);
+      if (cudaGetLastError() != cudaSuccess) return DQ_ECUDA;
+    }
+  }
+  return DQ_OK;
 }
 
 const char* dq_status_str(int status) {

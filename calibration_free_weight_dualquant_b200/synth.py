@@ -75,6 +75,33 @@ def llama_set_elements() -> int:
     return LLAMA31_8B_LAYERS * sum(r * c for _, r, c in LLAMA31_8B_LAYER)
 
 
+# The whole 224-matrix set, solved once per format (20 iterations each).
+LLAMA_SETS = {"llama31_8b_set_nvfp4": "nvfp4", "llama31_8b_set_mxint4": "mxint4"}
+
+
+def llama_set(fmt: str, iters: int = 20) -> list:
+    """The 224 matrices in layer-major order (layer 0: q, k, v, o, gate, up, down; layer 1: ...)."""
+    return [llama_set_workload(layer, pid, fmt, iters) for layer in range(LLAMA31_8B_LAYERS)
+            for pid in range(len(LLAMA31_8B_LAYER))]
+
+
+def make_weight_device(wl: Workload, device, seed: Optional[int] = None) -> torch.Tensor:
+    """A normal-law workload drawn directly on `device` with torch's Philox generator seeded per matrix
+    (the 14 GB Llama set is too large to draw on the host for every run).  Recipe: N(0, sigma^2) in fp32,
+    k = max(1, round_half_even(frac N)) outlier columns chosen by a CPU torch permutation with the same
+    seed and multiplied by the factor, then the round-to-nearest-even cast to bf16."""
+    if wl.dist != "normal":
+        raise ValueError("make_weight_device draws the normal law only")
+    s = wl.seed if seed is None else seed
+    gen = torch.Generator(device=device)
+    gen.manual_seed(s)
+    W = torch.randn((wl.rows, wl.cols), generator=gen, device=device, dtype=torch.float32) * wl.scale
+    k = max(1, _round_half_even(wl.outlier_frac * wl.cols))
+    cols = torch.randperm(wl.cols, generator=torch.Generator().manual_seed(s))[:k].to(device)
+    W[:, cols] *= wl.outlier_mult
+    return W.to(torch.bfloat16) if wl.wdtype == "bf16" else W
+
+
 def _round_half_even(x: float) -> int:
     return int(np.round(x))  # numpy rounds half to even
 

@@ -137,6 +137,31 @@ int dq_solve_host(const void* W_host, int w_dtype, int64_t rows, int64_t cols, i
  * Counts cover the BCD iterations only (not init or the final pass). */
 int dq_diagnostics(const void* workspace, void* stream, uint64_t out[4]);
 
+/* One matrix of a batched solve: W (device, row-major rows x cols, w_dtype)
+ * and its outputs (as for dq_solve, mse with iters+1 entries). */
+typedef struct {
+  const void* W;
+  int w_dtype;
+  int64_t rows;
+  int64_t cols;
+  dq_outputs out;
+} dq_matrix;
+
+/* dq_solve for `count` matrices with the same format, group, iteration count
+ * and column-scale dtype, enqueued one after another on `stream` and sharing
+ * one workspace (stream order keeps them apart).  This is how a whole model's
+ * linear layers are quantized in one call (the DualQuant summary, App. I and
+ * Table 12: the 224 linear layers of Llama-3.1-8B, each quantized on its
+ * own).  The workspace must hold
+ * dq_workspace_bytes() of the largest matrix.  Every matrix is validated
+ * before anything is enqueued; an invalid one returns its error and
+ * `*bad_index` (if non-NULL) receives its index.
+ *  status  optional device int[count]: after each matrix a stream-ordered
+ *          kernel stores its device-side status (DQ_OK, DQ_ENONFINITE or
+ *          DQ_ECUDA), so one non-finite matrix does not hide the others. */
+int dq_solve_batched(const dq_matrix* mats, int count, int format, int group, int iters, int col_dtype, int* status,
+                     void* workspace, size_t workspace_bytes, int* bad_index, void* stream);
+
 /* Size of the library-owned device scratch that dq_solve_static uses: 8 MiB.
  * A shape fits when dq_workspace_bytes(rows, cols, format, group) is at most
  * this; on a 148-SM B200 that holds every shape with cols <= 262144. */
