@@ -45,7 +45,7 @@ __host__ __device__ constexpr size_t iter_acc_bytes() {
 }
 __host__ __device__ constexpr size_t iter_smem_bytes(int es) {
   return (size_t)kRingBytes + iter_acc_bytes() + 2 * sizeof(uint64_t) * ring_stages(es) +
-         (2 + kStripMax + 4) * sizeof(int);
+         (2 + kStripMax + 4) * sizeof(int) + 2 * 4 * 32 * sizeof(unsigned long long);
 }
 
 // ---------------------------------------------------------------------------
@@ -114,12 +114,25 @@ __device__ __forceinline__ float a_load(const void* store, int64_t idx) {
   }
 }
 
+// Column table of the current strip in shared memory: colt[c][lane] holds
+// (b, cb) of column 8 lane + c as a float2 pair per column pair: entry
+// [(2 i) / 2][lane] = {b of pair i} and {cb of pair i}.  Loads are volatile so
+// the compiler re-reads the table at each use instead of holding 16 registers.
+__device__ __forceinline__ f2 col_ld(const f2* tab, int i, int lane) {
+  f2 v;
+  asm volatile("ld.shared.b64 %0, [%1];" : "=l"(v) : "r"(smem_u32(tab + i * 32 + lane)));
+  return v;
+}
+
 // Per-lane state of a column strip segment, as 4 column pairs: b, the
 // candidate factor cb = 1/b (times 1/s_T for NVFP4), fp32 column runs, and the
 // guard threshold per column (MXINT4 columns with a power-of-two b have an exact
 // candidate and need no guard).
 struct ColState {
-  f2 b2[4], cb2[4], cn2[4], cd2[4];
+  const f2* tb;   // shared table of b pairs [4][32]
+  const f2* tcb;  // shared table of cb pairs [4][32]
+  int lane;
+  f2 cn2[4], cd2[4];
   float thr[8];
   f2 res2;  // fp32 run of squared reconstruction residuals
   bool ok;
@@ -274,8 +287,9 @@ __device__ __forceinline__ void req_slow(const f2 w2[4], const f2 u2[4], float a
     w[2 * i + 1] = hi_of(w2[i]);
     u[2 * i] = lo_of(u2[i]);
     u[2 * i + 1] = hi_of(u2[i]);
-    b[2 * i] = lo_of(cs.b2[i]);
-    b[2 * i + 1] = hi_of(cs.b2[i]);
+    const f2 bi = col_ld(cs.tb, i, cs.lane);
+    b[2 * i] = lo_of(bi);
+    b[2 * i + 1] = hi_of(bi);
   }
   if (!ok) {
 #pragma unroll
@@ -408,7 +422,7 @@ __device__ __forceinline__ void row_sums(const f2 w2[4], const f2 q2[4], float a
   f2 num2 = 0ull, den2 = 0ull;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const f2 pq = mul2(q2[i], cs.b2[i]);
+    const f2 pq = mul2(q2[i], col_ld(cs.tb, i, cs.lane));
     num2 = fma2(w2[i], pq, num2);
     den2 = fma2(pq, pq, den2);
     const f2 e = mul2(fma2(pq, na2, w2[i]), rscale2);  // residual times a power of two (range)
@@ -425,7 +439,7 @@ __device__ __forceinline__ void row_sums64(const f2 w2[4], const f2 q2[4], const
   d64 = 0.0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const f2 pq = mul2(q2[i], cs.b2[i]);  // exact products
+    const f2 pq = mul2(q2[i], col_ld(cs.tb, i, cs.lane));  // exact products
     n64 = fma((double)lo_of(w2[i]), (double)lo_of(pq), n64);
     d64 = fma((double)lo_of(pq), (double)lo_of(pq), d64);
     n64 = fma((double)hi_of(w2[i]), (double)hi_of(pq), n64);
@@ -451,8 +465,9 @@ __device__ __forceinline__ void row_pair(const Problem& p, const f2 wx[4], float
   f2 ux[4], uy[4], qx[4], qy[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    ux[i] = mul2(wx[i], cs.cb2[i]);
-    uy[i] = mul2(wy[i], cs.cb2[i]);
+    const f2 cbi = col_ld(cs.tcb, i, cs.lane);
+    ux[i] = mul2(wx[i], cbi);
+    uy[i] = mul2(wy[i], cbi);
   }
   req_pair<FMT>(wx, ux, ax_old, actx, wy, uy, ay_old, acty, cs, sT, sTd, qx, qy, s_cnt);
   float nx, dx, ny, dy;
@@ -491,8 +506,9 @@ __device__ __forceinline__ void row_pair(const Problem& p, const f2 wx[4], float
     // recomputed rather than kept live across the block update (registers)
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      ux[i] = mul2(wx[i], cs.cb2[i]);
-      uy[i] = mul2(wy[i], cs.cb2[i]);
+      const f2 cbi = col_ld(cs.tcb, i, cs.lane);
+      ux[i] = mul2(wx[i], cbi);
+      uy[i] = mul2(wy[i], cbi);
     }
     req_pair<FMT>(wx, ux, anx, actx, wy, uy, any, acty, cs, sT, sTd, qx, qy, s_cnt);
   }
@@ -541,6 +557,7 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t, cons
   uint64_t* empty = full + S;
   int* s_misc = reinterpret_cast<int*>(empty + S);  // [0] ticket result, [1] #ambiguous, [2..] columns
   unsigned* s_cnt = reinterpret_cast<unsigned*>(s_misc + 2 + kStripMax);  // exact-path counters
+  f2* ctab = reinterpret_cast<f2*>(s_cnt + 4);  // column table of the strip: b pairs, then cb pairs
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row_bytes = p.TS * ES;  // ring slot per row
   const int stage_bytes = kRowsPerTile * row_bytes;
@@ -636,6 +653,10 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t, cons
     const int64_t blk_col = col / p.G;
 
     ColState cs;
+    cs.tb = ctab;
+    cs.tcb = ctab + 128;
+    cs.lane = lane;
+    consumer_sync(kConsumers);  // the previous segment's readers of the table are done
     cs.ok = sT_ok;
     cs.res2 = 0ull;
     int b_bits = 1;  // longest odd significand among the lane's column scales
@@ -657,12 +678,15 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t, cons
         }
         acc[(warp * 8 + c) * 32 + lane] = make_double2(0.0, 0.0);
       }
-      cs.b2[i] = pk(bj[0], bj[1]);
-      cs.cb2[i] = pk(cb[0], cb[1]);
+      if (warp == 0) {
+        ctab[i * 32 + lane] = pk(bj[0], bj[1]);
+        ctab[128 + i * 32 + lane] = pk(cb[0], cb[1]);
+      }
       cs.cn2[i] = cs.cd2[i] = 0ull;
     }
     // odd part of a b: E4M3 e has at most 4 significant bits, 2^k has 1
     cs.tie_ok = tie_certified<FMT, WDT>(FMT == FMT_NVFP4 ? sT_bits + 4 + b_bits : b_bits);
+    consumer_sync(kConsumers);  // the column table is written
     int run = 0;
     // block scales of this warp's rows, one tile ahead
     const int64_t a_step = (int64_t)kRowsPerTile * p.nb;
