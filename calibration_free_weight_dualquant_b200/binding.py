@@ -79,6 +79,8 @@ def load_library():
     lib.dq_solve_static.restype = I
     lib.dq_solve_batched.argtypes = [ctypes.POINTER(_Matrix), I, I, I, I, I, P, P, SZ, ctypes.POINTER(I), P]
     lib.dq_solve_batched.restype = I
+    lib.dq_act_quant.argtypes = [P, I, I64, I64, P, I, I, I, ctypes.POINTER(_Outputs), P, SZ, P]
+    lib.dq_act_quant.restype = I
     lib.dq_status_str.argtypes = [I]
     lib.dq_status_str.restype = ctypes.c_char_p
     _lib = lib
@@ -248,6 +250,43 @@ def dq_solve_batched(Ws, fmt, group: Optional[int] = None, iters: int = 0, col_d
     for o in outs:
         o["workspace"] = workspace
     return outs
+
+
+ACT_WORKSPACE_BYTES = 256
+
+
+def dq_act_quant(X: torch.Tensor, col_scales: torch.Tensor, fmt, group: Optional[int] = None,
+                 out: Optional[dict] = None, workspace: Optional[torch.Tensor] = None, stream=None,
+                 check: bool = True) -> dict:
+    """Enqueue dq_act_quant: X [tokens, cols] (bf16/f16 CUDA) times the column inverse scales, quantized
+    row-wise in the format (codes, group scales, NVFP4 tensor scale)."""
+    lib = load_library()
+    f = _fmt(fmt)
+    g = DEFAULT_GROUP[f] if group is None else group
+    if not X.is_cuda or X.dtype not in (torch.bfloat16, torch.float16) or not X.is_contiguous() or X.dim() != 2:
+        raise DQError(1, "dq_act_quant: X must be a contiguous 2-D bf16/f16 CUDA tensor")
+    if col_scales.dtype not in (torch.bfloat16, torch.float16) or not col_scales.is_cuda:
+        raise DQError(1, "dq_act_quant: col_scales must be a bf16/f16 CUDA tensor")
+    rows, cols = X.shape
+    if out is None:
+        out = {"codes": torch.empty((rows, cols // 2), dtype=torch.uint8, device=X.device),
+               "block_scales": torch.empty((rows, cols // g), dtype=torch.float16 if f == Format.INT4 else torch.uint8,
+                                           device=X.device),
+               "tensor_scale": torch.empty(1, dtype=torch.float32, device=X.device)}
+    if workspace is None:
+        workspace = torch.empty(ACT_WORKSPACE_BYTES, dtype=torch.uint8, device=X.device)
+    o = _Outputs(out["codes"].data_ptr(), out["block_scales"].data_ptr(), out["tensor_scale"].data_ptr(), None, None)
+    st = lib.dq_act_quant(X.data_ptr(), _DTYPES[X.dtype], rows, cols, col_scales.data_ptr(),
+                          _DTYPES[col_scales.dtype], int(f), g, ctypes.byref(o), workspace.data_ptr(),
+                          workspace.numel(), _stream_ptr(stream))
+    if st != 0:
+        raise DQError(st, "dq_act_quant")
+    if check:
+        st = lib.dq_sync_status(workspace.data_ptr(), _stream_ptr(stream))
+        if st != 0:
+            raise DQError(st, "dq_act_quant (device)")
+    out["workspace"] = workspace
+    return out
 
 
 def dq_rtn(W: torch.Tensor, fmt, group: Optional[int] = None, col_dtype: Optional[str] = None, **kw) -> dict:

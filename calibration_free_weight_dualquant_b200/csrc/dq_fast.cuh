@@ -51,7 +51,7 @@ __device__ __forceinline__ float qfast_int4(float u, float ia, float thr, bool& 
 // a*b is exact in fp32 (fp16*fp16, fp16*bf16 or 2^k*bf16), and w - h*a*b is
 // formed exactly inside one fma, so its sign says on which side of the
 // boundary h nearest the candidate W/(a b) lies; zero is a tie (to even).
-__device__ __noinline__ float qexact32_int4(float w, float u, float ia, float ab) {
+static __device__ __noinline__ float qexact32_int4(float w, float u, float ia, float ab) {
   const float xt = u * ia;
   const float qu = __fsub_rn(__fadd_rn(xt, 12582912.f), 12582912.f);
   const float h = qu + copysignf(0.5f, xt - qu);
@@ -69,7 +69,7 @@ __device__ __noinline__ float qexact32_int4(float w, float u, float ia, float ab
 
 // Exact E2M1 decision in fp32: a*b = c1 * sT with c1 = e*b exact (<= 15 bits),
 // h*c1 exact, and |w| - (h*c1)*sT formed exactly inside one fma.
-__device__ __noinline__ float qexact32_e2m1(float w, float u, float ia, float c1, float sT) {
+static __device__ __noinline__ float qexact32_e2m1(float w, float u, float ia, float c1, float sT) {
   const float xt = u * ia;
   const float ax = fminf(fabsf(xt), 6.f);
   const float p2 = __uint_as_float(max(__float_as_uint(ax) & 0x7F800000u, 0x3F800000u));

@@ -144,3 +144,22 @@ def to_oracle_input(W: torch.Tensor):
     if W.dtype == torch.float16:
         return W.contiguous().numpy(), "f16"
     return W.contiguous().numpy().astype(np.float32, copy=False), "f32"
+
+
+def make_activations(tokens: int, cols: int, seed: int, outlier_frac: float = 0.01,
+                     outlier_mult: float = 20.0) -> torch.Tensor:
+    """Synthetic activations for the activation quantizer: N(0, 1) in fp32 (numpy PCG64), with
+    k = max(1, round_half_even(frac * cols)) outlier channels (seeded permutation) multiplied by the
+    factor -- the channel outliers that make activation quantization hard -- then cast to bf16 (RNE)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    X = rng.standard_normal((tokens, cols), dtype=np.float32)
+    k = max(1, _round_half_even(outlier_frac * cols))
+    X[:, rng.permutation(cols)[:k]] *= np.float32(outlier_mult)
+    return torch.from_numpy(X).to(torch.bfloat16)
+
+
+def make_col_scales(cols: int, seed: int) -> torch.Tensor:
+    """Synthetic column inverse scales for the activation quantizer: exp(N(0, 0.3^2)) cast to bf16 (the
+    solver's column scales stay within a small factor of 1)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    return torch.from_numpy(np.exp(rng.normal(0.0, 0.3, cols)).astype(np.float32)).to(torch.bfloat16)

@@ -162,6 +162,29 @@ typedef struct {
 int dq_solve_batched(const dq_matrix* mats, int count, int format, int group, int iters, int col_dtype, int* status,
                      void* workspace, size_t workspace_bytes, int* bad_index, void* stream);
 
+/* Workspace bytes of dq_act_quant (header: flags and the NVFP4 amax). */
+#define DQ_ACT_WORKSPACE_BYTES 256u
+
+/* The beta-folded activation quantizer (DualQuant summary §4.4 "Inference-time
+ * procedure and overhead"; reproduction README flowchart, "Scale X by column
+ * inverse scales, then quantize"): with W ~ D_a Q D_b, X W^T = (X D_b) Q^T D_a,
+ * so the activations X [rows][cols] (rows = tokens, cols = input features) are
+ * multiplied per channel by the solver's column inverse scales b [cols] and
+ * quantized row-wise in the format's own way, in one kernel:
+ *   x'   = x * b[col]                      exact in fp32 (bf16/fp16 x and b)
+ *   a    = Proj_Fa(max|x'| over the group / qmax), 1 for an all-zero group
+ *          (NVFP4: a = s_T * e with s_T = fp32(amax|X'| / 2688), one per call)
+ *   q    = Q(x' / a)                       nearest grid value, ties to even
+ * Outputs as for dq_solve: out->codes [rows][cols/2], out->block_scales
+ * [rows][cols/group], out->tensor_scale (NVFP4; 1.0 otherwise, may be NULL
+ * then); col_scales and mse of `out` are not used.  x_dtype is DQ_BF16 or
+ * DQ_F16, col_dtype the dtype of `col_scales` (DQ_BF16 or DQ_F16).  The
+ * workspace (DQ_ACT_WORKSPACE_BYTES, 256-byte aligned) reports a non-finite
+ * X * b through dq_sync_status. */
+int dq_act_quant(const void* X, int x_dtype, int64_t rows, int64_t cols, const void* col_scales, int col_dtype,
+                 int format, int group, const dq_outputs* out, void* workspace, size_t workspace_bytes,
+                 void* stream);
+
 /* Size of the library-owned device scratch that dq_solve_static uses: 8 MiB.
  * A shape fits when dq_workspace_bytes(rows, cols, format, group) is at most
  * this; on a 148-SM B200 that holds every shape with cols <= 262144. */

@@ -140,6 +140,29 @@ def rtn(W: np.ndarray, wdtype: str, fmt: str, group: int, col_dtype: str, want_q
     return solve(W, wdtype, fmt, group, 0, col_dtype, want_q=want_q)
 
 
+def values(W: np.ndarray, wdtype: str) -> np.ndarray:
+    """Exact fp64 values of an input array given as the oracle takes it."""
+    if wdtype == "bf16":
+        return (np.ascontiguousarray(W, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    if wdtype == "f16":
+        return (W.view(np.float16) if W.dtype == np.uint16 else W.astype(np.float16)).astype(np.float64)
+    return np.asarray(W, dtype=np.float32).astype(np.float64)
+
+
+def act_quant(X: np.ndarray, xdtype: str, b: np.ndarray, fmt: str, group: int) -> dict:
+    """Beta-folded activation quantization (DualQuant summary §4.4 'Inference-time procedure and
+    overhead'; reproduction README flowchart, 'Scale X by column inverse scales, then quantize'):
+    X' = X diag(b), formed exactly in fp64, then the format's row-wise absmax round-to-nearest of X'
+    (`rtn`: group scale Proj(absmax/qmax), 1 for an all-zero group, NVFP4 tensor scale
+    fp32(amax/2688)).  With bf16/fp16 X and b every x*b has at most 22 significant bits, so the f32
+    copy handed to `rtn` is exact (checked)."""
+    Xp = values(X, xdtype) * np.asarray(b, dtype=np.float64)[None, :]
+    Xp32 = Xp.astype(np.float32)
+    if not np.array_equal(Xp32.astype(np.float64), Xp):
+        raise OracleError("x * b is not exact in fp32")
+    return rtn(Xp32, "f32", fmt, group, "bf16")
+
+
 def requant(W, wdtype, fmt, group, col_dtype, sT, a, b) -> np.ndarray:
     """Q(W/(a b)) for every element -> grid values [M, N]."""
     lib = _load()

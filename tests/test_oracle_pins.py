@@ -451,3 +451,36 @@ def test_nonfinite_rejected():
     W[1, 5] = np.inf
     with pytest.raises(oracle.OracleError):
         oracle.rtn(W, "f32", "int4", 64, "f16")
+
+
+@pytest.mark.parametrize("fmt,G", [("int4", 64), ("mxint4", 32), ("nvfp4", 16), ("int4", 16)])
+def test_act_quant_brute_force(fmt, G):
+    """Beta-folded activation quantization (DualQuant §4.4; README flowchart 'Scale X by column inverse
+    scales, then quantize'): codes, group scales and tensor scale re-derived by brute force from
+    X' = X diag(b) -- the product formed as an exact rational, scales by enumerating the admissible
+    set, codes by enumerating the grid."""
+    rows, cols = 3, 4 * G
+    bits, xdt, Xv = tiny_matrix(rows, cols, "bf16", seed=G * 7 + len(fmt))
+    rng = np.random.Generator(np.random.PCG64(G))
+    b_bits = bf16_bits(np.exp(rng.normal(0.0, 0.5, cols)).astype(np.float32))
+    b = bf16_values(b_bits)
+    Xv = Xv.copy()
+    Xv[1, :G] = 0.0  # an all-zero group gets scale 1
+    bits = bf16_bits(Xv.astype(np.float32))
+    out = oracle.act_quant(bits, "bf16", b, fmt, G)
+    Xp = [[Fraction(float(Xv[i, j])) * Fraction(float(b[j])) for j in range(cols)] for i in range(rows)]
+    qmax = Fraction(6 if fmt == "nvfp4" else 7)
+    sT = 1.0
+    if fmt == "nvfp4":
+        amax = max(abs(v) for row in Xp for v in row)
+        sT = float(np.float32(float(amax / 2688)))
+        assert out["sT"] == sT
+    for i in range(rows):
+        for g in range(cols // G):
+            m = max(abs(v) for v in Xp[i][g * G:(g + 1) * G])
+            want = bf.nearest_admissible(A_KIND[fmt], float(m / qmax) / sT) if m > 0 else 1.0
+            assert out["a"][i, g] == want, (i, g)
+            av = Fraction(float(want)) * Fraction(sT)
+            for j in range(g * G, (g + 1) * G):
+                q = bf.grid_argmin(fmt, float(Xp[i][j]), av)
+                assert bf.decode_codes(fmt, out["codes"])[i, j] == q, (i, j)
