@@ -227,6 +227,94 @@ def config_of(wl, world) -> dict:
             "l2": "flushed before each step (512 MB write, untimed)", "parallelism": "replicas x%d" % world}
 
 
+# beta-folded activation quantization of a prefill batch: (format, group, tokens, in-features)
+ACT_WORKLOADS = {
+    "act_nvfp4_8192x4096": ("nvfp4", 16, 8192, 4096),
+    "act_mxint4_8192x14336": ("mxint4", 32, 8192, 14336),
+    "act_int4_8192x4096": ("int4", 64, 8192, 4096),
+}
+
+
+def run_act(args, name, rank, world, local, dist):
+    """dq_act_quant on a synthetic prefill batch (X [tokens, cols] bf16, b [cols] bf16); a step is one call.
+    The oracle arm (--impl reference) times oracle.act_quant on a row sample."""
+    fmt, g, T, K = ACT_WORKLOADS[name]
+    cfg = {"workload": name, "tokens": T, "cols": K, "format": fmt, "group": g, "x_dtype": "bf16",
+           "col_dtype": "bf16", "l2": "flushed before each step (512 MB write, untimed)",
+           "parallelism": "replicas x%d" % world}
+    metric, unit = "activation elems/sec", "elem/s"
+    X = synth.make_activations(T, K, seed=77 + rank)
+    b = synth.make_col_scales(K, seed=78)
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        import oracle
+        rows = max(1, min(T, 256))
+        Xin, xdt = synth.to_oracle_input(X[:rows].contiguous())
+        bv = b.to(torch.float64).numpy()
+        for _ in range(args.warmup):
+            oracle.act_quant(Xin, xdt, bv, fmt, g)
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            oracle.act_quant(Xin, xdt, bv, fmt, g)
+        dt = time.perf_counter() - t0
+        value = rows * K * args.steps / dt
+        line = {"impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": cfg,
+                "cpu_baseline": {"value": value, "unit": unit, "cores": oracle.num_threads(), "kind": "oracle",
+                                 "sample": "first %d of %d tokens per step" % (rows, T)},
+                "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    binding.load_library()
+    Xd, bd = X.to(dev), b.to(dev)
+    out = binding.dq_act_quant(Xd, bd, fmt, g)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(steps):
+        ts = []
+        for _ in range(steps):
+            flush.fill_(1)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            binding.dq_act_quant(Xd, bd, fmt, g, out=out, workspace=out["workspace"], stream=stream, check=False)
+            e1.record(stream)
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return ts
+
+    timed(args.warmup)
+    barrier(dist)
+    torch.cuda.synchronize()
+    with ClockSampler(dev) as clk:
+        ts = timed(args.steps)
+    barrier(dist)
+    total_ms = max_over_ranks(sum(ts), dist)
+    med_ms = max_over_ranks(statistics.median(ts), dist)
+    if rank != 0:
+        return
+    asz = 2 if fmt == "int4" else 1
+    alg = T * K * 2 + T * K // 2 + T * (K // g) * asz + K * 2  # X read once, codes and scales written
+    peaks = measured_peaks()
+    achieved = alg / (med_ms * 1e-3) / 1e9
+    line = {"metric": metric, "value": world * T * K * args.steps / (total_ms * 1e-3), "unit": unit,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": cfg,
+            "roofline": {"bound": "hbm", "kernel": "k_act_amax+k_act", "achieved": achieved,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                         "traffic": None, "algorithmic_bytes_per_launch": alg, "peak_source": peaks["source"],
+                         "note": "one call = amax pass + quantize pass; algorithmic bytes count one read of X"},
+            "e2e": None, "gpu_launches": 2 * args.steps, "clocks": clk.summary()}
+    print(json.dumps(line), flush=True)
+
+
 def set_config(name, world) -> dict:
     fmt = synth.LLAMA_SETS[name]
     wl = synth.llama_set(fmt)[0]
@@ -247,7 +335,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS) + sorted(synth.LLAMA_SETS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=sorted(synth.WORKLOADS) + sorted(synth.LLAMA_SETS) + sorted(ACT_WORKLOADS))
     ap.add_argument("--impl", default="dq", choices=["dq", "reference"])
     ap.add_argument("--ref-rows", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -256,6 +345,14 @@ def main():
     ap.add_argument("--cols", type=int, help="override the workload's cols (profiling cases)")
     ap.add_argument("--iters", type=int, help="override the workload's BCD iterations")
     args = ap.parse_args()
+    if args.workload in ACT_WORKLOADS:
+        rank, world, local, dist = dist_setup(args.gpus)
+        try:
+            run_act(args, args.workload, rank, world, local, dist)
+        finally:
+            if dist is not None:
+                dist.destroy_process_group()
+        return
     if args.workload in synth.LLAMA_SETS:
         rank, world, local, dist = dist_setup(args.gpus)
         try:

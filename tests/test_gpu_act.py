@@ -72,9 +72,10 @@ def test_act_zeros_and_nonfinite():
     assert bool((gpu["codes"][0] == 0).all())
     Xn = X.clone().cuda()
     Xn[5, 100] = float("nan")
-    with pytest.raises(binding.DQError) as e:
-        binding.dq_act_quant(Xn, b.cuda(), "nvfp4", 16)
-    assert e.value.status == 4
+    for fmt, g in (("nvfp4", 16), ("mxint4", 32), ("int4", 64)):
+        with pytest.raises(binding.DQError) as e:
+            binding.dq_act_quant(Xn, b.cuda(), fmt, g)
+        assert e.value.status == 4, fmt
 
 
 def test_act_argument_checks():
