@@ -72,6 +72,8 @@ def _load():
         lib.dqo_absmax_scale.restype = D
         lib.dqo_num_threads.argtypes = []
         lib.dqo_num_threads.restype = I
+        lib.dqo_set_num_threads.argtypes = [I]
+        lib.dqo_set_num_threads.restype = None
         _lib = lib
     return _lib
 
@@ -257,3 +259,8 @@ def absmax_scale(w, qmax: float) -> float:
 
 def num_threads() -> int:
     return int(_load().dqo_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Threads of the oracle's later parallel loops (e.g. 1 to time it on one core)."""
+    _load().dqo_set_num_threads(int(n))

@@ -552,3 +552,13 @@ int dqo_num_threads(void) {
   return 1;
 #endif
 }
+
+/* threads of later parallel loops (timing the oracle on one core) */
+void dqo_set_num_threads(int n) {
+#ifdef _OPENMP
+  extern void omp_set_num_threads(int);
+  omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
