@@ -58,6 +58,8 @@ def _load():
         D = ctypes.c_double
         lib.dqo_solve.argtypes = [P, I, I64, I64, I, I, I, I, P, P, P, P, P, P, P, P]
         lib.dqo_solve.restype = I
+        lib.dqo_solve_mode.argtypes = [P, I, I64, I64, I, I, I, I, I, P, P, P, P, P, P, P, P]
+        lib.dqo_solve_mode.restype = I
         lib.dqo_step.argtypes = [P, I, I64, I64, I, I, I, D, I, P, P, P, P, P, P]
         lib.dqo_step.restype = I
         lib.dqo_project.argtypes = [I, D]
@@ -103,9 +105,14 @@ def _check(st: int):
         raise OracleError("oracle status %d" % st)
 
 
+MODES = {"dual": 0, "row": 1, "col": 2}
+
+
 def solve(W: np.ndarray, wdtype: str, fmt: str, group: int, iters: int, col_dtype: str,
-          want_q: bool = False, trace: bool = False) -> dict:
+          want_q: bool = False, trace: bool = False, mode: str = "dual") -> dict:
     """Run the full solver.  W is [M, N] (float32, float16, or uint16 bf16 bits).
+    ``mode``: "dual" (the BCD iteration), or the ablation modes of DualQuant §5.3 / Table 4:
+    "row" (block scales only, b stays 1) and "col" (column scales only, a stays at RTN).
 
     Returns codes [M, N/2] uint8, a [M, N/G] (stored block-scale values: fp16
     value, 2^k, or E4M3 value e for NVFP4), b [N], sT (NVFP4 tensor scale, 1
@@ -124,9 +131,9 @@ def solve(W: np.ndarray, wdtype: str, fmt: str, group: int, iters: int, col_dtyp
     q = np.zeros((M, N), np.float64) if want_q else None
     ta = np.zeros((iters + 1, M, nb), np.float64) if trace else None
     tb = np.zeros((iters + 1, N), np.float64) if trace else None
-    st = lib.dqo_solve(_ptr(Win), WDTYPES[wdtype], M, N, FORMATS[fmt], group, iters,
-                       WDTYPES[col_dtype], _ptr(codes), _ptr(a), _ptr(b), _ptr(sT), _ptr(mse),
-                       _ptr(q), _ptr(ta), _ptr(tb))
+    st = lib.dqo_solve_mode(_ptr(Win), WDTYPES[wdtype], M, N, FORMATS[fmt], group, iters,
+                            WDTYPES[col_dtype], MODES[mode], _ptr(codes), _ptr(a), _ptr(b), _ptr(sT), _ptr(mse),
+                            _ptr(q), _ptr(ta), _ptr(tb))
     _check(st)
     out = {"codes": codes, "a": a, "b": b, "sT": float(sT[0]), "mse": mse}
     if want_q:

@@ -428,10 +428,18 @@ static void pack_codes(const problem* p, const double* q, uint8_t* codes) {
  *   trace_a    [(iters+1)][M][N/G] block scales after init and each iteration
  *   trace_b    [(iters+1)][N]
  */
-int dqo_solve(const void* W, int wdt, int64_t M, int64_t N, int fmt, int G, int iters, int col_dt, uint8_t* codes,
-              double* a_out, double* b_out, double* sT_out, double* mse, double* q_out, double* trace_a,
-              double* trace_b) {
-  if (iters < 0) return DQO_EINVAL;
+/*
+ * The solver.  mode 0: the dual-scale BCD iteration (row update, requantize,
+ * column update, requantize).  The ablation modes of the DualQuant summary
+ * (§5.3, Table 4: row scaling alone, column scaling alone) keep the other
+ * scale at its initial value:  mode 1 = row (block) scales only, b stays 1
+ * (row update, requantize);  mode 2 = column scales only, a stays at the RTN
+ * initialization (column update, requantize).
+ */
+int dqo_solve_mode(const void* W, int wdt, int64_t M, int64_t N, int fmt, int G, int iters, int col_dt, int mode,
+                   uint8_t* codes, double* a_out, double* b_out, double* sT_out, double* mse, double* q_out,
+                   double* trace_a, double* trace_b) {
+  if (iters < 0 || mode < 0 || mode > 2) return DQO_EINVAL;
   problem p;
   double* Wd = NULL;
   int st = load_problem(&p, W, wdt, M, N, fmt, G, col_dt, &Wd);
@@ -453,10 +461,14 @@ int dqo_solve(const void* W, int wdt, int64_t M, int64_t N, int fmt, int G, int 
   if (trace_a) memcpy(trace_a, a, sizeof(double) * (size_t)nA);
   if (trace_b) memcpy(trace_b, b, sizeof(double) * (size_t)N);
   for (int t = 1; t <= iters; ++t) {
-    dqo_row_update_impl(&p, q, b, a, NULL);
-    dqo_requant_impl(&p, a, b, q);
-    dqo_col_update_impl(&p, q, a, b, NULL);
-    dqo_requant_impl(&p, a, b, q);
+    if (mode != 2) {
+      dqo_row_update_impl(&p, q, b, a, NULL);
+      dqo_requant_impl(&p, a, b, q);
+    }
+    if (mode != 1) {
+      dqo_col_update_impl(&p, q, a, b, NULL);
+      dqo_requant_impl(&p, a, b, q);
+    }
     if (mse) mse[t] = dqo_mse_impl(&p, q, a, b);
     if (trace_a) memcpy(trace_a + (size_t)t * nA, a, sizeof(double) * (size_t)nA);
     if (trace_b) memcpy(trace_b + (size_t)t * N, b, sizeof(double) * (size_t)N);
@@ -471,6 +483,13 @@ int dqo_solve(const void* W, int wdt, int64_t M, int64_t N, int fmt, int G, int 
   free(q);
   free(Wd);
   return DQO_OK;
+}
+
+int dqo_solve(const void* W, int wdt, int64_t M, int64_t N, int fmt, int G, int iters, int col_dt, uint8_t* codes,
+              double* a_out, double* b_out, double* sT_out, double* mse, double* q_out, double* trace_a,
+              double* trace_b) {
+  return dqo_solve_mode(W, wdt, M, N, fmt, G, iters, col_dt, 0, codes, a_out, b_out, sT_out, mse, q_out, trace_a,
+                        trace_b);
 }
 
 /* RTN = the solver's initial iterate ([R5]: RTN with beta = 1 is the start). */

@@ -484,3 +484,36 @@ def test_act_quant_brute_force(fmt, G):
             for j in range(g * G, (g + 1) * G):
                 q = bf.grid_argmin(fmt, float(Xp[i][j]), av)
                 assert bf.decode_codes(fmt, out["codes"])[i, j] == q, (i, j)
+
+
+@pytest.mark.parametrize("mode", ["row", "col"])
+@pytest.mark.parametrize("fmt,G,col_dt,M,N,wdt,iters", TINY[:4])
+def test_ablation_modes_brute_force(mode, fmt, G, col_dt, M, N, wdt, iters):
+    """Ablation modes (DualQuant §5.3, Table 4): 'row' updates only the block scales (b stays 1),
+    'col' only the column scales (a stays at its RTN value); each step re-derived by brute force, and
+    the MSE never increases."""
+    Win, wdtype, Wv = tiny_matrix(M, N, wdt, seed=hash((mode, fmt, G, M, N)) & 0xFFFF)
+    out = oracle.solve(Win, wdtype, fmt, G, iters, col_dt, want_q=True, trace=True, mode=mode)
+    sf = out["sT"] if fmt == "nvfp4" else 1.0
+    akind = A_KIND[fmt]
+    for t in range(iters):
+        a_t, b_t = out["trace_a"][t], out["trace_b"][t]
+        q_t = brute_codes(fmt, Wv, a_t * sf, b_t, G)
+        a_n, b_n = out["trace_a"][t + 1], out["trace_b"][t + 1]
+        if mode == "row":
+            assert np.all(b_n == 1.0)
+            for i in range(M):
+                for g in range(N // G):
+                    sl = slice(g * G, (g + 1) * G)
+                    R = q_t[i, sl] * b_t[sl]
+                    want = 1.0 if np.all(R == 0) else bf.argmin_scale_objective(akind, Wv[i, sl], R, sf)
+                    assert a_n[i, g] == want, (t, i, g)
+        else:
+            assert np.array_equal(a_n, out["trace_a"][0])
+            S = np.repeat(a_t * sf, G, axis=1) * q_t
+            for j in range(N):
+                want = 1.0 if np.all(S[:, j] == 0) else bf.argmin_scale_objective(col_dt, Wv[:, j], S[:, j])
+                assert b_n[j] == want, (t, j)
+    q_T = brute_codes(fmt, Wv, out["trace_a"][iters] * sf, out["trace_b"][iters], G)
+    np.testing.assert_array_equal(out["q"], q_T)
+    assert np.all(out["mse"][1:] <= out["mse"][:-1] * (1 + 1e-12))
