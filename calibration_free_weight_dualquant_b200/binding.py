@@ -67,6 +67,8 @@ def load_library():
     lib.dq_rtn.restype = I
     lib.dq_solve.argtypes = [P, I, I64, I64, I, I, I, I, ctypes.POINTER(_Outputs), P, SZ, P]
     lib.dq_solve.restype = I
+    lib.dq_solve_mode.argtypes = [P, I, I64, I64, I, I, I, I, I, ctypes.POINTER(_Outputs), P, SZ, P]
+    lib.dq_solve_mode.restype = I
     lib.dq_sync_status.argtypes = [P, P]
     lib.dq_sync_status.restype = I
     lib.dq_host_workspace_bytes.argtypes = [I64, I64, I, I, I, I]
@@ -129,9 +131,12 @@ def _stream_ptr(stream) -> int:
     return s.cuda_stream
 
 
+MODES = {"dual": 0, "row": 1, "col": 2}
+
+
 def dq_solve(W: torch.Tensor, fmt, group: Optional[int] = None, iters: int = 0, col_dtype: Optional[str] = None,
              out: Optional[dict] = None, workspace: Optional[torch.Tensor] = None, stream=None,
-             check: bool = True) -> dict:
+             check: bool = True, mode: str = "dual") -> dict:
     """Enqueue dq_solve on a CUDA tensor W [rows, cols]; returns the output tensors.
 
     ``check`` waits for the stream and raises on a device-reported status
@@ -154,9 +159,13 @@ def dq_solve(W: torch.Tensor, fmt, group: Optional[int] = None, iters: int = 0, 
             raise DQError(1, "dq_workspace_bytes")
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
     o = _outputs_struct(out)
-    st = lib.dq_solve(W.data_ptr(), _DTYPES[W.dtype], rows, cols, int(f), g, iters, 0 if cd == "f32" else
-                      (2 if cd == "f16" else 1), ctypes.byref(o), workspace.data_ptr(), workspace.numel(),
-                      _stream_ptr(stream))
+    cdt = 2 if cd == "f16" else 1
+    if mode == "dual":
+        st = lib.dq_solve(W.data_ptr(), _DTYPES[W.dtype], rows, cols, int(f), g, iters, cdt, ctypes.byref(o),
+                          workspace.data_ptr(), workspace.numel(), _stream_ptr(stream))
+    else:
+        st = lib.dq_solve_mode(W.data_ptr(), _DTYPES[W.dtype], rows, cols, int(f), g, iters, cdt, MODES[mode],
+                               ctypes.byref(o), workspace.data_ptr(), workspace.numel(), _stream_ptr(stream))
     if st != 0:
         raise DQError(st, "dq_solve")
     if check:

@@ -84,9 +84,11 @@ int check_outputs(const dq_outputs* out, int format, int col_dtype) {
 namespace dq {
 
 int solve_impl(const void* W, int w_dtype, int64_t rows, int64_t cols, int format, int group, int iters,
-               int col_dtype, const dq_outputs* out, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+               int col_dtype, const dq_outputs* out, void* workspace, size_t workspace_bytes, cudaStream_t stream,
+               int mode) {
   int st = check_shape(rows, cols, format, group);
   if (st != DQ_OK) return st;
+  if (mode < DQ_MODE_DUAL || mode > DQ_MODE_COL) return DQ_EINVAL;
   if (w_dtype < DQ_F32 || w_dtype > DQ_F16) return DQ_EINVAL;
   if (col_dtype != DQ_F16 && col_dtype != DQ_BF16) return DQ_EUNSUPPORTED;
   if (iters < 0) return DQ_EINVAL;
@@ -117,6 +119,7 @@ int solve_impl(const void* W, int w_dtype, int64_t rows, int64_t cols, int forma
   p.P_final = pl.P_final;
   p.segmax_final = pl.segmax_final;
   p.L = pl.L;
+  p.mode = mode;
   p.codes = out->codes;
   p.a_store = out->block_scales;
   p.b_store = out->col_scales;
@@ -154,6 +157,13 @@ int dq_solve(const void* W, int w_dtype, int64_t rows, int64_t cols, int format,
              const dq_outputs* out, void* workspace, size_t workspace_bytes, void* stream) {
   return dq::solve_impl(W, w_dtype, rows, cols, format, group, iters, col_dtype, out, workspace, workspace_bytes,
                     static_cast<cudaStream_t>(stream));
+}
+
+int dq_solve_mode(const void* W, int w_dtype, int64_t rows, int64_t cols, int format, int group, int iters,
+                  int col_dtype, int mode, const dq_outputs* out, void* workspace, size_t workspace_bytes,
+                  void* stream) {
+  return dq::solve_impl(W, w_dtype, rows, cols, format, group, iters, col_dtype, out, workspace, workspace_bytes,
+                        static_cast<cudaStream_t>(stream), mode);
 }
 
 int dq_rtn(const void* W, int w_dtype, int64_t rows, int64_t cols, int format, int group, int col_dtype,

@@ -53,6 +53,7 @@ struct Problem {
   double2* col_part;        // [P * segmax][TS] (sum W a q, sum (a q)^2)
   double* cta_part;         // [max(P, P_final)]
   int use_tmap;             // W streamed by 2-D tensor copies (else one bulk copy per row)
+  int mode;                 // DQ_MODE_DUAL, DQ_MODE_ROW (b stays 1) or DQ_MODE_COL (a stays at RTN)
 };
 
 cudaError_t launch_solve(const Problem& p, int iters, int stats_ctas, cudaStream_t st);
@@ -61,6 +62,6 @@ cudaError_t launch_solve(const Problem& p, int iters, int stats_ctas, cudaStream
 // of dq_solve; `workspace` is a device address of at least the planned size).
 int solve_impl(const void* W, int w_dtype, int64_t rows, int64_t cols, int format, int group, int iters,
                int col_dtype, const dq_outputs* out, void* workspace, size_t workspace_bytes,
-               cudaStream_t stream);
+               cudaStream_t stream, int mode = DQ_MODE_DUAL);
 
 }  // namespace dq

@@ -484,6 +484,11 @@ __device__ __forceinline__ void row_pair(const Problem& p, const f2 wx[4], float
   float any = a_fast<FMT>(ny, dy, isT, amby);
   ambx = ambx && actx;
   amby = amby && acty;
+  if (p.mode == DQ_MODE_COL) {  // column scales only: the block scales keep their values
+    anx = ax_old;
+    any = ay_old;
+    ambx = amby = false;
+  }
   if (__any_sync(0xffffffffu, ambx || amby)) {
     double n64, d64;
     row_sums64(wx, qx, cs, lpb, n64, d64);
@@ -755,7 +760,9 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t, cons
       s_misc[1] = 0;
     }
     consumer_sync(kConsumers);
-    if (s_misc[0]) {
+    if (s_misc[0] && p.mode == DQ_MODE_ROW) {  // block scales only: b keeps its values
+      if (threadIdx.x == 0) p.strip_counter[s] = 0u;
+    } else if (s_misc[0]) {
       __threadfence();
       // totals in CTA order, certified projection
       double bnew = 1.0;

@@ -106,6 +106,19 @@ int dq_rtn(const void* W, int w_dtype, int64_t rows, int64_t cols, int format, i
 int dq_solve(const void* W, int w_dtype, int64_t rows, int64_t cols, int format, int group, int iters, int col_dtype,
              const dq_outputs* out, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Ablation modes of the solver (DualQuant summary §5.3, Table 4: row scaling
+ * alone, column scaling alone). */
+typedef enum {
+  DQ_MODE_DUAL = 0,  /* the dual-scale BCD iteration (dq_solve) */
+  DQ_MODE_ROW = 1,   /* block scales only: row update and requantize; b stays 1 */
+  DQ_MODE_COL = 2    /* column scales only: column update and requantize; a stays at RTN */
+} dq_mode;
+
+/* dq_solve with an ablation mode (dq_mode); DQ_MODE_DUAL is dq_solve. */
+int dq_solve_mode(const void* W, int w_dtype, int64_t rows, int64_t cols, int format, int group, int iters,
+                  int col_dtype, int mode, const dq_outputs* out, void* workspace, size_t workspace_bytes,
+                  void* stream);
+
 /* Waits for `stream`, then reports what the device recorded in `workspace`
  * during the last dq_rtn / dq_solve that used it: DQ_OK, DQ_ENONFINITE, or
  * DQ_ECUDA if the wait itself failed. */

@@ -283,3 +283,19 @@ def test_mxint4_exact_ties(wdtype, col_dtype):
         assert d["quant_tie_lane_rows"] > 0, d
     else:
         assert d["quant_tie_lane_rows"] == 0, d
+
+
+@pytest.mark.parametrize("mode", ["row", "col"])
+@pytest.mark.parametrize("fmt,group,col_dtype", [("int4", 64, "f16"), ("mxint4", 32, "bf16"), ("nvfp4", 16, "bf16")])
+def test_ablation_modes_parity(mode, fmt, group, col_dtype):
+    """Row-only and column-only solves (DualQuant §5.3, Table 4) against the oracle's modes."""
+    wl = synth.WORKLOADS["nvfp4_g16_gateup_14336x4096"]
+    W = synth.make_weight(wl, 611, 1088, seed=91)
+    gpu = binding.dq_solve(W.cuda(), fmt, group, 5, col_dtype, mode=mode)
+    Win, wdt = synth.to_oracle_input(W)
+    orc = oracle.solve(Win, wdt, fmt, group, 5, col_dtype, mode=mode)
+    compare_with_oracle(fmt, gpu, orc, MSE_RTOL, mode)
+    if mode == "row":
+        assert bool((gpu["col_scales"].float() == 1).all())
+    else:
+        assert torch.equal(gpu["block_scales"], binding.dq_rtn(W.cuda(), fmt, group, col_dtype)["block_scales"])
