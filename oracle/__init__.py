@@ -28,10 +28,10 @@ _SRC = os.path.join(_HERE, "dq_oracle.c")
 _LIB_PATH = os.path.join(_HERE, "libdq_oracle.so")
 
 # numbering of formats, dtypes and projection kinds used by dq_oracle.c
-INT4, MXINT4, NVFP4 = 0, 1, 2
+INT4, MXINT4, NVFP4, MXFP4 = 0, 1, 2, 3
 F32, BF16, F16 = 0, 1, 2
 PROJ_F16, PROJ_BF16, PROJ_E4M3, PROJ_E8M0 = 0, 1, 2, 3
-FORMATS = {"int4": INT4, "mxint4": MXINT4, "nvfp4": NVFP4}
+FORMATS = {"int4": INT4, "mxint4": MXINT4, "nvfp4": NVFP4, "mxfp4": MXFP4}
 WDTYPES = {"f32": F32, "bf16": BF16, "f16": F16}
 
 _lib = None

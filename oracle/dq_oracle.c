@@ -51,6 +51,7 @@
 #define DQO_INT4 0
 #define DQO_MXINT4 1
 #define DQO_NVFP4 2
+#define DQO_MXFP4 3 /* E2M1 grid with E8M0 block scales (the MX family's FP4 member) */
 /* element dtypes */
 #define DQO_F32 0
 #define DQO_BF16 1
@@ -214,7 +215,10 @@ typedef struct {
   const double* W;
 } problem;
 
-static double qmax_of(int fmt) { return fmt == DQO_NVFP4 ? 6.0 : 7.0; }
+/* the formats on the E2M1 grid */
+static int e2m1_grid(int fmt) { return fmt == DQO_NVFP4 || fmt == DQO_MXFP4; }
+
+static double qmax_of(int fmt) { return e2m1_grid(fmt) ? 6.0 : 7.0; }
 
 /* block inverse scale value a from its stored factor (NVFP4 stores e, a = s_T*e) */
 static double a_value(const problem* p, double stored) { return p->fmt == DQO_NVFP4 ? p->sT * stored : stored; }
@@ -222,14 +226,14 @@ static double a_value(const problem* p, double stored) { return p->fmt == DQO_NV
 /* projection of an LS inverse-scale value onto F_a; returns the stored factor */
 static double project_a(const problem* p, double v) {
   if (p->fmt == DQO_INT4) return dqo_project(DQO_PROJ_F16, v);
-  if (p->fmt == DQO_MXINT4) return dqo_project(DQO_PROJ_E8M0, v);
+  if (p->fmt == DQO_MXINT4 || p->fmt == DQO_MXFP4) return dqo_project(DQO_PROJ_E8M0, v);
   return dqo_project(DQO_PROJ_E4M3, v / p->sT); /* nearest s_T*e to v */
 }
 
 /* Q(W/(a b)) -> grid value ([R5] flowchart "Black-box format grid Q") */
 static double quant_value(const problem* p, double w, double a, double b) {
   double ab = a * b;
-  if (p->fmt == DQO_NVFP4) return E2M1_GRID[dqo_quant_index(w, ab, E2M1_GRID, E2M1_EVEN, 15)];
+  if (e2m1_grid(p->fmt)) return E2M1_GRID[dqo_quant_index(w, ab, E2M1_GRID, E2M1_EVEN, 15)];
   return INT4_GRID[dqo_quant_index(w, ab, INT4_GRID, INT4_EVEN, 16)];
 }
 
@@ -356,7 +360,7 @@ static void init_scales(problem* p, double* astored, double* b) {
 static int load_problem(problem* p, const void* W, int wdt, int64_t M, int64_t N, int fmt, int G, int col_dt,
                         double** Wd_out) {
   if (!W || M <= 0 || N <= 0 || G <= 0 || N % G != 0 || N % 2 != 0) return DQO_EINVAL;
-  if (fmt < 0 || fmt > 2 || (col_dt != DQO_F16 && col_dt != DQO_BF16)) return DQO_EINVAL;
+  if (fmt < 0 || fmt > 3 || (col_dt != DQO_F16 && col_dt != DQO_BF16)) return DQO_EINVAL;
   double* Wd = (double*)malloc(sizeof(double) * (size_t)(M * N));
   if (!Wd) return DQO_ENOMEM;
   int bad = 0;
@@ -401,7 +405,7 @@ static void pack_codes(const problem* p, const double* q, uint8_t* codes) {
   for (int64_t i = 0; i < M; ++i)
     for (int64_t j = 0; j < N; j += 2) {
       uint8_t lo, hi;
-      if (p->fmt == DQO_NVFP4) {
+      if (e2m1_grid(p->fmt)) {
         lo = e2m1_nibble(q[i * N + j]);
         hi = e2m1_nibble(q[i * N + j + 1]);
       } else {
@@ -559,7 +563,7 @@ uint32_t dqo_encode(int kind, double v) {
 
 /* grid quantizer of a format on one value (for pins) -> grid value */
 double dqo_quant_value(int fmt, double w, double ab) {
-  if (fmt == DQO_NVFP4) return E2M1_GRID[dqo_quant_index(w, ab, E2M1_GRID, E2M1_EVEN, 15)];
+  if (e2m1_grid(fmt)) return E2M1_GRID[dqo_quant_index(w, ab, E2M1_GRID, E2M1_EVEN, 15)];
   return INT4_GRID[dqo_quant_index(w, ab, INT4_GRID, INT4_EVEN, 16)];
 }
 

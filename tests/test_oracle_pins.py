@@ -21,7 +21,7 @@ from calibration_free_weight_dualquant_b200 import synth
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 
 PROJ_KIND = {"f16": oracle.PROJ_F16, "bf16": oracle.PROJ_BF16, "e4m3": oracle.PROJ_E4M3, "e8m0": oracle.PROJ_E8M0}
-A_KIND = {"int4": "f16", "mxint4": "e8m0", "nvfp4": "e4m3"}
+A_KIND = {"int4": "f16", "mxint4": "e8m0", "nvfp4": "e4m3", "mxfp4": "e8m0"}
 
 
 def read_golden(name):
@@ -195,6 +195,8 @@ TINY = [
     ("mxint4", 32, "bf16", 6, 64, "bf16", 4),
     ("nvfp4", 16, "bf16", 6, 64, "bf16", 4),
     ("nvfp4", 16, "f16", 4, 32, "f32", 3),
+    ("mxfp4", 32, "bf16", 6, 64, "bf16", 4),
+    ("mxfp4", 32, "f16", 4, 64, "f32", 3),
 ]
 
 
@@ -227,7 +229,7 @@ def test_iterations_brute_force(fmt, G, col_dt, M, N, wdt, iters):
     sT = out["sT"]
     akind = A_KIND[fmt]
     # init: absmax RTN with beta = 1; NVFP4 tensor scale fp32(amax / (6*448))
-    qmax = 6.0 if fmt == "nvfp4" else 7.0
+    qmax = 6.0 if fmt in ("nvfp4", "mxfp4") else 7.0
     if fmt == "nvfp4":
         assert sT == float(np.float32(np.abs(Wv).max() / 2688.0))
     assert np.all(out["trace_b"][0] == 1.0)
@@ -248,8 +250,8 @@ def test_iterations_brute_force(fmt, G, col_dt, M, N, wdt, iters):
             np.testing.assert_array_equal(out["q"], q_t)
             np.testing.assert_array_equal(bf.decode_codes(fmt, out["codes"]), q_t)
             # a zero code is always the all-zero nibble (no E2M1 "-0")
-            assert not np.any((out["codes"] & 0xF) == 8) or fmt != "nvfp4"
-            assert not np.any((out["codes"] >> 4) == 8) or fmt != "nvfp4"
+            assert not np.any((out["codes"] & 0xF) == 8) or fmt not in ("nvfp4", "mxfp4")
+            assert not np.any((out["codes"] >> 4) == 8) or fmt not in ("nvfp4", "mxfp4")
             break
         # row update with codes fixed: projected LS minimiser over the enumerated set
         a_next = out["trace_a"][t + 1]
@@ -453,7 +455,7 @@ def test_nonfinite_rejected():
         oracle.rtn(W, "f32", "int4", 64, "f16")
 
 
-@pytest.mark.parametrize("fmt,G", [("int4", 64), ("mxint4", 32), ("nvfp4", 16), ("int4", 16)])
+@pytest.mark.parametrize("fmt,G", [("int4", 64), ("mxint4", 32), ("nvfp4", 16), ("int4", 16), ("mxfp4", 32)])
 def test_act_quant_brute_force(fmt, G):
     """Beta-folded activation quantization (DualQuant §4.4; README flowchart 'Scale X by column inverse
     scales, then quantize'): codes, group scales and tensor scale re-derived by brute force from
@@ -469,7 +471,7 @@ def test_act_quant_brute_force(fmt, G):
     bits = bf16_bits(Xv.astype(np.float32))
     out = oracle.act_quant(bits, "bf16", b, fmt, G)
     Xp = [[Fraction(float(Xv[i, j])) * Fraction(float(b[j])) for j in range(cols)] for i in range(rows)]
-    qmax = Fraction(6 if fmt == "nvfp4" else 7)
+    qmax = Fraction(6 if fmt in ("nvfp4", "mxfp4") else 7)
     sT = 1.0
     if fmt == "nvfp4":
         amax = max(abs(v) for row in Xp for v in row)
@@ -487,7 +489,7 @@ def test_act_quant_brute_force(fmt, G):
 
 
 @pytest.mark.parametrize("mode", ["row", "col"])
-@pytest.mark.parametrize("fmt,G,col_dt,M,N,wdt,iters", TINY[:4])
+@pytest.mark.parametrize("fmt,G,col_dt,M,N,wdt,iters", TINY[:4] + TINY[5:6])
 def test_ablation_modes_brute_force(mode, fmt, G, col_dt, M, N, wdt, iters):
     """Ablation modes (DualQuant §5.3, Table 4): 'row' updates only the block scales (b stays 1),
     'col' only the column scales (a stays at its RTN value); each step re-derived by brute force, and
