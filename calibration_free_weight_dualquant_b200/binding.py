@@ -24,13 +24,14 @@ class Format(enum.IntEnum):
     INT4 = 0
     MXINT4 = 1
     NVFP4 = 2
+    MXFP4 = 3
 
 
-_FMT_NAMES = {"int4": Format.INT4, "mxint4": Format.MXINT4, "nvfp4": Format.NVFP4}
+_FMT_NAMES = {"int4": Format.INT4, "mxint4": Format.MXINT4, "nvfp4": Format.NVFP4, "mxfp4": Format.MXFP4}
 _DTYPES = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
 _COL_DTYPES = {"f16": torch.float16, "bf16": torch.bfloat16}
-DEFAULT_GROUP = {Format.INT4: 64, Format.MXINT4: 32, Format.NVFP4: 16}
-DEFAULT_COL_DTYPE = {Format.INT4: "f16", Format.MXINT4: "bf16", Format.NVFP4: "bf16"}
+DEFAULT_GROUP = {Format.INT4: 64, Format.MXINT4: 32, Format.NVFP4: 16, Format.MXFP4: 32}
+DEFAULT_COL_DTYPE = {Format.INT4: "f16", Format.MXINT4: "bf16", Format.NVFP4: "bf16", Format.MXFP4: "bf16"}
 
 
 class DQError(RuntimeError):

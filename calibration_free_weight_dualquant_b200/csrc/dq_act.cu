@@ -137,7 +137,7 @@ __global__ void __launch_bounds__(kActThreads) k_act(ActProblem p) {
   const double sTd = (double)sT;
   const float isT = FMT == FMT_NVFP4 ? __frcp_rn(sT) : 1.f;
   const bool sT_ok = FMT != FMT_NVFP4 || in_range(isT);
-  const float qmax = FMT == FMT_NVFP4 ? 6.f : 7.f;
+  const float qmax = fmt_e2m1(FMT) ? 6.f : 7.f;
   const int lpg = p.G / 8;  // lanes per group
   const bool leader = (lane & (lpg - 1)) == 0;
   bool bad = false;
@@ -158,7 +158,7 @@ __global__ void __launch_bounds__(kActThreads) k_act(ActProblem p) {
     const bool ok = sT_ok && in_range(ia) && in_range(isT);
     uint32_t packed = 0;
     bool near = !ok;
-    if (FMT == FMT_NVFP4) {
+    if (fmt_e2m1(FMT)) {
       // hardware E2M1 codes of a +-2^-20 relative bracket of the candidate; the
       // lower bracket's code word is already the packed nibbles (element 2i in
       // the low nibble of byte i)
@@ -226,8 +226,8 @@ extern "C" int dq_act_quant(const void* X, int x_dtype, int64_t rows, int64_t co
                             int col_dtype, int format, int group, const dq_outputs* out, void* workspace,
                             size_t workspace_bytes, void* stream) {
   if (rows <= 0 || cols <= 0 || group <= 0 || cols % group != 0) return DQ_EINVAL;
-  if (format < DQ_INT4 || format > DQ_NVFP4) return DQ_EINVAL;
-  if (format == DQ_MXINT4 && group != 32) return DQ_EUNSUPPORTED;
+  if (format < DQ_INT4 || format > DQ_MXFP4) return DQ_EINVAL;
+  if ((format == DQ_MXINT4 || format == DQ_MXFP4) && group != 32) return DQ_EUNSUPPORTED;
   if (format == DQ_NVFP4 && group != 16) return DQ_EUNSUPPORTED;
   if (group < 8 || group > 256 || (group & (group - 1)) != 0) return DQ_EUNSUPPORTED;
   if (x_dtype != DQ_BF16 && x_dtype != DQ_F16) return DQ_EUNSUPPORTED;  // x b exact in fp32 needs <= 11-bit x
@@ -264,6 +264,7 @@ extern "C" int dq_act_quant(const void* X, int x_dtype, int64_t rows, int64_t co
   switch (format) {
     case DQ_INT4: e = dq::act_fmt<dq::FMT_INT4>(p, x_dtype, ctas, st); break;
     case DQ_MXINT4: e = dq::act_fmt<dq::FMT_MXINT4>(p, x_dtype, ctas, st); break;
+    case DQ_MXFP4: e = dq::act_fmt<dq::FMT_MXFP4>(p, x_dtype, ctas, st); break;
     default: e = dq::act_fmt<dq::FMT_NVFP4>(p, x_dtype, ctas, st); break;
   }
   return e == cudaSuccess ? DQ_OK : DQ_ECUDA;

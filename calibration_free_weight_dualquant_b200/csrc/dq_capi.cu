@@ -21,9 +21,9 @@ struct Plan {
 // Argument checks that do not touch memory.  Returns DQ_OK or an error code.
 int check_shape(int64_t rows, int64_t cols, int format, int group) {
   if (rows <= 0 || cols <= 0 || (cols & 1) || group <= 0) return DQ_EINVAL;
-  if (format < DQ_INT4 || format > DQ_NVFP4) return DQ_EINVAL;
+  if (format < DQ_INT4 || format > DQ_MXFP4) return DQ_EINVAL;
   if (cols % group != 0) return DQ_EINVAL;
-  if (format == DQ_MXINT4 && group != 32) return DQ_EUNSUPPORTED;
+  if ((format == DQ_MXINT4 || format == DQ_MXFP4) && group != 32) return DQ_EUNSUPPORTED;
   if (format == DQ_NVFP4 && group != 16) return DQ_EUNSUPPORTED;
   // a block spans group/8 lanes of a warp: a power of two from 1 to 32
   if (group < 8 || group > dq::kStripMax || (group & (group - 1)) != 0) return DQ_EUNSUPPORTED;

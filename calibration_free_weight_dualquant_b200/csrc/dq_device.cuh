@@ -20,7 +20,10 @@
 
 namespace dq {
 
-enum : int { FMT_INT4 = 0, FMT_MXINT4 = 1, FMT_NVFP4 = 2 };
+enum : int { FMT_INT4 = 0, FMT_MXINT4 = 1, FMT_NVFP4 = 2, FMT_MXFP4 = 3 };
+// formats on the E2M1 grid, and formats with power-of-two (E8M0) block scales
+__host__ __device__ constexpr bool fmt_e2m1(int f) { return f == FMT_NVFP4 || f == FMT_MXFP4; }
+__host__ __device__ constexpr bool fmt_pow2(int f) { return f == FMT_MXINT4 || f == FMT_MXFP4; }
 enum : int { DT_F32 = 0, DT_BF16 = 1, DT_F16 = 2 };
 
 // Distance (in grid units) from a rounding boundary inside which the fast fp32
@@ -88,7 +91,7 @@ template <int FMT>
 __device__ __forceinline__ float a_decode(const void* store, int64_t idx) {
   if (FMT == FMT_INT4) {
     return __half2float(reinterpret_cast<const __half*>(store)[idx]);
-  } else if (FMT == FMT_MXINT4) {
+  } else if (fmt_pow2(FMT)) {
     return __uint_as_float((uint32_t)reinterpret_cast<const uint8_t*>(store)[idx] << 23);
   } else {
     return e4m3_value(reinterpret_cast<const uint8_t*>(store)[idx]);
@@ -99,7 +102,7 @@ template <int FMT>
 __device__ __forceinline__ void a_encode(void* store, int64_t idx, double v) {
   if (FMT == FMT_INT4) {
     reinterpret_cast<__half*>(store)[idx] = __double2half(v);
-  } else if (FMT == FMT_MXINT4) {
+  } else if (fmt_pow2(FMT)) {
     reinterpret_cast<uint8_t*>(store)[idx] = (uint8_t)(ilogb(v) + 127);
   } else {
     reinterpret_cast<uint8_t*>(store)[idx] = e4m3_bits(v);
@@ -111,7 +114,7 @@ __device__ __forceinline__ void a_encode(void* store, int64_t idx, double v) {
 template <int FMT>
 __device__ __forceinline__ double a_project(double v, double sT) {
   if (FMT == FMT_INT4) return proj_f16(v);
-  if (FMT == FMT_MXINT4) return proj_pow2(v);
+  if (fmt_pow2(FMT)) return proj_pow2(v);
   return proj_e4m3(v / sT);
 }
 
@@ -195,14 +198,14 @@ __device__ __forceinline__ float quant(float w, float u, float ia, bool ok, floa
   } else {
     xt = (float)((double)w / ab_exact<FMT>(a, b, sTd));
   }
-  if (FMT == FMT_NVFP4) return q_e2m1<FMT>(xt, w, a, b, sTd);
+  if (fmt_e2m1(FMT)) return q_e2m1<FMT>(xt, w, a, b, sTd);
   return q_int4<FMT>(xt, w, a, b, sTd);
 }
 
 // 4-bit code of a grid value (zero is always the 0x0 nibble).
 template <int FMT>
 __device__ __forceinline__ uint32_t nibble(float q) {
-  if (FMT != FMT_NVFP4) return (uint32_t)((int)q) & 15u;
+  if (!fmt_e2m1(FMT)) return (uint32_t)((int)q) & 15u;
   const float m = fabsf(q);
   if (m == 0.f) return 0u;
   // magnitude code: 0.5->1, 1->2, 1.5->3, 2->4, 3->5, 4->6, 6->7

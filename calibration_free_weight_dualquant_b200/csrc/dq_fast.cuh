@@ -113,7 +113,7 @@ __device__ __forceinline__ float a_fast(float num, float den, float isT, bool& a
   }
   float v = num * rcp_approx(den);
   if (FMT == FMT_INT4) return proj_fast<10>(v, 0x1p-14f, 65504.f, amb);
-  if (FMT == FMT_MXINT4) return proj_fast<0>(v, 0x1p-126f, 0x1p126f, amb);
+  if (fmt_pow2(FMT)) return proj_fast<0>(v, 0x1p-126f, 0x1p126f, amb);
   v *= isT;
   return proj_fast<3>(v, 0x1p-6f, 448.f, amb);
 }
@@ -122,7 +122,7 @@ template <int FMT>
 __device__ __forceinline__ void a_store_f(void* store, int64_t idx, float v) {
   if (FMT == FMT_INT4) {
     reinterpret_cast<__half*>(store)[idx] = __float2half_rn(v);
-  } else if (FMT == FMT_MXINT4) {
+  } else if (fmt_pow2(FMT)) {
     reinterpret_cast<uint8_t*>(store)[idx] = (uint8_t)(__float_as_uint(v) >> 23);
   } else {
     reinterpret_cast<uint8_t*>(store)[idx] = (uint8_t)__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3);

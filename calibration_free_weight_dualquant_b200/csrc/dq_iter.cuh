@@ -104,7 +104,7 @@ template <int FMT>
 __device__ __forceinline__ float a_load(const void* store, int64_t idx) {
   if (FMT == FMT_INT4) {
     return __half2float(__ldg(reinterpret_cast<const __half*>(store) + idx));
-  } else if (FMT == FMT_MXINT4) {
+  } else if (fmt_pow2(FMT)) {
     return __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned char*>(store) + idx) << 23);
   } else {
     const unsigned short v = __ldg(reinterpret_cast<const unsigned char*>(store) + idx);
@@ -163,7 +163,7 @@ __device__ __forceinline__ int sig_bits(float v) {
 template <int FMT, int WDT>
 __device__ __forceinline__ bool tie_certified(int k_bits) {
   if (WDT == DT_F32 || FMT == FMT_INT4) return false;  // INT4: fp16 a and b give k up to 22
-  return FMT == FMT_NVFP4 ? k_bits <= 15 : k_bits <= 12;
+  return fmt_e2m1(FMT) ? k_bits <= 15 : k_bits <= 12;
 }
 
 // Exact fp64 decision for one element (factors outside the fast range).
@@ -171,7 +171,7 @@ template <int FMT>
 __device__ __noinline__ float qexact64(float w, float a, float b, double sTd) {
   const double ab = ab_exact<FMT>(a, b, sTd);
   const float xt = (float)((double)w / ab);
-  if (FMT == FMT_NVFP4) return q_e2m1<FMT>(xt, w, a, b, sTd);
+  if (fmt_e2m1(FMT)) return q_e2m1<FMT>(xt, w, a, b, sTd);
   return q_int4<FMT>(xt, w, a, b, sTd);
 }
 
@@ -185,7 +185,7 @@ __device__ __forceinline__ void req_fast(const f2 u2[4], float a, const ColState
   ok = cs.ok && in_range(ia);
   near = !ok;
   tie = false;
-  if (FMT == FMT_NVFP4) {
+  if (fmt_e2m1(FMT)) {
     const f2 ilo = splat(ia * (1.f - kRelGuard)), ihi = splat(ia * (1.f + kRelGuard));
     f2 lo[4], hi[4];
 #pragma unroll
@@ -294,7 +294,7 @@ __device__ __forceinline__ void req_slow(const f2 w2[4], const f2 u2[4], float a
   if (!ok) {
 #pragma unroll
     for (int c = 0; c < 8; ++c) q[c] = qexact64<FMT>(w[c], a, b[c], sTd);
-  } else if (FMT == FMT_NVFP4) {
+  } else if (fmt_e2m1(FMT)) {
     const float ilo = ia * (1.f - kRelGuard), ihi = ia * (1.f + kRelGuard);
 #pragma unroll
     for (int c = 0; c < 8; c += 2) {
@@ -364,7 +364,7 @@ __device__ double2 column_exact(const Problem& p, int64_t j, float bj, double sT
       a = __half2float(__ushort_as_half(__ldcg(reinterpret_cast<const unsigned short*>(p.a_store) + bidx)));
     } else {
       const uint32_t v = __ldcg(reinterpret_cast<const unsigned char*>(p.a_store) + bidx);
-      a = FMT == FMT_MXINT4 ? __uint_as_float(v << 23) : e4m3_value(v);
+      a = fmt_pow2(FMT) ? __uint_as_float(v << 23) : e4m3_value(v);
     }
     const float ia = __frcp_rn(a);
     const bool ok = in_range(cb) && in_range(ia);

@@ -54,6 +54,10 @@ WORKLOADS = {
     "nvfp4_g16_gateup_14336x4096": Workload(
         "nvfp4_g16_gateup_14336x4096", 14336, 4096, "bf16", "nvfp4", 16, "bf16", 30, "laplace", 0.012, 0.01, 10.0,
         1004),
+    # the MX family's FP4 member on the down_proj recipe (a solver variant beyond the five configs)
+    "mxfp4_g32_downproj_4096x14336": Workload(
+        "mxfp4_g32_downproj_4096x14336", 4096, 14336, "bf16", "mxfp4", 32, "bf16", 20, "student_t", 0.015, 0.005,
+        20.0, 1006),
 }
 
 # Llama-3.1-8B per-layer linear shapes (rows = out features, cols = in features)

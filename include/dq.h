@@ -53,8 +53,10 @@ typedef enum {
  *            [-126,126] stored as E8M0 bytes (k+127).
  *  DQ_NVFP4  E2M1 grid {0,+-0.5,+-1,+-1.5,+-2,+-3,+-4,+-6}, group 16, block
  *            inverse scale a = s_T * e with e an FP8 E4M3 value (stored as the
- *            E4M3 byte) and one fp32 tensor scale s_T = fp32(amax|W| / 2688). */
-typedef enum { DQ_INT4 = 0, DQ_MXINT4 = 1, DQ_NVFP4 = 2 } dq_format;
+ *            E4M3 byte) and one fp32 tensor scale s_T = fp32(amax|W| / 2688).
+ *  DQ_MXFP4  E2M1 grid, group 32, block inverse scales 2^k stored as E8M0 bytes
+ *            (the MX family's FP4 member; no tensor scale). */
+typedef enum { DQ_INT4 = 0, DQ_MXINT4 = 1, DQ_NVFP4 = 2, DQ_MXFP4 = 3 } dq_format;
 
 typedef enum { DQ_F32 = 0, DQ_BF16 = 1, DQ_F16 = 2 } dq_dtype;
 

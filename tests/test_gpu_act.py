@@ -37,7 +37,7 @@ def run_both(X: torch.Tensor, b: torch.Tensor, fmt: str, group: int, label: str)
     return gpu, orc
 
 
-@pytest.mark.parametrize("fmt,group", [("nvfp4", 16), ("mxint4", 32), ("int4", 64), ("int4", 128)])
+@pytest.mark.parametrize("fmt,group", [("nvfp4", 16), ("mxint4", 32), ("int4", 64), ("int4", 128), ("mxfp4", 32)])
 @pytest.mark.parametrize("tokens,cols,xdt,bdt", [
     (1, 256, torch.bfloat16, torch.bfloat16),
     (37, 4096, torch.bfloat16, torch.bfloat16),
@@ -50,7 +50,7 @@ def test_act_parity(fmt, group, tokens, cols, xdt, bdt):
     run_both(X, b, fmt, group, "act")
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "mxint4", "int4"])
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxint4", "int4", "mxfp4"])
 def test_act_with_unit_scales_is_the_solvers_rtn(fmt):
     """With b = 1 the activation quantizer is the solver's RTN initial iterate (dq_rtn)."""
     X = synth.make_activations(96, 1024, seed=5).cuda()
@@ -72,7 +72,7 @@ def test_act_zeros_and_nonfinite():
     assert bool((gpu["codes"][0] == 0).all())
     Xn = X.clone().cuda()
     Xn[5, 100] = float("nan")
-    for fmt, g in (("nvfp4", 16), ("mxint4", 32), ("int4", 64)):
+    for fmt, g in (("nvfp4", 16), ("mxint4", 32), ("int4", 64), ("mxfp4", 32)):
         with pytest.raises(binding.DQError) as e:
             binding.dq_act_quant(Xn, b.cuda(), fmt, g)
         assert e.value.status == 4, fmt

@@ -39,6 +39,7 @@ SMALL = {
     "int4_g64_qproj_4096x4096": (333, 704),
     "mxint4_g32_downproj_4096x14336": (301, 608),
     "nvfp4_g16_gateup_14336x4096": (339, 528),
+    "mxfp4_g32_downproj_4096x14336": (301, 608),
 }
 
 
@@ -53,6 +54,7 @@ def test_parity_small_workload_recipe(name):
 
 
 @pytest.mark.parametrize("fmt,group,col_dtype,M,N,iters", [
+    ("mxfp4", 32, "bf16", 999, 1088, 6),
     ("int4", 64, "f16", 1000, 1344, 6),
     ("mxint4", 32, "bf16", 777, 1056, 6),
     ("nvfp4", 16, "bf16", 1203, 800, 6),
@@ -64,6 +66,8 @@ def test_parity_many_ctas(fmt, group, col_dtype, M, N, iters):
 
 
 @pytest.mark.parametrize("fmt,group,col_dtype,M,N,wdtype", [
+    ("mxfp4", 32, "bf16", 3, 32, torch.bfloat16),
+    ("mxfp4", 32, "f16", 41, 288, torch.float32),
     ("int4", 8, "f16", 1, 8, torch.float32),
     ("int4", 256, "bf16", 5, 512, torch.bfloat16),
     ("int4", 128, "f16", 7, 384, torch.float16),
@@ -77,7 +81,10 @@ def test_parity_edge_shapes_and_dtypes(fmt, group, col_dtype, M, N, wdtype):
     run_both(W, fmt, group, 5, col_dtype, "edge")
 
 
-@pytest.mark.parametrize("fmt,group,col_dtype", [("int4", 64, "f16"), ("mxint4", 32, "bf16"), ("nvfp4", 16, "bf16")])
+FOUR = [("int4", 64, "f16"), ("mxint4", 32, "bf16"), ("nvfp4", 16, "bf16"), ("mxfp4", 32, "bf16")]
+
+
+@pytest.mark.parametrize("fmt,group,col_dtype", FOUR)
 def test_parity_zero_slices(fmt, group, col_dtype):
     g = torch.Generator().manual_seed(5)
     W = torch.randn(40, 4 * group, generator=g) * 0.02
@@ -88,7 +95,7 @@ def test_parity_zero_slices(fmt, group, col_dtype):
     run_both(torch.zeros(9, 2 * group, dtype=torch.bfloat16), fmt, group, 3, col_dtype, "all_zero")
 
 
-@pytest.mark.parametrize("fmt,group,col_dtype", [("int4", 64, "f16"), ("mxint4", 32, "bf16"), ("nvfp4", 16, "bf16")])
+@pytest.mark.parametrize("fmt,group,col_dtype", FOUR)
 def test_parity_exact_ties(fmt, group, col_dtype):
     """Weights on a coarse dyadic lattice make exact rounding ties frequent."""
     g = torch.Generator().manual_seed(9)
@@ -97,7 +104,7 @@ def test_parity_exact_ties(fmt, group, col_dtype):
     run_both(W.to(torch.bfloat16), fmt, group, 8, col_dtype, "ties")
 
 
-@pytest.mark.parametrize("fmt,group,col_dtype", [("int4", 64, "f16"), ("mxint4", 32, "bf16"), ("nvfp4", 16, "bf16")])
+@pytest.mark.parametrize("fmt,group,col_dtype", FOUR)
 @pytest.mark.parametrize("mag", [1e-33, 1e-12, 1e4, 1e30])
 def test_parity_extreme_magnitudes(fmt, group, col_dtype, mag):
     """Scales at the ends of the admissible sets (saturation, smallest values, fp64 fallback of the candidate)."""
@@ -107,7 +114,7 @@ def test_parity_extreme_magnitudes(fmt, group, col_dtype, mag):
     run_both(W.float(), fmt, group, 4, col_dtype, "mag%g" % mag)
 
 
-@pytest.mark.parametrize("fmt", ["int4", "mxint4", "nvfp4"])
+@pytest.mark.parametrize("fmt", ["int4", "mxint4", "nvfp4", "mxfp4"])
 def test_zero_iterations_is_rtn_and_deterministic(fmt):
     wl = synth.WORKLOADS["nvfp4_g16_gateup_14336x4096"]
     W = synth.make_weight(wl, 250, 1024, seed=3).cuda()
@@ -286,7 +293,7 @@ def test_mxint4_exact_ties(wdtype, col_dtype):
 
 
 @pytest.mark.parametrize("mode", ["row", "col"])
-@pytest.mark.parametrize("fmt,group,col_dtype", [("int4", 64, "f16"), ("mxint4", 32, "bf16"), ("nvfp4", 16, "bf16")])
+@pytest.mark.parametrize("fmt,group,col_dtype", FOUR)
 def test_ablation_modes_parity(mode, fmt, group, col_dtype):
     """Row-only and column-only solves (DualQuant §5.3, Table 4) against the oracle's modes."""
     wl = synth.WORKLOADS["nvfp4_g16_gateup_14336x4096"]
@@ -299,3 +306,13 @@ def test_ablation_modes_parity(mode, fmt, group, col_dtype):
         assert bool((gpu["col_scales"].float() == 1).all())
     else:
         assert torch.equal(gpu["block_scales"], binding.dq_rtn(W.cuda(), fmt, group, col_dtype)["block_scales"])
+
+
+def test_mxfp4_exact_ties():
+    """MXFP4 on few-bit weights: W / (2^k b) hits E2M1 boundaries exactly; bf16 W and b make every
+    flagged element a certified tie."""
+    g = torch.Generator().manual_seed(14)
+    W = (torch.randint(-48, 49, (389, 672), generator=g).float() * 2.0 ** -6).to(torch.bfloat16)
+    gpu, _ = run_both(W, "mxfp4", 32, 6, "bf16", "mxfp4_ties")
+    d = binding.diagnostics(gpu["workspace"])
+    assert d["quant_tie_lane_rows"] > 0, d
