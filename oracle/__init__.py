@@ -60,6 +60,10 @@ def _load():
         lib.dqo_solve.restype = I
         lib.dqo_solve_mode.argtypes = [P, I, I64, I64, I, I, I, I, I, P, P, P, P, P, P, P, P]
         lib.dqo_solve_mode.restype = I
+        lib.dqo_solve_ex.argtypes = [P, I, I64, I64, I, I, I, I, I, I, P, P, D, P, P, P, P, P, P, P, P, P]
+        lib.dqo_solve_ex.restype = I
+        lib.dqo_exact_abs_sum.argtypes = [P, I64]
+        lib.dqo_exact_abs_sum.restype = D
         lib.dqo_step.argtypes = [P, I, I64, I64, I, I, I, D, I, P, P, P, P, P, P]
         lib.dqo_step.restype = I
         lib.dqo_project.argtypes = [I, D]
@@ -106,18 +110,26 @@ def _check(st: int):
 
 
 MODES = {"dual": 0, "row": 1, "col": 2}
+INITS = {"rtn": 0, "l1": 1, "given": 2}
 
 
 def solve(W: np.ndarray, wdtype: str, fmt: str, group: int, iters: int, col_dtype: str,
-          want_q: bool = False, trace: bool = False, mode: str = "dual") -> dict:
+          want_q: bool = False, trace: bool = False, mode: str = "dual", init: str = "rtn",
+          a0: Optional[np.ndarray] = None, b0: Optional[np.ndarray] = None, sT0: float = 1.0,
+          changes: bool = False) -> dict:
     """Run the full solver.  W is [M, N] (float32, float16, or uint16 bf16 bits).
     ``mode``: "dual" (the BCD iteration), or the ablation modes of DualQuant §5.3 / Table 4:
-    "row" (block scales only, b stays 1) and "col" (column scales only, a stays at RTN).
+    "row" (block scales only, b keeps its initial value) and "col" (column scales only, a keeps
+    its initial value).
+    ``init``: "rtn" (absmax RTN, b = 1), "l1" (per-column L1-norm column scales, DualQuant §5.3),
+    or "given" (warm start from stored block scales a0 [M, N/G], column scales b0 [N] and, for
+    NVFP4, the tensor scale sT0).
 
     Returns codes [M, N/2] uint8, a [M, N/G] (stored block-scale values: fp16
     value, 2^k, or E4M3 value e for NVFP4), b [N], sT (NVFP4 tensor scale, 1
-    otherwise), mse [iters+1]; optionally q [M, N] grid values and per-iteration
-    traces of a and b.
+    otherwise), mse [iters+1]; optionally q [M, N] grid values, per-iteration
+    traces of a and b, and changes [iters+1] (elements whose grid value changed
+    in each iteration).
     """
     lib = _load()
     Win = _as_input(W, wdtype)
@@ -131,9 +143,12 @@ def solve(W: np.ndarray, wdtype: str, fmt: str, group: int, iters: int, col_dtyp
     q = np.zeros((M, N), np.float64) if want_q else None
     ta = np.zeros((iters + 1, M, nb), np.float64) if trace else None
     tb = np.zeros((iters + 1, N), np.float64) if trace else None
-    st = lib.dqo_solve_mode(_ptr(Win), WDTYPES[wdtype], M, N, FORMATS[fmt], group, iters,
-                            WDTYPES[col_dtype], MODES[mode], _ptr(codes), _ptr(a), _ptr(b), _ptr(sT), _ptr(mse),
-                            _ptr(q), _ptr(ta), _ptr(tb))
+    ch = np.zeros(iters + 1, np.uint64) if changes else None
+    a0c = None if a0 is None else np.ascontiguousarray(a0, np.float64).reshape(M, nb)
+    b0c = None if b0 is None else np.ascontiguousarray(b0, np.float64).reshape(N)
+    st = lib.dqo_solve_ex(_ptr(Win), WDTYPES[wdtype], M, N, FORMATS[fmt], group, iters,
+                          WDTYPES[col_dtype], MODES[mode], INITS[init], _ptr(a0c), _ptr(b0c), float(sT0),
+                          _ptr(codes), _ptr(a), _ptr(b), _ptr(sT), _ptr(mse), _ptr(q), _ptr(ta), _ptr(tb), _ptr(ch))
     _check(st)
     out = {"codes": codes, "a": a, "b": b, "sT": float(sT[0]), "mse": mse}
     if want_q:
@@ -141,7 +156,15 @@ def solve(W: np.ndarray, wdtype: str, fmt: str, group: int, iters: int, col_dtyp
     if trace:
         out["trace_a"] = ta
         out["trace_b"] = tb
+    if changes:
+        out["changes"] = ch
     return out
+
+
+def exact_abs_sum(x: np.ndarray) -> float:
+    """sum |x_k| of fp32-representable values, exact and rounded once to fp64."""
+    xd = np.ascontiguousarray(x, np.float64).reshape(-1)
+    return float(_load().dqo_exact_abs_sum(_ptr(xd), xd.size))
 
 
 def rtn(W: np.ndarray, wdtype: str, fmt: str, group: int, col_dtype: str, want_q: bool = False) -> dict:

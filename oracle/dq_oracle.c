@@ -35,7 +35,8 @@
  *  - "Scale 1 for an all-zero code slice": a = 1 (INT4, MXINT4), e = 1 (NVFP4),
  *    b = 1.
  *  - Init: b = 1 and a = Proj(absmax(block) / qmax), qmax = 7 (INT4 grid
- *    [-8,7]) or 6 (E2M1); an all-zero block gets scale 1.
+ *    [-8,7]) or 6 (E2M1); an all-zero block gets scale 1.  Variants: the
+ *    per-column L1-norm init (init_l1) and a warm start from given scales.
  */
 #include <math.h>
 #include <stdint.h>
@@ -326,24 +327,27 @@ double dqo_mse_impl(const problem* p, const double* q, const double* astored, co
   return tot / ((double)M * (double)N);
 }
 
+/* NVFP4 tensor scale from the largest magnitude the block scales must cover:
+ * s_T = fp32(amax / (6*448)), 1 when amax = 0, the least positive fp32 when it
+ * rounds to zero.  1 for the other formats. */
+static void set_tensor_scale(problem* p, double amax) {
+  if (p->fmt != DQO_NVFP4 || amax == 0.0) {
+    p->sT = 1.0;
+    return;
+  }
+  float s = (float)(amax / 2688.0);
+  if (s == 0.0f) s = ldexpf(1.0f, -149); /* nearest positive fp32 */
+  p->sT = (double)s;
+}
+
 /* Absmax RTN init ([T4] absmax; [P2] §3 symmetric scale; spec config:
  * beta = 1).  NVFP4 first fixes s_T = fp32(amax / (6*448)). */
 static void init_scales(problem* p, double* astored, double* b) {
   int64_t M = p->M, N = p->N;
-  if (p->fmt == DQO_NVFP4) {
-    double amax = 0.0;
-    for (int64_t k = 0; k < M * N; ++k)
-      if (fabs(p->W[k]) > amax) amax = fabs(p->W[k]);
-    if (amax == 0.0) {
-      p->sT = 1.0;
-    } else {
-      float s = (float)(amax / 2688.0);
-      if (s == 0.0f) s = ldexpf(1.0f, -149); /* nearest positive fp32 */
-      p->sT = (double)s;
-    }
-  } else {
-    p->sT = 1.0;
-  }
+  double amax = 0.0;
+  for (int64_t k = 0; k < M * N; ++k)
+    if (fabs(p->W[k]) > amax) amax = fabs(p->W[k]);
+  set_tensor_scale(p, amax);
   double qmax = qmax_of(p->fmt);
 #pragma omp parallel for schedule(static)
   for (int64_t i = 0; i < M; ++i)
@@ -352,6 +356,135 @@ static void init_scales(problem* p, double* astored, double* b) {
       astored[i * p->nb + g] = (m == 0.0) ? 1.0 : project_a(p, m / qmax);
     }
   for (int64_t j = 0; j < N; ++j) b[j] = 1.0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Exact sums of magnitudes.  Every input value (fp32, bf16 or fp16) is an
+ * integer multiple of 2^-149 below 2^128, so a sum of fewer than 2^63 of them
+ * is an integer below 2^340 in units of 2^-149.  It is held exactly in a
+ * 384-bit unsigned integer and rounded once to fp64, to nearest with ties to
+ * even. */
+#define XS_LIMBS 6
+typedef struct {
+  uint64_t limb[XS_LIMBS]; /* little-endian 64-bit limbs, units of 2^-149 */
+} xsum;
+
+static void xsum_add(xsum* s, double v) { /* v >= 0, a multiple of 2^-149 below 2^128 */
+  if (v == 0.0) return;
+  int e;
+  double f = frexp(v, &e);             /* v = f * 2^e with 0.5 <= f < 1 */
+  uint64_t m = (uint64_t)ldexp(f, 53); /* v = m * 2^(e-53), m < 2^53 */
+  int sh = e - 53 + 149;               /* v = m * 2^sh units */
+  if (sh < 0) {                        /* m has at least -sh trailing zero bits */
+    m >>= -sh;
+    sh = 0;
+  }
+  int li = sh / 64, bo = sh % 64;
+  uint64_t lo = m << bo, hi = bo ? m >> (64 - bo) : 0;
+  uint64_t old = s->limb[li];
+  s->limb[li] += lo;
+  uint64_t carry = s->limb[li] < old;
+  for (int k = li + 1; k < XS_LIMBS && (hi || carry); ++k) {
+    old = s->limb[k];
+    s->limb[k] += hi + carry; /* hi < 2^53: no overflow of the addend */
+    carry = s->limb[k] < old;
+    hi = 0;
+  }
+}
+
+static int xsum_bit(const xsum* s, int i) { return (int)((s->limb[i / 64] >> (i % 64)) & 1u); }
+
+static double xsum_round(const xsum* s) {
+  int top = -1;
+  for (int i = 64 * XS_LIMBS - 1; i >= 0; --i)
+    if (xsum_bit(s, i)) {
+      top = i;
+      break;
+    }
+  if (top < 0) return 0.0;
+  if (top < 53) return ldexp((double)s->limb[0], -149); /* fewer than 54 bits: exact */
+  int low = top - 52; /* keep bits low..top */
+  uint64_t mant = 0;
+  for (int i = 0; i < 53; ++i) mant |= (uint64_t)xsum_bit(s, low + i) << i;
+  int rbit = xsum_bit(s, low - 1), sticky = 0;
+  for (int i = 0; i < low - 1; ++i) sticky |= xsum_bit(s, i);
+  if (rbit && (sticky || (mant & 1u))) mant += 1; /* 2^53 is still exact */
+  return ldexp((double)mant, low - 149);
+}
+
+/* sum of |x_k| over n values, exact then rounded once to fp64 (x_k must be
+ * fp32-representable) */
+double dqo_exact_abs_sum(const double* x, int64_t n) {
+  xsum s;
+  memset(&s, 0, sizeof s);
+  for (int64_t k = 0; k < n; ++k) xsum_add(&s, fabs(x[k]));
+  return xsum_round(&s);
+}
+
+/*
+ * Per-column L1-norm init ([P2] §5.3: format-native row absmax scales and
+ * per-column L1-norm scales).  The pages name the norm only; readings taken:
+ *  - the column scale is the column's L1 norm relative to the mean column L1
+ *    norm: b_j = Proj_Fb(c_j / mu), c_j = sum_i |W_ij|, mu = (sum_ij |W_ij|) / N,
+ *    each sum exact and rounded once to fp64; b_j = 1 for an all-zero column;
+ *  - the block scales are the absmax RTN scales of the column-scaled matrix
+ *    W D_b^-1: a = Proj_Fa(max_j (|W_ij| / b_j) / qmax), 1 for an all-zero block;
+ *  - NVFP4: s_T is taken from the same matrix, fp32(max_ij (|W_ij| / b_j) / 2688).
+ * Every quotient is one correctly rounded fp64 division.  With all b_j = 1 this
+ * is exactly the absmax RTN init.
+ */
+static void init_l1(problem* p, double* astored, double* b) {
+  int64_t M = p->M, N = p->N;
+  double mu = dqo_exact_abs_sum(p->W, M * N) / (double)N;
+#pragma omp parallel for schedule(static)
+  for (int64_t j = 0; j < N; ++j) {
+    xsum c;
+    memset(&c, 0, sizeof c);
+    for (int64_t i = 0; i < M; ++i) xsum_add(&c, fabs(p->W[i * N + j]));
+    double cj = xsum_round(&c);
+    b[j] = (cj == 0.0 || mu == 0.0) ? 1.0 : dqo_project(p->col_kind, cj / mu);
+  }
+  double amax = 0.0;
+  for (int64_t k = 0; k < M * N; ++k) {
+    double v = fabs(p->W[k]) / b[k % N];
+    if (v > amax) amax = v;
+  }
+  set_tensor_scale(p, amax);
+  double qmax = qmax_of(p->fmt);
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < M; ++i)
+    for (int g = 0; g < p->nb; ++g) {
+      double m = 0.0;
+      for (int jj = 0; jj < p->G; ++jj) {
+        int64_t j = (int64_t)g * p->G + jj;
+        double v = fabs(p->W[i * N + j]) / b[j];
+        if (v > m) m = v;
+      }
+      astored[i * p->nb + g] = (m == 0.0) ? 1.0 : project_a(p, m / qmax);
+    }
+}
+
+/* Warm start: the caller's scales are the initial iterate.  Each must be
+ * admissible (an element of its set, so projection leaves it unchanged), and
+ * the NVFP4 tensor scale a positive finite fp32 value. */
+static int init_given(problem* p, const double* a0, const double* b0, double sT0, double* astored, double* b) {
+  if (!a0 || !b0) return DQO_EINVAL;
+  if (p->fmt == DQO_NVFP4) {
+    if (!(sT0 > 0.0) || !isfinite(sT0) || (double)(float)sT0 != sT0) return DQO_EINVAL;
+    p->sT = sT0;
+  } else {
+    p->sT = 1.0;
+  }
+  int akind = p->fmt == DQO_INT4 ? DQO_PROJ_F16 : (p->fmt == DQO_NVFP4 ? DQO_PROJ_E4M3 : DQO_PROJ_E8M0);
+  for (int64_t k = 0; k < p->M * p->nb; ++k) {
+    if (!(a0[k] > 0.0) || dqo_project(akind, a0[k]) != a0[k]) return DQO_EINVAL;
+    astored[k] = a0[k];
+  }
+  for (int64_t j = 0; j < p->N; ++j) {
+    if (!(b0[j] > 0.0) || dqo_project(p->col_kind, b0[j]) != b0[j]) return DQO_EINVAL;
+    b[j] = b0[j];
+  }
+  return DQO_OK;
 }
 
 /* ------------------------------------------------------------------------ */
@@ -436,14 +569,22 @@ static void pack_codes(const problem* p, const double* q, uint8_t* codes) {
  * The solver.  mode 0: the dual-scale BCD iteration (row update, requantize,
  * column update, requantize).  The ablation modes of the DualQuant summary
  * (§5.3, Table 4: row scaling alone, column scaling alone) keep the other
- * scale at its initial value:  mode 1 = row (block) scales only, b stays 1
- * (row update, requantize);  mode 2 = column scales only, a stays at the RTN
- * initialization (column update, requantize).
+ * scale at its initial value:  mode 1 = row (block) scales only, b keeps its
+ * initial value (row update, requantize);  mode 2 = column scales only, a
+ * keeps its initial value (column update, requantize).
+ * init 0: absmax RTN with b = 1; init 1: per-column L1-norm column scales
+ * (init_l1); init 2: warm start from the stored scales a0 [M][N/G], b0 [N] and
+ * (NVFP4) sT0.
+ * changes (optional, [iters+1]): changes[0] = 0 and changes[t] = the number of
+ * elements whose grid value differs between the iterates after iterations t-1
+ * and t ([P2] §4.3, App. B: the quantized matrix stabilizes; the relative
+ * change of Q is changes[t] / (M N)).
  */
-int dqo_solve_mode(const void* W, int wdt, int64_t M, int64_t N, int fmt, int G, int iters, int col_dt, int mode,
-                   uint8_t* codes, double* a_out, double* b_out, double* sT_out, double* mse, double* q_out,
-                   double* trace_a, double* trace_b) {
-  if (iters < 0 || mode < 0 || mode > 2) return DQO_EINVAL;
+int dqo_solve_ex(const void* W, int wdt, int64_t M, int64_t N, int fmt, int G, int iters, int col_dt, int mode,
+                 int init, const double* a0, const double* b0, double sT0, uint8_t* codes, double* a_out,
+                 double* b_out, double* sT_out, double* mse, double* q_out, double* trace_a, double* trace_b,
+                 uint64_t* changes) {
+  if (iters < 0 || mode < 0 || mode > 2 || init < 0 || init > 2) return DQO_EINVAL;
   problem p;
   double* Wd = NULL;
   int st = load_problem(&p, W, wdt, M, N, fmt, G, col_dt, &Wd);
@@ -452,41 +593,66 @@ int dqo_solve_mode(const void* W, int wdt, int64_t M, int64_t N, int fmt, int G,
   double* a = (double*)malloc(sizeof(double) * (size_t)nA);
   double* b = (double*)malloc(sizeof(double) * (size_t)N);
   double* q = (double*)malloc(sizeof(double) * (size_t)(M * N));
-  if (!a || !b || !q) {
+  double* qprev = changes ? (double*)malloc(sizeof(double) * (size_t)(M * N)) : NULL;
+  if (!a || !b || !q || (changes && !qprev)) {
     free(a);
     free(b);
     free(q);
+    free(qprev);
     free(Wd);
     return DQO_ENOMEM;
   }
-  init_scales(&p, a, b);
-  dqo_requant_impl(&p, a, b, q);
-  if (mse) mse[0] = dqo_mse_impl(&p, q, a, b);
-  if (trace_a) memcpy(trace_a, a, sizeof(double) * (size_t)nA);
-  if (trace_b) memcpy(trace_b, b, sizeof(double) * (size_t)N);
-  for (int t = 1; t <= iters; ++t) {
-    if (mode != 2) {
-      dqo_row_update_impl(&p, q, b, a, NULL);
-      dqo_requant_impl(&p, a, b, q);
-    }
-    if (mode != 1) {
-      dqo_col_update_impl(&p, q, a, b, NULL);
-      dqo_requant_impl(&p, a, b, q);
-    }
-    if (mse) mse[t] = dqo_mse_impl(&p, q, a, b);
-    if (trace_a) memcpy(trace_a + (size_t)t * nA, a, sizeof(double) * (size_t)nA);
-    if (trace_b) memcpy(trace_b + (size_t)t * N, b, sizeof(double) * (size_t)N);
+  if (init == 0) {
+    init_scales(&p, a, b);
+  } else if (init == 1) {
+    init_l1(&p, a, b);
+  } else {
+    st = init_given(&p, a0, b0, sT0, a, b);
   }
-  if (codes) pack_codes(&p, q, codes);
-  if (a_out) memcpy(a_out, a, sizeof(double) * (size_t)nA);
-  if (b_out) memcpy(b_out, b, sizeof(double) * (size_t)N);
-  if (sT_out) *sT_out = p.sT;
-  if (q_out) memcpy(q_out, q, sizeof(double) * (size_t)(M * N));
+  if (st == DQO_OK) {
+    dqo_requant_impl(&p, a, b, q);
+    if (mse) mse[0] = dqo_mse_impl(&p, q, a, b);
+    if (changes) changes[0] = 0;
+    if (trace_a) memcpy(trace_a, a, sizeof(double) * (size_t)nA);
+    if (trace_b) memcpy(trace_b, b, sizeof(double) * (size_t)N);
+    for (int t = 1; t <= iters; ++t) {
+      if (changes) memcpy(qprev, q, sizeof(double) * (size_t)(M * N));
+      if (mode != 2) {
+        dqo_row_update_impl(&p, q, b, a, NULL);
+        dqo_requant_impl(&p, a, b, q);
+      }
+      if (mode != 1) {
+        dqo_col_update_impl(&p, q, a, b, NULL);
+        dqo_requant_impl(&p, a, b, q);
+      }
+      if (mse) mse[t] = dqo_mse_impl(&p, q, a, b);
+      if (changes) {
+        uint64_t n = 0;
+        for (int64_t k = 0; k < M * N; ++k) n += q[k] != qprev[k];
+        changes[t] = n;
+      }
+      if (trace_a) memcpy(trace_a + (size_t)t * nA, a, sizeof(double) * (size_t)nA);
+      if (trace_b) memcpy(trace_b + (size_t)t * N, b, sizeof(double) * (size_t)N);
+    }
+    if (codes) pack_codes(&p, q, codes);
+    if (a_out) memcpy(a_out, a, sizeof(double) * (size_t)nA);
+    if (b_out) memcpy(b_out, b, sizeof(double) * (size_t)N);
+    if (sT_out) *sT_out = p.sT;
+    if (q_out) memcpy(q_out, q, sizeof(double) * (size_t)(M * N));
+  }
   free(a);
   free(b);
   free(q);
+  free(qprev);
   free(Wd);
-  return DQO_OK;
+  return st;
+}
+
+int dqo_solve_mode(const void* W, int wdt, int64_t M, int64_t N, int fmt, int G, int iters, int col_dt, int mode,
+                   uint8_t* codes, double* a_out, double* b_out, double* sT_out, double* mse, double* q_out,
+                   double* trace_a, double* trace_b) {
+  return dqo_solve_ex(W, wdt, M, N, fmt, G, iters, col_dt, mode, 0, NULL, NULL, 1.0, codes, a_out, b_out, sT_out, mse,
+                      q_out, trace_a, trace_b, NULL);
 }
 
 int dqo_solve(const void* W, int wdt, int64_t M, int64_t N, int fmt, int G, int iters, int col_dt, uint8_t* codes,

@@ -8,6 +8,7 @@ invariants of the method.
 from __future__ import annotations
 
 import os
+import zlib
 from fractions import Fraction
 
 import numpy as np
@@ -200,6 +201,11 @@ TINY = [
 ]
 
 
+def stable_seed(*key) -> int:
+    """A seed from a key that is the same in every process (str hashes are randomised)."""
+    return zlib.crc32(repr(key).encode()) & 0xFFFF
+
+
 def tiny_matrix(rows, cols, wdt, seed):
     rng = np.random.Generator(np.random.PCG64(seed))
     W = (rng.laplace(0, 0.02, (rows, cols))).astype(np.float32)
@@ -224,8 +230,8 @@ def brute_codes(fmt, Wv, a_val, b, G):
 def test_iterations_brute_force(fmt, G, col_dt, M, N, wdt, iters):
     """Every step of every iteration re-derived by brute force from the previous state
     (reproduction README flowchart and 'Core equations'; DualQuant §4.3, App. B)."""
-    Win, wdtype, Wv = tiny_matrix(M, N, wdt, seed=hash((fmt, G, M, N)) & 0xFFFF)
-    out = oracle.solve(Win, wdtype, fmt, G, iters, col_dt, want_q=True, trace=True)
+    Win, wdtype, Wv = tiny_matrix(M, N, wdt, seed=stable_seed(fmt, G, M, N))
+    out = oracle.solve(Win, wdtype, fmt, G, iters, col_dt, want_q=True, trace=True, changes=True)
     sT = out["sT"]
     akind = A_KIND[fmt]
     # init: absmax RTN with beta = 1; NVFP4 tensor scale fp32(amax / (6*448))
@@ -238,11 +244,23 @@ def test_iterations_brute_force(fmt, G, col_dt, M, N, wdt, iters):
             m = np.abs(Wv[i, g * G:(g + 1) * G]).max()
             want = bf.nearest_admissible(akind, (m / qmax) / sT) if m > 0 else 1.0
             assert out["trace_a"][0][i, g] == want
+    check_iterations(out, fmt, G, col_dt, Wv, iters)
+
+
+def check_iterations(out, fmt, G, col_dt, Wv, iters):
+    """Re-derive every step of every iteration by brute force from the traced state."""
+    M, N = Wv.shape
+    sT = out["sT"]
+    akind = A_KIND[fmt]
     scale_factor = sT if fmt == "nvfp4" else 1.0
+    q_prev = None
     for t in range(iters + 1):
         a_t = out["trace_a"][t]
         b_t = out["trace_b"][t]
         q_t = brute_codes(fmt, Wv, a_t * scale_factor, b_t, G)
+        if "changes" in out:  # elements whose grid value changed in iteration t
+            assert int(out["changes"][t]) == (0 if t == 0 else int(np.sum(q_t != q_prev))), t
+        q_prev = q_t
         # MSE definition: mean (W - a q b)^2
         rec = np.repeat(a_t * scale_factor, G, axis=1) * q_t * b_t[None, :]
         np.testing.assert_allclose(out["mse"][t], np.mean((Wv - rec) ** 2), rtol=1e-12)
@@ -494,7 +512,7 @@ def test_ablation_modes_brute_force(mode, fmt, G, col_dt, M, N, wdt, iters):
     """Ablation modes (DualQuant §5.3, Table 4): 'row' updates only the block scales (b stays 1),
     'col' only the column scales (a stays at its RTN value); each step re-derived by brute force, and
     the MSE never increases."""
-    Win, wdtype, Wv = tiny_matrix(M, N, wdt, seed=hash((mode, fmt, G, M, N)) & 0xFFFF)
+    Win, wdtype, Wv = tiny_matrix(M, N, wdt, seed=stable_seed(mode, fmt, G, M, N))
     out = oracle.solve(Win, wdtype, fmt, G, iters, col_dt, want_q=True, trace=True, mode=mode)
     sf = out["sT"] if fmt == "nvfp4" else 1.0
     akind = A_KIND[fmt]
@@ -519,3 +537,178 @@ def test_ablation_modes_brute_force(mode, fmt, G, col_dt, M, N, wdt, iters):
     q_T = brute_codes(fmt, Wv, out["trace_a"][iters] * sf, out["trace_b"][iters], G)
     np.testing.assert_array_equal(out["q"], q_T)
     assert np.all(out["mse"][1:] <= out["mse"][:-1] * (1 + 1e-12))
+
+
+# ---------------------------------------------------------------------------
+# Init variants: per-column L1-norm column scales (DualQuant §5.3) and warm start
+
+
+def test_exact_abs_sum_is_fsum():
+    """The exact magnitude sum, rounded once, equals math.fsum (Shewchuk's correctly rounded sum)."""
+    import math
+    rng = np.random.Generator(np.random.PCG64(7))
+    # (2^64 - 1) * 2^-85 + (2^64 - 1) * 2^-149 in six fp32 values, then 2^-149: the last unit
+    # carries through two full 64-bit words of 2^-149 units; the exact sum is 2^-21
+    carry = np.array([(2 ** 24 - 1) * 2.0 ** -45, (2 ** 24 - 1) * 2.0 ** -69, (2 ** 16 - 1) * 2.0 ** -85,
+                      (2 ** 24 - 1) * 2.0 ** -109, (2 ** 24 - 1) * 2.0 ** -133, (2 ** 16 - 1) * 2.0 ** -149,
+                      2.0 ** -149], np.float32)
+    cases = [
+        rng.standard_normal(5000).astype(np.float32),
+        (rng.standard_normal(3000) * np.exp2(rng.integers(-140, 120, 3000))).astype(np.float32),
+        np.array([1.0, 2.0 ** -53], np.float32),                 # exact tie: stays at 1
+        np.array([1.0, 2.0 ** -53, 2.0 ** -149], np.float32),    # just above the tie: rounds up
+        np.array([1.0, 2.0 ** -52, 2.0 ** -53], np.float32),     # tie with an odd last bit: rounds up to even
+        carry,
+        np.array([2.0 ** 127, 2.0 ** 127, 2.0 ** -149], np.float32),
+        np.full(70000, 2.0 ** -149, np.float32),                 # fp32 subnormals only
+        np.zeros(9, np.float32),
+    ]
+    for x in cases:
+        want = math.fsum(np.abs(x.astype(np.float64)))
+        assert oracle.exact_abs_sum(x) == want, x[:4]
+    assert oracle.exact_abs_sum(carry) == 2.0 ** -21
+    bits = bf16_bits(rng.laplace(0, 0.01, 4096).astype(np.float32))
+    v = bf16_values(bits)
+    assert oracle.exact_abs_sum(v) == math.fsum(np.abs(v))
+
+
+def l1_expected_init(Wv, fmt, G, col_dt):
+    """The L1-norm init re-derived with independent primitives: math.fsum for the exact norms,
+    enumeration of the admissible sets for every projection."""
+    import math
+    M, N = Wv.shape
+    mu = math.fsum(np.abs(Wv).ravel()) / N
+    b = np.ones(N)
+    for j in range(N):
+        c = math.fsum(np.abs(Wv[:, j]))
+        if c != 0.0 and mu != 0.0:
+            b[j] = bf.nearest_admissible(col_dt, c / mu)
+    Q = np.abs(Wv) / b[None, :]
+    amax = Q.max()
+    sT = 1.0
+    if fmt == "nvfp4" and amax > 0:
+        sT = float(np.float32(amax / 2688.0))
+    qmax = 6.0 if fmt in ("nvfp4", "mxfp4") else 7.0
+    a = np.ones((M, N // G))
+    for i in range(M):
+        for g in range(N // G):
+            m = Q[i, g * G:(g + 1) * G].max()
+            if m > 0:
+                a[i, g] = bf.nearest_admissible(A_KIND[fmt], (m / qmax) / sT) if fmt == "nvfp4" else \
+                    bf.nearest_admissible(A_KIND[fmt], m / qmax)
+    return a, b, sT
+
+
+@pytest.mark.parametrize("fmt,G,col_dt,M,N,wdt,iters", TINY[:4] + TINY[5:6])
+def test_l1_init_brute_force(fmt, G, col_dt, M, N, wdt, iters):
+    """L1-norm init re-derived independently, then every iteration by brute force; MSE non-increasing."""
+    Win, wdtype, Wv = tiny_matrix(M, N, wdt, seed=stable_seed("l1", fmt, G, M, N))
+    out = oracle.solve(Win, wdtype, fmt, G, iters, col_dt, want_q=True, trace=True, init="l1", changes=True)
+    a0, b0, sT = l1_expected_init(Wv, fmt, G, col_dt)
+    assert out["sT"] == sT
+    np.testing.assert_array_equal(out["trace_b"][0], b0)
+    np.testing.assert_array_equal(out["trace_a"][0], a0)
+    assert not np.all(b0 == 1.0)  # the outlier columns get larger column scales
+    check_iterations(out, fmt, G, col_dt, Wv, iters)
+    assert np.all(out["mse"][1:] <= out["mse"][:-1] * (1 + 1e-12))
+
+
+def equal_norm_matrix(M, N, seed):
+    """Every column a signed permutation of one vector: all column L1 norms are equal."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    v = rng.laplace(0, 0.02, M).astype(np.float32)
+    cols = [rng.permutation(v) * rng.choice(np.array([-1, 1], np.float32), M) for _ in range(N)]
+    return np.ascontiguousarray(np.stack(cols, axis=1))
+
+
+@pytest.mark.parametrize("fmt,G,col_dt", [("int4", 64, "f16"), ("mxint4", 32, "bf16"), ("nvfp4", 16, "bf16"),
+                                          ("mxfp4", 32, "bf16")])
+def test_l1_init_with_equal_column_norms_is_rtn(fmt, G, col_dt):
+    """Equal column L1 norms give b = 1, and then the L1 init is the absmax RTN init bit for bit."""
+    W = equal_norm_matrix(24, 4 * G, seed=11)
+    r = oracle.solve(W, "f32", fmt, G, 5, col_dt)
+    s = oracle.solve(W, "f32", fmt, G, 5, col_dt, init="l1")
+    for k in ("codes", "a", "b", "mse"):
+        np.testing.assert_array_equal(r[k], s[k])
+    assert r["sT"] == s["sT"]
+
+
+@pytest.mark.parametrize("fmt,G,col_dt", [("int4", 64, "f16"), ("mxint4", 32, "bf16"), ("nvfp4", 16, "bf16"),
+                                          ("mxfp4", 32, "bf16")])
+def test_l1_init_power_of_two_columns(fmt, G, col_dt):
+    """Columns of an equal-norm matrix B scaled by s_j in {1, 1, 2, 4} (mean 2): the L1 init gives
+    b = s/2 exactly and sees W D_b^-1 = 2B, so its block scales, tensor scale and codes are those of
+    the absmax RTN init of 2B."""
+    B = equal_norm_matrix(16, 4 * G, seed=12)
+    s = np.tile(np.array([1, 1, 2, 4], np.float32), G)
+    o = oracle.solve(B * s[None, :], "f32", fmt, G, 0, col_dt, init="l1")
+    r = oracle.solve(B * np.float32(2), "f32", fmt, G, 0, col_dt)
+    np.testing.assert_array_equal(o["b"], s / 2)
+    np.testing.assert_array_equal(o["a"], r["a"])
+    np.testing.assert_array_equal(o["codes"], r["codes"])
+    assert o["sT"] == r["sT"]
+
+
+@pytest.mark.parametrize("fmt,G,col_dt", [("int4", 64, "f16"), ("nvfp4", 16, "bf16")])
+def test_l1_init_zero_columns_and_power_of_two_scaling(fmt, G, col_dt):
+    """An all-zero column keeps b = 1 (zero-slice rule); an all-zero W gives scale 1 everywhere;
+    W -> 4W leaves b and the codes unchanged under the L1 init."""
+    Win, _, _ = tiny_matrix(12, 4 * G, "f32", seed=13)
+    Win = Win.copy()
+    Win[:, 5] = 0.0
+    o = oracle.solve(Win, "f32", fmt, G, 4, col_dt, init="l1", want_q=True)
+    assert o["b"][5] == 1.0 and np.all(o["q"][:, 5] == 0)
+    z = oracle.solve(np.zeros((4, 2 * G), np.float32), "f32", fmt, G, 2, col_dt, init="l1")
+    assert z["sT"] == 1.0 and np.all(z["a"] == 1.0) and np.all(z["b"] == 1.0) and np.all(z["mse"] == 0)
+    o4 = oracle.solve(Win * np.float32(4), "f32", fmt, G, 4, col_dt, init="l1", want_q=True)
+    np.testing.assert_array_equal(o["b"], o4["b"])
+    np.testing.assert_array_equal(o["q"], o4["q"])
+
+
+@pytest.mark.parametrize("init", ["rtn", "l1"])
+@pytest.mark.parametrize("fmt,G,col_dt", [("int4", 64, "f16"), ("mxint4", 32, "bf16"), ("nvfp4", 16, "bf16"),
+                                          ("mxfp4", 32, "bf16")])
+def test_warm_start_continues_the_iteration(init, fmt, G, col_dt):
+    """The iterate is the pair of scales (codes are a function of them), so T1 iterations followed by a
+    warm start of T2 more equal T1 + T2 iterations: every output, and the MSE sequence from T1 on."""
+    wl, (Win, wdt) = small_workload("nvfp4_g16_gateup_14336x4096", 40, 4 * 64, 17)
+    full = oracle.solve(Win, wdt, fmt, G, 7, col_dt, init=init, changes=True)
+    first = oracle.solve(Win, wdt, fmt, G, 3, col_dt, init=init)
+    warm = oracle.solve(Win, wdt, fmt, G, 4, col_dt, init="given", a0=first["a"], b0=first["b"],
+                        sT0=first["sT"], changes=True)
+    for k in ("codes", "a", "b"):
+        np.testing.assert_array_equal(full[k], warm[k])
+    assert full["sT"] == warm["sT"]
+    np.testing.assert_array_equal(full["mse"][3:], warm["mse"])
+    np.testing.assert_array_equal(full["changes"][4:], warm["changes"][1:])
+
+
+@pytest.mark.parametrize("fmt,G,col_dt", [("int4", 64, "f16"), ("mxint4", 32, "bf16"), ("nvfp4", 16, "bf16")])
+def test_warm_start_rejects_inadmissible_scales(fmt, G, col_dt):
+    """A warm start takes only admissible scales: elements of F_a and F_b, a positive fp32 s_T."""
+    wl, (Win, wdt) = small_workload("nvfp4_g16_gateup_14336x4096", 8, 2 * 64, 19)
+    r = oracle.rtn(Win, wdt, fmt, G, col_dt)
+    ok = dict(a0=r["a"], b0=r["b"], sT0=r["sT"])
+    oracle.solve(Win, wdt, fmt, G, 1, col_dt, init="given", **ok)
+    bad_a = {"int4": 1.0 + 2.0 ** -12, "mxint4": 0.75, "nvfp4": 1.0625}[fmt]
+    cases = [dict(ok, a0=np.where(np.arange(r["a"].size).reshape(r["a"].shape) == 3, bad_a, r["a"])),
+             dict(ok, a0=-r["a"]), dict(ok, a0=r["a"] * 0.0),
+             dict(ok, b0=np.where(np.arange(r["b"].size) == 2, 1.0 + 2.0 ** -14, r["b"])),
+             dict(ok, b0=np.full_like(r["b"], np.nan))]
+    if fmt == "nvfp4":
+        cases += [dict(ok, sT0=0.0), dict(ok, sT0=0.1), dict(ok, sT0=float("inf"))]
+    for c in cases:
+        with pytest.raises(oracle.OracleError):
+            oracle.solve(Win, wdt, fmt, G, 1, col_dt, init="given", **c)
+
+
+def test_changes_vanish_at_a_fixed_point():
+    """Once the iterate stops moving no code changes: the count is 0 from then on."""
+    wl, (Win, wdt) = small_workload("mxint4_g32_downproj_4096x14336", 16, 128, 23)
+    o = oracle.solve(Win, wdt, "mxint4", 32, 60, "bf16", trace=True, changes=True)
+    still = [t for t in range(1, 61) if np.array_equal(o["trace_a"][t], o["trace_a"][t - 1])
+             and np.array_equal(o["trace_b"][t], o["trace_b"][t - 1])]
+    assert still, "no fixed point reached"
+    for t in still:
+        assert o["changes"][t] == 0
+    assert o["changes"][0] == 0 and o["changes"][1] > 0
