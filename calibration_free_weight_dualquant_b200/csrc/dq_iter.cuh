@@ -529,6 +529,49 @@ __device__ __forceinline__ void row_pair(const Problem& p, const f2 wx[4], float
   }
 }
 
+// Final pass: the 8 codes of a lane's row packed into one word (even column in
+// the low nibble; zero is always the 0x0 nibble).
+template <int FMT>
+__device__ __forceinline__ uint32_t pack8(const f2 q2[4]) {
+  uint32_t r = 0u;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float lo = __fadd_rn(lo_of(q2[i]), 0.f), hi = __fadd_rn(hi_of(q2[i]), 0.f);  // -0 becomes +0
+    uint32_t byte;
+    if (fmt_e2m1(FMT)) {
+      byte = cvt_e2m1x2(hi, lo);  // grid values convert exactly
+    } else {  // q + 1.5 * 2^23 holds the integer q in its low mantissa bits (two's complement mod 16)
+      byte = (__float_as_uint(lo + 12582912.f) & 15u) | ((__float_as_uint(hi + 12582912.f) & 15u) << 4);
+    }
+    r |= byte << (8 * i);
+  }
+  return r;
+}
+
+// Final pass for two rows of a lane (x = row rx, y = row rx + kConsumerWarps,
+// possibly absent): codes of the final iterate, written packed, and the
+// residuals of that iterate for its MSE.
+template <int FMT>
+__device__ __forceinline__ void final_pair(const Problem& p, const f2 wx[4], float ax, int64_t rx, const f2 wy[4],
+                                           float ay, bool has_y, bool active, int64_t col, ColState& cs, float sT,
+                                           double sTd, f2 rscale2, unsigned* s_cnt) {
+  const bool actx = active, acty = active && has_y;
+  f2 ux[4], uy[4], qx[4], qy[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const f2 cbi = col_ld(cs.tcb, i, cs.lane);
+    ux[i] = mul2(wx[i], cbi);
+    uy[i] = mul2(wy[i], cbi);
+  }
+  req_pair<FMT>(wx, ux, ax, actx, wy, uy, ay, acty, cs, sT, sTd, qx, qy, s_cnt);
+  float n, d;  // block sums: not needed here
+  row_sums<FMT>(wx, qx, ax, cs, sT, rscale2, n, d, cs.res2);
+  row_sums<FMT>(wy, qy, ay, cs, sT, rscale2, n, d, cs.res2);
+  uint32_t* codes = reinterpret_cast<uint32_t*>(p.codes);
+  if (actx) codes[(rx * p.N + col) >> 3] = pack8<FMT>(qx);
+  if (acty) codes[((rx + kConsumerWarps) * p.N + col) >> 3] = pack8<FMT>(qy);
+}
+
 // fp32 runs into the warp's fp64 accumulators (layout [warp][c][lane], then
 // [warp][lane] for the residuals).
 __device__ __forceinline__ void flush_runs(ColState& cs, double2* acc, double* racc, int warp, int lane,
@@ -549,7 +592,10 @@ __device__ __forceinline__ void flush_runs(ColState& cs, double2* acc, double* r
   cs.res2 = 0ull;
 }
 
-template <int FMT, int WDT>
+// One pass over W.  FIN = false: BCD iteration t (writes mse[t - 1], the MSE of
+// the incoming iterate).  FIN = true: the final pass after T iterations, called
+// with t = T + 1: the codes of the final iterate, packed, and mse[T].
+template <int FMT, int WDT, bool FIN>
 __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t, const __grid_constant__ CUtensorMap wmap) {
   if (p.hdr->flags & kFlagNonFinite) return;
   constexpr int ES = WDT == DT_F32 ? 4 : 2;
@@ -722,8 +768,12 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t, cons
 #pragma unroll
           for (int i = 0; i < 4; ++i) wb[i] = 0ull;  // absent row: zeros contribute nothing
         }
-        row_pair<FMT>(p, wa, aa, aidx, wb, ab, aidx + kConsumerWarps * p.nb, has_b, active, leader, lpb, cs, sT, isT,
-                      sTd, rscale2, s_cnt);
+        if (FIN) {
+          final_pair<FMT>(p, wa, aa, ra, wb, ab, has_b, active, col, cs, sT, sTd, rscale2, s_cnt);
+        } else {
+          row_pair<FMT>(p, wa, aa, aidx, wb, ab, aidx + kConsumerWarps * p.nb, has_b, active, leader, lpb, cs, sT,
+                        isT, sTd, rscale2, s_cnt);
+        }
         run += has_b ? 2 : 1;
       }
       if (run >= kRun) {
@@ -732,6 +782,10 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t, cons
       }
     }
     flush_runs(cs, acc, racc, warp, lane, active);
+    if (FIN) {  // no column update in the final pass
+      u = (s + 1) * p.M;
+      continue;
+    }
 
     // CTA reduction of the column sums over the consumer warps, fixed order.
     // Thread t sums entry (c, l) = (t / 32, t % 32), i.e. column 8 (t % 32) + t / 32.
@@ -810,7 +864,10 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t, cons
   }
 
   // MSE of the incoming iterate: per-thread residual sums, CTA tree, then the
-  // CTA-ordered total (the residual accumulators are not reused above).
+  // CTA-ordered total (the residual accumulators are not reused above).  The
+  // tree reuses the column accumulators: in the final pass no barrier follows
+  // the last flush into them, so wait for every consumer warp here.
+  if (FIN) consumer_sync(kConsumers);
   double* mred = reinterpret_cast<double*>(acc);
   mred[threadIdx.x] = racc[threadIdx.x];
   consumer_sync(kConsumers);

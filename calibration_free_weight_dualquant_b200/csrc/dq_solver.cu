@@ -10,22 +10,14 @@
 //     b <- Proj_Fb(sum W a q' / sum (a q')^2) per column, codes fixed
 //   scale 1 for an all-zero code slice; codes are a function of (W, a, b).
 //
-// HBM layout and schedule.  One pass over W per iteration: kernel k_iter
-// fuses, for every element, the requantization of the current iterate, the
-// block sums (reduced over the G/8 lanes of a block with xor shuffles, which
-// give every lane the bit-identical total), the block update, the
-// requantization with the new block scale and the column sums.  Columns are
-// cut into strips of TS <= 256 columns; the (strip, row) pairs are laid out
-// strip-major and split evenly into P contiguous ranges, one per CTA
-// (P = 2 CTAs per SM), so every CTA streams the same number of rows.  A CTA
-// keeps its columns' sums in registers, reduces them over its 8 warps in
-// shared memory and writes one fp64 partial per (CTA, strip) it touched; the
-// last CTA to finish a strip (atomic ticket, no waiting) sums the partials of
-// that strip in CTA order -- a fixed order, so the result is deterministic --
-// and writes the new column scales.  The reconstruction MSE of the iterate
-// entering iteration t is accumulated from the residuals W - a q b of the
-// requantized incoming iterate (fp32 runs into fp64), per CTA, then summed in
-// CTA order by the last CTA.
+// Launches per solve: k_stats (non-finite check, max |W|), k_init (scales of
+// the initial iterate), T x k_iter (one BCD iteration each, one read of W), and
+// k_iter in its final mode (codes of the final iterate and the last MSE, one
+// more read of W).  k_iter (dq_iter.cuh) runs one persistent CTA per SM over
+// contiguous ranges of strip-major (strip, row) units, so every CTA streams
+// the same number of rows; the column totals and the MSE are summed in CTA
+// order by the last CTA to arrive (an atomic ticket, never a wait), so every
+// result is deterministic.
 #include <cudaTypedefs.h>  // PFN_cuTensorMapEncodeTiled
 
 #include <climits>
@@ -116,75 +108,6 @@ __global__ void __launch_bounds__(kThreads) k_init(Problem p) {
 }
 
 // ---------------------------------------------------------------------------
-// Final pass: codes of the final iterate, nibble packing, direct MSE.
-template <int FMT, int WDT>
-__global__ void __launch_bounds__(kThreads) k_final(Problem p, int T) {
-  if (p.hdr->flags & kFlagNonFinite) return;
-  __shared__ double mred[kThreads];
-  __shared__ int s_last;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const float sT = p.hdr->sT;
-  const double sTd = (double)sT;
-  const float isT = FMT == FMT_NVFP4 ? 1.f / sT : 1.f;
-  const bool sT_ok = FMT != FMT_NVFP4 || in_range(isT);
-  const int64_t k = blockIdx.x;
-  const int64_t u_begin = range_begin(k, p.P, p.L), u_end = range_begin(k + 1, p.P, p.L);
-  double acc = 0.0;
-  for (int64_t u = u_begin; u < u_end;) {
-    const int64_t s = u / p.M;
-    const int64_t r0 = u - s * p.M;
-    const int64_t r1 = min(p.M, r0 + (u_end - u));
-    const int64_t c0 = s * p.TS;
-    const int width = (int)min((int64_t)p.TS, p.N - c0);
-    const bool active = lane * 8 < width;
-    const int64_t col = c0 + lane * 8;
-    if (active) {
-      float bj[8], cb[8];
-      bool col_ok = sT_ok;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        bj[c] = b_decode(p.b_store, p.col_dt, col + c);
-        cb[c] = __frcp_rn(bj[c]) * isT;
-        col_ok = col_ok && in_range(cb[c]);
-      }
-      for (int64_t r = r0 + warp; r < r1; r += kWarps) {
-        float w[8];
-        load8<WDT>(p.W, r * p.N + col, w);
-        const float a = a_decode<FMT>(p.a_store, r * p.nb + col / p.G);
-        const float ia = __frcp_rn(a);
-        const bool ok = col_ok && in_range(ia);
-        const double aval = FMT == FMT_NVFP4 ? sTd * (double)a : (double)a;
-        uint32_t packed = 0;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const float q = quant<FMT>(w[c], w[c] * cb[c], ia, ok, a, bj[c], sTd);
-          packed |= nibble<FMT>(q) << (4 * c);
-          const double res = (double)w[c] - aval * (double)q * (double)bj[c];
-          acc = fma(res, res, acc);
-        }
-        reinterpret_cast<uint32_t*>(p.codes)[(r * p.N + col) / 8] = packed;
-      }
-    }
-    u = (s + 1) * p.M;
-  }
-  mred[threadIdx.x] = acc;
-  __syncthreads();
-  for (int o = kThreads / 2; o > 0; o >>= 1) {
-    if (threadIdx.x < o) mred[threadIdx.x] += mred[threadIdx.x + o];
-    __syncthreads();
-  }
-  if (threadIdx.x == 0) p.cta_part[k] = mred[0];
-  if (arrive_last(&p.hdr->cta_counter, (unsigned)p.P, &s_last)) {
-    if (threadIdx.x == 0) {
-      double tot = 0.0;
-      for (int64_t kk = 0; kk < p.P; ++kk) tot += __ldcg(&p.cta_part[kk]);
-      p.mse[T] = tot / ((double)p.M * (double)p.N);
-      p.hdr->cta_counter = 0u;
-    }
-  }
-}
-
-// ---------------------------------------------------------------------------
 // Host-side launch of the whole solve on one stream.
 
 // The driver's tensor-map encoder, looked up once through the runtime.
@@ -226,7 +149,9 @@ template <int FMT, int WDT>
 static cudaError_t run_typed(const Problem& p, int iters, int stats_ctas, cudaStream_t st) {
   constexpr int ES = WDT == DT_F32 ? 4 : 2;
   const size_t smem = iter_smem_bytes(ES);
-  cudaError_t e = cudaFuncSetAttribute(k_iter<FMT, WDT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(k_iter<FMT, WDT, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(k_iter<FMT, WDT, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   CUtensorMap wmap;
   Problem pi = p;
@@ -236,8 +161,8 @@ static cudaError_t run_typed(const Problem& p, int iters, int stats_ctas, cudaSt
   pf.segmax = p.segmax_final;
   k_stats<WDT><<<stats_ctas, kThreads, 0, st>>>(pf);
   k_init<FMT, WDT><<<stats_ctas, kThreads, 0, st>>>(pf);
-  for (int t = 1; t <= iters; ++t) k_iter<FMT, WDT><<<(unsigned)p.P, kIterThreads, smem, st>>>(pi, t, wmap);
-  k_final<FMT, WDT><<<(unsigned)pf.P, kThreads, 0, st>>>(pf, iters);
+  for (int t = 1; t <= iters; ++t) k_iter<FMT, WDT, false><<<(unsigned)p.P, kIterThreads, smem, st>>>(pi, t, wmap);
+  k_iter<FMT, WDT, true><<<(unsigned)p.P, kIterThreads, smem, st>>>(pi, iters + 1, wmap);
   return cudaGetLastError();
 }
 
