@@ -45,6 +45,10 @@ class _Outputs(ctypes.Structure):
                 ("col_scales", ctypes.c_void_p), ("mse", ctypes.c_void_p)]
 
 
+class _Options(ctypes.Structure):
+    _fields_ = [("mode", ctypes.c_int), ("init", ctypes.c_int), ("code_changes", ctypes.c_void_p)]
+
+
 class _Matrix(ctypes.Structure):
     _fields_ = [("W", ctypes.c_void_p), ("w_dtype", ctypes.c_int), ("rows", ctypes.c_int64),
                 ("cols", ctypes.c_int64), ("out", _Outputs)]
@@ -70,6 +74,11 @@ def load_library():
     lib.dq_solve.restype = I
     lib.dq_solve_mode.argtypes = [P, I, I64, I64, I, I, I, I, I, ctypes.POINTER(_Outputs), P, SZ, P]
     lib.dq_solve_mode.restype = I
+    lib.dq_workspace_bytes_ex.argtypes = [I64, I64, I, I, ctypes.POINTER(_Options)]
+    lib.dq_workspace_bytes_ex.restype = SZ
+    lib.dq_solve_ex.argtypes = [P, I, I64, I64, I, I, I, I, ctypes.POINTER(_Options), ctypes.POINTER(_Outputs), P,
+                                SZ, P]
+    lib.dq_solve_ex.restype = I
     lib.dq_sync_status.argtypes = [P, P]
     lib.dq_sync_status.restype = I
     lib.dq_host_workspace_bytes.argtypes = [I64, I64, I, I, I, I]
@@ -133,16 +142,24 @@ def _stream_ptr(stream) -> int:
 
 
 MODES = {"dual": 0, "row": 1, "col": 2}
+INITS = {"rtn": 0, "l1": 1, "given": 2}
 
 
 def dq_solve(W: torch.Tensor, fmt, group: Optional[int] = None, iters: int = 0, col_dtype: Optional[str] = None,
              out: Optional[dict] = None, workspace: Optional[torch.Tensor] = None, stream=None,
-             check: bool = True, mode: str = "dual") -> dict:
+             check: bool = True, mode: str = "dual", init: str = "rtn", init_scales: Optional[dict] = None,
+             changes: bool = False) -> dict:
     """Enqueue dq_solve on a CUDA tensor W [rows, cols]; returns the output tensors.
 
     ``check`` waits for the stream and raises on a device-reported status
-    (non-finite W).  Pass preallocated ``out`` / ``workspace`` to avoid
-    allocations (e.g. when timing)."""
+    (non-finite W, inadmissible warm-start scales).  Pass preallocated ``out`` /
+    ``workspace`` to avoid allocations (e.g. when timing).  ``mode``: "dual",
+    "row" or "col" (dq_mode).  ``init``: "rtn", "l1" or "given" (dq_init); with
+    "given" the initial scales are ``init_scales`` ({"block_scales",
+    "col_scales", "tensor_scale"} in storage format, e.g. a previous call's
+    outputs), copied into ``out`` first, or whatever ``out`` already holds.
+    ``changes`` adds out["code_changes"] (int64 [iters+1], changed codes per
+    iteration)."""
     lib = load_library()
     if not W.is_cuda:
         raise DQError(1, "dq_solve: W must be a CUDA tensor (use solve() for host tensors)")
@@ -154,14 +171,30 @@ def dq_solve(W: torch.Tensor, fmt, group: Optional[int] = None, iters: int = 0, 
         raise DQError(1, "dq_solve: W must be contiguous f32/bf16/f16")
     if out is None:
         out = alloc_outputs(rows, cols, f, g, cd, iters, W.device)
+    extended = init != "rtn" or changes
+    opts = None
+    if extended:
+        if init == "given" and init_scales is not None:
+            for k in ("block_scales", "col_scales", "tensor_scale"):
+                if k in init_scales:
+                    out[k].view(-1).copy_(init_scales[k].reshape(-1))
+        if changes:
+            out["code_changes"] = torch.empty(iters + 1, dtype=torch.int64, device=W.device)
+        opts = _Options(MODES[mode], INITS[init], out["code_changes"].data_ptr() if changes else None)
     if workspace is None:
-        nbytes = lib.dq_workspace_bytes(rows, cols, int(f), g)
+        if extended:
+            nbytes = lib.dq_workspace_bytes_ex(rows, cols, int(f), g, ctypes.byref(opts))
+        else:
+            nbytes = lib.dq_workspace_bytes(rows, cols, int(f), g)
         if nbytes == 0:
             raise DQError(1, "dq_workspace_bytes")
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
     o = _outputs_struct(out)
     cdt = 2 if cd == "f16" else 1
-    if mode == "dual":
+    if extended:
+        st = lib.dq_solve_ex(W.data_ptr(), _DTYPES[W.dtype], rows, cols, int(f), g, iters, cdt, ctypes.byref(opts),
+                             ctypes.byref(o), workspace.data_ptr(), workspace.numel(), _stream_ptr(stream))
+    elif mode == "dual":
         st = lib.dq_solve(W.data_ptr(), _DTYPES[W.dtype], rows, cols, int(f), g, iters, cdt, ctypes.byref(o),
                           workspace.data_ptr(), workspace.numel(), _stream_ptr(stream))
     else:

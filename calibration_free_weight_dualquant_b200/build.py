@@ -16,7 +16,7 @@ INCLUDE = os.path.join(ROOT, "include")
 OUT_DIR = os.path.join(PKG, "lib")
 LIB = os.path.join(OUT_DIR, "libdq.so")
 SOURCES = ["dq_capi.cu", "dq_solver.cu", "dq_static.cu", "dq_act.cu"]
-HEADERS = ["dq_device.cuh", "dq_fast.cuh", "dq_internal.h", "dq_iter.cuh"]
+HEADERS = ["dq_device.cuh", "dq_fast.cuh", "dq_init.cuh", "dq_internal.h", "dq_iter.cuh"]
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "--expt-relaxed-constexpr",

@@ -16,6 +16,8 @@ struct Plan {
   int TS, n_strips, P, segmax, P_final, segmax_final, nb;
   int64_t L;
   size_t off_counters, off_col_part, off_cta_part, total;
+  size_t l1_zero_bytes;  // L1 init: digit counters to zero (start of the col_part region)
+  size_t off_l1_tot, off_l1_norm;
 };
 
 // Argument checks that do not touch memory.  Returns DQ_OK or an error code.
@@ -40,7 +42,7 @@ int device_sms(int* sms) {
 }
 
 // Schedule and workspace layout for the current device.
-int make_plan(int64_t M, int64_t N, int group, Plan* pl) {
+int make_plan(int64_t M, int64_t N, int group, int init, Plan* pl) {
   int sms = 0;
   int st = device_sms(&sms);
   if (st != DQ_OK) return st;
@@ -60,7 +62,17 @@ int make_plan(int64_t M, int64_t N, int group, Plan* pl) {
   pl->off_counters = off;
   off += align_up(sizeof(unsigned) * (size_t)pl->n_strips);
   pl->off_col_part = off;
-  off += align_up(sizeof(double2) * (size_t)pl->P * (size_t)pl->segmax * (size_t)pl->TS);
+  // the L1-init scratch overlays the column partials (the init kernels run
+  // before the first iteration): per-column digits, the total's digits, norms;
+  // only the L1 init asks for it
+  const size_t dig_bytes = align_up(sizeof(unsigned long long) * dq::kXDigits * (size_t)N);
+  const size_t tot_bytes = align_up(sizeof(unsigned long long) * dq::kXDigits);
+  pl->off_l1_tot = off + dig_bytes;
+  pl->off_l1_norm = pl->off_l1_tot + tot_bytes;
+  pl->l1_zero_bytes = dig_bytes + tot_bytes;
+  const size_t l1_bytes = dig_bytes + tot_bytes + align_up(sizeof(double) * (size_t)N);
+  const size_t part_bytes = align_up(sizeof(double2) * (size_t)pl->P * (size_t)pl->segmax * (size_t)pl->TS);
+  off += (init == DQ_INIT_L1 && l1_bytes > part_bytes) ? l1_bytes : part_bytes;
   pl->off_cta_part = off;
   off += align_up(sizeof(double) * (size_t)(pl->P > pl->P_final ? pl->P : pl->P_final));
   pl->total = off;
@@ -85,10 +97,15 @@ namespace dq {
 
 int solve_impl(const void* W, int w_dtype, int64_t rows, int64_t cols, int format, int group, int iters,
                int col_dtype, const dq_outputs* out, void* workspace, size_t workspace_bytes, cudaStream_t stream,
-               int mode) {
+               const dq_options* opt) {
   int st = check_shape(rows, cols, format, group);
   if (st != DQ_OK) return st;
+  const int mode = opt ? opt->mode : DQ_MODE_DUAL;
+  const int init = opt ? opt->init : DQ_INIT_RTN;
+  unsigned long long* changes = opt ? reinterpret_cast<unsigned long long*>(opt->code_changes) : nullptr;
   if (mode < DQ_MODE_DUAL || mode > DQ_MODE_COL) return DQ_EINVAL;
+  if (init < DQ_INIT_RTN || init > DQ_INIT_GIVEN) return DQ_EINVAL;
+  if (changes != nullptr) return DQ_EUNSUPPORTED;
   if (w_dtype < DQ_F32 || w_dtype > DQ_F16) return DQ_EINVAL;
   if (col_dtype != DQ_F16 && col_dtype != DQ_BF16) return DQ_EUNSUPPORTED;
   if (iters < 0) return DQ_EINVAL;
@@ -97,7 +114,7 @@ int solve_impl(const void* W, int w_dtype, int64_t rows, int64_t cols, int forma
   if (st != DQ_OK) return st;
   if (!workspace || !aligned(workspace, kAlign)) return DQ_EINVAL;
   Plan pl;
-  st = make_plan(rows, cols, group, &pl);
+  st = make_plan(rows, cols, group, init, &pl);
   if (st != DQ_OK) return st;
   if (workspace_bytes < pl.total) return DQ_EWORKSPACE;
 
@@ -120,6 +137,11 @@ int solve_impl(const void* W, int w_dtype, int64_t rows, int64_t cols, int forma
   p.segmax_final = pl.segmax_final;
   p.L = pl.L;
   p.mode = mode;
+  p.init = init;
+  p.changes = changes;
+  p.l1_dig = reinterpret_cast<unsigned long long*>(ws + pl.off_col_part);
+  p.l1_tot = reinterpret_cast<unsigned long long*>(ws + pl.off_l1_tot);
+  p.l1_norm = reinterpret_cast<double*>(ws + pl.off_l1_norm);
   p.codes = out->codes;
   p.a_store = out->block_scales;
   p.b_store = out->col_scales;
@@ -132,6 +154,8 @@ int solve_impl(const void* W, int w_dtype, int64_t rows, int64_t cols, int forma
 
   // header and arrival counters start at zero; the partial buffers need no init
   if (cudaMemsetAsync(ws, 0, pl.off_col_part, stream) != cudaSuccess) return DQ_ECUDA;
+  if (init == DQ_INIT_L1 && cudaMemsetAsync(ws + pl.off_col_part, 0, pl.l1_zero_bytes, stream) != cudaSuccess)
+    return DQ_ECUDA;
   if (dq::launch_solve(p, iters, pl.P_final, stream) != cudaSuccess) return DQ_ECUDA;
   return DQ_OK;
 }
@@ -139,7 +163,10 @@ int solve_impl(const void* W, int w_dtype, int64_t rows, int64_t cols, int forma
 // Device-side status of the solve that used `ws`, as a dq_status.
 __global__ void k_ws_status(const WsHeader* ws, int* status) {
   const unsigned f = ws->flags;
-  *status = (f & kFlagNonFinite) ? DQ_ENONFINITE : ((f & kFlagTimeout) ? DQ_ECUDA : DQ_OK);
+  *status = (f & kFlagNonFinite) ? DQ_ENONFINITE
+           : (f & kFlagBadInit)  ? DQ_EINVAL
+           : (f & kFlagTimeout)  ? DQ_ECUDA
+                                 : DQ_OK;
 }
 
 }  // namespace dq
@@ -149,7 +176,14 @@ extern "C" {
 size_t dq_workspace_bytes(int64_t rows, int64_t cols, int format, int group) {
   if (check_shape(rows, cols, format, group) != DQ_OK) return 0;
   Plan pl;
-  if (make_plan(rows, cols, group, &pl) != DQ_OK) return 0;
+  if (make_plan(rows, cols, group, DQ_INIT_RTN, &pl) != DQ_OK) return 0;
+  return pl.total;
+}
+
+size_t dq_workspace_bytes_ex(int64_t rows, int64_t cols, int format, int group, const dq_options* options) {
+  if (check_shape(rows, cols, format, group) != DQ_OK) return 0;
+  Plan pl;
+  if (make_plan(rows, cols, group, options ? options->init : DQ_INIT_RTN, &pl) != DQ_OK) return 0;
   return pl.total;
 }
 
@@ -162,8 +196,18 @@ int dq_solve(const void* W, int w_dtype, int64_t rows, int64_t cols, int format,
 int dq_solve_mode(const void* W, int w_dtype, int64_t rows, int64_t cols, int format, int group, int iters,
                   int col_dtype, int mode, const dq_outputs* out, void* workspace, size_t workspace_bytes,
                   void* stream) {
+  dq_options opt;
+  std::memset(&opt, 0, sizeof(opt));
+  opt.mode = mode;
   return dq::solve_impl(W, w_dtype, rows, cols, format, group, iters, col_dtype, out, workspace, workspace_bytes,
-                        static_cast<cudaStream_t>(stream), mode);
+                        static_cast<cudaStream_t>(stream), &opt);
+}
+
+int dq_solve_ex(const void* W, int w_dtype, int64_t rows, int64_t cols, int format, int group, int iters,
+                int col_dtype, const dq_options* options, const dq_outputs* out, void* workspace,
+                size_t workspace_bytes, void* stream) {
+  return dq::solve_impl(W, w_dtype, rows, cols, format, group, iters, col_dtype, out, workspace, workspace_bytes,
+                        static_cast<cudaStream_t>(stream), options);
 }
 
 int dq_rtn(const void* W, int w_dtype, int64_t rows, int64_t cols, int format, int group, int col_dtype,
@@ -178,6 +222,7 @@ int dq_sync_status(const void* workspace, void* stream) {
   unsigned flags = 0;
   if (cudaMemcpy(&flags, workspace, sizeof(flags), cudaMemcpyDeviceToHost) != cudaSuccess) return DQ_ECUDA;
   if (flags & dq::kFlagNonFinite) return DQ_ENONFINITE;
+  if (flags & dq::kFlagBadInit) return DQ_EINVAL;
   return (flags & dq::kFlagTimeout) ? DQ_ECUDA : DQ_OK;
 }
 
@@ -277,7 +322,7 @@ int dq_solve_batched(const dq_matrix* mats, int count, int format, int group, in
     if (st == DQ_OK) st = check_outputs(&m.out, format, col_dtype);
     if (st == DQ_OK) {
       Plan pl;
-      st = make_plan(m.rows, m.cols, group, &pl);
+      st = make_plan(m.rows, m.cols, group, DQ_INIT_RTN, &pl);
       if (st == DQ_OK && workspace_bytes < pl.total) st = DQ_EWORKSPACE;
     }
     if (st != DQ_OK) {

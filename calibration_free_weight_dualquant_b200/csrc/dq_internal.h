@@ -14,12 +14,17 @@ constexpr int kStripMax = 256;  // columns per strip (8 per lane, 32 lanes)
 constexpr int kCtasPerSm = 1;        // per-iteration pass: one 544-thread CTA per SM
 constexpr int kFinalCtasPerSm = 4;   // one-time passes
 constexpr int64_t kMinRowsPerCta = 64;
+// 32-bit digits of an exact magnitude sum in units of 2^-149 (L1 init): one
+// value reaches bit 277, a sum of up to 2^31 values bit 308
+constexpr int kXDigits = 10;
 constexpr unsigned kFlagNonFinite = 1u;
 constexpr unsigned kFlagTimeout = 2u;  // a bounded pipeline wait gave up (results invalid)
+constexpr unsigned kFlagBadInit = 4u;  // a warm start was given an inadmissible scale
+constexpr unsigned kFlagAbort = kFlagNonFinite | kFlagBadInit;  // later kernels do nothing
 
 // Device workspace header (first 256 bytes of the workspace).
 struct WsHeader {
-  unsigned flags;        // kFlagNonFinite
+  unsigned flags;        // kFlagNonFinite, kFlagTimeout, kFlagBadInit
   unsigned amax_bits;    // max |W| as fp32 bits
   unsigned cta_counter;  // arrival ticket for CTA-ordered totals
   float sT;              // NVFP4 tensor scale (1 otherwise)
@@ -28,6 +33,7 @@ struct WsHeader {
   unsigned long long n_quant_exact;  // lane-rows (8 elements) decided on the exact path
   unsigned long long n_block_exact;  // block updates taken in fp64
   unsigned long long n_col_exact;    // column updates recomputed exactly over all rows
+  unsigned long long amax_scaled;    // L1 init, NVFP4: max |W_ij| / b_j as the bits of a double
 };
 
 // Everything a kernel needs, passed by value.
@@ -53,15 +59,22 @@ struct Problem {
   double2* col_part;        // [P * segmax][TS] (sum W a q, sum (a q)^2)
   double* cta_part;         // [max(P, P_final)]
   int use_tmap;             // W streamed by 2-D tensor copies (else one bulk copy per row)
-  int mode;                 // DQ_MODE_DUAL, DQ_MODE_ROW (b stays 1) or DQ_MODE_COL (a stays at RTN)
+  int mode;                 // DQ_MODE_DUAL, DQ_MODE_ROW (b keeps its initial value) or DQ_MODE_COL
+  int init;                 // DQ_INIT_RTN, DQ_INIT_L1 or DQ_INIT_GIVEN
+  // L1 init scratch (overlays col_part, which the init kernels do not use)
+  unsigned long long* l1_dig;   // [N][10] digit counters of the column magnitude sums (zeroed)
+  unsigned long long* l1_tot;   // [10] digit counters of the total (zeroed)
+  double* l1_norm;              // [N] column L1 norms rounded to fp64
+  unsigned long long* changes;  // NULL, or [iters + 1] changed-code counts
 };
 
 cudaError_t launch_solve(const Problem& p, int iters, int stats_ctas, cudaStream_t st);
 
 // Host-side validation, workspace layout and enqueue of a whole solve (the body
 // of dq_solve; `workspace` is a device address of at least the planned size).
+// `opt` NULL means the defaults (dual mode, RTN init, no change counts).
 int solve_impl(const void* W, int w_dtype, int64_t rows, int64_t cols, int format, int group, int iters,
                int col_dtype, const dq_outputs* out, void* workspace, size_t workspace_bytes,
-               cudaStream_t stream, int mode = DQ_MODE_DUAL);
+               cudaStream_t stream, const dq_options* opt = nullptr);
 
 }  // namespace dq

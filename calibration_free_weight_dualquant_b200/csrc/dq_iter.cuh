@@ -415,17 +415,25 @@ __device__ __forceinline__ void smem_row(const unsigned char* src, f2 w2[4]) {
 }
 
 // Block sums, residuals of the incoming iterate, for one row of one lane.
+// The residual W - a q b is taken with the product q b a exact inside fmas:
+// q b is exact in fp32, and so is a for INT4/MX; the NVFP4 factor a = e s_T is
+// split as hi + lo (hi = fl(e s_T), lo its exact rounding error), so the only
+// rounding is that of the (small) residual itself.
 template <int FMT>
 __device__ __forceinline__ void row_sums(const f2 w2[4], const f2 q2[4], float aold, const ColState& cs, float sT,
                                          f2 rscale2, float& num, float& den, f2& res2) {
-  const f2 na2 = splat(FMT == FMT_NVFP4 ? -(aold * sT) : -aold);
+  const float ahi = FMT == FMT_NVFP4 ? aold * sT : aold;
+  const f2 na2 = splat(-ahi);
+  const f2 nlo2 = splat(FMT == FMT_NVFP4 ? -fmaf(aold, sT, -ahi) : 0.f);
   f2 num2 = 0ull, den2 = 0ull;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const f2 pq = mul2(q2[i], col_ld(cs.tb, i, cs.lane));
     num2 = fma2(w2[i], pq, num2);
     den2 = fma2(pq, pq, den2);
-    const f2 e = mul2(fma2(pq, na2, w2[i]), rscale2);  // residual times a power of two (range)
+    f2 r = fma2(pq, na2, w2[i]);
+    if (FMT == FMT_NVFP4) r = fma2(pq, nlo2, r);
+    const f2 e = mul2(r, rscale2);  // residual times a power of two (range)
     res2 = fma2(e, e, res2);
   }
   num = lo_of(num2) + hi_of(num2);
@@ -597,7 +605,7 @@ __device__ __forceinline__ void flush_runs(ColState& cs, double2* acc, double* r
 // with t = T + 1: the codes of the final iterate, packed, and mse[T].
 template <int FMT, int WDT, bool FIN>
 __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t, const __grid_constant__ CUtensorMap wmap) {
-  if (p.hdr->flags & kFlagNonFinite) return;
+  if (p.hdr->flags & kFlagAbort) return;
   constexpr int ES = WDT == DT_F32 ? 4 : 2;
   constexpr int S = ring_stages(ES);
   extern __shared__ __align__(128) unsigned char smem[];

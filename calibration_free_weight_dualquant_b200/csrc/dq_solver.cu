@@ -20,11 +20,13 @@
 // result is deterministic.
 #include <cudaTypedefs.h>  // PFN_cuTensorMapEncodeTiled
 
+#include <algorithm>
 #include <climits>
 #include <cstring>
 
 #include "dq_device.cuh"
 #include "dq_fast.cuh"
+#include "dq_init.cuh"
 #include "dq_internal.h"
 #include "dq_iter.cuh"
 
@@ -70,14 +72,17 @@ __global__ void __launch_bounds__(kThreads) k_stats(Problem p) {
 
 // ---------------------------------------------------------------------------
 // Init: s_T (NVFP4), a = Proj(absmax/qmax) per block (1 for an all-zero
-// block), b = 1.
+// block), b = 1.  With the L1-norm init (dq_init.cuh) the column scales are
+// already set and the absmax is taken of |W_ij| / b_j (fp64 quotients).
 template <int FMT, int WDT>
 __global__ void __launch_bounds__(kThreads) k_init(Problem p) {
-  if (p.hdr->flags & kFlagNonFinite) return;
+  if (p.hdr->flags & kFlagAbort) return;
+  const bool l1 = p.init == DQ_INIT_L1;
   double sTd = 1.0;
   if (FMT == FMT_NVFP4) {
-    const float amax = __uint_as_float(p.hdr->amax_bits);
-    float s = amax == 0.f ? 1.f : __double2float_rn((double)amax / 2688.0);
+    const double amax = l1 ? __longlong_as_double((long long)p.hdr->amax_scaled)
+                           : (double)__uint_as_float(p.hdr->amax_bits);
+    float s = amax == 0.0 ? 1.f : __double2float_rn(amax / 2688.0);
     if (s == 0.f) s = 0x1p-149f;
     sTd = (double)s;
     if (blockIdx.x == 0 && threadIdx.x == 0) {
@@ -94,17 +99,31 @@ __global__ void __launch_bounds__(kThreads) k_init(Problem p) {
   for (int64_t blk = (int64_t)blockIdx.x * kThreads + threadIdx.x; blk < nblocks; blk += stride) {
     const int64_t i = blk / p.nb, g = blk % p.nb;
     const int64_t off = i * p.N + g * p.G;
-    float m = 0.f;
-    for (int c = 0; c < p.G; c += 8) {
-      float w[8];
-      load8<WDT>(p.W, off + c, w);
+    double m = 0.0;
+    if (l1) {
+      for (int c = 0; c < p.G; c += 8) {
+        float w[8];
+        load8<WDT>(p.W, off + c, w);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) m = fmaxf(m, fabsf(w[k]));
+        for (int k = 0; k < 8; ++k)
+          m = fmax(m, (double)fabsf(w[k]) / (double)b_decode(p.b_store, p.col_dt, g * p.G + c + k));
+      }
+    } else {
+      float mf = 0.f;
+      for (int c = 0; c < p.G; c += 8) {
+        float w[8];
+        load8<WDT>(p.W, off + c, w);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mf = fmaxf(mf, fabsf(w[k]));
+      }
+      m = (double)mf;
     }
-    const double a = (m == 0.f) ? 1.0 : a_project<FMT>((double)m / qmax, sTd);
+    const double a = (m == 0.0) ? 1.0 : a_project<FMT>(m / qmax, sTd);
     a_encode<FMT>(p.a_store, blk, a);
   }
-  for (int64_t j = (int64_t)blockIdx.x * kThreads + threadIdx.x; j < p.N; j += stride) b_encode(p.b_store, p.col_dt, j, 1.0);
+  if (!l1)
+    for (int64_t j = (int64_t)blockIdx.x * kThreads + threadIdx.x; j < p.N; j += stride)
+      b_encode(p.b_store, p.col_dt, j, 1.0);
 }
 
 // ---------------------------------------------------------------------------
@@ -160,7 +179,23 @@ static cudaError_t run_typed(const Problem& p, int iters, int stats_ctas, cudaSt
   pf.P = p.P_final;
   pf.segmax = p.segmax_final;
   k_stats<WDT><<<stats_ctas, kThreads, 0, st>>>(pf);
-  k_init<FMT, WDT><<<stats_ctas, kThreads, 0, st>>>(pf);
+  if (p.init == DQ_INIT_GIVEN) {
+    k_check_given<FMT><<<stats_ctas, kThreads, 0, st>>>(pf);
+  } else {
+    if (p.init == DQ_INIT_L1) {
+      // exact column sums: 32 columns per CTA, rows split so the grid fills the GPU
+      const int64_t gx = (p.N + 31) / 32;
+      int64_t gy = std::max<int64_t>(1, std::min<int64_t>((8 * (int64_t)stats_ctas + gx - 1) / gx,
+                                                          (p.M + kMinRowsPerCta - 1) / kMinRowsPerCta));
+      const int64_t rows_per_cta = (p.M + gy - 1) / gy;
+      gy = (p.M + rows_per_cta - 1) / rows_per_cta;
+      k_l1_sums<WDT><<<dim3((unsigned)gx, (unsigned)gy), kThreads, 0, st>>>(pf, rows_per_cta);
+      k_l1_cols<<<(unsigned)((p.N + kThreads - 1) / kThreads), kThreads, 0, st>>>(pf);
+      k_l1_b<<<(unsigned)std::min<int64_t>(stats_ctas, (p.N + kThreads - 1) / kThreads), kThreads, 0, st>>>(pf);
+      if (FMT == FMT_NVFP4) k_amax_scaled<WDT><<<stats_ctas, kThreads, 0, st>>>(pf);
+    }
+    k_init<FMT, WDT><<<stats_ctas, kThreads, 0, st>>>(pf);
+  }
   for (int t = 1; t <= iters; ++t) k_iter<FMT, WDT, false><<<(unsigned)p.P, kIterThreads, smem, st>>>(pi, t, wmap);
   k_iter<FMT, WDT, true><<<(unsigned)p.P, kIterThreads, smem, st>>>(pi, iters + 1, wmap);
   return cudaGetLastError();

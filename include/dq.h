@@ -112,8 +112,8 @@ int dq_solve(const void* W, int w_dtype, int64_t rows, int64_t cols, int format,
  * alone, column scaling alone). */
 typedef enum {
   DQ_MODE_DUAL = 0,  /* the dual-scale BCD iteration (dq_solve) */
-  DQ_MODE_ROW = 1,   /* block scales only: row update and requantize; b stays 1 */
-  DQ_MODE_COL = 2    /* column scales only: column update and requantize; a stays at RTN */
+  DQ_MODE_ROW = 1,   /* block scales only: row update and requantize; b keeps its initial value */
+  DQ_MODE_COL = 2    /* column scales only: column update and requantize; a keeps its initial value */
 } dq_mode;
 
 /* dq_solve with an ablation mode (dq_mode); DQ_MODE_DUAL is dq_solve. */
@@ -121,9 +121,59 @@ int dq_solve_mode(const void* W, int w_dtype, int64_t rows, int64_t cols, int fo
                   int col_dtype, int mode, const dq_outputs* out, void* workspace, size_t workspace_bytes,
                   void* stream);
 
+/* Initial iterate of the solver.
+ *  DQ_INIT_RTN    absmax RTN block scales, column scales 1 (what dq_solve uses).
+ *  DQ_INIT_L1     per-column L1-norm column scales (DualQuant summary §5.3: the
+ *                 initialization uses format-native row absmax scales and
+ *                 per-column L1-norm scales).  The pages name the norm only; the
+ *                 reading implemented: b_j = Proj_Fb(c_j / mu) with
+ *                 c_j = sum_i |W_ij| and mu = (sum_ij |W_ij|) / cols, each sum
+ *                 exact and rounded once to fp64, b_j = 1 for an all-zero column;
+ *                 then the absmax RTN scales of W D_b^-1:
+ *                 a = Proj_Fa(max_j (|W_ij| / b_j) / qmax) (1 for a zero block) and,
+ *                 for NVFP4, s_T = fp32(max_ij (|W_ij| / b_j) / 2688).  With every
+ *                 b_j = 1 this is DQ_INIT_RTN.
+ *  DQ_INIT_GIVEN  warm start: the scales already in out->block_scales,
+ *                 out->col_scales and (NVFP4) out->tensor_scale, in their storage
+ *                 formats, are the initial iterate.  Each must be admissible:
+ *                 positive and finite (E8M0 bytes 1..253, E4M3 bytes 0x01..0x7E,
+ *                 fp16 0x0001..0x7BFF, bf16 0x0001..0x7F7F, s_T a positive finite
+ *                 float).  A violation is found on the device: dq_sync_status then
+ *                 returns DQ_EINVAL and nothing but the given scales is written.
+ *                 T1 iterations followed by a warm start of T2 more give exactly the
+ *                 outputs of T1 + T2 iterations (mse[0] of the second call is mse[T1]
+ *                 of the whole). */
+typedef enum { DQ_INIT_RTN = 0, DQ_INIT_L1 = 1, DQ_INIT_GIVEN = 2 } dq_init;
+
+/* Options of dq_solve_ex.  A NULL options pointer means all defaults. */
+typedef struct {
+  int mode;                /* dq_mode (default DQ_MODE_DUAL = 0) */
+  int init;                /* dq_init (default DQ_INIT_RTN = 0) */
+  uint64_t* code_changes;  /* NULL, or a device array of iters+1 counters: code_changes[0] = 0 and
+                            * code_changes[t] = the number of elements whose code differs between
+                            * the iterates after iterations t-1 and t (DualQuant summary §4.3 and
+                            * App. B: the quantized matrix stabilizes; the relative change of Q is
+                            * code_changes[t] / (rows*cols)).  The solver keeps the codes of the
+                            * previous iterate in out->codes meanwhile. */
+} dq_options;
+
+/* Device workspace bytes dq_solve_ex needs with these options (0 on invalid
+ * arguments).  Equal to dq_workspace_bytes except for DQ_INIT_L1, whose exact
+ * column sums need 88 bytes per column of scratch, and more for very wide
+ * matrices. */
+size_t dq_workspace_bytes_ex(int64_t rows, int64_t cols, int format, int group, const dq_options* options);
+
+/* The solver with options: ablation mode, initial iterate, changed-code
+ * counts.  dq_solve is dq_solve_ex with NULL options.  DQ_EINVAL for an
+ * unknown mode or init; DQ_EWORKSPACE below dq_workspace_bytes_ex. */
+int dq_solve_ex(const void* W, int w_dtype, int64_t rows, int64_t cols, int format, int group, int iters,
+                int col_dtype, const dq_options* options, const dq_outputs* out, void* workspace,
+                size_t workspace_bytes, void* stream);
+
 /* Waits for `stream`, then reports what the device recorded in `workspace`
- * during the last dq_rtn / dq_solve that used it: DQ_OK, DQ_ENONFINITE, or
- * DQ_ECUDA if the wait itself failed. */
+ * during the last dq_rtn / dq_solve that used it: DQ_OK, DQ_ENONFINITE,
+ * DQ_EINVAL (a warm start with an inadmissible scale), or DQ_ECUDA if the
+ * wait itself failed or a bounded pipeline wait gave up. */
 int dq_sync_status(const void* workspace, void* stream);
 
 /* Device bytes dq_solve_host needs: room for a device copy of W, the outputs
