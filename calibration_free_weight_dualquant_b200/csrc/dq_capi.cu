@@ -105,7 +105,7 @@ int solve_impl(const void* W, int w_dtype, int64_t rows, int64_t cols, int forma
   unsigned long long* changes = opt ? reinterpret_cast<unsigned long long*>(opt->code_changes) : nullptr;
   if (mode < DQ_MODE_DUAL || mode > DQ_MODE_COL) return DQ_EINVAL;
   if (init < DQ_INIT_RTN || init > DQ_INIT_GIVEN) return DQ_EINVAL;
-  if (changes != nullptr) return DQ_EUNSUPPORTED;
+  if (changes != nullptr && !aligned(changes, 8)) return DQ_EINVAL;
   if (w_dtype < DQ_F32 || w_dtype > DQ_F16) return DQ_EINVAL;
   if (col_dtype != DQ_F16 && col_dtype != DQ_BF16) return DQ_EUNSUPPORTED;
   if (iters < 0) return DQ_EINVAL;
@@ -155,6 +155,8 @@ int solve_impl(const void* W, int w_dtype, int64_t rows, int64_t cols, int forma
   // header and arrival counters start at zero; the partial buffers need no init
   if (cudaMemsetAsync(ws, 0, pl.off_col_part, stream) != cudaSuccess) return DQ_ECUDA;
   if (init == DQ_INIT_L1 && cudaMemsetAsync(ws + pl.off_col_part, 0, pl.l1_zero_bytes, stream) != cudaSuccess)
+    return DQ_ECUDA;
+  if (changes && cudaMemsetAsync(changes, 0, sizeof(unsigned long long) * (size_t)(iters + 1), stream) != cudaSuccess)
     return DQ_ECUDA;
   if (dq::launch_solve(p, iters, pl.P_final, stream) != cudaSuccess) return DQ_ECUDA;
   return DQ_OK;

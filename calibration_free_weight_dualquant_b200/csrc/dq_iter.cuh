@@ -28,6 +28,10 @@ constexpr int kIterThreads = kConsumers + 32;
 constexpr int kConsumerTreeTop = 256;  // largest power of two below kConsumers
 static_assert(kConsumerTreeTop < kConsumers && 2 * kConsumerTreeTop >= kConsumers, "tree reduction shape");
 constexpr int kRowsPerWarp = 2;
+// kinds of k_iter pass: a BCD iteration; a BCD iteration that also tracks the
+// codes between iterates (changed-code counts); the final pass (codes of the
+// final iterate and the last MSE)
+enum : int { PASS_ITER = 0, PASS_COUNT = 1, PASS_FINAL = 2 };
 constexpr int kRowsPerTile = kConsumerWarps * kRowsPerWarp;
 constexpr int kRun = 8;
 constexpr int kRingBytes = 96 * 1024;
@@ -459,16 +463,62 @@ __device__ __forceinline__ void row_sums64(const f2 w2[4], const f2 q2[4], const
   }
 }
 
+// The 8 codes of a lane's row packed into one word (even column in the low
+// nibble; zero is always the 0x0 nibble).
+template <int FMT>
+__device__ __forceinline__ uint32_t pack8(const f2 q2[4]) {
+  uint32_t r = 0u;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float lo = __fadd_rn(lo_of(q2[i]), 0.f), hi = __fadd_rn(hi_of(q2[i]), 0.f);  // -0 becomes +0
+    uint32_t byte;
+    if (fmt_e2m1(FMT)) {
+      byte = cvt_e2m1x2(hi, lo);  // grid values convert exactly
+    } else {  // q + 1.5 * 2^23 holds the integer q in its low mantissa bits (two's complement mod 16)
+      byte = (__float_as_uint(lo + 12582912.f) & 15u) | ((__float_as_uint(hi + 12582912.f) & 15u) << 4);
+    }
+    r |= byte << (8 * i);
+  }
+  return r;
+}
+
+// Number of nonzero nibbles of x (codes that differ, for x = new ^ old).
+__device__ __forceinline__ uint32_t changed_nibbles(uint32_t x) {
+  x |= x >> 1;
+  x |= x >> 2;
+  return (uint32_t)__popc(x & 0x11111111u);
+}
+
+// Code tracking for two rows of a lane: the packed codes replace the words at
+// cix (row x) and cix + kConsumerWarps rows (row y); with `cmp` the nibbles
+// that differ from the previous words oldx, oldy are counted into nchg.
+template <int FMT>
+__device__ __forceinline__ void track_codes(const Problem& p, const f2 qx[4], const f2 qy[4], bool actx, bool acty,
+                                            int64_t cix, uint32_t oldx, uint32_t oldy, bool cmp, unsigned& nchg) {
+  uint32_t* codes = reinterpret_cast<uint32_t*>(p.codes);
+  if (actx) {
+    const uint32_t c = pack8<FMT>(qx);
+    if (cmp) nchg += changed_nibbles(c ^ oldx);
+    codes[cix] = c;
+  }
+  if (acty) {
+    const uint32_t c = pack8<FMT>(qy);
+    if (cmp) nchg += changed_nibbles(c ^ oldy);
+    codes[cix + (int64_t)kConsumerWarps * (p.N >> 3)] = c;
+  }
+}
+
 // Two rows of one lane (x = row a, y = row b; y may be absent, then its data
 // are zero and nothing of it is written): requantize the incoming iterate;
 // block sums, residuals and block updates; requantize with the new block
 // scales where they changed; column sums.  Warp-collective (shuffles and
 // votes); `active` lanes hold real columns and alone write results.
-template <int FMT>
+template <int FMT, int PASS>
 __device__ __forceinline__ void row_pair(const Problem& p, const f2 wx[4], float ax_old, int64_t bidx_x,
                                          const f2 wy[4], float ay_old, int64_t bidx_y, bool has_y, bool active,
                                          bool leader, int lpb, ColState& cs, float sT, float isT, double sTd,
-                                         f2 rscale2, unsigned* s_cnt) {
+                                         f2 rscale2, unsigned* s_cnt, int64_t cix, uint32_t oldx, uint32_t oldy,
+                                         bool cmp, unsigned& nchg) {
   const bool actx = active, acty = active && has_y;
   f2 ux[4], uy[4], qx[4], qy[4];
 #pragma unroll
@@ -478,6 +528,7 @@ __device__ __forceinline__ void row_pair(const Problem& p, const f2 wx[4], float
     uy[i] = mul2(wy[i], cbi);
   }
   req_pair<FMT>(wx, ux, ax_old, actx, wy, uy, ay_old, acty, cs, sT, sTd, qx, qy, s_cnt);
+  if (PASS == PASS_COUNT) track_codes<FMT>(p, qx, qy, actx, acty, cix, oldx, oldy, cmp, nchg);
   float nx, dx, ny, dy;
   row_sums<FMT>(wx, qx, ax_old, cs, sT, rscale2, nx, dx, cs.res2);
   row_sums<FMT>(wy, qy, ay_old, cs, sT, rscale2, ny, dy, cs.res2);
@@ -537,32 +588,14 @@ __device__ __forceinline__ void row_pair(const Problem& p, const f2 wx[4], float
   }
 }
 
-// Final pass: the 8 codes of a lane's row packed into one word (even column in
-// the low nibble; zero is always the 0x0 nibble).
-template <int FMT>
-__device__ __forceinline__ uint32_t pack8(const f2 q2[4]) {
-  uint32_t r = 0u;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float lo = __fadd_rn(lo_of(q2[i]), 0.f), hi = __fadd_rn(hi_of(q2[i]), 0.f);  // -0 becomes +0
-    uint32_t byte;
-    if (fmt_e2m1(FMT)) {
-      byte = cvt_e2m1x2(hi, lo);  // grid values convert exactly
-    } else {  // q + 1.5 * 2^23 holds the integer q in its low mantissa bits (two's complement mod 16)
-      byte = (__float_as_uint(lo + 12582912.f) & 15u) | ((__float_as_uint(hi + 12582912.f) & 15u) << 4);
-    }
-    r |= byte << (8 * i);
-  }
-  return r;
-}
-
 // Final pass for two rows of a lane (x = row rx, y = row rx + kConsumerWarps,
 // possibly absent): codes of the final iterate, written packed, and the
 // residuals of that iterate for its MSE.
 template <int FMT>
-__device__ __forceinline__ void final_pair(const Problem& p, const f2 wx[4], float ax, int64_t rx, const f2 wy[4],
-                                           float ay, bool has_y, bool active, int64_t col, ColState& cs, float sT,
-                                           double sTd, f2 rscale2, unsigned* s_cnt) {
+__device__ __forceinline__ void final_pair(const Problem& p, const f2 wx[4], float ax, const f2 wy[4], float ay,
+                                           bool has_y, bool active, ColState& cs, float sT, double sTd, f2 rscale2,
+                                           unsigned* s_cnt, int64_t cix, uint32_t oldx, uint32_t oldy, bool cmp,
+                                           unsigned& nchg) {
   const bool actx = active, acty = active && has_y;
   f2 ux[4], uy[4], qx[4], qy[4];
 #pragma unroll
@@ -575,9 +608,7 @@ __device__ __forceinline__ void final_pair(const Problem& p, const f2 wx[4], flo
   float n, d;  // block sums: not needed here
   row_sums<FMT>(wx, qx, ax, cs, sT, rscale2, n, d, cs.res2);
   row_sums<FMT>(wy, qy, ay, cs, sT, rscale2, n, d, cs.res2);
-  uint32_t* codes = reinterpret_cast<uint32_t*>(p.codes);
-  if (actx) codes[(rx * p.N + col) >> 3] = pack8<FMT>(qx);
-  if (acty) codes[((rx + kConsumerWarps) * p.N + col) >> 3] = pack8<FMT>(qy);
+  track_codes<FMT>(p, qx, qy, actx, acty, cix, oldx, oldy, cmp, nchg);
 }
 
 // fp32 runs into the warp's fp64 accumulators (layout [warp][c][lane], then
@@ -600,10 +631,13 @@ __device__ __forceinline__ void flush_runs(ColState& cs, double2* acc, double* r
   cs.res2 = 0ull;
 }
 
-// One pass over W.  FIN = false: BCD iteration t (writes mse[t - 1], the MSE of
-// the incoming iterate).  FIN = true: the final pass after T iterations, called
-// with t = T + 1: the codes of the final iterate, packed, and mse[T].
-template <int FMT, int WDT, bool FIN>
+// One pass over W.  PASS_ITER: BCD iteration t (writes mse[t - 1], the MSE of
+// the incoming iterate).  PASS_COUNT: the same, and the incoming iterate's codes
+// replace those of the iterate before it in p.codes, the changed ones counted
+// into changes[t - 1] (t >= 2).  PASS_FINAL: the final pass after T iterations,
+// called with t = T + 1: the codes of the final iterate, packed, and mse[T]
+// (and changes[T] when counting, T >= 1).
+template <int FMT, int WDT, int PASS>
 __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t, const __grid_constant__ CUtensorMap wmap) {
   if (p.hdr->flags & kFlagAbort) return;
   constexpr int ES = WDT == DT_F32 ? 4 : 2;
@@ -700,6 +734,12 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t, cons
   const int64_t s_first = u_begin / p.M;
   int st = 0;
   unsigned par = 0u;
+  constexpr bool FIN = PASS == PASS_FINAL;
+  // compare with the previous iterate's codes (kept in p.codes by the pass before)
+  const bool cmp = (PASS == PASS_COUNT || (FIN && p.changes != nullptr)) && t > 1;
+  const uint32_t* codes_old = reinterpret_cast<const uint32_t*>(p.codes);
+  const int64_t code_step = (int64_t)kConsumerWarps * (p.N >> 3);  // code words between a warp's two rows
+  unsigned nchg = 0u;
 
   for (int64_t u = u_begin; u < u_end;) {
     const int64_t s = u / p.M;
@@ -760,6 +800,12 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t, cons
       const float aa = an0, ab = an1;
       if (active && ra + kRowsPerTile < r1) an0 = a_load<FMT>(p.a_store, aidx + a_step);
       if (active && rb + kRowsPerTile < r1) an1 = a_load<FMT>(p.a_store, aidx + a_step + kConsumerWarps * p.nb);
+      const int64_t cix = (ra * p.N + col) >> 3;  // code word of row ra, this lane's 8 columns
+      uint32_t oldx = 0u, oldy = 0u;
+      if (PASS != PASS_ITER && cmp && active) {  // issued before the wait: the latency hides behind it
+        if (has_a) oldx = __ldcg(codes_old + cix);
+        if (has_b) oldy = __ldcg(codes_old + cix + code_step);
+      }
       mbar_wait(&full[st], par, &p.hdr->flags);
       f2 wa[4], wb[4];
       const unsigned char* base = ring + st * stage_bytes + lane * 8 * ES;
@@ -777,10 +823,10 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t, cons
           for (int i = 0; i < 4; ++i) wb[i] = 0ull;  // absent row: zeros contribute nothing
         }
         if (FIN) {
-          final_pair<FMT>(p, wa, aa, ra, wb, ab, has_b, active, col, cs, sT, sTd, rscale2, s_cnt);
+          final_pair<FMT>(p, wa, aa, wb, ab, has_b, active, cs, sT, sTd, rscale2, s_cnt, cix, oldx, oldy, cmp, nchg);
         } else {
-          row_pair<FMT>(p, wa, aa, aidx, wb, ab, aidx + kConsumerWarps * p.nb, has_b, active, leader, lpb, cs, sT,
-                        isT, sTd, rscale2, s_cnt);
+          row_pair<FMT, PASS>(p, wa, aa, aidx, wb, ab, aidx + kConsumerWarps * p.nb, has_b, active, leader, lpb, cs,
+                              sT, isT, sTd, rscale2, s_cnt, cix, oldx, oldy, cmp, nchg);
         }
         run += has_b ? 2 : 1;
       }
@@ -869,6 +915,11 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t, cons
     }
     consumer_sync(kConsumers);
     u = (s + 1) * p.M;
+  }
+
+  if (PASS != PASS_ITER && cmp) {  // changed codes of this warp, one atomic per warp
+    for (int o = 16; o > 0; o >>= 1) nchg += __shfl_xor_sync(0xffffffffu, nchg, o);
+    if (lane == 0 && nchg) atomicAdd(&p.changes[t - 1], (unsigned long long)nchg);
   }
 
   // MSE of the incoming iterate: per-thread residual sums, CTA tree, then the

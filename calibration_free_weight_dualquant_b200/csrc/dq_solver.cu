@@ -168,9 +168,10 @@ template <int FMT, int WDT>
 static cudaError_t run_typed(const Problem& p, int iters, int stats_ctas, cudaStream_t st) {
   constexpr int ES = WDT == DT_F32 ? 4 : 2;
   const size_t smem = iter_smem_bytes(ES);
-  cudaError_t e = cudaFuncSetAttribute(k_iter<FMT, WDT, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const auto iter_kernel = p.changes ? k_iter<FMT, WDT, PASS_COUNT> : k_iter<FMT, WDT, PASS_ITER>;
+  cudaError_t e = cudaFuncSetAttribute(iter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(k_iter<FMT, WDT, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  e = cudaFuncSetAttribute(k_iter<FMT, WDT, PASS_FINAL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   CUtensorMap wmap;
   Problem pi = p;
@@ -196,8 +197,8 @@ static cudaError_t run_typed(const Problem& p, int iters, int stats_ctas, cudaSt
     }
     k_init<FMT, WDT><<<stats_ctas, kThreads, 0, st>>>(pf);
   }
-  for (int t = 1; t <= iters; ++t) k_iter<FMT, WDT, false><<<(unsigned)p.P, kIterThreads, smem, st>>>(pi, t, wmap);
-  k_iter<FMT, WDT, true><<<(unsigned)p.P, kIterThreads, smem, st>>>(pi, iters + 1, wmap);
+  for (int t = 1; t <= iters; ++t) iter_kernel<<<(unsigned)p.P, kIterThreads, smem, st>>>(pi, t, wmap);
+  k_iter<FMT, WDT, PASS_FINAL><<<(unsigned)p.P, kIterThreads, smem, st>>>(pi, iters + 1, wmap);
   return cudaGetLastError();
 }
 
