@@ -15,7 +15,7 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 struct Plan {
   int TS, n_strips, P, segmax, P_final, segmax_final, nb;
   int64_t L;
-  size_t off_counters, off_col_part, off_cta_part, total;
+  size_t off_counters, off_amb_tick, off_col_part, off_cta_part, off_amb_list, total;
   size_t l1_zero_bytes;  // L1 init: digit counters to zero (start of the col_part region)
   size_t off_l1_tot, off_l1_norm;
 };
@@ -61,6 +61,8 @@ int make_plan(int64_t M, int64_t N, int group, int init, Plan* pl) {
   size_t off = align_up(sizeof(dq::WsHeader));
   pl->off_counters = off;
   off += align_up(sizeof(unsigned) * (size_t)pl->n_strips);
+  pl->off_amb_tick = off;
+  off += align_up(sizeof(unsigned) * (size_t)N);
   pl->off_col_part = off;
   // the L1-init scratch overlays the column partials (the init kernels run
   // before the first iteration): per-column digits, the total's digits, norms;
@@ -75,6 +77,8 @@ int make_plan(int64_t M, int64_t N, int group, int init, Plan* pl) {
   off += (init == DQ_INIT_L1 && l1_bytes > part_bytes) ? l1_bytes : part_bytes;
   pl->off_cta_part = off;
   off += align_up(sizeof(double) * (size_t)(pl->P > pl->P_final ? pl->P : pl->P_final));
+  pl->off_amb_list = off;
+  off += align_up(sizeof(int) * (size_t)N);
   pl->total = off;
   return DQ_OK;
 }
@@ -151,8 +155,11 @@ int solve_impl(const void* W, int w_dtype, int64_t rows, int64_t cols, int forma
   p.strip_counter = reinterpret_cast<unsigned*>(ws + pl.off_counters);
   p.col_part = reinterpret_cast<double2*>(ws + pl.off_col_part);
   p.cta_part = reinterpret_cast<double*>(ws + pl.off_cta_part);
+  p.amb_list = reinterpret_cast<int*>(ws + pl.off_amb_list);
+  p.amb_tick = reinterpret_cast<unsigned*>(ws + pl.off_amb_tick);
 
-  // header and arrival counters start at zero; the partial buffers need no init
+  // header and arrival counters (strips, listed columns) start at zero; the
+  // partial buffers and the column list need no init
   if (cudaMemsetAsync(ws, 0, pl.off_col_part, stream) != cudaSuccess) return DQ_ECUDA;
   if (init == DQ_INIT_L1 && cudaMemsetAsync(ws + pl.off_col_part, 0, pl.l1_zero_bytes, stream) != cudaSuccess)
     return DQ_ECUDA;

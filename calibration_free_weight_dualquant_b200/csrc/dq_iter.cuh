@@ -346,53 +346,6 @@ __device__ __forceinline__ void req_pair(const f2 wx[4], const f2 ux[4], float f
 }
 
 // ---------------------------------------------------------------------------
-// Exact fp64 column sums of one column over all rows (ambiguous-projection
-// fallback), run by the consumer threads of the finalizing CTA.
-template <int FMT, int WDT>
-__device__ double2 column_exact(const Problem& p, int64_t j, float bj, double sTd, double* scratch) {
-  const float isT = FMT == FMT_NVFP4 ? (float)(1.0 / sTd) : 1.f;
-  const float cb = __frcp_rn(bj) * isT;
-  double cn = 0.0, cd = 0.0;
-  for (int64_t i = threadIdx.x; i < p.M; i += kConsumers) {
-    float w;
-    if (WDT == DT_F32) {
-      w = __ldg(reinterpret_cast<const float*>(p.W) + i * p.N + j);
-    } else if (WDT == DT_BF16) {
-      w = __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short*>(p.W) + i * p.N + j) << 16);
-    } else {
-      w = __half2float(__ushort_as_half(__ldg(reinterpret_cast<const unsigned short*>(p.W) + i * p.N + j)));
-    }
-    const int64_t bidx = i * p.nb + j / p.G;
-    float a;
-    if (FMT == FMT_INT4) {
-      a = __half2float(__ushort_as_half(__ldcg(reinterpret_cast<const unsigned short*>(p.a_store) + bidx)));
-    } else {
-      const uint32_t v = __ldcg(reinterpret_cast<const unsigned char*>(p.a_store) + bidx);
-      a = fmt_pow2(FMT) ? __uint_as_float(v << 23) : e4m3_value(v);
-    }
-    const float ia = __frcp_rn(a);
-    const bool ok = in_range(cb) && in_range(ia);
-    const float q = quant<FMT>(w, w * cb, ia, ok, a, bj, sTd);
-    const double sv = (double)q * (double)a;
-    cn = fma((double)w, sv, cn);
-    cd = fma(sv, sv, cd);
-  }
-  scratch[2 * threadIdx.x] = cn;
-  scratch[2 * threadIdx.x + 1] = cd;
-  consumer_sync(kConsumers);
-  for (int o = kConsumerTreeTop; o > 0; o >>= 1) {  // fixed-order tree
-    if (threadIdx.x < o && threadIdx.x + o < kConsumers) {
-      scratch[2 * threadIdx.x] += scratch[2 * (threadIdx.x + o)];
-      scratch[2 * threadIdx.x + 1] += scratch[2 * (threadIdx.x + o) + 1];
-    }
-    consumer_sync(kConsumers);
-  }
-  const double2 r = make_double2(scratch[0], scratch[1]);
-  consumer_sync(kConsumers);
-  return r;
-}
-
-// ---------------------------------------------------------------------------
 // One row of W for one lane (8 elements as 4 pairs, exact fp32 values).
 template <int WDT>
 __device__ __forceinline__ void smem_row(const unsigned char* src, f2 w2[4]) {
@@ -874,8 +827,10 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t, cons
       __threadfence();
       // totals in CTA order, certified projection
       double bnew = 1.0;
+      bool amb = false;
       if (threadIdx.x < width) {
         double2 tot = make_double2(0.0, 0.0);
+#pragma unroll 4
         for (int64_t kk = k_first; kk <= k_last; ++kk) {
           const int64_t sl = kk * p.segmax + (s - range_begin(kk, p.P, p.L) / p.M);
           const double2 v = __ldcg(&p.col_part[sl * p.TS + threadIdx.x]);
@@ -892,25 +847,17 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t, cons
         if (lo == hi) {
           bnew = lo;
         } else {
-          const int slot_a = atomicAdd(&s_misc[1], 1);
-          s_misc[2 + slot_a] = threadIdx.x;
+          // ambiguous: listed for k_col_exact, which recomputes the column's
+          // sums exactly over all rows and writes its scale (b keeps its value
+          // until then)
+          amb = true;
+          atomicAdd(&s_misc[1], 1);
+          p.amb_list[atomicAdd(&p.hdr->amb_n, 1u)] = (int)(c0 + threadIdx.x);
         }
       }
       consumer_sync(kConsumers);
-      const int namb = s_misc[1];
-      if (threadIdx.x == 0) s_cnt[2] += (unsigned)namb;
-      double* scratch = reinterpret_cast<double*>(acc);
-      for (int ia = 0; ia < namb; ++ia) {
-        const int cidx = s_misc[2 + ia];
-        const float bold = b_decode(p.b_store, p.col_dt, c0 + cidx);
-        const double2 ex = column_exact<FMT, WDT>(p, c0 + cidx, bold, sTd, scratch);
-        if (threadIdx.x == cidx) {
-          const double v = FMT == FMT_NVFP4 ? (ex.x / ex.y) / sTd : ex.x / ex.y;
-          bnew = ex.y == 0.0 ? 1.0 : b_project(v, p.col_dt);
-        }
-      }
-      consumer_sync(kConsumers);
-      if (threadIdx.x < width) b_encode(p.b_store, p.col_dt, c0 + threadIdx.x, bnew);
+      if (threadIdx.x == 0) s_cnt[2] += (unsigned)s_misc[1];
+      if (threadIdx.x < width && !amb) b_encode(p.b_store, p.col_dt, c0 + threadIdx.x, bnew);
       if (threadIdx.x == 0) p.strip_counter[s] = 0u;
     }
     consumer_sync(kConsumers);
@@ -942,11 +889,128 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t, cons
     p.cta_part[k] = mred[0];
     __threadfence();
     const unsigned prev = atomicAdd(&p.hdr->cta_counter, 1u);
-    if (prev == (unsigned)p.P - 1u) {
+    s_misc[0] = prev == (unsigned)p.P - 1u ? 1 : 0;
+  }
+  consumer_sync(kConsumers);
+  if (s_misc[0]) {
+    // the last CTA: the per-CTA partials in a fixed-order tree (one load per
+    // thread in flight at once, instead of a chain of P dependent additions)
+    __threadfence();
+    double v = 0.0;
+    for (int64_t kk = threadIdx.x; kk < p.P; kk += kConsumers) v += __ldcg(&p.cta_part[kk]);
+    mred[threadIdx.x] = v;
+    consumer_sync(kConsumers);
+    for (int o = kConsumerTreeTop; o > 0; o >>= 1) {
+      if (threadIdx.x < o && threadIdx.x + o < kConsumers) mred[threadIdx.x] += mred[threadIdx.x + o];
+      consumer_sync(kConsumers);
+    }
+    if (threadIdx.x == 0) {
+      p.mse[t - 1] = mred[0] / (rscale_d * rscale_d) / ((double)p.M * (double)p.N);
+      p.hdr->cta_counter = 0u;
+    }
+  }
+}
+
+
+// ---------------------------------------------------------------------------
+// Exact column update of the columns that the k_iter launch just before listed
+// (their certified projection was ambiguous and their scale still holds the
+// value of the iterate): sum W a q' and sum (a q')^2 in fp64 over all rows,
+// then b = Proj_Fb(ratio), 1 for a zero sum.  Each listed column is cut into R
+// row chunks; a CTA takes (column, chunk) items, each thread keeps the loads
+// of kXRows rows in flight, and the chunk total is a fixed-order tree.  The
+// last chunk of a column to arrive adds the R chunk totals in chunk order, so
+// the result does not depend on the schedule.  With an empty list every CTA
+// returns at once.  The last CTA to finish empties the list.
+constexpr int kXThreads = 256;
+constexpr int kXRows = 8;
+
+template <int FMT, int WDT>
+__global__ void __launch_bounds__(kXThreads) k_col_exact(Problem p) {
+  __shared__ double s_red[2][kXThreads];
+  __shared__ int s_last;
+  const unsigned n = p.hdr->amb_n;
+  if (n == 0u) return;
+  const double sTd = (double)p.hdr->sT;
+  const float isT = FMT == FMT_NVFP4 ? (float)(1.0 / sTd) : 1.f;
+  // R chunks per column: about kXThreads * kXRows rows each, and n * R
+  // partials must fit the column-partial buffer of k_iter (free by now)
+  const int64_t cap = (int64_t)p.P * p.segmax * p.TS;
+  const int64_t chunk_want = (int64_t)kXThreads * kXRows;
+  const int64_t R = max((int64_t)1, min((p.M + chunk_want - 1) / chunk_want, cap / (int64_t)n));
+  const int64_t chunk = (p.M + R - 1) / R;
+  for (int64_t it = blockIdx.x; it < (int64_t)n * R; it += gridDim.x) {
+    const int64_t ci = it / R, r = it - ci * R;
+    const int64_t j = p.amb_list[ci];
+    const float bj = b_decode(p.b_store, p.col_dt, j);
+    const float cb = __frcp_rn(bj) * isT;
+    const int64_t i_end = min(p.M, (r + 1) * chunk);
+    double cn = 0.0, cd = 0.0;
+    for (int64_t i0 = r * chunk + threadIdx.x; i0 < i_end; i0 += (int64_t)kXRows * kXThreads) {
+      float w[kXRows], a[kXRows];
+#pragma unroll
+      for (int k = 0; k < kXRows; ++k) {  // all loads first
+        const int64_t i = i0 + (int64_t)k * kXThreads;
+        w[k] = 0.f;
+        a[k] = 1.f;
+        if (i < i_end) {
+          const int64_t e = i * p.N + j;
+          if (WDT == DT_F32) {
+            w[k] = __ldg(reinterpret_cast<const float*>(p.W) + e);
+          } else if (WDT == DT_BF16) {
+            w[k] = __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short*>(p.W) + e) << 16);
+          } else {
+            w[k] = __half2float(__ushort_as_half(__ldg(reinterpret_cast<const unsigned short*>(p.W) + e)));
+          }
+          a[k] = a_decode<FMT>(p.a_store, i * p.nb + j / p.G);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < kXRows; ++k) {  // absent rows hold w = 0, which adds nothing
+        const float ia = __frcp_rn(a[k]);
+        const bool ok = in_range(cb) && in_range(ia);
+        const float q = quant<FMT>(w[k], w[k] * cb, ia, ok, a[k], bj, sTd);
+        const double sv = (double)q * (double)a[k];
+        cn = fma((double)w[k], sv, cn);
+        cd = fma(sv, sv, cd);
+      }
+    }
+    s_red[0][threadIdx.x] = cn;
+    s_red[1][threadIdx.x] = cd;
+    __syncthreads();
+    for (int o = kXThreads / 2; o > 0; o >>= 1) {
+      if (threadIdx.x < o) {
+        s_red[0][threadIdx.x] += s_red[0][threadIdx.x + o];
+        s_red[1][threadIdx.x] += s_red[1][threadIdx.x + o];
+      }
+      __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+      p.col_part[it] = make_double2(s_red[0][0], s_red[1][0]);
       __threadfence();
-      double tot = 0.0;
-      for (int64_t kk = 0; kk < p.P; ++kk) tot += __ldcg(&p.cta_part[kk]);
-      p.mse[t - 1] = tot / (rscale_d * rscale_d) / ((double)p.M * (double)p.N);
+      const unsigned prev = atomicAdd(&p.amb_tick[ci], 1u);
+      if (prev == (unsigned)R - 1u) {  // last chunk of this column: totals in chunk order
+        __threadfence();
+        double2 tot = make_double2(0.0, 0.0);
+        for (int64_t k = 0; k < R; ++k) {
+          const double2 v = __ldcg(&p.col_part[ci * R + k]);
+          tot.x += v.x;
+          tot.y += v.y;
+        }
+        const double v = FMT == FMT_NVFP4 ? (tot.x / tot.y) / sTd : tot.x / tot.y;
+        b_encode(p.b_store, p.col_dt, j, tot.y == 0.0 ? 1.0 : b_project(v, p.col_dt));
+        p.amb_tick[ci] = 0u;
+      }
+    }
+    __syncthreads();  // s_red is reused by the next item
+  }
+  // every CTA read n before arriving here; the last one empties the list
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const unsigned prev = atomicAdd(&p.hdr->cta_counter, 1u);
+    s_last = prev == gridDim.x - 1u ? 1 : 0;
+    if (s_last) {
+      p.hdr->amb_n = 0u;
       p.hdr->cta_counter = 0u;
     }
   }

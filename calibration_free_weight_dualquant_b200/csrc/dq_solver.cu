@@ -197,7 +197,11 @@ static cudaError_t run_typed(const Problem& p, int iters, int stats_ctas, cudaSt
     }
     k_init<FMT, WDT><<<stats_ctas, kThreads, 0, st>>>(pf);
   }
-  for (int t = 1; t <= iters; ++t) iter_kernel<<<(unsigned)p.P, kIterThreads, smem, st>>>(pi, t, wmap);
+  for (int t = 1; t <= iters; ++t) {
+    iter_kernel<<<(unsigned)p.P, kIterThreads, smem, st>>>(pi, t, wmap);
+    // the columns whose projection was ambiguous (usually none)
+    if (p.mode != DQ_MODE_ROW) k_col_exact<FMT, WDT><<<(unsigned)p.P, kXThreads, 0, st>>>(pi);
+  }
   k_iter<FMT, WDT, PASS_FINAL><<<(unsigned)p.P, kIterThreads, smem, st>>>(pi, iters + 1, wmap);
   return cudaGetLastError();
 }
