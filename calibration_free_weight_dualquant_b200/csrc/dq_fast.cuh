@@ -198,6 +198,16 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const void* map, int x, i
       : "memory");
 }
 
+// Programmatic dependent launch.  A grid launched with programmatic stream
+// serialization may start while the grid before it in the stream is still
+// running; griddep_wait() returns once every grid it depends on has completed
+// and its memory operations are visible, so it must come before the first
+// read of anything an earlier kernel wrote, in every CTA (a CTA that exits
+// without it would let the next grid overtake the unfinished one).
+// griddep_launch_dependents() lets the next grid begin launching early.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void consumer_sync(int nthreads) {
   asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
 }

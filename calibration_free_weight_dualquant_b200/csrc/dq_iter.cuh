@@ -186,7 +186,8 @@ template <int FMT>
 __device__ __forceinline__ void req_fast(const f2 u2[4], float a, const ColState& cs, float& ia, bool& ok, f2 q2[4],
                                          bool& near, bool& tie) {
   ia = rcp_approx(a);
-  ok = cs.ok && in_range(ia);
+  // fp16 a (INT4) and E4M3 e (NVFP4) keep 1/a inside [2^-50, 2^50]; 2^k may not
+  ok = cs.ok && (!fmt_pow2(FMT) || in_range(ia));
   near = !ok;
   tie = false;
   if (fmt_e2m1(FMT)) {
@@ -324,15 +325,14 @@ __device__ __forceinline__ void req_slow(const f2 w2[4], const f2 u2[4], float a
 template <int FMT>
 __device__ __forceinline__ void req_pair(const f2 wx[4], const f2 ux[4], float fa, bool actx, const f2 wy[4],
                                          const f2 uy[4], float fb, bool acty, const ColState& cs, float sT, double sTd,
-                                         f2 qx[4], f2 qy[4], unsigned* s_cnt) {
+                                         f2 qx[4], f2 qy[4], unsigned* s_cnt, unsigned& tcnt) {
   float iax, iay;
   bool okx, oky, nx, ny, tx, ty;
   req_fast<FMT>(ux, fa, cs, iax, okx, qx, nx, tx);
   req_fast<FMT>(uy, fb, cs, iay, oky, qy, ny, ty);
   nx = nx && actx;
   ny = ny && acty;
-  const int ties = __popc(__ballot_sync(0xffffffffu, tx && actx)) + __popc(__ballot_sync(0xffffffffu, ty && acty));
-  if (ties && (threadIdx.x & 31) == 0) atomicAdd(&s_cnt[3], (unsigned)ties);
+  tcnt += (unsigned)(tx && actx) + (unsigned)(ty && acty);  // lane-rows settled as certified ties
   if (nx || ny) {
     if (nx) {
       atomicAdd(&s_cnt[0], 1u);
@@ -371,30 +371,48 @@ __device__ __forceinline__ void smem_row(const unsigned char* src, f2 w2[4]) {
   }
 }
 
-// Block sums, residuals of the incoming iterate, for one row of one lane.
-// The residual W - a q b is taken with the product q b a exact inside fmas:
-// q b is exact in fp32, and so is a for INT4/MX; the NVFP4 factor a = e s_T is
-// split as hi + lo (hi = fl(e s_T), lo its exact rounding error), so the only
-// rounding is that of the (small) residual itself.
+// Block sums and residuals of the incoming iterate for the two rows of a lane
+// (x, y; an absent row holds zeros and adds nothing).  The residual W - a q b
+// is taken with the product q b a exact inside fmas: q b is exact in fp32, and
+// so is a for INT4/MX; the NVFP4 factor a = e s_T is split as hi + lo (hi =
+// fl(e s_T), lo its exact rounding error), so the only rounding is that of the
+// (small) residual itself.  With `scaled` the residual is multiplied by the
+// power of two rscale before it is squared (a W whose max |W| is far from 1);
+// otherwise its square cannot leave the fp32 range.
 template <int FMT>
-__device__ __forceinline__ void row_sums(const f2 w2[4], const f2 q2[4], float aold, const ColState& cs, float sT,
-                                         f2 rscale2, float& num, float& den, f2& res2) {
-  const float ahi = FMT == FMT_NVFP4 ? aold * sT : aold;
-  const f2 na2 = splat(-ahi);
-  const f2 nlo2 = splat(FMT == FMT_NVFP4 ? -fmaf(aold, sT, -ahi) : 0.f);
-  f2 num2 = 0ull, den2 = 0ull;
+__device__ __forceinline__ void row_sums2(const f2 wx[4], const f2 qx[4], float ax, const f2 wy[4], const f2 qy[4],
+                                          float ay, const ColState& cs, float sT, bool scaled, f2 rscale2, float& nx,
+                                          float& dx, float& ny, float& dy, f2& res2) {
+  const float axh = FMT == FMT_NVFP4 ? ax * sT : ax;
+  const float ayh = FMT == FMT_NVFP4 ? ay * sT : ay;
+  const f2 nax2 = splat(-axh), nay2 = splat(-ayh);
+  const f2 nlox2 = splat(FMT == FMT_NVFP4 ? -fmaf(ax, sT, -axh) : 0.f);
+  const f2 nloy2 = splat(FMT == FMT_NVFP4 ? -fmaf(ay, sT, -ayh) : 0.f);
+  f2 nx2 = 0ull, dx2 = 0ull, ny2 = 0ull, dy2 = 0ull;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const f2 pq = mul2(q2[i], col_ld(cs.tb, i, cs.lane));
-    num2 = fma2(w2[i], pq, num2);
-    den2 = fma2(pq, pq, den2);
-    f2 r = fma2(pq, na2, w2[i]);
-    if (FMT == FMT_NVFP4) r = fma2(pq, nlo2, r);
-    const f2 e = mul2(r, rscale2);  // residual times a power of two (range)
-    res2 = fma2(e, e, res2);
+    const f2 bi = col_ld(cs.tb, i, cs.lane);
+    const f2 px = mul2(qx[i], bi), py = mul2(qy[i], bi);
+    nx2 = fma2(wx[i], px, nx2);
+    dx2 = fma2(px, px, dx2);
+    ny2 = fma2(wy[i], py, ny2);
+    dy2 = fma2(py, py, dy2);
+    f2 rx = fma2(px, nax2, wx[i]), ry = fma2(py, nay2, wy[i]);
+    if (FMT == FMT_NVFP4) {
+      rx = fma2(px, nlox2, rx);
+      ry = fma2(py, nloy2, ry);
+    }
+    if (scaled) {
+      rx = mul2(rx, rscale2);
+      ry = mul2(ry, rscale2);
+    }
+    res2 = fma2(rx, rx, res2);
+    res2 = fma2(ry, ry, res2);
   }
-  num = lo_of(num2) + hi_of(num2);
-  den = lo_of(den2) + hi_of(den2);
+  nx = lo_of(nx2) + hi_of(nx2);
+  dx = lo_of(dx2) + hi_of(dx2);
+  ny = lo_of(ny2) + hi_of(ny2);
+  dy = lo_of(dy2) + hi_of(dy2);
 }
 
 // Exact fp64 block sums of one row of one lane (warp-collective reduction).
@@ -470,8 +488,8 @@ template <int FMT, int PASS>
 __device__ __forceinline__ void row_pair(const Problem& p, const f2 wx[4], float ax_old, int64_t bidx_x,
                                          const f2 wy[4], float ay_old, int64_t bidx_y, bool has_y, bool active,
                                          bool leader, int lpb, ColState& cs, float sT, float isT, double sTd,
-                                         f2 rscale2, unsigned* s_cnt, int64_t cix, uint32_t oldx, uint32_t oldy,
-                                         bool cmp, unsigned& nchg) {
+                                         bool scaled, f2 rscale2, unsigned* s_cnt, unsigned& tcnt, int64_t cix,
+                                         uint32_t oldx, uint32_t oldy, bool cmp, unsigned& nchg) {
   const bool actx = active, acty = active && has_y;
   f2 ux[4], uy[4], qx[4], qy[4];
 #pragma unroll
@@ -480,39 +498,61 @@ __device__ __forceinline__ void row_pair(const Problem& p, const f2 wx[4], float
     ux[i] = mul2(wx[i], cbi);
     uy[i] = mul2(wy[i], cbi);
   }
-  req_pair<FMT>(wx, ux, ax_old, actx, wy, uy, ay_old, acty, cs, sT, sTd, qx, qy, s_cnt);
+  req_pair<FMT>(wx, ux, ax_old, actx, wy, uy, ay_old, acty, cs, sT, sTd, qx, qy, s_cnt, tcnt);
   if (PASS == PASS_COUNT) track_codes<FMT>(p, qx, qy, actx, acty, cix, oldx, oldy, cmp, nchg);
   float nx, dx, ny, dy;
-  row_sums<FMT>(wx, qx, ax_old, cs, sT, rscale2, nx, dx, cs.res2);
-  row_sums<FMT>(wy, qy, ay_old, cs, sT, rscale2, ny, dy, cs.res2);
-  for (int o = 1; o < lpb; o <<= 1) {
-    nx += __shfl_xor_sync(0xffffffffu, nx, o);
-    dx += __shfl_xor_sync(0xffffffffu, dx, o);
-    ny += __shfl_xor_sync(0xffffffffu, ny, o);
-    dy += __shfl_xor_sync(0xffffffffu, dy, o);
-  }
-  bool ambx = false, amby = false;
-  float anx = a_fast<FMT>(nx, dx, isT, ambx);
-  float any = a_fast<FMT>(ny, dy, isT, amby);
-  ambx = ambx && actx;
-  amby = amby && acty;
+  row_sums2<FMT>(wx, qx, ax_old, wy, qy, ay_old, cs, sT, scaled, rscale2, nx, dx, ny, dy, cs.res2);
+  float anx, any;
   if (p.mode == DQ_MODE_COL) {  // column scales only: the block scales keep their values
     anx = ax_old;
     any = ay_old;
-    ambx = amby = false;
-  }
-  if (__any_sync(0xffffffffu, ambx || amby)) {
-    double n64, d64;
-    row_sums64(wx, qx, cs, lpb, n64, d64);
-    if (ambx) {
-      if (leader) atomicAdd(&s_cnt[1], 1u);
-      anx = d64 == 0.0 ? 1.f : (float)a_project<FMT>(n64 / d64, sTd);
+  } else if (lpb == 1) {  // a block within one lane: both rows here
+    bool ambx = false, amby = false;
+    anx = a_fast<FMT>(nx, dx, isT, ambx);
+    any = a_fast<FMT>(ny, dy, isT, amby);
+    ambx = ambx && actx;
+    amby = amby && acty;
+    if (__any_sync(0xffffffffu, ambx || amby)) {
+      double n64, d64;
+      row_sums64(wx, qx, cs, lpb, n64, d64);
+      if (ambx) {
+        atomicAdd(&s_cnt[1], 1u);
+        anx = d64 == 0.0 ? 1.f : (float)a_project<FMT>(n64 / d64, sTd);
+      }
+      row_sums64(wy, qy, cs, lpb, n64, d64);
+      if (amby) {
+        atomicAdd(&s_cnt[1], 1u);
+        any = d64 == 0.0 ? 1.f : (float)a_project<FMT>(n64 / d64, sTd);
+      }
     }
-    row_sums64(wy, qy, cs, lpb, n64, d64);
-    if (amby) {
-      if (leader) atomicAdd(&s_cnt[1], 1u);
-      any = d64 == 0.0 ? 1.f : (float)a_project<FMT>(n64 / d64, sTd);
+  } else {
+    // the lanes of a block split the two rows: even lanes finish row x, odd
+    // lanes row y (one reduce-scatter step, then the usual xor tree), so each
+    // lane projects one block value; the partner's result comes back by shuffle
+    const bool odd = (cs.lane & 1) != 0;
+    float kn = odd ? ny : nx, kd = odd ? dy : dx;
+    kn += __shfl_xor_sync(0xffffffffu, odd ? nx : ny, 1);
+    kd += __shfl_xor_sync(0xffffffffu, odd ? dx : dy, 1);
+    for (int o = 2; o < lpb; o <<= 1) {
+      kn += __shfl_xor_sync(0xffffffffu, kn, o);
+      kd += __shfl_xor_sync(0xffffffffu, kd, o);
     }
+    bool amb = false;
+    float an = a_fast<FMT>(kn, kd, isT, amb);
+    amb = amb && (odd ? acty : actx);
+    if (__any_sync(0xffffffffu, amb)) {
+      double n64x, d64x, n64y, d64y;
+      row_sums64(wx, qx, cs, lpb, n64x, d64x);
+      row_sums64(wy, qy, cs, lpb, n64y, d64y);
+      if (amb) {
+        if ((cs.lane & (lpb - 1)) <= 1) atomicAdd(&s_cnt[1], 1u);  // once per block row
+        const double n64 = odd ? n64y : n64x, d64 = odd ? d64y : d64x;
+        an = d64 == 0.0 ? 1.f : (float)a_project<FMT>(n64 / d64, sTd);
+      }
+    }
+    const float ao = __shfl_xor_sync(0xffffffffu, an, 1);
+    anx = odd ? ao : an;
+    any = odd ? an : ao;
   }
   // the storage already holds the old factors; with a block scale unchanged the
   // codes are unchanged too (same a, same b), so requantize only where it changed
@@ -527,7 +567,7 @@ __device__ __forceinline__ void row_pair(const Problem& p, const f2 wx[4], float
       ux[i] = mul2(wx[i], cbi);
       uy[i] = mul2(wy[i], cbi);
     }
-    req_pair<FMT>(wx, ux, anx, actx, wy, uy, any, acty, cs, sT, sTd, qx, qy, s_cnt);
+    req_pair<FMT>(wx, ux, anx, actx, wy, uy, any, acty, cs, sT, sTd, qx, qy, s_cnt, tcnt);
   }
   const f2 anx2 = splat(anx), any2 = splat(any);
 #pragma unroll
@@ -546,9 +586,9 @@ __device__ __forceinline__ void row_pair(const Problem& p, const f2 wx[4], float
 // residuals of that iterate for its MSE.
 template <int FMT>
 __device__ __forceinline__ void final_pair(const Problem& p, const f2 wx[4], float ax, const f2 wy[4], float ay,
-                                           bool has_y, bool active, ColState& cs, float sT, double sTd, f2 rscale2,
-                                           unsigned* s_cnt, int64_t cix, uint32_t oldx, uint32_t oldy, bool cmp,
-                                           unsigned& nchg) {
+                                           bool has_y, bool active, ColState& cs, float sT, double sTd, bool scaled,
+                                           f2 rscale2, unsigned* s_cnt, unsigned& tcnt, int64_t cix, uint32_t oldx,
+                                           uint32_t oldy, bool cmp, unsigned& nchg) {
   const bool actx = active, acty = active && has_y;
   f2 ux[4], uy[4], qx[4], qy[4];
 #pragma unroll
@@ -557,10 +597,9 @@ __device__ __forceinline__ void final_pair(const Problem& p, const f2 wx[4], flo
     ux[i] = mul2(wx[i], cbi);
     uy[i] = mul2(wy[i], cbi);
   }
-  req_pair<FMT>(wx, ux, ax, actx, wy, uy, ay, acty, cs, sT, sTd, qx, qy, s_cnt);
-  float n, d;  // block sums: not needed here
-  row_sums<FMT>(wx, qx, ax, cs, sT, rscale2, n, d, cs.res2);
-  row_sums<FMT>(wy, qy, ay, cs, sT, rscale2, n, d, cs.res2);
+  req_pair<FMT>(wx, ux, ax, actx, wy, uy, ay, acty, cs, sT, sTd, qx, qy, s_cnt, tcnt);
+  float nx, dx, ny, dy;  // block sums: not needed here
+  row_sums2<FMT>(wx, qx, ax, wy, qy, ay, cs, sT, scaled, rscale2, nx, dx, ny, dy, cs.res2);
   track_codes<FMT>(p, qx, qy, actx, acty, cix, oldx, oldy, cmp, nchg);
 }
 
@@ -592,7 +631,6 @@ __device__ __forceinline__ void flush_runs(ColState& cs, double2* acc, double* r
 // (and changes[T] when counting, T >= 1).
 template <int FMT, int WDT, int PASS>
 __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t, const __grid_constant__ CUtensorMap wmap) {
-  if (p.hdr->flags & kFlagAbort) return;
   constexpr int ES = WDT == DT_F32 ? 4 : 2;
   constexpr int S = ring_stages(ES);
   extern __shared__ __align__(128) unsigned char smem[];
@@ -618,6 +656,11 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t, cons
   }
   if (threadIdx.x < kConsumers) racc[threadIdx.x] = 0.0;
   __syncthreads();
+  // launched with programmatic stream serialization: what the kernels before
+  // wrote (flags, scales, counters) is read only after this wait
+  griddep_wait();
+  griddep_launch_dependents();
+  if (p.hdr->flags & kFlagAbort) return;
 
   const int64_t k = blockIdx.x;
   const int64_t u_begin = range_begin(k, p.P, p.L), u_end = range_begin(k + 1, p.P, p.L);
@@ -672,11 +715,14 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t, cons
   // ---------------- consumer warps ----------------
   const int lpb = p.G / 8;  // lanes per block
   const bool leader = (lane & (lpb - 1)) == 0;
-  // residuals are squared after scaling by rscale = 2^-floor(log2 amax), which
-  // keeps every square inside the fp32 range whatever the magnitude of W
+  // residuals are squared as they are when max |W| lies in [2^-8, 2^41) (no
+  // square of a residual can overflow, and none that underflows matters at the
+  // MSE's tolerance), otherwise after scaling by rscale = 2^-floor(log2 amax),
+  // which keeps every square inside the fp32 range whatever the magnitude of W
   const uint32_t amax_bits = p.hdr->amax_bits;
   const int amax_exp = (amax_bits == 0u) ? 0 : (int)((amax_bits >> 23) & 0xFFu) - 127;
-  const float rscale = __uint_as_float((uint32_t)(127 - max(-126, min(126, amax_exp))) << 23);
+  const bool scaled = amax_exp < -8 || amax_exp > 40;
+  const float rscale = scaled ? __uint_as_float((uint32_t)(127 - max(-126, min(126, amax_exp))) << 23) : 1.f;
   const f2 rscale2 = splat(rscale);
   const double rscale_d = (double)rscale;
   const float sT = p.hdr->sT;
@@ -693,6 +739,7 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t, cons
   const uint32_t* codes_old = reinterpret_cast<const uint32_t*>(p.codes);
   const int64_t code_step = (int64_t)kConsumerWarps * (p.N >> 3);  // code words between a warp's two rows
   unsigned nchg = 0u;
+  unsigned tcnt = 0u;  // lane-rows settled as certified exact ties
 
   for (int64_t u = u_begin; u < u_end;) {
     const int64_t s = u / p.M;
@@ -776,10 +823,11 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t, cons
           for (int i = 0; i < 4; ++i) wb[i] = 0ull;  // absent row: zeros contribute nothing
         }
         if (FIN) {
-          final_pair<FMT>(p, wa, aa, wb, ab, has_b, active, cs, sT, sTd, rscale2, s_cnt, cix, oldx, oldy, cmp, nchg);
+          final_pair<FMT>(p, wa, aa, wb, ab, has_b, active, cs, sT, sTd, scaled, rscale2, s_cnt, tcnt, cix, oldx,
+                          oldy, cmp, nchg);
         } else {
           row_pair<FMT, PASS>(p, wa, aa, aidx, wb, ab, aidx + kConsumerWarps * p.nb, has_b, active, leader, lpb, cs,
-                              sT, isT, sTd, rscale2, s_cnt, cix, oldx, oldy, cmp, nchg);
+                              sT, isT, sTd, scaled, rscale2, s_cnt, tcnt, cix, oldx, oldy, cmp, nchg);
         }
         run += has_b ? 2 : 1;
       }
@@ -864,6 +912,8 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t, cons
     u = (s + 1) * p.M;
   }
 
+  for (int o = 16; o > 0; o >>= 1) tcnt += __shfl_xor_sync(0xffffffffu, tcnt, o);
+  if (lane == 0 && tcnt) atomicAdd(&s_cnt[3], tcnt);  // read by thread 0 after the barriers below
   if (PASS != PASS_ITER && cmp) {  // changed codes of this warp, one atomic per warp
     for (int o = 16; o > 0; o >>= 1) nchg += __shfl_xor_sync(0xffffffffu, nchg, o);
     if (lane == 0 && nchg) atomicAdd(&p.changes[t - 1], (unsigned long long)nchg);
@@ -928,7 +978,8 @@ constexpr int kXRows = 8;
 template <int FMT, int WDT>
 __global__ void __launch_bounds__(kXThreads) k_col_exact(Problem p) {
   __shared__ double s_red[2][kXThreads];
-  __shared__ int s_last;
+  griddep_wait();  // launched with programmatic stream serialization: k_iter's list is read after this
+  griddep_launch_dependents();
   const unsigned n = p.hdr->amb_n;
   if (n == 0u) return;
   const double sTd = (double)p.hdr->sT;
@@ -1008,8 +1059,7 @@ __global__ void __launch_bounds__(kXThreads) k_col_exact(Problem p) {
   if (threadIdx.x == 0) {
     __threadfence();
     const unsigned prev = atomicAdd(&p.hdr->cta_counter, 1u);
-    s_last = prev == gridDim.x - 1u ? 1 : 0;
-    if (s_last) {
+    if (prev == gridDim.x - 1u) {
       p.hdr->amb_n = 0u;
       p.hdr->cta_counter = 0u;
     }

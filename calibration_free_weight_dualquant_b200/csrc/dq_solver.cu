@@ -164,6 +164,26 @@ static bool encode_w_map(const Problem& p, CUtensorMap* map) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Launch with programmatic stream serialization: the grid may start while the
+// one before it in the stream finishes (its prologue overlaps that grid's
+// tail); the kernel waits (griddep_wait) before it reads earlier results.
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem, cudaStream_t st,
+                              Args... args) {
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 template <int FMT, int WDT>
 static cudaError_t run_typed(const Problem& p, int iters, int stats_ctas, cudaStream_t st) {
   constexpr int ES = WDT == DT_F32 ? 4 : 2;
@@ -198,11 +218,16 @@ static cudaError_t run_typed(const Problem& p, int iters, int stats_ctas, cudaSt
     k_init<FMT, WDT><<<stats_ctas, kThreads, 0, st>>>(pf);
   }
   for (int t = 1; t <= iters; ++t) {
-    iter_kernel<<<(unsigned)p.P, kIterThreads, smem, st>>>(pi, t, wmap);
+    e = launch_pdl(iter_kernel, (unsigned)p.P, kIterThreads, smem, st, pi, t, wmap);
+    if (e != cudaSuccess) return e;
     // the columns whose projection was ambiguous (usually none)
-    if (p.mode != DQ_MODE_ROW) k_col_exact<FMT, WDT><<<(unsigned)p.P, kXThreads, 0, st>>>(pi);
+    if (p.mode != DQ_MODE_ROW) {
+      e = launch_pdl(k_col_exact<FMT, WDT>, (unsigned)p.P, kXThreads, 0, st, pi);
+      if (e != cudaSuccess) return e;
+    }
   }
-  k_iter<FMT, WDT, PASS_FINAL><<<(unsigned)p.P, kIterThreads, smem, st>>>(pi, iters + 1, wmap);
+  e = launch_pdl(k_iter<FMT, WDT, PASS_FINAL>, (unsigned)p.P, kIterThreads, smem, st, pi, iters + 1, wmap);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
