@@ -103,19 +103,28 @@ __device__ __forceinline__ f2 dec_e2m1x2(uint32_t code) {  // low nibble -> low 
   return pk(f.x, f.y);
 }
 
-// Block-scale factor from storage, decoded with the hardware where it can.
+// Stored block scale as loaded (fp16 bits or an 8-bit code), fetched a tile
+// ahead of its use and decoded only there, so the warp does not wait for the
+// load right after issuing it.
 template <int FMT>
-__device__ __forceinline__ float a_load(const void* store, int64_t idx) {
-  if (FMT == FMT_INT4) {
-    return __half2float(__ldg(reinterpret_cast<const __half*>(store) + idx));
-  } else if (fmt_pow2(FMT)) {
-    return __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned char*>(store) + idx) << 23);
-  } else {
-    const unsigned short v = __ldg(reinterpret_cast<const unsigned char*>(store) + idx);
-    uint32_t h;
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(v));
-    return __half2float(__ushort_as_half((unsigned short)(h & 0xFFFFu)));
-  }
+__device__ __forceinline__ uint32_t a_fetch(const void* store, int64_t idx) {
+  if (FMT == FMT_INT4) return __ldg(reinterpret_cast<const unsigned short*>(store) + idx);
+  return __ldg(reinterpret_cast<const unsigned char*>(store) + idx);
+}
+
+// the stored form of the factor 1 (fp16 1.0, 2^0, E4M3 1.0)
+template <int FMT>
+__device__ __forceinline__ constexpr uint32_t a_raw_one() {
+  return FMT == FMT_INT4 ? 0x3C00u : (fmt_pow2(FMT) ? 127u : 0x38u);
+}
+
+template <int FMT>
+__device__ __forceinline__ float a_dec(uint32_t v) {
+  if (FMT == FMT_INT4) return __half2float(__ushort_as_half((unsigned short)v));
+  if (fmt_pow2(FMT)) return __uint_as_float(v << 23);
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"((unsigned short)v));
+  return __half2float(__ushort_as_half((unsigned short)(h & 0xFFFFu)));
 }
 
 // Column table of the current strip in shared memory: colt[c][lane] holds
@@ -790,16 +799,16 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t, cons
     // block scales of this warp's rows, one tile ahead
     const int64_t a_step = (int64_t)kRowsPerTile * p.nb;
     int64_t aidx = (r0 + warp) * p.nb + blk_col;
-    float an0 = 1.f, an1 = 1.f;
-    if (active && r0 + warp < r1) an0 = a_load<FMT>(p.a_store, aidx);
-    if (active && r0 + warp + kConsumerWarps < r1) an1 = a_load<FMT>(p.a_store, aidx + kConsumerWarps * p.nb);
+    uint32_t an0 = a_raw_one<FMT>(), an1 = a_raw_one<FMT>();
+    if (active && r0 + warp < r1) an0 = a_fetch<FMT>(p.a_store, aidx);
+    if (active && r0 + warp + kConsumerWarps < r1) an1 = a_fetch<FMT>(p.a_store, aidx + kConsumerWarps * p.nb);
 
     for (int64_t tr = r0; tr < r1; tr += kRowsPerTile, aidx += a_step) {
       const int64_t ra = tr + warp, rb = ra + kConsumerWarps;
       const bool has_a = ra < r1, has_b = rb < r1;  // warp-uniform
-      const float aa = an0, ab = an1;
-      if (active && ra + kRowsPerTile < r1) an0 = a_load<FMT>(p.a_store, aidx + a_step);
-      if (active && rb + kRowsPerTile < r1) an1 = a_load<FMT>(p.a_store, aidx + a_step + kConsumerWarps * p.nb);
+      const uint32_t ra_raw = an0, rb_raw = an1;
+      if (active && ra + kRowsPerTile < r1) an0 = a_fetch<FMT>(p.a_store, aidx + a_step);
+      if (active && rb + kRowsPerTile < r1) an1 = a_fetch<FMT>(p.a_store, aidx + a_step + kConsumerWarps * p.nb);
       const int64_t cix = (ra * p.N + col) >> 3;  // code word of row ra, this lane's 8 columns
       uint32_t oldx = 0u, oldy = 0u;
       if (PASS != PASS_ITER && cmp && active) {  // issued before the wait: the latency hides behind it
@@ -818,6 +827,7 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t, cons
         par ^= 1u;
       }
       if (has_a) {
+        const float aa = a_dec<FMT>(ra_raw), ab = a_dec<FMT>(rb_raw);  // fetched a tile ago
         if (!has_b) {
 #pragma unroll
           for (int i = 0; i < 4; ++i) wb[i] = 0ull;  // absent row: zeros contribute nothing
