@@ -76,9 +76,9 @@ int make_plan(int64_t M, int64_t N, int group, int init, Plan* pl) {
   const size_t part_bytes = align_up(sizeof(double2) * (size_t)pl->P * (size_t)pl->segmax * (size_t)pl->TS);
   off += (init == DQ_INIT_L1 && l1_bytes > part_bytes) ? l1_bytes : part_bytes;
   pl->off_cta_part = off;
-  off += align_up(sizeof(double) * (size_t)(pl->P > pl->P_final ? pl->P : pl->P_final));
+  off += align_up(sizeof(double) * 3 * (size_t)(pl->P > pl->P_final ? pl->P : pl->P_final));
   pl->off_amb_list = off;
-  off += align_up(sizeof(int) * (size_t)N);
+  off += align_up(sizeof(int) * 2 * (size_t)N);
   pl->total = off;
   return DQ_OK;
 }

@@ -27,7 +27,8 @@ struct WsHeader {
   unsigned flags;        // kFlagNonFinite, kFlagTimeout, kFlagBadInit
   unsigned amax_bits;    // max |W| as fp32 bits
   unsigned cta_counter;  // arrival ticket for CTA-ordered totals
-  unsigned amb_n;        // columns listed for the exact column update (k_col_exact)
+  unsigned amb_n[2];     // columns listed for the exact column update, by iteration parity
+  unsigned gbar;         // arrivals at k_iter's grid-wide barrier
   float sT;              // NVFP4 tensor scale (1 otherwise)
   unsigned long long n_quant_tie;    // lane-rows with a certified exact tie settled on the fast path
   // diagnostics: how often the exact paths ran in the per-iteration passes
@@ -59,7 +60,7 @@ struct Problem {
   unsigned* strip_counter;  // [n_strips]
   double2* col_part;        // [P * segmax][TS] (sum W a q, sum (a q)^2)
   double* cta_part;         // [max(P, P_final)]
-  int* amb_list;            // [N] columns whose certified projection was ambiguous
+  int* amb_list;            // [2][N] columns whose certified projection was ambiguous, by iteration parity
   unsigned* amb_tick;       // [N] arrival counters of their row chunks (zeroed)
   int use_tmap;             // W streamed by 2-D tensor copies (else one bulk copy per row)
   int mode;                 // DQ_MODE_DUAL, DQ_MODE_ROW (b keeps its initial value) or DQ_MODE_COL

@@ -106,10 +106,18 @@ __device__ __forceinline__ f2 dec_e2m1x2(uint32_t code) {  // low nibble -> low 
 // Stored block scale as loaded (fp16 bits or an 8-bit code), fetched a tile
 // ahead of its use and decoded only there, so the warp does not wait for the
 // load right after issuing it.
+// Block scales are rewritten inside the kernel, so the load goes to L2
+// (ld.global.cg), never through the read-only or L1 path.
 template <int FMT>
 __device__ __forceinline__ uint32_t a_fetch(const void* store, int64_t idx) {
-  if (FMT == FMT_INT4) return __ldg(reinterpret_cast<const unsigned short*>(store) + idx);
-  return __ldg(reinterpret_cast<const unsigned char*>(store) + idx);
+  if (FMT == FMT_INT4) return __ldcg(reinterpret_cast<const unsigned short*>(store) + idx);
+  return __ldcg(reinterpret_cast<const unsigned char*>(store) + idx);
+}
+
+// Column scale from storage through L2 (other CTAs rewrite it inside the kernel).
+__device__ __forceinline__ float b_decode_cg(const void* store, int col_dt, int64_t j) {
+  const unsigned short h = __ldcg(reinterpret_cast<const unsigned short*>(store) + j);
+  return col_dt == DT_F16 ? __half2float(__ushort_as_half(h)) : __uint_as_float((uint32_t)h << 16);
 }
 
 // the stored form of the factor 1 (fp16 1.0, 2^0, E4M3 1.0)
@@ -632,14 +640,218 @@ __device__ __forceinline__ void flush_runs(ColState& cs, double2* acc, double* r
   cs.res2 = 0ull;
 }
 
-// One pass over W.  PASS_ITER: BCD iteration t (writes mse[t - 1], the MSE of
-// the incoming iterate).  PASS_COUNT: the same, and the incoming iterate's codes
-// replace those of the iterate before it in p.codes, the changed ones counted
-// into changes[t - 1] (t >= 2).  PASS_FINAL: the final pass after T iterations,
-// called with t = T + 1: the codes of the final iterate, packed, and mse[T]
-// (and changes[T] when counting, T >= 1).
+// ---------------------------------------------------------------------------
+// Grid-wide barrier of the consumer threads of every CTA.  k_iter is launched
+// cooperatively, so all its CTAs are resident at once.  Arrivals are counted
+// in hdr->gbar over the whole solve; a use waits for the next multiple of the
+// grid size.  The wait is bounded: it gives up after kGridSpinLimit polls (or
+// at once when some wait already gave up), records kFlagTimeout and goes on.
+constexpr unsigned kGridSpinLimit = 1u << 24;
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* a) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
+  return v;
+}
+
+// MSE of a finished pass from its per-CTA residual totals `part` (P values):
+// a fixed-order tree over the CTA index, so the value does not depend on which
+// CTA sums it.  Run by the consumer threads of one CTA; `red` holds kConsumers
+// doubles.
+__device__ void mse_total(const Problem& p, const double* part, double* out, double rscale_d, double* red) {
+  double v = 0.0;
+  for (int64_t kk = threadIdx.x; kk < p.P; kk += kConsumers) v += __ldcg(part + kk);
+  red[threadIdx.x] = v;
+  consumer_sync(kConsumers);
+  for (int o = kConsumerTreeTop; o > 0; o >>= 1) {
+    if (threadIdx.x < o && threadIdx.x + o < kConsumers) red[threadIdx.x] += red[threadIdx.x + o];
+    consumer_sync(kConsumers);
+  }
+  if (threadIdx.x == 0) *out = red[0] / (rscale_d * rscale_d) / ((double)p.M * (double)p.N);
+  consumer_sync(kConsumers);
+}
+
+// Per-CTA residual totals of pass t live in cta_part[(t % 3) P + k]: three
+// buffers, so the totals of pass t - 1 stay intact while pass t + 1 runs.
+__device__ __forceinline__ double* mse_part(const Problem& p, int t) { return p.cta_part + (int64_t)(t % 3) * p.P; }
+
+// Grid barrier at the end of pass t.  The first CTA to arrive has the most
+// time to spare: it sums the MSE of pass t - 1 (all of whose totals were
+// written before the barrier that ended it) while the others finish.
+__device__ void grid_sync(const Problem& p, int t, double rscale_d, double* red, int* s_flag) {
+  WsHeader* hdr = p.hdr;
+  consumer_sync(kConsumers);
+  unsigned target = 0u;
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const unsigned ticket = atomicAdd(&hdr->gbar, 1u);
+    target = (ticket / gridDim.x + 1u) * gridDim.x;
+    *s_flag = (ticket % gridDim.x == 0u && t >= 2) ? 1 : 0;
+  }
+  consumer_sync(kConsumers);
+  if (*s_flag) mse_total(p, mse_part(p, t - 1), p.mse + (t - 2), rscale_d, red);
+  if (threadIdx.x == 0) {
+    for (unsigned i = 0;; ++i) {
+      if ((int)(ld_acquire_gpu(&hdr->gbar) - target) >= 0) break;
+      if (i >= kGridSpinLimit || (*reinterpret_cast<volatile unsigned*>(&hdr->flags) & kFlagTimeout)) {
+        atomicOr(&hdr->flags, kFlagTimeout);
+        break;
+      }
+      __nanosleep(64);
+    }
+    __threadfence();
+  }
+  consumer_sync(kConsumers);
+}
+
+// Plain grid barrier (no MSE duty).
+__device__ void grid_sync_plain(WsHeader* hdr) {
+  consumer_sync(kConsumers);
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const unsigned ticket = atomicAdd(&hdr->gbar, 1u);
+    const unsigned target = (ticket / gridDim.x + 1u) * gridDim.x;
+    for (unsigned i = 0;; ++i) {
+      if ((int)(ld_acquire_gpu(&hdr->gbar) - target) >= 0) break;
+      if (i >= kGridSpinLimit || (*reinterpret_cast<volatile unsigned*>(&hdr->flags) & kFlagTimeout)) {
+        atomicOr(&hdr->flags, kFlagTimeout);
+        break;
+      }
+      __nanosleep(64);
+    }
+    __threadfence();
+  }
+  consumer_sync(kConsumers);
+}
+
+// Exact column update, at the start of pass t, of the columns that the strip
+// finalizers of pass t - 1 listed (their certified projection was ambiguous and
+// their scale still holds the previous value): sum W a q' and sum (a q')^2 in
+// fp64 over all rows, then b = Proj_Fb(ratio), 1 for a zero sum.  Each listed
+// column is cut into R row chunks; the CTAs of the grid take (column, chunk)
+// items, each consumer thread keeping the loads of kXRows rows in flight, and
+// a chunk's total is a fixed-order tree.  The last chunk of a column to arrive
+// adds the R chunk totals in chunk order, so the result does not depend on the
+// schedule.  A grid barrier then makes every new scale visible.  With an empty
+// list (the usual case) nothing happens and nobody waits.  Run by the consumer
+// threads; `scratch` holds 2 * kConsumers doubles.
+constexpr int kXRows = 8;
+constexpr int64_t kXMinRows = 32;  // rows of the smallest chunk
+
+template <int FMT, int WDT>
+__device__ void exact_listed(const Problem& p, int t, double sTd, float isT, double* scratch, int* s_flag) {
+  const int lb = (t - 1) & 1;
+  const unsigned n = __ldcg(&p.hdr->amb_n[lb]);
+  if (n == 0u) return;  // the same value in every CTA
+  const int* list = p.amb_list + (int64_t)lb * p.N;
+  // R chunks per column: enough items for every CTA of the grid (one short
+  // round of loads each), chunks of at least kXMinRows rows, and n * R
+  // partials must fit the column-partial buffer (free until the strips finish)
+  const int64_t cap = (int64_t)p.P * p.segmax * p.TS;
+  const int64_t R = max((int64_t)1, min(min((p.M + kXMinRows - 1) / kXMinRows, max((int64_t)1, (int64_t)p.P / (int64_t)n)),
+                                        cap / (int64_t)n));
+  const int64_t chunk = (p.M + R - 1) / R;
+  for (int64_t it = blockIdx.x; it < (int64_t)n * R; it += gridDim.x) {
+    const int64_t ci = it / R, r = it - ci * R;
+    const int64_t j = __ldcg(list + ci);
+    const float bj = b_decode_cg(p.b_store, p.col_dt, j);
+    const float cb = __frcp_rn(bj) * isT;
+    const int64_t i_end = min(p.M, (r + 1) * chunk);
+    double cn = 0.0, cd = 0.0;
+    for (int64_t i0 = r * chunk + threadIdx.x; i0 < i_end; i0 += (int64_t)kXRows * kConsumers) {
+      float w[kXRows];
+      uint32_t araw[kXRows];
+#pragma unroll
+      for (int k = 0; k < kXRows; ++k) {  // all loads first
+        const int64_t i = i0 + (int64_t)k * kConsumers;
+        w[k] = 0.f;
+        araw[k] = a_raw_one<FMT>();
+        if (i < i_end) {
+          const int64_t e = i * p.N + j;
+          if (WDT == DT_F32) {
+            w[k] = __ldg(reinterpret_cast<const float*>(p.W) + e);
+          } else if (WDT == DT_BF16) {
+            w[k] = __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short*>(p.W) + e) << 16);
+          } else {
+            w[k] = __half2float(__ushort_as_half(__ldg(reinterpret_cast<const unsigned short*>(p.W) + e)));
+          }
+          araw[k] = a_fetch<FMT>(p.a_store, i * p.nb + j / p.G);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < kXRows; ++k) {  // absent rows hold w = 0, which adds nothing
+        const float a = a_dec<FMT>(araw[k]);
+        const float ia = __frcp_rn(a);
+        const bool ok = in_range(cb) && in_range(ia);
+        const float q = quant<FMT>(w[k], w[k] * cb, ia, ok, a, bj, sTd);
+        const double sv = (double)q * (double)a;
+        cn = fma((double)w[k], sv, cn);
+        cd = fma(sv, sv, cd);
+      }
+    }
+    scratch[threadIdx.x] = cn;
+    scratch[kConsumers + threadIdx.x] = cd;
+    consumer_sync(kConsumers);
+    for (int o = kConsumerTreeTop; o > 0; o >>= 1) {  // fixed-order tree
+      if (threadIdx.x < o && threadIdx.x + o < kConsumers) {
+        scratch[threadIdx.x] += scratch[threadIdx.x + o];
+        scratch[kConsumers + threadIdx.x] += scratch[kConsumers + threadIdx.x + o];
+      }
+      consumer_sync(kConsumers);
+    }
+    if (threadIdx.x == 0) {
+      p.col_part[it] = make_double2(scratch[0], scratch[kConsumers]);
+      __threadfence();
+      const unsigned prev = atomicAdd(&p.amb_tick[ci], 1u);
+      *s_flag = prev == (unsigned)R - 1u ? 1 : 0;
+    }
+    consumer_sync(kConsumers);
+    if (*s_flag) {  // last chunk of this column: the chunk totals in a fixed-order tree
+      __threadfence();
+      double2 v = make_double2(0.0, 0.0);
+      for (int64_t k = threadIdx.x; k < R; k += kConsumers) {
+        const double2 c = __ldcg(&p.col_part[ci * R + k]);
+        v.x += c.x;
+        v.y += c.y;
+      }
+      scratch[threadIdx.x] = v.x;
+      scratch[kConsumers + threadIdx.x] = v.y;
+      consumer_sync(kConsumers);
+      for (int o = kConsumerTreeTop; o > 0; o >>= 1) {
+        if (threadIdx.x < o && threadIdx.x + o < kConsumers) {
+          scratch[threadIdx.x] += scratch[threadIdx.x + o];
+          scratch[kConsumers + threadIdx.x] += scratch[kConsumers + threadIdx.x + o];
+        }
+        consumer_sync(kConsumers);
+      }
+      if (threadIdx.x == 0) {
+        const double tn = scratch[0], td = scratch[kConsumers];
+        const double v = FMT == FMT_NVFP4 ? (tn / td) / sTd : tn / td;
+        b_encode(p.b_store, p.col_dt, j, td == 0.0 ? 1.0 : b_project(v, p.col_dt));
+        p.amb_tick[ci] = 0u;
+      }
+    }
+    consumer_sync(kConsumers);  // the scratch and the flag are reused by the next item
+  }
+  grid_sync_plain(p.hdr);
+  // every CTA read n before the barrier; the list is written again two passes later
+  if (blockIdx.x == 0 && threadIdx.x == 0) p.hdr->amb_n[lb] = 0u;
+}
+
+// Passes t = t_first .. t_last over W, one read of W each, in one persistent
+// launch (cooperative: a grid barrier separates consecutive passes, so pass
+// t + 1 reads the scales that pass t wrote; the producer warp streams W on
+// across the barriers).  PASS_ITER: BCD iteration t (writes mse[t - 1], the
+// MSE of the incoming iterate).  PASS_COUNT: the same, and the incoming
+// iterate's codes replace those of the iterate before it in p.codes, the
+// changed ones counted into changes[t - 1] (t >= 2).  PASS_FINAL: the final
+// pass after T iterations, called with t_first = t_last = T + 1: the codes of
+// the final iterate, packed, and mse[T] (and changes[T] when counting, T >= 1).
+// Every pass starts with the exact update of the columns that the pass before
+// left ambiguous (exact_listed).
 template <int FMT, int WDT, int PASS>
-__global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t, const __grid_constant__ CUtensorMap wmap) {
+__global__ void __launch_bounds__(kIterThreads, 1)
+    k_iter(Problem p, int t_first, int t_last, const __grid_constant__ CUtensorMap wmap) {
   constexpr int ES = WDT == DT_F32 ? 4 : 2;
   constexpr int S = ring_stages(ES);
   extern __shared__ __align__(128) unsigned char smem[];
@@ -678,6 +890,7 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t, cons
     // ---------------- producer warp ----------------
     int st = 0;
     unsigned par = 1u;
+    for (int t = t_first; t <= t_last; ++t)  // the same tiles, pass after pass
     for (int64_t u = u_begin; u < u_end;) {
       const int64_t s = u / p.M;
       const int64_t r0 = u - s * p.M;
@@ -743,12 +956,21 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t, cons
   int st = 0;
   unsigned par = 0u;
   constexpr bool FIN = PASS == PASS_FINAL;
-  // compare with the previous iterate's codes (kept in p.codes by the pass before)
-  const bool cmp = (PASS == PASS_COUNT || (FIN && p.changes != nullptr)) && t > 1;
   const uint32_t* codes_old = reinterpret_cast<const uint32_t*>(p.codes);
   const int64_t code_step = (int64_t)kConsumerWarps * (p.N >> 3);  // code words between a warp's two rows
-  unsigned nchg = 0u;
   unsigned tcnt = 0u;  // lane-rows settled as certified exact ties
+
+  for (int t = t_first; t <= t_last; ++t) {
+  exact_listed<FMT, WDT>(p, t, sTd, isT, reinterpret_cast<double*>(acc), &s_misc[0]);
+  if (FIN && blockIdx.x == 0) {
+    // the MSE of the passes that no grid barrier of the iteration launch summed
+    for (int tp = max(1, t - 2); tp <= t - 1; ++tp)
+      mse_total(p, mse_part(p, tp), p.mse + (tp - 1), rscale_d, reinterpret_cast<double*>(acc));
+  }
+  racc[threadIdx.x] = 0.0;
+  // compare with the previous iterate's codes (kept in p.codes by the pass before)
+  const bool cmp = (PASS == PASS_COUNT || (FIN && p.changes != nullptr)) && t > 1;
+  unsigned nchg = 0u;
 
   for (int64_t u = u_begin; u < u_end;) {
     const int64_t s = u / p.M;
@@ -776,7 +998,7 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t, cons
         const int c = 2 * i + h;
         cs.thr[c] = 0.5f - kGuard;
         if (active) {
-          bj[h] = b_decode(p.b_store, p.col_dt, col + c);
+          bj[h] = b_decode_cg(p.b_store, p.col_dt, col + c);
           cb[h] = __frcp_rn(bj[h]) * isT;
           cs.ok = cs.ok && in_range(cb[h]);
           b_bits = max(b_bits, sig_bits(bj[h]));
@@ -905,12 +1127,12 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t, cons
         if (lo == hi) {
           bnew = lo;
         } else {
-          // ambiguous: listed for k_col_exact, which recomputes the column's
-          // sums exactly over all rows and writes its scale (b keeps its value
-          // until then)
+          // ambiguous: listed for the exact update at the start of the next
+          // pass (exact_listed), which recomputes the column's sums over all
+          // rows and writes its scale (b keeps its value until then)
           amb = true;
           atomicAdd(&s_misc[1], 1);
-          p.amb_list[atomicAdd(&p.hdr->amb_n, 1u)] = (int)(c0 + threadIdx.x);
+          p.amb_list[(int64_t)(t & 1) * p.N + atomicAdd(&p.hdr->amb_n[t & 1], 1u)] = (int)(c0 + threadIdx.x);
         }
       }
       consumer_sync(kConsumers);
@@ -922,8 +1144,6 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t, cons
     u = (s + 1) * p.M;
   }
 
-  for (int o = 16; o > 0; o >>= 1) tcnt += __shfl_xor_sync(0xffffffffu, tcnt, o);
-  if (lane == 0 && tcnt) atomicAdd(&s_cnt[3], tcnt);  // read by thread 0 after the barriers below
   if (PASS != PASS_ITER && cmp) {  // changed codes of this warp, one atomic per warp
     for (int o = 16; o > 0; o >>= 1) nchg += __shfl_xor_sync(0xffffffffu, nchg, o);
     if (lane == 0 && nchg) atomicAdd(&p.changes[t - 1], (unsigned long long)nchg);
@@ -942,138 +1162,36 @@ __global__ void __launch_bounds__(kIterThreads, 1) k_iter(Problem p, int t, cons
     consumer_sync(kConsumers);
   }
   if (threadIdx.x == 0) {
+    mse_part(p, t)[k] = mred[0];
+    if (FIN) {  // no barrier follows the final pass: the last CTA to finish sums its MSE
+      __threadfence();
+      const unsigned prev = atomicAdd(&p.hdr->cta_counter, 1u);
+      s_misc[0] = prev == (unsigned)p.P - 1u ? 1 : 0;
+    }
+  }
+  if (FIN) {
+    consumer_sync(kConsumers);
+    if (s_misc[0]) {
+      __threadfence();
+      mse_total(p, mse_part(p, t), p.mse + (t - 1), rscale_d, mred);
+      if (threadIdx.x == 0) p.hdr->cta_counter = 0u;
+    }
+  }
+  // the scales of pass t (except the listed columns) are final before pass
+  // t + 1 reads them
+  if (t < t_last) grid_sync(p, t, rscale_d, mred, &s_misc[0]);
+  }  // passes
+
+  for (int o = 16; o > 0; o >>= 1) tcnt += __shfl_xor_sync(0xffffffffu, tcnt, o);
+  if (lane == 0 && tcnt) atomicAdd(&s_cnt[3], tcnt);
+  consumer_sync(kConsumers);
+  if (threadIdx.x == 0) {
     if (s_cnt[0]) atomicAdd(&p.hdr->n_quant_exact, (unsigned long long)s_cnt[0]);
     if (s_cnt[1]) atomicAdd(&p.hdr->n_block_exact, (unsigned long long)s_cnt[1]);
     if (s_cnt[2]) atomicAdd(&p.hdr->n_col_exact, (unsigned long long)s_cnt[2]);
     if (s_cnt[3]) atomicAdd(&p.hdr->n_quant_tie, (unsigned long long)s_cnt[3]);
-    p.cta_part[k] = mred[0];
-    __threadfence();
-    const unsigned prev = atomicAdd(&p.hdr->cta_counter, 1u);
-    s_misc[0] = prev == (unsigned)p.P - 1u ? 1 : 0;
-  }
-  consumer_sync(kConsumers);
-  if (s_misc[0]) {
-    // the last CTA: the per-CTA partials in a fixed-order tree (one load per
-    // thread in flight at once, instead of a chain of P dependent additions)
-    __threadfence();
-    double v = 0.0;
-    for (int64_t kk = threadIdx.x; kk < p.P; kk += kConsumers) v += __ldcg(&p.cta_part[kk]);
-    mred[threadIdx.x] = v;
-    consumer_sync(kConsumers);
-    for (int o = kConsumerTreeTop; o > 0; o >>= 1) {
-      if (threadIdx.x < o && threadIdx.x + o < kConsumers) mred[threadIdx.x] += mred[threadIdx.x + o];
-      consumer_sync(kConsumers);
-    }
-    if (threadIdx.x == 0) {
-      p.mse[t - 1] = mred[0] / (rscale_d * rscale_d) / ((double)p.M * (double)p.N);
-      p.hdr->cta_counter = 0u;
-    }
   }
 }
 
-
-// ---------------------------------------------------------------------------
-// Exact column update of the columns that the k_iter launch just before listed
-// (their certified projection was ambiguous and their scale still holds the
-// value of the iterate): sum W a q' and sum (a q')^2 in fp64 over all rows,
-// then b = Proj_Fb(ratio), 1 for a zero sum.  Each listed column is cut into R
-// row chunks; a CTA takes (column, chunk) items, each thread keeps the loads
-// of kXRows rows in flight, and the chunk total is a fixed-order tree.  The
-// last chunk of a column to arrive adds the R chunk totals in chunk order, so
-// the result does not depend on the schedule.  With an empty list every CTA
-// returns at once.  The last CTA to finish empties the list.
-constexpr int kXThreads = 256;
-constexpr int kXRows = 8;
-
-template <int FMT, int WDT>
-__global__ void __launch_bounds__(kXThreads) k_col_exact(Problem p) {
-  __shared__ double s_red[2][kXThreads];
-  griddep_wait();  // launched with programmatic stream serialization: k_iter's list is read after this
-  griddep_launch_dependents();
-  const unsigned n = p.hdr->amb_n;
-  if (n == 0u) return;
-  const double sTd = (double)p.hdr->sT;
-  const float isT = FMT == FMT_NVFP4 ? (float)(1.0 / sTd) : 1.f;
-  // R chunks per column: about kXThreads * kXRows rows each, and n * R
-  // partials must fit the column-partial buffer of k_iter (free by now)
-  const int64_t cap = (int64_t)p.P * p.segmax * p.TS;
-  const int64_t chunk_want = (int64_t)kXThreads * kXRows;
-  const int64_t R = max((int64_t)1, min((p.M + chunk_want - 1) / chunk_want, cap / (int64_t)n));
-  const int64_t chunk = (p.M + R - 1) / R;
-  for (int64_t it = blockIdx.x; it < (int64_t)n * R; it += gridDim.x) {
-    const int64_t ci = it / R, r = it - ci * R;
-    const int64_t j = p.amb_list[ci];
-    const float bj = b_decode(p.b_store, p.col_dt, j);
-    const float cb = __frcp_rn(bj) * isT;
-    const int64_t i_end = min(p.M, (r + 1) * chunk);
-    double cn = 0.0, cd = 0.0;
-    for (int64_t i0 = r * chunk + threadIdx.x; i0 < i_end; i0 += (int64_t)kXRows * kXThreads) {
-      float w[kXRows], a[kXRows];
-#pragma unroll
-      for (int k = 0; k < kXRows; ++k) {  // all loads first
-        const int64_t i = i0 + (int64_t)k * kXThreads;
-        w[k] = 0.f;
-        a[k] = 1.f;
-        if (i < i_end) {
-          const int64_t e = i * p.N + j;
-          if (WDT == DT_F32) {
-            w[k] = __ldg(reinterpret_cast<const float*>(p.W) + e);
-          } else if (WDT == DT_BF16) {
-            w[k] = __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short*>(p.W) + e) << 16);
-          } else {
-            w[k] = __half2float(__ushort_as_half(__ldg(reinterpret_cast<const unsigned short*>(p.W) + e)));
-          }
-          a[k] = a_decode<FMT>(p.a_store, i * p.nb + j / p.G);
-        }
-      }
-#pragma unroll
-      for (int k = 0; k < kXRows; ++k) {  // absent rows hold w = 0, which adds nothing
-        const float ia = __frcp_rn(a[k]);
-        const bool ok = in_range(cb) && in_range(ia);
-        const float q = quant<FMT>(w[k], w[k] * cb, ia, ok, a[k], bj, sTd);
-        const double sv = (double)q * (double)a[k];
-        cn = fma((double)w[k], sv, cn);
-        cd = fma(sv, sv, cd);
-      }
-    }
-    s_red[0][threadIdx.x] = cn;
-    s_red[1][threadIdx.x] = cd;
-    __syncthreads();
-    for (int o = kXThreads / 2; o > 0; o >>= 1) {
-      if (threadIdx.x < o) {
-        s_red[0][threadIdx.x] += s_red[0][threadIdx.x + o];
-        s_red[1][threadIdx.x] += s_red[1][threadIdx.x + o];
-      }
-      __syncthreads();
-    }
-    if (threadIdx.x == 0) {
-      p.col_part[it] = make_double2(s_red[0][0], s_red[1][0]);
-      __threadfence();
-      const unsigned prev = atomicAdd(&p.amb_tick[ci], 1u);
-      if (prev == (unsigned)R - 1u) {  // last chunk of this column: totals in chunk order
-        __threadfence();
-        double2 tot = make_double2(0.0, 0.0);
-        for (int64_t k = 0; k < R; ++k) {
-          const double2 v = __ldcg(&p.col_part[ci * R + k]);
-          tot.x += v.x;
-          tot.y += v.y;
-        }
-        const double v = FMT == FMT_NVFP4 ? (tot.x / tot.y) / sTd : tot.x / tot.y;
-        b_encode(p.b_store, p.col_dt, j, tot.y == 0.0 ? 1.0 : b_project(v, p.col_dt));
-        p.amb_tick[ci] = 0u;
-      }
-    }
-    __syncthreads();  // s_red is reused by the next item
-  }
-  // every CTA read n before arriving here; the last one empties the list
-  if (threadIdx.x == 0) {
-    __threadfence();
-    const unsigned prev = atomicAdd(&p.hdr->cta_counter, 1u);
-    if (prev == gridDim.x - 1u) {
-      p.hdr->amb_n = 0u;
-      p.hdr->cta_counter = 0u;
-    }
-  }
-}
 
 }  // namespace dq

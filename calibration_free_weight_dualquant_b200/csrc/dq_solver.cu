@@ -11,13 +11,13 @@
 //   scale 1 for an all-zero code slice; codes are a function of (W, a, b).
 //
 // Launches per solve: k_stats (non-finite check, max |W|), k_init (scales of
-// the initial iterate), T x k_iter (one BCD iteration each, one read of W), and
-// k_iter in its final mode (codes of the final iterate and the last MSE, one
-// more read of W).  k_iter (dq_iter.cuh) runs one persistent CTA per SM over
-// contiguous ranges of strip-major (strip, row) units, so every CTA streams
-// the same number of rows; the column totals and the MSE are summed in CTA
-// order by the last CTA to arrive (an atomic ticket, never a wait), so every
-// result is deterministic.
+// the initial iterate), one k_iter running all T BCD iterations (one read of W
+// each, a grid barrier between them), and k_iter in its final mode (codes of
+// the final iterate and the last MSE, one more read of W).  k_iter
+// (dq_iter.cuh) runs one CTA per SM over contiguous ranges of strip-major
+// (strip, row) units, so every CTA streams the same number of rows; the column
+// totals and the MSE are summed in CTA order by the last CTA to arrive (an
+// atomic ticket), so every result is deterministic.
 #include <cudaTypedefs.h>  // PFN_cuTensorMapEncodeTiled
 
 #include <algorithm>
@@ -164,24 +164,34 @@ static bool encode_w_map(const Problem& p, CUtensorMap* map) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Launch with programmatic stream serialization: the grid may start while the
-// one before it in the stream finishes (its prologue overlaps that grid's
-// tail); the kernel waits (griddep_wait) before it reads earlier results.
+// Launch of k_iter: cooperative (all CTAs resident at once, for its grid
+// barrier) and with programmatic stream serialization (the grid may start while
+// the one before it in the stream finishes; the kernel waits, griddep_wait,
+// before it reads earlier results).  Where the runtime refuses the two
+// attributes together, the launch is cooperative alone.
 template <typename... KArgs, typename... Args>
-static cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem, cudaStream_t st,
-                              Args... args) {
+static cudaError_t launch_coop(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem, cudaStream_t st,
+                               Args... args) {
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(block);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, args...);
+  cfg.numAttrs = 2;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  if (e == cudaErrorInvalidValue || e == cudaErrorNotSupported) {
+    (void)cudaGetLastError();  // a refused configuration is not a sticky error
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  }
+  return e;
 }
 
 template <int FMT, int WDT>
@@ -217,16 +227,12 @@ static cudaError_t run_typed(const Problem& p, int iters, int stats_ctas, cudaSt
     }
     k_init<FMT, WDT><<<stats_ctas, kThreads, 0, st>>>(pf);
   }
-  for (int t = 1; t <= iters; ++t) {
-    e = launch_pdl(iter_kernel, (unsigned)p.P, kIterThreads, smem, st, pi, t, wmap);
+  // all BCD iterations in one persistent launch, then the final pass
+  if (iters > 0) {
+    e = launch_coop(iter_kernel, (unsigned)p.P, kIterThreads, smem, st, pi, 1, iters, wmap);
     if (e != cudaSuccess) return e;
-    // the columns whose projection was ambiguous (usually none)
-    if (p.mode != DQ_MODE_ROW) {
-      e = launch_pdl(k_col_exact<FMT, WDT>, (unsigned)p.P, kXThreads, 0, st, pi);
-      if (e != cudaSuccess) return e;
-    }
   }
-  e = launch_pdl(k_iter<FMT, WDT, PASS_FINAL>, (unsigned)p.P, kIterThreads, smem, st, pi, iters + 1, wmap);
+  e = launch_coop(k_iter<FMT, WDT, PASS_FINAL>, (unsigned)p.P, kIterThreads, smem, st, pi, iters + 1, iters + 1, wmap);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
