@@ -15,7 +15,7 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 struct Plan {
   int TS, n_strips, P, segmax, P_final, segmax_final, nb;
   int64_t L;
-  size_t off_counters, off_amb_tick, off_col_part, off_cta_part, off_amb_list, total;
+  size_t off_counters, off_amb_tick, off_sx_left, off_col_part, off_cta_part, off_amb_list, off_xpart, total;
   size_t l1_zero_bytes;  // L1 init: digit counters to zero (start of the col_part region)
   size_t off_l1_tot, off_l1_norm;
 };
@@ -63,6 +63,8 @@ int make_plan(int64_t M, int64_t N, int group, int init, Plan* pl) {
   off += align_up(sizeof(unsigned) * (size_t)pl->n_strips);
   pl->off_amb_tick = off;
   off += align_up(sizeof(unsigned) * (size_t)N);
+  pl->off_sx_left = off;
+  off += align_up(sizeof(unsigned) * (size_t)pl->n_strips);
   pl->off_col_part = off;
   // the L1-init scratch overlays the column partials (the init kernels run
   // before the first iteration): per-column digits, the total's digits, norms;
@@ -78,7 +80,9 @@ int make_plan(int64_t M, int64_t N, int group, int init, Plan* pl) {
   pl->off_cta_part = off;
   off += align_up(sizeof(double) * 3 * (size_t)(pl->P > pl->P_final ? pl->P : pl->P_final));
   pl->off_amb_list = off;
-  off += align_up(sizeof(int) * 2 * (size_t)N);
+  off += align_up(sizeof(int) * 3 * (size_t)N);
+  pl->off_xpart = off;
+  off += align_up(sizeof(double2) * (size_t)dq::kXPartCap);
   pl->total = off;
   return DQ_OK;
 }
@@ -157,6 +161,8 @@ int solve_impl(const void* W, int w_dtype, int64_t rows, int64_t cols, int forma
   p.cta_part = reinterpret_cast<double*>(ws + pl.off_cta_part);
   p.amb_list = reinterpret_cast<int*>(ws + pl.off_amb_list);
   p.amb_tick = reinterpret_cast<unsigned*>(ws + pl.off_amb_tick);
+  p.sx_left = reinterpret_cast<unsigned*>(ws + pl.off_sx_left);
+  p.xpart = reinterpret_cast<double2*>(ws + pl.off_xpart);
 
   // header and arrival counters (strips, listed columns) start at zero; the
   // partial buffers and the column list need no init

@@ -17,6 +17,7 @@ constexpr int64_t kMinRowsPerCta = 64;
 // 32-bit digits of an exact magnitude sum in units of 2^-149 (L1 init): one
 // value reaches bit 277, a sum of up to 2^31 values bit 308
 constexpr int kXDigits = 10;
+constexpr int64_t kXPartCap = 32768;  // entries of the exact-update partial buffer
 constexpr unsigned kFlagNonFinite = 1u;
 constexpr unsigned kFlagTimeout = 2u;  // a bounded pipeline wait gave up (results invalid)
 constexpr unsigned kFlagBadInit = 4u;  // a warm start was given an inadmissible scale
@@ -27,7 +28,7 @@ struct WsHeader {
   unsigned flags;        // kFlagNonFinite, kFlagTimeout, kFlagBadInit
   unsigned amax_bits;    // max |W| as fp32 bits
   unsigned cta_counter;  // arrival ticket for CTA-ordered totals
-  unsigned amb_n[2];     // columns listed for the exact column update, by iteration parity
+  unsigned amb_n[3];     // columns listed for the exact column update, by pass mod 3
   unsigned gbar;         // arrivals at k_iter's grid-wide barrier
   float sT;              // NVFP4 tensor scale (1 otherwise)
   unsigned long long n_quant_tie;    // lane-rows with a certified exact tie settled on the fast path
@@ -60,8 +61,10 @@ struct Problem {
   unsigned* strip_counter;  // [n_strips]
   double2* col_part;        // [P * segmax][TS] (sum W a q, sum (a q)^2)
   double* cta_part;         // [max(P, P_final)]
-  int* amb_list;            // [2][N] columns whose certified projection was ambiguous, by iteration parity
+  int* amb_list;            // [3][N] columns whose certified projection was ambiguous, by pass mod 3
   unsigned* amb_tick;       // [N] arrival counters of their row chunks (zeroed)
+  unsigned* sx_left;        // [n_strips] listed columns of a strip still awaiting their exact update (zeroed)
+  double2* xpart;           // [kXPartCap] per-CTA exact partial sums of the listed columns
   int use_tmap;             // W streamed by 2-D tensor copies (else one bulk copy per row)
   int mode;                 // DQ_MODE_DUAL, DQ_MODE_ROW (b keeps its initial value) or DQ_MODE_COL
   int init;                 // DQ_INIT_RTN, DQ_INIT_L1 or DQ_INIT_GIVEN

@@ -727,115 +727,167 @@ __device__ void grid_sync_plain(WsHeader* hdr) {
 // Exact column update, at the start of pass t, of the columns that the strip
 // finalizers of pass t - 1 listed (their certified projection was ambiguous and
 // their scale still holds the previous value): sum W a q' and sum (a q')^2 in
-// fp64 over all rows, then b = Proj_Fb(ratio), 1 for a zero sum.  Each listed
-// column is cut into R row chunks; the CTAs of the grid take (column, chunk)
-// items, each consumer thread keeping the loads of kXRows rows in flight, and
-// a chunk's total is a fixed-order tree.  The last chunk of a column to arrive
-// adds the R chunk totals in chunk order, so the result does not depend on the
-// schedule.  A grid barrier then makes every new scale visible.  With an empty
-// list (the usual case) nothing happens and nobody waits.  Run by the consumer
-// threads; `scratch` holds 2 * kConsumers doubles.
+// fp64 over all rows, then b = Proj_Fb(ratio), 1 for a zero sum.
+//
+// Each listed column is cut into R row chunks and the (column, chunk) items
+// are spread over all CTAs of the grid (about one each), so the update costs
+// one short round of loads per CTA.  A chunk's total is a fixed-order
+// reduction over the consumer threads; the last chunk of a column to arrive
+// adds the R chunk totals in chunk order (the result does not depend on the
+// schedule), writes the scale and counts the strip's p.sx_left down.  A CTA
+// reaching a strip with listed columns waits for that count to reach zero
+// (wait_strip); nobody else waits.  When the list is too long for p.xpart the
+// chunk totals go to p.col_part instead and a grid barrier follows (then no
+// strip waits).  Run by the consumer threads; `scratch` holds 2 * kConsumers
+// doubles.
 constexpr int kXRows = 8;
 constexpr int64_t kXMinRows = 32;  // rows of the smallest chunk
 
+// Fixed-order sum of one value per consumer thread (xor trees within the warps,
+// then the warp totals in warp order); the total is in red[0] afterwards.
+__device__ __forceinline__ void consumer_sum2(double x, double y, double* red) {
+  for (int o = 16; o > 0; o >>= 1) {
+    x += __shfl_xor_sync(0xffffffffu, x, o);
+    y += __shfl_xor_sync(0xffffffffu, y, o);
+  }
+  const int warp = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) {
+    red[2 + 2 * warp] = x;
+    red[3 + 2 * warp] = y;
+  }
+  consumer_sync(kConsumers);
+  if (threadIdx.x == 0) {
+    double sx = 0.0, sy = 0.0;
+    for (int w = 0; w < kConsumerWarps; ++w) {
+      sx += red[2 + 2 * w];
+      sy += red[3 + 2 * w];
+    }
+    red[0] = sx;
+    red[1] = sy;
+  }
+}
+
+// fp64 sums of W a q and (a q)^2 of column j over rows [i_begin, i_end)
+// (every load issued before any is used); the totals go to scratch[0], [1]
+// (thread 0; the caller synchronizes before others read them).
 template <int FMT, int WDT>
-__device__ void exact_listed(const Problem& p, int t, double sTd, float isT, double* scratch, int* s_flag) {
-  const int lb = (t - 1) & 1;
+__device__ void column_rows_exact(const Problem& p, int64_t j, int64_t i_begin, int64_t i_end, double sTd, float isT,
+                                  double* scratch) {
+  const unsigned short braw = __ldcg(reinterpret_cast<const unsigned short*>(p.b_store) + j);
+  double cn = 0.0, cd = 0.0;
+  for (int64_t i0 = i_begin + threadIdx.x; i0 < i_end; i0 += (int64_t)kXRows * kConsumers) {
+    float w[kXRows];
+    uint32_t araw[kXRows];
+#pragma unroll
+    for (int k = 0; k < kXRows; ++k) {
+      const int64_t i = i0 + (int64_t)k * kConsumers;
+      w[k] = 0.f;
+      araw[k] = a_raw_one<FMT>();
+      if (i < i_end) {
+        const int64_t e = i * p.N + j;
+        if (WDT == DT_F32) {
+          w[k] = __ldg(reinterpret_cast<const float*>(p.W) + e);
+        } else if (WDT == DT_BF16) {
+          w[k] = __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short*>(p.W) + e) << 16);
+        } else {
+          w[k] = __half2float(__ushort_as_half(__ldg(reinterpret_cast<const unsigned short*>(p.W) + e)));
+        }
+        araw[k] = a_fetch<FMT>(p.a_store, i * p.nb + j / p.G);
+      }
+    }
+    const float bj = p.col_dt == DT_F16 ? __half2float(__ushort_as_half(braw)) : __uint_as_float((uint32_t)braw << 16);
+    const float cb = __frcp_rn(bj) * isT;
+#pragma unroll
+    for (int k = 0; k < kXRows; ++k) {  // absent rows hold w = 0, which adds nothing
+      const float a = a_dec<FMT>(araw[k]);
+      const float ia = __frcp_rn(a);
+      const bool ok = in_range(cb) && in_range(ia);
+      const float q = quant<FMT>(w[k], w[k] * cb, ia, ok, a, bj, sTd);
+      const double sv = (double)q * (double)a;
+      cn = fma((double)w[k], sv, cn);
+      cd = fma(sv, sv, cd);
+    }
+  }
+  consumer_sum2(cn, cd, scratch);
+}
+
+// The last contributor to a listed column: adds the `cnt` chunk totals in
+// order and writes the projected scale (consumer threads; thread 0 writes).
+template <int FMT>
+__device__ void column_settle(const Problem& p, int64_t j, const double2* part, int64_t cnt, double sTd,
+                              double* scratch) {
+  double2 v = make_double2(0.0, 0.0);
+  for (int64_t k = threadIdx.x; k < cnt; k += kConsumers) {
+    const double2 c = __ldcg(part + k);
+    v.x += c.x;
+    v.y += c.y;
+  }
+  consumer_sum2(v.x, v.y, scratch);
+  if (threadIdx.x == 0) {
+    const double tn = scratch[0], td = scratch[1];
+    const double v2 = FMT == FMT_NVFP4 ? (tn / td) / sTd : tn / td;
+    b_encode(p.b_store, p.col_dt, j, td == 0.0 ? 1.0 : b_project(v2, p.col_dt));
+  }
+}
+
+// Returns true when strips with listed columns must be waited for (wait_strip).
+template <int FMT, int WDT>
+__device__ bool exact_listed(const Problem& p, int t, double sTd, float isT, double* scratch, int* s_flag) {
+  const int lb = (t - 1) % 3;
   const unsigned n = __ldcg(&p.hdr->amb_n[lb]);
-  if (n == 0u) return;  // the same value in every CTA
+  // the list of pass t + 1 was last read in pass t - 1: empty it for its writers
+  if (blockIdx.x == 0 && threadIdx.x == 0) p.hdr->amb_n[(t + 1) % 3] = 0u;
+  if (n == 0u) return false;  // the same value in every CTA
   const int* list = p.amb_list + (int64_t)lb * p.N;
-  // R chunks per column: enough items for every CTA of the grid (one short
-  // round of loads each), chunks of at least kXMinRows rows, and n * R
-  // partials must fit the column-partial buffer (free until the strips finish)
-  const int64_t cap = (int64_t)p.P * p.segmax * p.TS;
+  const bool own = (int64_t)n <= kXPartCap;  // chunk totals in p.xpart, no barrier
+  double2* part = own ? p.xpart : p.col_part;
+  const int64_t cap = own ? kXPartCap : (int64_t)p.P * p.segmax * p.TS;
   const int64_t R = max((int64_t)1, min(min((p.M + kXMinRows - 1) / kXMinRows, max((int64_t)1, (int64_t)p.P / (int64_t)n)),
                                         cap / (int64_t)n));
   const int64_t chunk = (p.M + R - 1) / R;
   for (int64_t it = blockIdx.x; it < (int64_t)n * R; it += gridDim.x) {
     const int64_t ci = it / R, r = it - ci * R;
     const int64_t j = __ldcg(list + ci);
-    const float bj = b_decode_cg(p.b_store, p.col_dt, j);
-    const float cb = __frcp_rn(bj) * isT;
-    const int64_t i_end = min(p.M, (r + 1) * chunk);
-    double cn = 0.0, cd = 0.0;
-    for (int64_t i0 = r * chunk + threadIdx.x; i0 < i_end; i0 += (int64_t)kXRows * kConsumers) {
-      float w[kXRows];
-      uint32_t araw[kXRows];
-#pragma unroll
-      for (int k = 0; k < kXRows; ++k) {  // all loads first
-        const int64_t i = i0 + (int64_t)k * kConsumers;
-        w[k] = 0.f;
-        araw[k] = a_raw_one<FMT>();
-        if (i < i_end) {
-          const int64_t e = i * p.N + j;
-          if (WDT == DT_F32) {
-            w[k] = __ldg(reinterpret_cast<const float*>(p.W) + e);
-          } else if (WDT == DT_BF16) {
-            w[k] = __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short*>(p.W) + e) << 16);
-          } else {
-            w[k] = __half2float(__ushort_as_half(__ldg(reinterpret_cast<const unsigned short*>(p.W) + e)));
-          }
-          araw[k] = a_fetch<FMT>(p.a_store, i * p.nb + j / p.G);
-        }
-      }
-#pragma unroll
-      for (int k = 0; k < kXRows; ++k) {  // absent rows hold w = 0, which adds nothing
-        const float a = a_dec<FMT>(araw[k]);
-        const float ia = __frcp_rn(a);
-        const bool ok = in_range(cb) && in_range(ia);
-        const float q = quant<FMT>(w[k], w[k] * cb, ia, ok, a, bj, sTd);
-        const double sv = (double)q * (double)a;
-        cn = fma((double)w[k], sv, cn);
-        cd = fma(sv, sv, cd);
-      }
-    }
-    scratch[threadIdx.x] = cn;
-    scratch[kConsumers + threadIdx.x] = cd;
-    consumer_sync(kConsumers);
-    for (int o = kConsumerTreeTop; o > 0; o >>= 1) {  // fixed-order tree
-      if (threadIdx.x < o && threadIdx.x + o < kConsumers) {
-        scratch[threadIdx.x] += scratch[threadIdx.x + o];
-        scratch[kConsumers + threadIdx.x] += scratch[kConsumers + threadIdx.x + o];
-      }
-      consumer_sync(kConsumers);
-    }
+    column_rows_exact<FMT, WDT>(p, j, r * chunk, min(p.M, (r + 1) * chunk), sTd, isT, scratch);
     if (threadIdx.x == 0) {
-      p.col_part[it] = make_double2(scratch[0], scratch[kConsumers]);
+      part[it] = make_double2(scratch[0], scratch[1]);
       __threadfence();
       const unsigned prev = atomicAdd(&p.amb_tick[ci], 1u);
       *s_flag = prev == (unsigned)R - 1u ? 1 : 0;
     }
     consumer_sync(kConsumers);
-    if (*s_flag) {  // last chunk of this column: the chunk totals in a fixed-order tree
+    if (*s_flag) {
       __threadfence();
-      double2 v = make_double2(0.0, 0.0);
-      for (int64_t k = threadIdx.x; k < R; k += kConsumers) {
-        const double2 c = __ldcg(&p.col_part[ci * R + k]);
-        v.x += c.x;
-        v.y += c.y;
-      }
-      scratch[threadIdx.x] = v.x;
-      scratch[kConsumers + threadIdx.x] = v.y;
-      consumer_sync(kConsumers);
-      for (int o = kConsumerTreeTop; o > 0; o >>= 1) {
-        if (threadIdx.x < o && threadIdx.x + o < kConsumers) {
-          scratch[threadIdx.x] += scratch[threadIdx.x + o];
-          scratch[kConsumers + threadIdx.x] += scratch[kConsumers + threadIdx.x + o];
-        }
-        consumer_sync(kConsumers);
-      }
+      column_settle<FMT>(p, j, part + ci * R, R, sTd, scratch);
       if (threadIdx.x == 0) {
-        const double tn = scratch[0], td = scratch[kConsumers];
-        const double v = FMT == FMT_NVFP4 ? (tn / td) / sTd : tn / td;
-        b_encode(p.b_store, p.col_dt, j, td == 0.0 ? 1.0 : b_project(v, p.col_dt));
         p.amb_tick[ci] = 0u;
+        __threadfence();  // the scale is visible before the count drops
+        if (own) {
+          atomicSub(&p.sx_left[j / p.TS], 1u);
+        } else {
+          p.sx_left[j / p.TS] = 0u;  // the barrier below orders it
+        }
       }
     }
-    consumer_sync(kConsumers);  // the scratch and the flag are reused by the next item
+    consumer_sync(kConsumers);  // the scratch and the flag are reused
   }
-  grid_sync_plain(p.hdr);
-  // every CTA read n before the barrier; the list is written again two passes later
-  if (blockIdx.x == 0 && threadIdx.x == 0) p.hdr->amb_n[lb] = 0u;
+  if (!own) grid_sync_plain(p.hdr);
+  return own;
+}
+
+// Before pass t uses the column scales of strip s: wait until the listed
+// columns of the strip are settled (bounded; gives up with kFlagTimeout).
+__device__ void wait_strip(const Problem& p, int64_t s) {
+  if (threadIdx.x == 0) {
+    for (unsigned i = 0;; ++i) {
+      if (ld_acquire_gpu(&p.sx_left[s]) == 0u) break;
+      if (i >= kGridSpinLimit || (*reinterpret_cast<volatile unsigned*>(&p.hdr->flags) & kFlagTimeout)) {
+        atomicOr(&p.hdr->flags, kFlagTimeout);
+        break;
+      }
+      __nanosleep(64);
+    }
+  }
 }
 
 // Passes t = t_first .. t_last over W, one read of W each, in one persistent
@@ -961,7 +1013,7 @@ __global__ void __launch_bounds__(kIterThreads, 1)
   unsigned tcnt = 0u;  // lane-rows settled as certified exact ties
 
   for (int t = t_first; t <= t_last; ++t) {
-  exact_listed<FMT, WDT>(p, t, sTd, isT, reinterpret_cast<double*>(acc), &s_misc[0]);
+  const bool strip_wait = exact_listed<FMT, WDT>(p, t, sTd, isT, reinterpret_cast<double*>(acc), &s_misc[0]);
   if (FIN && blockIdx.x == 0) {
     // the MSE of the passes that no grid barrier of the iteration launch summed
     for (int tp = max(1, t - 2); tp <= t - 1; ++tp)
@@ -986,6 +1038,7 @@ __global__ void __launch_bounds__(kIterThreads, 1)
     cs.tb = ctab;
     cs.tcb = ctab + 128;
     cs.lane = lane;
+    if (strip_wait) wait_strip(p, s);  // listed columns of this strip settled first
     consumer_sync(kConsumers);  // the previous segment's readers of the table are done
     cs.ok = sT_ok;
     cs.res2 = 0ull;
@@ -1132,11 +1185,14 @@ __global__ void __launch_bounds__(kIterThreads, 1)
           // rows and writes its scale (b keeps its value until then)
           amb = true;
           atomicAdd(&s_misc[1], 1);
-          p.amb_list[(int64_t)(t & 1) * p.N + atomicAdd(&p.hdr->amb_n[t & 1], 1u)] = (int)(c0 + threadIdx.x);
+          p.amb_list[(int64_t)(t % 3) * p.N + atomicAdd(&p.hdr->amb_n[t % 3], 1u)] = (int)(c0 + threadIdx.x);
         }
       }
       consumer_sync(kConsumers);
-      if (threadIdx.x == 0) s_cnt[2] += (unsigned)s_misc[1];
+      if (threadIdx.x == 0) {
+        s_cnt[2] += (unsigned)s_misc[1];
+        p.sx_left[s] = (unsigned)s_misc[1];  // listed columns the next pass must settle before using the strip
+      }
       if (threadIdx.x < width && !amb) b_encode(p.b_store, p.col_dt, c0 + threadIdx.x, bnew);
       if (threadIdx.x == 0) p.strip_counter[s] = 0u;
     }
