@@ -54,7 +54,15 @@ int make_plan(int64_t M, int64_t N, int group, int init, Plan* pl) {
   auto ctas = [&](int64_t want) { return (int)(byrows < want ? (byrows < 1 ? 1 : byrows) : want); };
   // a CTA's contiguous range of len rows touches at most ceil(len/M) + 1 strips
   auto segs = [&](int64_t P) { return (int)(((pl->L + P - 1) / P + M - 1) / M + 1); };
-  pl->P = ctas((int64_t)sms * dq::kCtasPerSm);
+  // a grid that is a multiple of the strip count (when that keeps at least
+  // 90% of the SMs) gives every CTA rows of a single strip: no CTA pays a
+  // second column-table setup and strip end inside a pass
+  int64_t want = (int64_t)sms * dq::kCtasPerSm;
+  if (pl->n_strips <= want) {
+    const int64_t aligned = want / pl->n_strips * pl->n_strips;
+    if (10 * aligned >= 9 * want) want = aligned;
+  }
+  pl->P = ctas(want);
   pl->segmax = segs(pl->P);
   pl->P_final = ctas((int64_t)sms * dq::kFinalCtasPerSm);
   pl->segmax_final = segs(pl->P_final);
