@@ -35,7 +35,9 @@ L2_FLUSH_BYTES = 512 << 20
 KERNEL_SOURCES = ["calibration_free_weight_dualquant_b200/csrc/dq_solver.cu",
                   "calibration_free_weight_dualquant_b200/csrc/dq_device.cuh",
                   "calibration_free_weight_dualquant_b200/csrc/dq_fast.cuh",
-                  "calibration_free_weight_dualquant_b200/csrc/dq_iter.cuh"]
+                  "calibration_free_weight_dualquant_b200/csrc/dq_iter.cuh",
+                  "calibration_free_weight_dualquant_b200/csrc/dq_internal.h",
+                  "calibration_free_weight_dualquant_b200/csrc/dq_capi.cu"]
 
 
 def kernel_hash() -> str:
@@ -56,7 +58,9 @@ def measured_peaks() -> dict:
 
 
 def profile_traffic(workload: str):
-    """dram bytes per k_iter launch from the committed ncu summary, if it matches the current kernel source."""
+    """DRAM bytes per pass of k_iter (one BCD iteration) from the committed ncu summary, if it was taken of
+    the current kernel source.  One k_iter launch runs all T passes, so the summary stores its launch's
+    dram bytes divided by the passes it ran."""
     path = os.path.join(ROOT, "profiles", "k_iter_%s.json" % workload)
     if not os.path.exists(path):
         return None
@@ -64,7 +68,7 @@ def profile_traffic(workload: str):
         d = json.load(f)
     if d.get("kernel_hash") != kernel_hash():
         return None
-    return d.get("dram_bytes_per_launch")
+    return d.get("dram_bytes_per_pass")
 
 
 class ClockSampler:
@@ -469,9 +473,10 @@ def run_dq(args, wl, rank, world, local, dist):
         "ms_per_iter": iter_ms,
         "roofline": {"bound": "hbm", "kernel": "k_iter", "achieved": achieved, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
-                     "algorithmic_bytes_per_launch": alg, "peak_source": peaks["source"]},
+                     "algorithmic_bytes_per_pass": alg, "passes_per_launch": T, "peak_source": peaks["source"]},
         "e2e": e2e_line,
-        "gpu_launches": args.steps * (T + 3),
+        # per solve: k_stats, k_init, one k_iter for all T iterations, the final k_iter pass
+        "gpu_launches": args.steps * (4 if T > 0 else 3),
         "exact_paths_last_step": exact_paths,
         "clocks": clk.summary(),
     }
@@ -538,10 +543,10 @@ def run_dq_set(args, name, rank, world, local, dist):
         "ms_per_iter": iter_ms,
         "roofline": {"bound": "hbm", "kernel": "k_iter", "achieved": achieved, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
-                     "algorithmic_bytes_per_launch": alg, "peak_source": peaks["source"],
+                     "algorithmic_bytes_per_pass": alg, "passes_per_launch": T, "peak_source": peaks["source"],
                      "note": "per iteration of the whole set (224 launches of k_iter)"},
         "e2e": None,
-        "gpu_launches": args.steps * len(wls) * (T + 3),
+        "gpu_launches": args.steps * len(wls) * (4 if T > 0 else 3),
         "clocks": clk.summary(),
     }
     if world == 1 and not args.no_cpu_baseline:

@@ -252,7 +252,7 @@ int dq_act_quant(const void* X, int x_dtype, int64_t rows, int64_t cols, const v
 
 /* Size of the library-owned device scratch that dq_solve_static uses: 8 MiB.
  * A shape fits when dq_workspace_bytes(rows, cols, format, group) is at most
- * this; on a 148-SM B200 that holds every shape with cols <= 262144. */
+ * this; on a 148-SM B200 that holds every shape with cols <= 196608. */
 #define DQ_STATIC_SCRATCH_BYTES (8u << 20)
 
 /* dq_solve without a workspace argument, for callers that cannot allocate
