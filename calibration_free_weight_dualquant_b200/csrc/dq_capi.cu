@@ -58,6 +58,7 @@ int make_plan(int64_t M, int64_t N, int group, int init, Plan* pl) {
   // 90% of the SMs) gives every CTA rows of a single strip: no CTA pays a
   // second column-table setup and strip end inside a pass
   int64_t want = (int64_t)sms * dq::kCtasPerSm;
+  if (want > dq::kMaxGrid) want = dq::kMaxGrid;
   if (pl->n_strips <= want) {
     const int64_t aligned = want / pl->n_strips * pl->n_strips;
     if (10 * aligned >= 9 * want) want = aligned;

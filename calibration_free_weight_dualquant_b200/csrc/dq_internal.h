@@ -11,7 +11,8 @@ namespace dq {
 constexpr int kThreads = 256;   // 8 warps per CTA
 constexpr int kWarps = kThreads / 32;
 constexpr int kStripMax = 256;  // columns per strip (8 per lane, 32 lanes)
-constexpr int kCtasPerSm = 1;        // per-iteration pass: one 544-thread CTA per SM
+constexpr int kCtasPerSm = 1;        // per-iteration pass: one 512-thread CTA per SM
+constexpr int kMaxGrid = 1024;       // CTAs of the per-iteration pass at most
 constexpr int kFinalCtasPerSm = 4;   // one-time passes
 constexpr int64_t kMinRowsPerCta = 64;
 // 32-bit digits of an exact magnitude sum in units of 2^-149 (L1 init): one

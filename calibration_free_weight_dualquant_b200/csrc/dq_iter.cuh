@@ -49,7 +49,7 @@ __host__ __device__ constexpr size_t iter_acc_bytes() {
 }
 __host__ __device__ constexpr size_t iter_smem_bytes(int es) {
   return (size_t)kRingBytes + iter_acc_bytes() + 2 * sizeof(uint64_t) * ring_stages(es) +
-         (2 + kStripMax + 4) * sizeof(int) + 2 * 4 * 32 * sizeof(unsigned long long);
+         (2 + kStripMax + 4) * sizeof(int) + 2 * 4 * 32 * sizeof(unsigned long long) + kMaxGrid * sizeof(int);
 }
 
 // ---------------------------------------------------------------------------
@@ -915,6 +915,7 @@ __global__ void __launch_bounds__(kIterThreads, 1)
   int* s_misc = reinterpret_cast<int*>(empty + S);  // [0] ticket result, [1] #ambiguous, [2..] columns
   unsigned* s_cnt = reinterpret_cast<unsigned*>(s_misc + 2 + kStripMax);  // exact-path counters
   f2* ctab = reinterpret_cast<f2*>(s_cnt + 4);  // column table of the strip: b pairs, then cb pairs
+  int* s_sfirst = reinterpret_cast<int*>(ctab + 2 * 4 * 32);  // [P] first strip of each CTA's range
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row_bytes = p.TS * ES;  // ring slot per row
   const int stage_bytes = kRowsPerTile * row_bytes;
@@ -934,6 +935,9 @@ __global__ void __launch_bounds__(kIterThreads, 1)
   griddep_wait();
   griddep_launch_dependents();
   if (p.hdr->flags & kFlagAbort) return;
+  // first strip of every CTA's range (the strip finalizers index partials by it)
+  for (int kk = threadIdx.x; kk < p.P; kk += kIterThreads) s_sfirst[kk] = (int)(range_begin(kk, p.P, p.L) / p.M);
+  __syncthreads();
 
   const int64_t k = blockIdx.x;
   const int64_t u_begin = range_begin(k, p.P, p.L), u_end = range_begin(k + 1, p.P, p.L);
@@ -1074,17 +1078,20 @@ __global__ void __launch_bounds__(kIterThreads, 1)
     // block scales of this warp's rows, one tile ahead
     const int64_t a_step = (int64_t)kRowsPerTile * p.nb;
     int64_t aidx = (r0 + warp) * p.nb + blk_col;
+    const int64_t y_off = (int64_t)kConsumerWarps * p.nb;  // block-scale offset of the warp's second row
+    // rows relative to the segment start, in 32 bits (a segment has fewer than 2^31 rows)
+    const int nrows = (int)(r1 - r0);
     uint32_t an0 = a_raw_one<FMT>(), an1 = a_raw_one<FMT>();
-    if (active && r0 + warp < r1) an0 = a_fetch<FMT>(p.a_store, aidx);
-    if (active && r0 + warp + kConsumerWarps < r1) an1 = a_fetch<FMT>(p.a_store, aidx + kConsumerWarps * p.nb);
+    if (active && warp < nrows) an0 = a_fetch<FMT>(p.a_store, aidx);
+    if (active && warp + kConsumerWarps < nrows) an1 = a_fetch<FMT>(p.a_store, aidx + y_off);
 
-    for (int64_t tr = r0; tr < r1; tr += kRowsPerTile, aidx += a_step) {
-      const int64_t ra = tr + warp, rb = ra + kConsumerWarps;
-      const bool has_a = ra < r1, has_b = rb < r1;  // warp-uniform
+    for (int tr = 0; tr < nrows; tr += kRowsPerTile, aidx += a_step) {
+      const int ra = tr + warp, rb = ra + kConsumerWarps;
+      const bool has_a = ra < nrows, has_b = rb < nrows;  // warp-uniform
       const uint32_t ra_raw = an0, rb_raw = an1;
-      if (active && ra + kRowsPerTile < r1) an0 = a_fetch<FMT>(p.a_store, aidx + a_step);
-      if (active && rb + kRowsPerTile < r1) an1 = a_fetch<FMT>(p.a_store, aidx + a_step + kConsumerWarps * p.nb);
-      const int64_t cix = (ra * p.N + col) >> 3;  // code word of row ra, this lane's 8 columns
+      if (active && ra + kRowsPerTile < nrows) an0 = a_fetch<FMT>(p.a_store, aidx + a_step);
+      if (active && rb + kRowsPerTile < nrows) an1 = a_fetch<FMT>(p.a_store, aidx + a_step + y_off);
+      const int64_t cix = ((r0 + ra) * p.N + col) >> 3;  // code word of row ra, this lane's 8 columns
       uint32_t oldx = 0u, oldy = 0u;
       if (PASS != PASS_ITER && cmp && active) {  // issued before the wait: the latency hides behind it
         if (has_a) oldx = __ldcg(codes_old + cix);
@@ -1111,7 +1118,7 @@ __global__ void __launch_bounds__(kIterThreads, 1)
           final_pair<FMT>(p, wa, aa, wb, ab, has_b, active, cs, sT, sTd, scaled, rscale2, s_cnt, tcnt, cix, oldx,
                           oldy, cmp, nchg);
         } else {
-          row_pair<FMT, PASS>(p, wa, aa, aidx, wb, ab, aidx + kConsumerWarps * p.nb, has_b, active, leader, lpb, cs,
+          row_pair<FMT, PASS>(p, wa, aa, aidx, wb, ab, aidx + y_off, has_b, active, leader, lpb, cs,
                               sT, isT, sTd, scaled, rscale2, s_cnt, tcnt, cix, oldx, oldy, cmp, nchg);
         }
         run += has_b ? 2 : 1;
@@ -1163,12 +1170,19 @@ __global__ void __launch_bounds__(kIterThreads, 1)
       bool amb = false;
       if (threadIdx.x < width) {
         double2 tot = make_double2(0.0, 0.0);
-#pragma unroll 4
-        for (int64_t kk = k_first; kk <= k_last; ++kk) {
-          const int64_t sl = kk * p.segmax + (s - range_begin(kk, p.P, p.L) / p.M);
-          const double2 v = __ldcg(&p.col_part[sl * p.TS + threadIdx.x]);
-          tot.x += v.x;
-          tot.y += v.y;
+        for (int64_t kb = k_first; kb <= k_last; kb += 8) {  // 8 loads in flight, added in CTA order
+          double2 v[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int64_t kk = kb + q;
+            v[q] = make_double2(0.0, 0.0);
+            if (kk <= k_last) v[q] = __ldcg(&p.col_part[(kk * p.segmax + (s - s_sfirst[kk])) * p.TS + threadIdx.x]);
+          }
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            tot.x += v[q].x;
+            tot.y += v[q].y;
+          }
         }
         // certified only when the fp32 runs stayed well inside the normal
         // range (no overflow; underflowed terms negligible); a zero total may
