@@ -774,6 +774,7 @@ template <int FMT, int WDT>
 __device__ void column_rows_exact(const Problem& p, int64_t j, int64_t i_begin, int64_t i_end, double sTd, float isT,
                                   double* scratch) {
   const unsigned short braw = __ldcg(reinterpret_cast<const unsigned short*>(p.b_store) + j);
+  const int64_t jb = j / p.G;  // block column
   double cn = 0.0, cd = 0.0;
   for (int64_t i0 = i_begin + threadIdx.x; i0 < i_end; i0 += (int64_t)kXRows * kConsumers) {
     float w[kXRows];
@@ -792,7 +793,7 @@ __device__ void column_rows_exact(const Problem& p, int64_t j, int64_t i_begin, 
         } else {
           w[k] = __half2float(__ushort_as_half(__ldg(reinterpret_cast<const unsigned short*>(p.W) + e)));
         }
-        araw[k] = a_fetch<FMT>(p.a_store, i * p.nb + j / p.G);
+        araw[k] = a_fetch<FMT>(p.a_store, i * p.nb + jb);
       }
     }
     const float bj = p.col_dt == DT_F16 ? __half2float(__ushort_as_half(braw)) : __uint_as_float((uint32_t)braw << 16);
