@@ -96,8 +96,15 @@ __global__ void __launch_bounds__(kThreads) k_init(Problem p) {
   const double qmax = fmt_e2m1(FMT) ? 6.0 : 7.0;
   const int64_t nblocks = p.M * p.nb;
   const int64_t stride = (int64_t)gridDim.x * kThreads;
-  for (int64_t blk = (int64_t)blockIdx.x * kThreads + threadIdx.x; blk < nblocks; blk += stride) {
-    const int64_t i = blk / p.nb, g = blk % p.nb;
+  // (row i, block g) of blk, advanced incrementally (no division per block)
+  const int64_t blk0 = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  const int64_t sq = stride / p.nb, sr = stride % p.nb;
+  int64_t i = blk0 / p.nb, g = blk0 % p.nb;
+  for (int64_t blk = blk0; blk < nblocks; blk += stride, i += sq, g += sr) {
+    if (g >= p.nb) {
+      g -= p.nb;
+      ++i;
+    }
     const int64_t off = i * p.N + g * p.G;
     double m = 0.0;
     if (l1) {
