@@ -87,6 +87,8 @@ def load_library():
     lib.dq_solve_host.restype = I
     lib.dq_diagnostics.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint64)]
     lib.dq_diagnostics.restype = I
+    lib.dq_wait_selftest.argtypes = [P, SZ, P]
+    lib.dq_wait_selftest.restype = I
     lib.dq_solve_static.argtypes = [P, I, I64, I64, I, I, I, I, ctypes.POINTER(_Outputs), P, P]
     lib.dq_solve_static.restype = I
     lib.dq_solve_batched.argtypes = [ctypes.POINTER(_Matrix), I, I, I, I, I, P, P, SZ, ctypes.POINTER(I), P]
@@ -394,6 +396,16 @@ def solve(W: torch.Tensor, fmt="nvfp4", group: Optional[int] = None, iters: int 
 def rtn(W: torch.Tensor, fmt="nvfp4", group: Optional[int] = None, col_dtype: Optional[str] = None) -> dict:
     """User-level absmax RTN (the 0-iteration solve)."""
     return solve(W, fmt, group, 0, col_dtype)
+
+
+def wait_selftest(workspace: torch.Tensor, stream=None) -> int:
+    """Run the library's bounded-wait self-test on ``workspace`` (device, >= 512 bytes) and return the
+    device status it leaves (dq_sync_status): DQ_ECUDA (5) when the wait gave up as it should."""
+    lib = load_library()
+    st = lib.dq_wait_selftest(workspace.data_ptr(), workspace.numel(), _stream_ptr(stream))
+    if st != 0:
+        raise DQError(st, "dq_wait_selftest")
+    return lib.dq_sync_status(workspace.data_ptr(), _stream_ptr(stream))
 
 
 def diagnostics(workspace: torch.Tensor, stream=None) -> dict:

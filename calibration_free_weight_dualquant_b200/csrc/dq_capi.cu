@@ -250,6 +250,13 @@ int dq_sync_status(const void* workspace, void* stream) {
   return (flags & dq::kFlagTimeout) ? DQ_ECUDA : DQ_OK;
 }
 
+int dq_wait_selftest(void* workspace, size_t workspace_bytes, void* stream) {
+  if (!workspace || !aligned(workspace, kAlign)) return DQ_EINVAL;
+  if (workspace_bytes < 512) return DQ_EWORKSPACE;
+  if (dq::launch_wait_selftest(workspace, static_cast<cudaStream_t>(stream)) != cudaSuccess) return DQ_ECUDA;
+  return DQ_OK;
+}
+
 int dq_diagnostics(const void* workspace, void* stream, uint64_t out[4]) {
   if (!workspace || !out) return DQ_EINVAL;
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DQ_ECUDA;

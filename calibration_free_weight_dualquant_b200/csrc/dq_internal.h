@@ -77,6 +77,8 @@ struct Problem {
 };
 
 cudaError_t launch_solve(const Problem& p, int iters, int stats_ctas, cudaStream_t st);
+// Runs the bounded-wait self-test on `workspace` (>= 512 bytes).
+cudaError_t launch_wait_selftest(void* workspace, cudaStream_t st);
 
 // Host-side validation, workspace layout and enqueue of a whole solve (the body
 // of dq_solve; `workspace` is a device address of at least the planned size).

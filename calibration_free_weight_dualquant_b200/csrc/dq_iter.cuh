@@ -644,9 +644,26 @@ __device__ __forceinline__ void flush_runs(ColState& cs, double2* acc, double* r
 // Grid-wide barrier of the consumer threads of every CTA.  k_iter is launched
 // cooperatively, so all its CTAs are resident at once.  Arrivals are counted
 // in hdr->gbar over the whole solve; a use waits for the next multiple of the
-// grid size.  The wait is bounded: it gives up after kGridSpinLimit polls (or
-// at once when some wait already gave up), records kFlagTimeout and goes on.
-constexpr unsigned kGridSpinLimit = 1u << 24;
+// grid size.  The wait is bounded: it gives up after kWaitLimitNs of wall
+// time (or at once when some wait already gave up), records kFlagTimeout and
+// goes on.
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s
+
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// True when a bounded wait begun at t0 must give up (its time is over, or some
+// other wait already gave up); then kFlagTimeout is recorded.
+__device__ __forceinline__ bool wait_expired(unsigned* flags, unsigned long long t0) {
+  if (global_ns() - t0 > kWaitLimitNs || (*reinterpret_cast<volatile unsigned*>(flags) & kFlagTimeout)) {
+    atomicOr(flags, kFlagTimeout);
+    return true;
+  }
+  return false;
+}
 
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* a) {
   unsigned v;
@@ -691,12 +708,10 @@ __device__ void grid_sync(const Problem& p, int t, double rscale_d, double* red,
   consumer_sync(kConsumers);
   if (*s_flag) mse_total(p, mse_part(p, t - 1), p.mse + (t - 2), rscale_d, red);
   if (threadIdx.x == 0) {
-    for (unsigned i = 0;; ++i) {
+    const unsigned long long t0 = global_ns();
+    for (;;) {
       if ((int)(ld_acquire_gpu(&hdr->gbar) - target) >= 0) break;
-      if (i >= kGridSpinLimit || (*reinterpret_cast<volatile unsigned*>(&hdr->flags) & kFlagTimeout)) {
-        atomicOr(&hdr->flags, kFlagTimeout);
-        break;
-      }
+      if (wait_expired(&hdr->flags, t0)) break;
       __nanosleep(64);
     }
     __threadfence();
@@ -711,12 +726,10 @@ __device__ void grid_sync_plain(WsHeader* hdr) {
     __threadfence();
     const unsigned ticket = atomicAdd(&hdr->gbar, 1u);
     const unsigned target = (ticket / gridDim.x + 1u) * gridDim.x;
-    for (unsigned i = 0;; ++i) {
+    const unsigned long long t0 = global_ns();
+    for (;;) {
       if ((int)(ld_acquire_gpu(&hdr->gbar) - target) >= 0) break;
-      if (i >= kGridSpinLimit || (*reinterpret_cast<volatile unsigned*>(&hdr->flags) & kFlagTimeout)) {
-        atomicOr(&hdr->flags, kFlagTimeout);
-        break;
-      }
+      if (wait_expired(&hdr->flags, t0)) break;
       __nanosleep(64);
     }
     __threadfence();
@@ -880,12 +893,10 @@ __device__ bool exact_listed(const Problem& p, int t, double sTd, float isT, dou
 // columns of the strip are settled (bounded; gives up with kFlagTimeout).
 __device__ void wait_strip(const Problem& p, int64_t s) {
   if (threadIdx.x == 0) {
-    for (unsigned i = 0;; ++i) {
+    const unsigned long long t0 = global_ns();
+    for (;;) {
       if (ld_acquire_gpu(&p.sx_left[s]) == 0u) break;
-      if (i >= kGridSpinLimit || (*reinterpret_cast<volatile unsigned*>(&p.hdr->flags) & kFlagTimeout)) {
-        atomicOr(&p.hdr->flags, kFlagTimeout);
-        break;
-      }
+      if (wait_expired(&p.hdr->flags, t0)) break;
       __nanosleep(64);
     }
   }

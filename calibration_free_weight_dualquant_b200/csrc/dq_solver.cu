@@ -96,15 +96,8 @@ __global__ void __launch_bounds__(kThreads) k_init(Problem p) {
   const double qmax = fmt_e2m1(FMT) ? 6.0 : 7.0;
   const int64_t nblocks = p.M * p.nb;
   const int64_t stride = (int64_t)gridDim.x * kThreads;
-  // (row i, block g) of blk, advanced incrementally (no division per block)
-  const int64_t blk0 = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-  const int64_t sq = stride / p.nb, sr = stride % p.nb;
-  int64_t i = blk0 / p.nb, g = blk0 % p.nb;
-  for (int64_t blk = blk0; blk < nblocks; blk += stride, i += sq, g += sr) {
-    if (g >= p.nb) {
-      g -= p.nb;
-      ++i;
-    }
+  for (int64_t blk = (int64_t)blockIdx.x * kThreads + threadIdx.x; blk < nblocks; blk += stride) {
+    const int64_t i = blk / p.nb, g = blk % p.nb;
     const int64_t off = i * p.N + g * p.G;
     double m = 0.0;
     if (l1) {
@@ -260,6 +253,30 @@ cudaError_t launch_solve(const Problem& p, int iters, int stats_ctas, cudaStream
     case FMT_MXFP4: return run_fmt<FMT_MXFP4>(p, iters, stats_ctas, st);
     default: return run_fmt<FMT_NVFP4>(p, iters, stats_ctas, st);
   }
+}
+
+// Self-test of the bounded waits: strip 0's pending count is set to 1 and
+// never released, so wait_strip gives up after its time limit and records
+// kFlagTimeout; nothing faults and the context stays usable.
+__global__ void k_wait_selftest(Problem p) {
+  if (threadIdx.x == 0) {
+    p.hdr->flags = 0u;
+    p.sx_left[0] = 1u;
+    __threadfence();
+  }
+  __syncthreads();
+  wait_strip(p, 0);
+  __syncthreads();
+  if (threadIdx.x == 0) p.sx_left[0] = 0u;
+}
+
+cudaError_t launch_wait_selftest(void* workspace, cudaStream_t st) {
+  Problem p;
+  std::memset(&p, 0, sizeof(p));
+  p.hdr = reinterpret_cast<WsHeader*>(workspace);
+  p.sx_left = reinterpret_cast<unsigned*>(static_cast<char*>(workspace) + 256);
+  k_wait_selftest<<<1, 32, 0, st>>>(p);
+  return cudaGetLastError();
 }
 
 }  // namespace dq

@@ -202,6 +202,19 @@ int dq_solve_host(const void* W_host, int w_dtype, int64_t rows, int64_t cols, i
  * Counts cover the BCD iterations only (not init or the final pass). */
 int dq_diagnostics(const void* workspace, void* stream, uint64_t out[4]);
 
+/* Self-test of the solver's bounded device waits (no counterpart in the
+ * method; failure detection).  Every wait of the per-iteration kernel (the
+ * tile pipeline, the grid barrier between BCD passes, the wait for a strip's
+ * exactly updated column scales) gives up after a time limit (about 1 s),
+ * records a timeout in the workspace header and lets the kernel finish, so a
+ * lost arrival ends in a status instead of a hung GPU.  This call enqueues one
+ * such wait on a counter that nothing releases: afterwards dq_sync_status on
+ * the same workspace returns DQ_ECUDA, and the context stays usable (the next
+ * dq_solve clears the header).  `workspace`: device, 256-byte aligned, at least
+ * 512 bytes, overwritten.  Returns DQ_EINVAL / DQ_EWORKSPACE / DQ_ECUDA on bad
+ * arguments or a failed launch. */
+int dq_wait_selftest(void* workspace, size_t workspace_bytes, void* stream);
+
 /* One matrix of a batched solve: W (device, row-major rows x cols, w_dtype)
  * and its outputs (as for dq_solve, mse with iters+1 entries). */
 typedef struct {
