@@ -35,8 +35,13 @@
  *  - "Scale 1 for an all-zero code slice": a = 1 (INT4, MXINT4), e = 1 (NVFP4),
  *    b = 1.
  *  - Init: b = 1 and a = Proj(absmax(block) / qmax), qmax = 7 (INT4 grid
- *    [-8,7]) or 6 (E2M1); an all-zero block gets scale 1.  Variants: the
- *    per-column L1-norm init (init_l1) and a warm start from given scales.
+ *    [-8,7]), 127 (INT8 grid [-128,127]) or 6 (E2M1); an all-zero block gets
+ *    scale 1.  Variants: the per-column L1-norm init (init_l1) and a warm
+ *    start from given scales.
+ *  - MXINT8 ([P2] App. G.2, 8-bit W+A quantization with MXINT8 and MXFP8): the INT8
+ *    codebook [-128,127] with E8M0 power-of-two block scales, group 32, one
+ *    byte per code; the OCP element's fixed 2^-6 factor is a power of two and
+ *    is absorbed into the block scale.
  */
 #include <math.h>
 #include <stdint.h>
@@ -53,6 +58,7 @@
 #define DQO_MXINT4 1
 #define DQO_NVFP4 2
 #define DQO_MXFP4 3 /* E2M1 grid with E8M0 block scales (the MX family's FP4 member) */
+#define DQO_MXINT8 4 /* INT8 grid [-128,127] with E8M0 block scales (the MX family's INT8 member) */
 /* element dtypes */
 #define DQO_F32 0
 #define DQO_BF16 1
@@ -72,6 +78,15 @@ static const unsigned char INT4_EVEN[16] = {1, 0, 1, 0, 1, 0, 1, 0, 1, 0, 1, 0, 
  * magnitudes 0,0.5,1,1.5,2,3,4,6 have encodings 000,001,010,011,100,101,110,111 */
 static const double E2M1_GRID[15] = {-6, -4, -3, -2, -1.5, -1, -0.5, 0, 0.5, 1, 1.5, 2, 3, 4, 6};
 static const unsigned char E2M1_EVEN[15] = {0, 1, 0, 1, 0, 1, 0, 1, 0, 1, 0, 1, 0, 1, 0};
+/* INT8 codebook -128..127 and its even flags, filled once by int8_grid_init() */
+static double INT8_GRID[256];
+static unsigned char INT8_EVEN[256];
+static void int8_grid_init(void) {
+  for (int k = 0; k < 256; ++k) {
+    INT8_GRID[k] = (double)(k - 128);
+    INT8_EVEN[k] = (unsigned char)((k - 128) % 2 == 0);
+  }
+}
 
 /*
  * Nearest grid value to w/scale ([L1] Ch. 2 round-to-nearest then clip;
@@ -219,7 +234,10 @@ typedef struct {
 /* the formats on the E2M1 grid */
 static int e2m1_grid(int fmt) { return fmt == DQO_NVFP4 || fmt == DQO_MXFP4; }
 
-static double qmax_of(int fmt) { return e2m1_grid(fmt) ? 6.0 : 7.0; }
+static double qmax_of(int fmt) { return e2m1_grid(fmt) ? 6.0 : (fmt == DQO_MXINT8 ? 127.0 : 7.0); }
+
+/* formats with 8-bit codes (one byte per element) */
+static int byte_codes(int fmt) { return fmt == DQO_MXINT8; }
 
 /* block inverse scale value a from its stored factor (NVFP4 stores e, a = s_T*e) */
 static double a_value(const problem* p, double stored) { return p->fmt == DQO_NVFP4 ? p->sT * stored : stored; }
@@ -227,7 +245,7 @@ static double a_value(const problem* p, double stored) { return p->fmt == DQO_NV
 /* projection of an LS inverse-scale value onto F_a; returns the stored factor */
 static double project_a(const problem* p, double v) {
   if (p->fmt == DQO_INT4) return dqo_project(DQO_PROJ_F16, v);
-  if (p->fmt == DQO_MXINT4 || p->fmt == DQO_MXFP4) return dqo_project(DQO_PROJ_E8M0, v);
+  if (p->fmt == DQO_MXINT4 || p->fmt == DQO_MXFP4 || p->fmt == DQO_MXINT8) return dqo_project(DQO_PROJ_E8M0, v);
   return dqo_project(DQO_PROJ_E4M3, v / p->sT); /* nearest s_T*e to v */
 }
 
@@ -235,6 +253,7 @@ static double project_a(const problem* p, double v) {
 static double quant_value(const problem* p, double w, double a, double b) {
   double ab = a * b;
   if (e2m1_grid(p->fmt)) return E2M1_GRID[dqo_quant_index(w, ab, E2M1_GRID, E2M1_EVEN, 15)];
+  if (p->fmt == DQO_MXINT8) return INT8_GRID[dqo_quant_index(w, ab, INT8_GRID, INT8_EVEN, 256)];
   return INT4_GRID[dqo_quant_index(w, ab, INT4_GRID, INT4_EVEN, 16)];
 }
 
@@ -493,7 +512,8 @@ static int init_given(problem* p, const double* a0, const double* b0, double sT0
 static int load_problem(problem* p, const void* W, int wdt, int64_t M, int64_t N, int fmt, int G, int col_dt,
                         double** Wd_out) {
   if (!W || M <= 0 || N <= 0 || G <= 0 || N % G != 0 || N % 2 != 0) return DQO_EINVAL;
-  if (fmt < 0 || fmt > 3 || (col_dt != DQO_F16 && col_dt != DQO_BF16)) return DQO_EINVAL;
+  if (fmt < 0 || fmt > 4 || (col_dt != DQO_F16 && col_dt != DQO_BF16)) return DQO_EINVAL;
+  int8_grid_init();
   double* Wd = (double*)malloc(sizeof(double) * (size_t)(M * N));
   if (!Wd) return DQO_ENOMEM;
   int bad = 0;
@@ -535,6 +555,10 @@ static int load_problem(problem* p, const void* W, int wdt, int64_t M, int64_t N
 
 static void pack_codes(const problem* p, const double* q, uint8_t* codes) {
   int64_t M = p->M, N = p->N;
+  if (byte_codes(p->fmt)) { /* one two's-complement byte per element */
+    for (int64_t k = 0; k < M * N; ++k) codes[k] = (uint8_t)((int)q[k] & 0xFF);
+    return;
+  }
   for (int64_t i = 0; i < M; ++i)
     for (int64_t j = 0; j < N; j += 2) {
       uint8_t lo, hi;
@@ -556,7 +580,8 @@ static void pack_codes(const problem* p, const double* q, uint8_t* codes) {
  *     row update (codes fixed) -> project -> requantize
  *     column update (codes fixed) -> project -> requantize; mse[t]
  * Outputs (any may be NULL except mse when iters >= 0 is wanted):
- *   codes      [M][N/2] packed nibbles, even column in the low nibble
+ *   codes      [M][N/2] packed nibbles, even column in the low nibble (MXINT8:
+ *              [M][N], one two's-complement byte per element)
  *   a_out      [M][N/G] stored block scale values (fp16 value / 2^k / E4M3 e)
  *   b_out      [N] column inverse scales
  *   sT_out     NVFP4 tensor scale (1 for the other formats)
@@ -730,6 +755,10 @@ uint32_t dqo_encode(int kind, double v) {
 /* grid quantizer of a format on one value (for pins) -> grid value */
 double dqo_quant_value(int fmt, double w, double ab) {
   if (e2m1_grid(fmt)) return E2M1_GRID[dqo_quant_index(w, ab, E2M1_GRID, E2M1_EVEN, 15)];
+  if (fmt == DQO_MXINT8) {
+    int8_grid_init();
+    return INT8_GRID[dqo_quant_index(w, ab, INT8_GRID, INT8_EVEN, 256)];
+  }
   return INT4_GRID[dqo_quant_index(w, ab, INT4_GRID, INT4_EVEN, 16)];
 }
 

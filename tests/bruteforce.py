@@ -14,17 +14,25 @@ import numpy as np
 import torch
 
 INT4_VALUES = list(range(-8, 8))
+INT8_VALUES = list(range(-128, 128))
 E2M1_MAGS = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]  # encodings 0..7
 E2M1_VALUES = sorted(set([-m for m in E2M1_MAGS] + E2M1_MAGS))
 
 
 def grid_values(fmt: str):
+    if fmt == "mxint8":
+        return INT8_VALUES
     return INT4_VALUES if fmt in ("int4", "mxint4") else E2M1_VALUES
+
+
+def grid_qmax(fmt: str) -> int:
+    """qmax of the absmax init: largest positive grid value."""
+    return {"mxint8": 127, "nvfp4": 6, "mxfp4": 6}.get(fmt, 7)
 
 
 def grid_is_even(fmt: str, v: float) -> bool:
     """Tie winner flag: even integer (INT4) or even mantissa bit of the E2M1 encoding."""
-    if fmt in ("int4", "mxint4"):
+    if fmt in ("int4", "mxint4", "mxint8"):
         return int(v) % 2 == 0
     return E2M1_MAGS.index(abs(v)) % 2 == 0
 
@@ -122,7 +130,10 @@ def argmin_scale_objective(kind: str, W: np.ndarray, R: np.ndarray, scale_factor
 
 
 def decode_codes(fmt: str, codes: np.ndarray) -> np.ndarray:
-    """Unpack nibble codes [M, N/2] -> grid values [M, N] (even column in the low nibble)."""
+    """Unpack nibble codes [M, N/2] -> grid values [M, N] (even column in the low nibble);
+    MXINT8 codes [M, N] are one two's-complement byte each."""
+    if fmt == "mxint8":
+        return codes.view(np.int8).astype(np.float64)
     lo = codes & 0xF
     hi = codes >> 4
     nib = np.stack([lo, hi], axis=-1).reshape(codes.shape[0], -1).astype(np.int64)

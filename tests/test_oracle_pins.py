@@ -22,7 +22,7 @@ from calibration_free_weight_dualquant_b200 import synth
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 
 PROJ_KIND = {"f16": oracle.PROJ_F16, "bf16": oracle.PROJ_BF16, "e4m3": oracle.PROJ_E4M3, "e8m0": oracle.PROJ_E8M0}
-A_KIND = {"int4": "f16", "mxint4": "e8m0", "nvfp4": "e4m3", "mxfp4": "e8m0"}
+A_KIND = {"int4": "f16", "mxint4": "e8m0", "nvfp4": "e4m3", "mxfp4": "e8m0", "mxint8": "e8m0"}
 
 
 def read_golden(name):
@@ -118,7 +118,7 @@ def test_storage_sizes():
 # Grid quantizer Q against exact rationals
 
 
-@pytest.mark.parametrize("fmt", ["int4", "nvfp4"])
+@pytest.mark.parametrize("fmt", ["int4", "nvfp4", "mxint8"])
 def test_quantizer_exact_rational(fmt):
     """Q = nearest grid value, ties to even, clip (DualQuant §3; reproduction README 'Local reproduction')."""
     rng = np.random.Generator(np.random.PCG64(11))
@@ -134,7 +134,8 @@ def test_quantizer_exact_rational(fmt):
             h = (Fraction(g[k]) + Fraction(g[k + 1])) / 2
             w = float(h * ab)
         else:
-            w = float(rng.uniform(-10, 10) * a * b)
+            span = 200 if fmt == "mxint8" else 10  # past both ends of the grid
+            w = float(rng.uniform(-span, span) * a * b)
         got = oracle.quant_value(fmt, w, float(ab))
         assert got == bf.grid_argmin(fmt, w, ab), (w, a, b)
 
@@ -198,6 +199,7 @@ TINY = [
     ("nvfp4", 16, "f16", 4, 32, "f32", 3),
     ("mxfp4", 32, "bf16", 6, 64, "bf16", 4),
     ("mxfp4", 32, "f16", 4, 64, "f32", 3),
+    ("mxint8", 32, "bf16", 4, 64, "bf16", 3),
 ]
 
 
@@ -235,7 +237,7 @@ def test_iterations_brute_force(fmt, G, col_dt, M, N, wdt, iters):
     sT = out["sT"]
     akind = A_KIND[fmt]
     # init: absmax RTN with beta = 1; NVFP4 tensor scale fp32(amax / (6*448))
-    qmax = 6.0 if fmt in ("nvfp4", "mxfp4") else 7.0
+    qmax = float(bf.grid_qmax(fmt))
     if fmt == "nvfp4":
         assert sT == float(np.float32(np.abs(Wv).max() / 2688.0))
     assert np.all(out["trace_b"][0] == 1.0)
@@ -293,7 +295,8 @@ def check_iterations(out, fmt, G, col_dt, Wv, iters):
                 assert b_next[j] == bf.argmin_scale_objective(col_dt, Wv[:, j], S[:, j]), (t, j)
 
 
-@pytest.mark.parametrize("fmt,G,col_dt", [("int4", 64, "f16"), ("mxint4", 32, "bf16"), ("nvfp4", 16, "bf16")])
+@pytest.mark.parametrize("fmt,G,col_dt", [("int4", 64, "f16"), ("mxint4", 32, "bf16"), ("nvfp4", 16, "bf16"),
+                                          ("mxint8", 32, "bf16")])
 def test_closed_form_is_least_squares(fmt, G, col_dt):
     """With codes fixed the unprojected update is the 1-D least-squares solution
     (reproduction README 'Core equations'; DualQuant App. B)."""
@@ -347,7 +350,8 @@ def test_zero_iterations_is_rtn_and_mse_monotone(name):
     assert s["mse"][-1] < s["mse"][0]
 
 
-@pytest.mark.parametrize("fmt,G,col_dt", [("int4", 64, "f16"), ("mxint4", 32, "bf16"), ("nvfp4", 16, "bf16")])
+@pytest.mark.parametrize("fmt,G,col_dt", [("int4", 64, "f16"), ("mxint4", 32, "bf16"), ("nvfp4", 16, "bf16"),
+                                          ("mxint8", 32, "bf16")])
 def test_half_steps_monotone(fmt, G, col_dt):
     """Objective non-increasing after every half-step, not only after codes settle."""
     Win, wdtype, _ = tiny_matrix(32, 4 * G, "bf16", seed=31)
@@ -393,7 +397,8 @@ def test_fixed_point_is_stationary(fmt, G, col_dt):
                 assert a[i, g] == bf.argmin_scale_objective(A_KIND[fmt], Wv[i, sl], R, sf)
 
 
-@pytest.mark.parametrize("fmt,G,col_dt", [("int4", 64, "f16"), ("mxint4", 32, "bf16"), ("nvfp4", 16, "bf16")])
+@pytest.mark.parametrize("fmt,G,col_dt", [("int4", 64, "f16"), ("mxint4", 32, "bf16"), ("nvfp4", 16, "bf16"),
+                                          ("mxint8", 32, "bf16")])
 def test_zero_slices(fmt, G, col_dt):
     """'Use scale 1 for an all-zero code slice' (reproduction README 'Core equations')."""
     Win, wdtype, Wv = tiny_matrix(8, 4 * G, "f32", seed=51)
@@ -409,7 +414,8 @@ def test_zero_slices(fmt, G, col_dt):
     assert np.all(z["codes"] == 0) and np.all(z["mse"] == 0.0)
 
 
-@pytest.mark.parametrize("fmt,G,col_dt", [("int4", 64, "f16"), ("mxint4", 32, "bf16"), ("nvfp4", 16, "bf16")])
+@pytest.mark.parametrize("fmt,G,col_dt", [("int4", 64, "f16"), ("mxint4", 32, "bf16"), ("nvfp4", 16, "bf16"),
+                                          ("mxint8", 32, "bf16")])
 def test_power_of_two_equivariance(fmt, G, col_dt):
     """W -> 2^k W scales the block inverse scales (or s_T) by 2^k and leaves codes and b unchanged."""
     Win, _, _ = tiny_matrix(16, 4 * G, "f32", seed=61)
@@ -588,7 +594,7 @@ def l1_expected_init(Wv, fmt, G, col_dt):
     sT = 1.0
     if fmt == "nvfp4" and amax > 0:
         sT = float(np.float32(amax / 2688.0))
-    qmax = 6.0 if fmt in ("nvfp4", "mxfp4") else 7.0
+    qmax = float(bf.grid_qmax(fmt))
     a = np.ones((M, N // G))
     for i in range(M):
         for g in range(N // G):
@@ -683,14 +689,15 @@ def test_warm_start_continues_the_iteration(init, fmt, G, col_dt):
     np.testing.assert_array_equal(full["changes"][4:], warm["changes"][1:])
 
 
-@pytest.mark.parametrize("fmt,G,col_dt", [("int4", 64, "f16"), ("mxint4", 32, "bf16"), ("nvfp4", 16, "bf16")])
+@pytest.mark.parametrize("fmt,G,col_dt", [("int4", 64, "f16"), ("mxint4", 32, "bf16"), ("nvfp4", 16, "bf16"),
+                                          ("mxint8", 32, "bf16")])
 def test_warm_start_rejects_inadmissible_scales(fmt, G, col_dt):
     """A warm start takes only admissible scales: elements of F_a and F_b, a positive fp32 s_T."""
     wl, (Win, wdt) = small_workload("nvfp4_g16_gateup_14336x4096", 8, 2 * 64, 19)
     r = oracle.rtn(Win, wdt, fmt, G, col_dt)
     ok = dict(a0=r["a"], b0=r["b"], sT0=r["sT"])
     oracle.solve(Win, wdt, fmt, G, 1, col_dt, init="given", **ok)
-    bad_a = {"int4": 1.0 + 2.0 ** -12, "mxint4": 0.75, "nvfp4": 1.0625}[fmt]
+    bad_a = {"int4": 1.0 + 2.0 ** -12, "mxint4": 0.75, "nvfp4": 1.0625, "mxint8": 0.75}[fmt]
     cases = [dict(ok, a0=np.where(np.arange(r["a"].size).reshape(r["a"].shape) == 3, bad_a, r["a"])),
              dict(ok, a0=-r["a"]), dict(ok, a0=r["a"] * 0.0),
              dict(ok, b0=np.where(np.arange(r["b"].size) == 2, 1.0 + 2.0 ** -14, r["b"])),
