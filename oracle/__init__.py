@@ -31,9 +31,9 @@ _LIB_PATH = os.path.join(_HERE, "libdq_oracle.so")
 INT4, MXINT4, NVFP4, MXFP4 = 0, 1, 2, 3
 F32, BF16, F16 = 0, 1, 2
 PROJ_F16, PROJ_BF16, PROJ_E4M3, PROJ_E8M0 = 0, 1, 2, 3
-MXINT8 = 4
-FORMATS = {"int4": INT4, "mxint4": MXINT4, "nvfp4": NVFP4, "mxfp4": MXFP4, "mxint8": MXINT8}
-BYTE_CODE_FORMATS = ("mxint8",)  # one byte per code; the others pack two nibbles per byte
+MXINT8, MXFP8 = 4, 5
+FORMATS = {"int4": INT4, "mxint4": MXINT4, "nvfp4": NVFP4, "mxfp4": MXFP4, "mxint8": MXINT8, "mxfp8": MXFP8}
+BYTE_CODE_FORMATS = ("mxint8", "mxfp8")  # one byte per code; the others pack two nibbles per byte
 WDTYPES = {"f32": F32, "bf16": BF16, "f16": F16}
 
 _lib = None
@@ -127,7 +127,7 @@ def solve(W: np.ndarray, wdtype: str, fmt: str, group: int, iters: int, col_dtyp
     or "given" (warm start from stored block scales a0 [M, N/G], column scales b0 [N] and, for
     NVFP4, the tensor scale sT0).
 
-    Returns codes [M, N/2] uint8 ([M, N] for MXINT8), a [M, N/G] (stored block-scale values: fp16
+    Returns codes [M, N/2] uint8 ([M, N] for MXINT8 and MXFP8), a [M, N/G] (stored block-scale values: fp16
     value, 2^k, or E4M3 value e for NVFP4), b [N], sT (NVFP4 tensor scale, 1
     otherwise), mse [iters+1]; optionally q [M, N] grid values, per-iteration
     traces of a and b, and changes [iters+1] (elements whose grid value changed

@@ -42,6 +42,11 @@
  *    codebook [-128,127] with E8M0 power-of-two block scales, group 32, one
  *    byte per code; the OCP element's fixed 2^-6 factor is a power of two and
  *    is absorbed into the block scale.
+ *  - MXFP8 (the same passage): the FP8 E4M3 codebook (1 sign, 4 exponent bits
+ *    with bias 7, 3 mantissa bits, subnormals, largest finite value 448, no
+ *    infinities) with E8M0 power-of-two block scales, group 32, absmax qmax
+ *    448, ties to the value with an even mantissa bit, one byte per code (the
+ *    E4M3 bit pattern; zero is always 0x00).
  */
 #include <math.h>
 #include <stdint.h>
@@ -59,6 +64,7 @@
 #define DQO_NVFP4 2
 #define DQO_MXFP4 3 /* E2M1 grid with E8M0 block scales (the MX family's FP4 member) */
 #define DQO_MXINT8 4 /* INT8 grid [-128,127] with E8M0 block scales (the MX family's INT8 member) */
+#define DQO_MXFP8 5  /* FP8 E4M3 grid with E8M0 block scales (the MX family's FP8 E4M3 member) */
 /* element dtypes */
 #define DQO_F32 0
 #define DQO_BF16 1
@@ -78,13 +84,38 @@ static const unsigned char INT4_EVEN[16] = {1, 0, 1, 0, 1, 0, 1, 0, 1, 0, 1, 0, 
  * magnitudes 0,0.5,1,1.5,2,3,4,6 have encodings 000,001,010,011,100,101,110,111 */
 static const double E2M1_GRID[15] = {-6, -4, -3, -2, -1.5, -1, -0.5, 0, 0.5, 1, 1.5, 2, 3, 4, 6};
 static const unsigned char E2M1_EVEN[15] = {0, 1, 0, 1, 0, 1, 0, 1, 0, 1, 0, 1, 0, 1, 0};
-/* INT8 codebook -128..127 and its even flags, filled once by int8_grid_init() */
+/* INT8 codebook -128..127 and its even flags (filled by grids_init(), with the E4M3 table) */
 static double INT8_GRID[256];
 static unsigned char INT8_EVEN[256];
-static void int8_grid_init(void) {
+/* E4M3 values in ascending order (253: +-126 nonzero magnitudes and zero) and
+ * whether each has mantissa bit 0; the magnitude with exponent field e and
+ * mantissa m is m * 2^-9 for e = 0 and (1 + m/8) * 2^(e-7) otherwise, the
+ * pattern e = 15, m = 7 being NaN. */
+static double E4M3_GRID[253];
+static unsigned char E4M3_EVEN[253];
+static void grids_init(void) {
   for (int k = 0; k < 256; ++k) {
     INT8_GRID[k] = (double)(k - 128);
     INT8_EVEN[k] = (unsigned char)((k - 128) % 2 == 0);
+  }
+  double mag[127];
+  unsigned char ev[127];
+  int n = 0;
+  for (int e = 0; e < 16; ++e)
+    for (int m = 0; m < 8; ++m) {
+      if (e == 15 && m == 7) continue;
+      mag[n] = (e == 0) ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+      ev[n] = (unsigned char)(m % 2 == 0);
+      ++n;
+    }
+  /* mag[] ascends with the bit pattern; mirror it for the negative half */
+  for (int k = 0; k < 126; ++k) {
+    E4M3_GRID[k] = -mag[126 - k];
+    E4M3_EVEN[k] = ev[126 - k];
+  }
+  for (int k = 0; k < 127; ++k) {
+    E4M3_GRID[126 + k] = mag[k];
+    E4M3_EVEN[126 + k] = ev[k];
   }
 }
 
@@ -234,10 +265,15 @@ typedef struct {
 /* the formats on the E2M1 grid */
 static int e2m1_grid(int fmt) { return fmt == DQO_NVFP4 || fmt == DQO_MXFP4; }
 
-static double qmax_of(int fmt) { return e2m1_grid(fmt) ? 6.0 : (fmt == DQO_MXINT8 ? 127.0 : 7.0); }
+static double qmax_of(int fmt) {
+  if (e2m1_grid(fmt)) return 6.0;
+  if (fmt == DQO_MXINT8) return 127.0;
+  if (fmt == DQO_MXFP8) return 448.0;
+  return 7.0;
+}
 
 /* formats with 8-bit codes (one byte per element) */
-static int byte_codes(int fmt) { return fmt == DQO_MXINT8; }
+static int byte_codes(int fmt) { return fmt == DQO_MXINT8 || fmt == DQO_MXFP8; }
 
 /* block inverse scale value a from its stored factor (NVFP4 stores e, a = s_T*e) */
 static double a_value(const problem* p, double stored) { return p->fmt == DQO_NVFP4 ? p->sT * stored : stored; }
@@ -245,7 +281,8 @@ static double a_value(const problem* p, double stored) { return p->fmt == DQO_NV
 /* projection of an LS inverse-scale value onto F_a; returns the stored factor */
 static double project_a(const problem* p, double v) {
   if (p->fmt == DQO_INT4) return dqo_project(DQO_PROJ_F16, v);
-  if (p->fmt == DQO_MXINT4 || p->fmt == DQO_MXFP4 || p->fmt == DQO_MXINT8) return dqo_project(DQO_PROJ_E8M0, v);
+  if (p->fmt == DQO_MXINT4 || p->fmt == DQO_MXFP4 || p->fmt == DQO_MXINT8 || p->fmt == DQO_MXFP8)
+    return dqo_project(DQO_PROJ_E8M0, v);
   return dqo_project(DQO_PROJ_E4M3, v / p->sT); /* nearest s_T*e to v */
 }
 
@@ -254,6 +291,7 @@ static double quant_value(const problem* p, double w, double a, double b) {
   double ab = a * b;
   if (e2m1_grid(p->fmt)) return E2M1_GRID[dqo_quant_index(w, ab, E2M1_GRID, E2M1_EVEN, 15)];
   if (p->fmt == DQO_MXINT8) return INT8_GRID[dqo_quant_index(w, ab, INT8_GRID, INT8_EVEN, 256)];
+  if (p->fmt == DQO_MXFP8) return E4M3_GRID[dqo_quant_index(w, ab, E4M3_GRID, E4M3_EVEN, 253)];
   return INT4_GRID[dqo_quant_index(w, ab, INT4_GRID, INT4_EVEN, 16)];
 }
 
@@ -512,8 +550,8 @@ static int init_given(problem* p, const double* a0, const double* b0, double sT0
 static int load_problem(problem* p, const void* W, int wdt, int64_t M, int64_t N, int fmt, int G, int col_dt,
                         double** Wd_out) {
   if (!W || M <= 0 || N <= 0 || G <= 0 || N % G != 0 || N % 2 != 0) return DQO_EINVAL;
-  if (fmt < 0 || fmt > 4 || (col_dt != DQO_F16 && col_dt != DQO_BF16)) return DQO_EINVAL;
-  int8_grid_init();
+  if (fmt < 0 || fmt > 5 || (col_dt != DQO_F16 && col_dt != DQO_BF16)) return DQO_EINVAL;
+  grids_init();
   double* Wd = (double*)malloc(sizeof(double) * (size_t)(M * N));
   if (!Wd) return DQO_ENOMEM;
   int bad = 0;
@@ -555,8 +593,13 @@ static int load_problem(problem* p, const void* W, int wdt, int64_t M, int64_t N
 
 static void pack_codes(const problem* p, const double* q, uint8_t* codes) {
   int64_t M = p->M, N = p->N;
-  if (byte_codes(p->fmt)) { /* one two's-complement byte per element */
+  if (p->fmt == DQO_MXINT8) { /* one two's-complement byte per element */
     for (int64_t k = 0; k < M * N; ++k) codes[k] = (uint8_t)((int)q[k] & 0xFF);
+    return;
+  }
+  if (p->fmt == DQO_MXFP8) { /* one E4M3 bit pattern per element, zero as 0x00 */
+    for (int64_t k = 0; k < M * N; ++k)
+      codes[k] = (q[k] == 0.0) ? 0 : (uint8_t)((q[k] < 0 ? 0x80 : 0) | encode_float_bits(fabs(q[k]), 3, -6, 4));
     return;
   }
   for (int64_t i = 0; i < M; ++i)
@@ -581,7 +624,8 @@ static void pack_codes(const problem* p, const double* q, uint8_t* codes) {
  *     column update (codes fixed) -> project -> requantize; mse[t]
  * Outputs (any may be NULL except mse when iters >= 0 is wanted):
  *   codes      [M][N/2] packed nibbles, even column in the low nibble (MXINT8:
- *              [M][N], one two's-complement byte per element)
+ *              [M][N], one two's-complement byte per element; MXFP8: [M][N],
+ *              one E4M3 bit pattern per element)
  *   a_out      [M][N/G] stored block scale values (fp16 value / 2^k / E4M3 e)
  *   b_out      [N] column inverse scales
  *   sT_out     NVFP4 tensor scale (1 for the other formats)
@@ -756,8 +800,12 @@ uint32_t dqo_encode(int kind, double v) {
 double dqo_quant_value(int fmt, double w, double ab) {
   if (e2m1_grid(fmt)) return E2M1_GRID[dqo_quant_index(w, ab, E2M1_GRID, E2M1_EVEN, 15)];
   if (fmt == DQO_MXINT8) {
-    int8_grid_init();
+    grids_init();
     return INT8_GRID[dqo_quant_index(w, ab, INT8_GRID, INT8_EVEN, 256)];
+  }
+  if (fmt == DQO_MXFP8) {
+    grids_init();
+    return E4M3_GRID[dqo_quant_index(w, ab, E4M3_GRID, E4M3_EVEN, 253)];
   }
   return INT4_GRID[dqo_quant_index(w, ab, INT4_GRID, INT4_EVEN, 16)];
 }

@@ -19,21 +19,38 @@ E2M1_MAGS = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]  # encodings 0..7
 E2M1_VALUES = sorted(set([-m for m in E2M1_MAGS] + E2M1_MAGS))
 
 
+@lru_cache(maxsize=None)
+def e4m3_values():
+    """Every finite FP8 E4M3 value (torch float8_e4m3fn bit patterns 0x00..0x7E and their negatives,
+    zero once), ascending, with the mantissa-bit-even flag of its encoding."""
+    bits = np.arange(0, 0x7F, dtype=np.uint8)
+    mags = torch.from_numpy(bits).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    even = {}
+    for b, m in zip(bits.tolist(), mags.tolist()):
+        even[m] = even[-m] = (b & 1) == 0
+    vals = sorted(set(mags.tolist()) | set((-mags).tolist()))
+    return vals, even
+
+
 def grid_values(fmt: str):
     if fmt == "mxint8":
         return INT8_VALUES
+    if fmt == "mxfp8":
+        return e4m3_values()[0]
     return INT4_VALUES if fmt in ("int4", "mxint4") else E2M1_VALUES
 
 
 def grid_qmax(fmt: str) -> int:
     """qmax of the absmax init: largest positive grid value."""
-    return {"mxint8": 127, "nvfp4": 6, "mxfp4": 6}.get(fmt, 7)
+    return {"mxint8": 127, "nvfp4": 6, "mxfp4": 6, "mxfp8": 448}.get(fmt, 7)
 
 
 def grid_is_even(fmt: str, v: float) -> bool:
-    """Tie winner flag: even integer (INT4) or even mantissa bit of the E2M1 encoding."""
+    """Tie winner flag: even integer (INT4/INT8) or even mantissa bit of the E2M1 / E4M3 encoding."""
     if fmt in ("int4", "mxint4", "mxint8"):
         return int(v) % 2 == 0
+    if fmt == "mxfp8":
+        return e4m3_values()[1][float(v)]
     return E2M1_MAGS.index(abs(v)) % 2 == 0
 
 
@@ -131,9 +148,11 @@ def argmin_scale_objective(kind: str, W: np.ndarray, R: np.ndarray, scale_factor
 
 def decode_codes(fmt: str, codes: np.ndarray) -> np.ndarray:
     """Unpack nibble codes [M, N/2] -> grid values [M, N] (even column in the low nibble);
-    MXINT8 codes [M, N] are one two's-complement byte each."""
+    MXINT8 codes [M, N] are one two's-complement byte each, MXFP8 codes [M, N] one E4M3 pattern each."""
     if fmt == "mxint8":
         return codes.view(np.int8).astype(np.float64)
+    if fmt == "mxfp8":
+        return torch.from_numpy(np.ascontiguousarray(codes)).view(torch.float8_e4m3fn).to(torch.float64).numpy()
     lo = codes & 0xF
     hi = codes >> 4
     nib = np.stack([lo, hi], axis=-1).reshape(codes.shape[0], -1).astype(np.int64)

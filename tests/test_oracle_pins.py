@@ -22,7 +22,7 @@ from calibration_free_weight_dualquant_b200 import synth
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 
 PROJ_KIND = {"f16": oracle.PROJ_F16, "bf16": oracle.PROJ_BF16, "e4m3": oracle.PROJ_E4M3, "e8m0": oracle.PROJ_E8M0}
-A_KIND = {"int4": "f16", "mxint4": "e8m0", "nvfp4": "e4m3", "mxfp4": "e8m0", "mxint8": "e8m0"}
+A_KIND = {"int4": "f16", "mxint4": "e8m0", "nvfp4": "e4m3", "mxfp4": "e8m0", "mxint8": "e8m0", "mxfp8": "e8m0"}
 
 
 def read_golden(name):
@@ -118,7 +118,7 @@ def test_storage_sizes():
 # Grid quantizer Q against exact rationals
 
 
-@pytest.mark.parametrize("fmt", ["int4", "nvfp4", "mxint8"])
+@pytest.mark.parametrize("fmt", ["int4", "nvfp4", "mxint8", "mxfp8"])
 def test_quantizer_exact_rational(fmt):
     """Q = nearest grid value, ties to even, clip (DualQuant §3; reproduction README 'Local reproduction')."""
     rng = np.random.Generator(np.random.PCG64(11))
@@ -134,8 +134,11 @@ def test_quantizer_exact_rational(fmt):
             h = (Fraction(g[k]) + Fraction(g[k + 1])) / 2
             w = float(h * ab)
         else:
-            span = 200 if fmt == "mxint8" else 10  # past both ends of the grid
-            w = float(rng.uniform(-span, span) * a * b)
+            span = {"mxint8": 200, "mxfp8": 600}.get(fmt, 10)  # past both ends of the grid
+            x = rng.uniform(-span, span)
+            if fmt == "mxfp8" and trial % 3 == 1:  # every binade, subnormals included
+                x = float(np.sign(x)) * 2.0 ** rng.uniform(-12, 9.5)
+            w = float(x * a * b)
         got = oracle.quant_value(fmt, w, float(ab))
         assert got == bf.grid_argmin(fmt, w, ab), (w, a, b)
 
@@ -148,6 +151,26 @@ def test_quantizer_tie_cases():
     cases_fp4 = {0.25: 0, 0.75: 1, 1.25: 1, 1.75: 2, 2.5: 2, 3.5: 4, 5.0: 4, 7.0: 6, -5.0: -4, -0.25: 0}
     for x, q in cases_fp4.items():
         assert oracle.quant_value("nvfp4", x, 1.0) == q
+
+
+def test_quantizer_e4m3_matches_library_cast():
+    """The MXFP8 element grid is FP8 E4M3: inside its range, Q(x) with unit scale equals torch's
+    round-to-nearest-even cast to float8_e4m3fn (binade interiors, midpoints, subnormals); beyond
+    448 it clips.  Midpoint cases: 1.0625 lies between 1 (mantissa 0) and 1.125 (mantissa 1) -> 1;
+    1.1875 -> 1.25; the subnormal midpoint 3 * 2^-10 -> 2^-8; 2^-10 -> 0."""
+    rng = np.random.Generator(np.random.PCG64(21))
+    xs = np.concatenate([np.sign(rng.uniform(-1, 1, 3000)) * 2.0 ** rng.uniform(-12, np.log2(448), 3000),
+                         rng.uniform(-448, 448, 1000)]).astype(np.float32)
+    vals, _ = bf.e4m3_values()
+    v = np.array(vals)
+    mids = ((v[:-1] + v[1:]) / 2).astype(np.float32)   # exact in fp32
+    xs = np.concatenate([xs, mids, -mids, np.float32([0.0, 448.0, -448.0])])
+    want = torch.from_numpy(xs).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    for x, w in zip(xs.tolist(), want.tolist()):
+        assert oracle.quant_value("mxfp8", x, 1.0) == w, (x, w)
+    for x, q in {1.0625: 1.0, 1.1875: 1.25, 3 * 2.0 ** -10: 2.0 ** -8, 2.0 ** -10: 0.0, 464.0: 448.0,
+                 1e6: 448.0, -1e6: -448.0, -2.0 ** -10: 0.0}.items():
+        assert oracle.quant_value("mxfp8", x, 1.0) == q, x
 
 
 # ---------------------------------------------------------------------------
@@ -200,6 +223,8 @@ TINY = [
     ("mxfp4", 32, "bf16", 6, 64, "bf16", 4),
     ("mxfp4", 32, "f16", 4, 64, "f32", 3),
     ("mxint8", 32, "bf16", 4, 64, "bf16", 3),
+    ("mxfp8", 32, "bf16", 4, 64, "bf16", 3),
+    ("mxfp8", 32, "f16", 4, 64, "f32", 3),
 ]
 
 
@@ -296,7 +321,7 @@ def check_iterations(out, fmt, G, col_dt, Wv, iters):
 
 
 @pytest.mark.parametrize("fmt,G,col_dt", [("int4", 64, "f16"), ("mxint4", 32, "bf16"), ("nvfp4", 16, "bf16"),
-                                          ("mxint8", 32, "bf16")])
+                                          ("mxint8", 32, "bf16"), ("mxfp8", 32, "bf16")])
 def test_closed_form_is_least_squares(fmt, G, col_dt):
     """With codes fixed the unprojected update is the 1-D least-squares solution
     (reproduction README 'Core equations'; DualQuant App. B)."""
@@ -351,7 +376,7 @@ def test_zero_iterations_is_rtn_and_mse_monotone(name):
 
 
 @pytest.mark.parametrize("fmt,G,col_dt", [("int4", 64, "f16"), ("mxint4", 32, "bf16"), ("nvfp4", 16, "bf16"),
-                                          ("mxint8", 32, "bf16")])
+                                          ("mxint8", 32, "bf16"), ("mxfp8", 32, "bf16")])
 def test_half_steps_monotone(fmt, G, col_dt):
     """Objective non-increasing after every half-step, not only after codes settle."""
     Win, wdtype, _ = tiny_matrix(32, 4 * G, "bf16", seed=31)
@@ -398,7 +423,7 @@ def test_fixed_point_is_stationary(fmt, G, col_dt):
 
 
 @pytest.mark.parametrize("fmt,G,col_dt", [("int4", 64, "f16"), ("mxint4", 32, "bf16"), ("nvfp4", 16, "bf16"),
-                                          ("mxint8", 32, "bf16")])
+                                          ("mxint8", 32, "bf16"), ("mxfp8", 32, "bf16")])
 def test_zero_slices(fmt, G, col_dt):
     """'Use scale 1 for an all-zero code slice' (reproduction README 'Core equations')."""
     Win, wdtype, Wv = tiny_matrix(8, 4 * G, "f32", seed=51)
@@ -415,7 +440,7 @@ def test_zero_slices(fmt, G, col_dt):
 
 
 @pytest.mark.parametrize("fmt,G,col_dt", [("int4", 64, "f16"), ("mxint4", 32, "bf16"), ("nvfp4", 16, "bf16"),
-                                          ("mxint8", 32, "bf16")])
+                                          ("mxint8", 32, "bf16"), ("mxfp8", 32, "bf16")])
 def test_power_of_two_equivariance(fmt, G, col_dt):
     """W -> 2^k W scales the block inverse scales (or s_T) by 2^k and leaves codes and b unchanged."""
     Win, _, _ = tiny_matrix(16, 4 * G, "f32", seed=61)
@@ -690,14 +715,14 @@ def test_warm_start_continues_the_iteration(init, fmt, G, col_dt):
 
 
 @pytest.mark.parametrize("fmt,G,col_dt", [("int4", 64, "f16"), ("mxint4", 32, "bf16"), ("nvfp4", 16, "bf16"),
-                                          ("mxint8", 32, "bf16")])
+                                          ("mxint8", 32, "bf16"), ("mxfp8", 32, "bf16")])
 def test_warm_start_rejects_inadmissible_scales(fmt, G, col_dt):
     """A warm start takes only admissible scales: elements of F_a and F_b, a positive fp32 s_T."""
     wl, (Win, wdt) = small_workload("nvfp4_g16_gateup_14336x4096", 8, 2 * 64, 19)
     r = oracle.rtn(Win, wdt, fmt, G, col_dt)
     ok = dict(a0=r["a"], b0=r["b"], sT0=r["sT"])
     oracle.solve(Win, wdt, fmt, G, 1, col_dt, init="given", **ok)
-    bad_a = {"int4": 1.0 + 2.0 ** -12, "mxint4": 0.75, "nvfp4": 1.0625, "mxint8": 0.75}[fmt]
+    bad_a = {"int4": 1.0 + 2.0 ** -12, "mxint4": 0.75, "nvfp4": 1.0625, "mxint8": 0.75, "mxfp8": 0.75}[fmt]
     cases = [dict(ok, a0=np.where(np.arange(r["a"].size).reshape(r["a"].shape) == 3, bad_a, r["a"])),
              dict(ok, a0=-r["a"]), dict(ok, a0=r["a"] * 0.0),
              dict(ok, b0=np.where(np.arange(r["b"].size) == 2, 1.0 + 2.0 ** -14, r["b"])),
