@@ -25,13 +25,23 @@ class Format(enum.IntEnum):
     MXINT4 = 1
     NVFP4 = 2
     MXFP4 = 3
+    MXINT8 = 4
+    MXFP8 = 5
 
 
-_FMT_NAMES = {"int4": Format.INT4, "mxint4": Format.MXINT4, "nvfp4": Format.NVFP4, "mxfp4": Format.MXFP4}
+_FMT_NAMES = {"int4": Format.INT4, "mxint4": Format.MXINT4, "nvfp4": Format.NVFP4, "mxfp4": Format.MXFP4,
+              "mxint8": Format.MXINT8, "mxfp8": Format.MXFP8}
 _DTYPES = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
 _COL_DTYPES = {"f16": torch.float16, "bf16": torch.bfloat16}
-DEFAULT_GROUP = {Format.INT4: 64, Format.MXINT4: 32, Format.NVFP4: 16, Format.MXFP4: 32}
-DEFAULT_COL_DTYPE = {Format.INT4: "f16", Format.MXINT4: "bf16", Format.NVFP4: "bf16", Format.MXFP4: "bf16"}
+DEFAULT_GROUP = {Format.INT4: 64, Format.MXINT4: 32, Format.NVFP4: 16, Format.MXFP4: 32, Format.MXINT8: 32,
+                 Format.MXFP8: 32}
+DEFAULT_COL_DTYPE = {Format.INT4: "f16", Format.MXINT4: "bf16", Format.NVFP4: "bf16", Format.MXFP4: "bf16",
+                     Format.MXINT8: "bf16", Format.MXFP8: "bf16"}
+
+
+def code_cols(cols: int, fmt) -> int:
+    """Bytes of codes per row: one per element on the INT8 and E4M3 grids, two nibbles per byte otherwise."""
+    return cols if _fmt(fmt) in (Format.MXINT8, Format.MXFP8) else cols // 2
 
 
 class DQError(RuntimeError):
@@ -110,7 +120,7 @@ def output_nbytes(rows: int, cols: int, fmt, group: Optional[int] = None, col_dt
     f = _fmt(fmt)
     g = DEFAULT_GROUP[f] if group is None else group
     cd = DEFAULT_COL_DTYPE[f] if col_dtype is None else col_dtype
-    return {"codes": rows * cols // 2, "block_scales": rows * (cols // g) * (2 if f == Format.INT4 else 1),
+    return {"codes": rows * code_cols(cols, f), "block_scales": rows * (cols // g) * (2 if f == Format.INT4 else 1),
             "col_scales": cols * 2, "tensor_scale": 4 if f == Format.NVFP4 else 0}
 
 
@@ -124,7 +134,7 @@ def alloc_outputs(rows: int, cols: int, fmt, group: int, col_dtype: str, iters: 
     f = _fmt(fmt)
     nb = cols // group
     return {
-        "codes": torch.empty((rows, cols // 2), dtype=torch.uint8, device=device),
+        "codes": torch.empty((rows, code_cols(cols, f)), dtype=torch.uint8, device=device),
         "block_scales": torch.empty((rows, nb), dtype=torch.float16 if f == Format.INT4 else torch.uint8,
                                     device=device),
         "tensor_scale": torch.empty(1, dtype=torch.float32, device=device),

@@ -226,7 +226,8 @@ extern "C" int dq_act_quant(const void* X, int x_dtype, int64_t rows, int64_t co
                             int col_dtype, int format, int group, const dq_outputs* out, void* workspace,
                             size_t workspace_bytes, void* stream) {
   if (rows <= 0 || cols <= 0 || group <= 0 || cols % group != 0) return DQ_EINVAL;
-  if (format < DQ_INT4 || format > DQ_MXFP4) return DQ_EINVAL;
+  if (format < DQ_INT4 || format > DQ_MXFP8) return DQ_EINVAL;
+  if (format == DQ_MXINT8 || format == DQ_MXFP8) return DQ_EUNSUPPORTED;  // 4-bit codes only
   if ((format == DQ_MXINT4 || format == DQ_MXFP4) && group != 32) return DQ_EUNSUPPORTED;
   if (format == DQ_NVFP4 && group != 16) return DQ_EUNSUPPORTED;
   if (group < 8 || group > 256 || (group & (group - 1)) != 0) return DQ_EUNSUPPORTED;

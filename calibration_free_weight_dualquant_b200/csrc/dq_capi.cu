@@ -23,9 +23,10 @@ struct Plan {
 // Argument checks that do not touch memory.  Returns DQ_OK or an error code.
 int check_shape(int64_t rows, int64_t cols, int format, int group) {
   if (rows <= 0 || cols <= 0 || (cols & 1) || group <= 0) return DQ_EINVAL;
-  if (format < DQ_INT4 || format > DQ_MXFP4) return DQ_EINVAL;
+  if (format < DQ_INT4 || format > DQ_MXFP8) return DQ_EINVAL;
   if (cols % group != 0) return DQ_EINVAL;
-  if ((format == DQ_MXINT4 || format == DQ_MXFP4) && group != 32) return DQ_EUNSUPPORTED;
+  if ((format == DQ_MXINT4 || format == DQ_MXFP4 || format == DQ_MXINT8 || format == DQ_MXFP8) && group != 32)
+    return DQ_EUNSUPPORTED;
   if (format == DQ_NVFP4 && group != 16) return DQ_EUNSUPPORTED;
   // a block spans group/8 lanes of a warp: a power of two from 1 to 32
   if (group < 8 || group > dq::kStripMax || (group & (group - 1)) != 0) return DQ_EUNSUPPORTED;
@@ -98,10 +99,13 @@ int make_plan(int64_t M, int64_t N, int group, int init, Plan* pl) {
 
 bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
+// formats with one byte per code
+bool byte_code_format(int format) { return format == DQ_MXINT8 || format == DQ_MXFP8; }
+
 int check_outputs(const dq_outputs* out, int format, int col_dtype) {
   if (!out || !out->codes || !out->block_scales || !out->col_scales || !out->mse) return DQ_EINVAL;
   if (format == DQ_NVFP4 && !out->tensor_scale) return DQ_EINVAL;
-  if (!aligned(out->codes, 4) || !aligned(out->block_scales, 2) || !aligned(out->col_scales, 2) ||
+  if (!aligned(out->codes, byte_code_format(format) ? 8 : 4) || !aligned(out->block_scales, 2) || !aligned(out->col_scales, 2) ||
       !aligned(out->mse, 8) || (out->tensor_scale && !aligned(out->tensor_scale, 4)))
     return DQ_EINVAL;
   (void)col_dtype;
@@ -270,6 +274,10 @@ int dq_diagnostics(const void* workspace, void* stream, uint64_t out[4]) {
 }
 
 static size_t wsize(int dt) { return dt == DQ_F32 ? 4 : 2; }
+// bytes of the codes: one per element on the INT8 and E4M3 grids, else two per byte
+static size_t code_bytes(int64_t rows, int64_t cols, int format) {
+  return byte_code_format(format) ? (size_t)rows * cols : (size_t)rows * cols / 2;
+}
 
 size_t dq_host_workspace_bytes(int64_t rows, int64_t cols, int w_dtype, int format, int group, int iters) {
   if (w_dtype < DQ_F32 || w_dtype > DQ_F16 || iters < 0) return 0;
@@ -277,7 +285,7 @@ size_t dq_host_workspace_bytes(int64_t rows, int64_t cols, int w_dtype, int form
   if (solver == 0) return 0;
   const size_t nb = (size_t)(cols / group);
   size_t tot = align_up((size_t)rows * cols * wsize(w_dtype));
-  tot += align_up((size_t)rows * cols / 2);
+  tot += align_up(code_bytes(rows, cols, format));
   tot += align_up((size_t)rows * nb * (format == DQ_INT4 ? 2 : 1));
   tot += kAlign;  // tensor scale
   tot += align_up((size_t)cols * 2);
@@ -299,7 +307,7 @@ int dq_solve_host(const void* W_host, int w_dtype, int64_t rows, int64_t cols, i
   char* base = static_cast<char*>(device_workspace);
   const size_t nb = (size_t)(cols / group);
   const size_t bytes_w = (size_t)rows * cols * wsize(w_dtype);
-  const size_t bytes_codes = (size_t)rows * cols / 2;
+  const size_t bytes_codes = code_bytes(rows, cols, format);
   const size_t bytes_a = (size_t)rows * nb * (format == DQ_INT4 ? 2 : 1);
   const size_t bytes_b = (size_t)cols * 2;
   const size_t bytes_mse = (size_t)(iters + 1) * sizeof(double);

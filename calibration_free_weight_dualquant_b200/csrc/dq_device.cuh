@@ -1,5 +1,5 @@
 // dq_device.cuh -- device-side format helpers of the B200 DualQuant solver:
-// grid quantizers Q (INT4 [-8,7] and E2M1), projections of inverse scales onto
+// grid quantizers Q (INT4 [-8,7], INT8 [-128,127], E2M1 and E4M3), projections of inverse scales onto
 // the admissible sets (fp16, bf16, E4M3, E8M0 power of two), and storage
 // decode/encode of block and column scales.
 //
@@ -20,17 +20,33 @@
 
 namespace dq {
 
-enum : int { FMT_INT4 = 0, FMT_MXINT4 = 1, FMT_NVFP4 = 2, FMT_MXFP4 = 3 };
+enum : int { FMT_INT4 = 0, FMT_MXINT4 = 1, FMT_NVFP4 = 2, FMT_MXFP4 = 3, FMT_MXINT8 = 4, FMT_MXFP8 = 5 };
 // formats on the E2M1 grid, and formats with power-of-two (E8M0) block scales
 __host__ __device__ constexpr bool fmt_e2m1(int f) { return f == FMT_NVFP4 || f == FMT_MXFP4; }
-__host__ __device__ constexpr bool fmt_pow2(int f) { return f == FMT_MXINT4 || f == FMT_MXFP4; }
+__host__ __device__ constexpr bool fmt_pow2(int f) {
+  return f == FMT_MXINT4 || f == FMT_MXFP4 || f == FMT_MXINT8 || f == FMT_MXFP8;
+}
+// the FP8 E4M3 grid (MXFP8)
+__host__ __device__ constexpr bool fmt_e4m3(int f) { return f == FMT_MXFP8; }
+// integer grids with power-of-two block scales (MXINT4, MXINT8)
+__host__ __device__ constexpr bool fmt_mxint(int f) { return f == FMT_MXINT4 || f == FMT_MXINT8; }
+// one byte per code (INT8 and E4M3 grids) instead of two nibbles per byte
+__host__ __device__ constexpr bool fmt_byte_codes(int f) { return f == FMT_MXINT8 || f == FMT_MXFP8; }
+// ends of the integer grids, and qmax of the absmax initialization
+__host__ __device__ constexpr float grid_lo(int f) { return f == FMT_MXINT8 ? -128.f : -8.f; }
+__host__ __device__ constexpr float grid_hi(int f) { return f == FMT_MXINT8 ? 127.f : 7.f; }
+__host__ __device__ constexpr double grid_qmax(int f) {
+  return fmt_e2m1(f) ? 6.0 : (f == FMT_MXINT8 ? 127.0 : (f == FMT_MXFP8 ? 448.0 : 7.0));
+}
 enum : int { DT_F32 = 0, DT_BF16 = 1, DT_F16 = 2 };
 
 // Distance (in grid units) from a rounding boundary inside which the fast fp32
 // candidate x~ = (W * (1/b)) * (1/a) is not trusted and the decision is taken
 // exactly.  The candidate's relative error is below 6 * 2^-24 (at most six
 // correctly rounded fp32 operations), i.e. below 3.1e-6 grid units for
-// |x| <= 8.5, far inside this guard.
+// |x| <= 8.5, far inside this guard, and below 4.6e-5 grid units for
+// |x| <= 128.5 (INT8 grid; boundaries further out separate two values that
+// clip to the same grid end), still inside it.
 constexpr float kGuard = 0x1p-14f;
 
 // ---------------------------------------------------------------------------
@@ -151,7 +167,7 @@ __device__ __forceinline__ double ab_exact(float astored, float b, double sTd) {
 
 template <int FMT>
 __device__ __forceinline__ float q_int4(float xt, float w, float a, float b, double sTd) {
-  const float c = fminf(fmaxf(xt, -8.f), 7.f);
+  const float c = fminf(fmaxf(xt, grid_lo(FMT)), grid_hi(FMT));
   float q = __fsub_rn(__fadd_rn(c, 12582912.f), 12582912.f);  // round half even
   const float r = c - q;
   if (fabsf(r) > 0.5f - kGuard) {
@@ -159,7 +175,7 @@ __device__ __forceinline__ float q_int4(float xt, float w, float a, float b, dou
     const double d = fma(-(double)h, ab_exact<FMT>(a, b, sTd), (double)w);
     const float lo = h - 0.5f, hi = h + 0.5f;
     q = d > 0.0 ? hi : (d < 0.0 ? lo : (fmodf(lo, 2.f) == 0.f ? lo : hi));
-    q = fminf(fmaxf(q, -8.f), 7.f);
+    q = fminf(fmaxf(q, grid_lo(FMT)), grid_hi(FMT));
   }
   return q;
 }
@@ -186,6 +202,31 @@ __device__ __forceinline__ float q_e2m1(float xt, float w, float a, float b, dou
   return copysignf(qm, xt);
 }
 
+// FP8 E4M3 magnitudes: binade [2^E, 2^(E+1)) with E >= -6 has spacing 2^(E-3),
+// below 2^-6 the subnormal spacing 2^-9; 448 is the largest value and larger
+// magnitudes clip to it.  Rounding to a multiple of the local spacing with
+// half-even gives the even-mantissa tie rule (the spacing's multiples
+// alternate mantissa parity, across binade ends too).  Near a boundary h the
+// side is the sign of |w| - h*a*b, formed in fp64 (h has 5 significant bits).
+template <int FMT>
+__device__ __forceinline__ float q_e4m3(float xt, float w, float a, float b, double sTd) {
+  const float ax = fminf(fabsf(xt), 448.f);
+  const float p2 = __uint_as_float(max(__float_as_uint(ax) & 0x7F800000u, 0x3C800000u));  // binade base, >= 2^-6
+  const float magic = p2 * 1572864.f;  // 1.5 * 2^23 * (p2 / 8)
+  float qm = __fsub_rn(__fadd_rn(ax, magic), magic);
+  const float half = p2 * 0.0625f;
+  const float r = ax - qm;
+  if (fabsf(r) > half - p2 * 0x1p-14f) {
+    const float h = qm + copysignf(half, r);
+    const float lo = h - half, hi = h + half;
+    const double d = fma(-(double)h, ab_exact<FMT>(a, b, sTd), fabs((double)w));
+    const bool lo_even = fmodf(lo / (2.f * half), 2.f) == 0.f;
+    qm = d > 0.0 ? hi : (d < 0.0 ? lo : (lo_even ? lo : hi));
+    qm = fminf(qm, 448.f);
+  }
+  return copysignf(qm, xt);
+}
+
 // Q(W/(a b)) for one element.  u = W * cb is the weight times the column
 // factor (1/b, and 1/s_T for NVFP4), ia = 1/a (1/e for NVFP4); `ok` says the
 // fast fp32 candidate u*ia is trustworthy, otherwise it comes from an fp64
@@ -199,6 +240,7 @@ __device__ __forceinline__ float quant(float w, float u, float ia, bool ok, floa
     xt = (float)((double)w / ab_exact<FMT>(a, b, sTd));
   }
   if (fmt_e2m1(FMT)) return q_e2m1<FMT>(xt, w, a, b, sTd);
+  if (fmt_e4m3(FMT)) return q_e4m3<FMT>(xt, w, a, b, sTd);
   return q_int4<FMT>(xt, w, a, b, sTd);
 }
 

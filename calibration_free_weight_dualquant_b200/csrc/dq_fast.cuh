@@ -36,22 +36,13 @@ __device__ __forceinline__ float rcp_approx(float x) {
   return r;
 }
 
-// INT4 grid [-8,7]: round half to even by the 1.5*2^23 trick inside one fma.
-// `thr` is 0.5 - kGuard, or above 0.5 where the candidate is known to be exact
-// (then its own round-half-even is the answer, ties included).
-__device__ __forceinline__ float qfast_int4(float u, float ia, float thr, bool& near) {
-  const float y = fmaf(u, ia, 12582912.f);
-  const float qu = y - 12582912.f;
-  const float r = fmaf(u, ia, -qu);
-  near |= fabsf(r) > thr;
-  return fminf(fmaxf(qu, -8.f), 7.f);
-}
-
-// Exact INT4-grid decision in fp32 for an element the fast path flagged.  ab =
-// a*b is exact in fp32 (fp16*fp16, fp16*bf16 or 2^k*bf16), and w - h*a*b is
-// formed exactly inside one fma, so its sign says on which side of the
-// boundary h nearest the candidate W/(a b) lies; zero is a tie (to even).
-static __device__ __noinline__ float qexact32_int4(float w, float u, float ia, float ab) {
+// Exact integer-grid decision in fp32 for an element the fast path flagged.
+// ab = a*b is exact in fp32 (fp16*fp16, fp16*bf16 or 2^k*bf16), h*ab too (h
+// has at most 9 significant bits on the INT8 grid), and w - h*a*b is formed
+// inside one fma, so its sign says on which side of the boundary h nearest the
+// candidate W/(a b) lies; zero is a tie (to even).
+template <int FMT>
+static __device__ __noinline__ float qexact32_int(float w, float u, float ia, float ab) {
   const float xt = u * ia;
   const float qu = __fsub_rn(__fadd_rn(xt, 12582912.f), 12582912.f);
   const float h = qu + copysignf(0.5f, xt - qu);
@@ -64,7 +55,7 @@ static __device__ __noinline__ float qexact32_int4(float w, float u, float ia, f
   } else {
     q = __fsub_rn(__fadd_rn(h, 12582912.f), 12582912.f);  // the even neighbour
   }
-  return fminf(fmaxf(q, -8.f), 7.f);
+  return fminf(fmaxf(q, grid_lo(FMT)), grid_hi(FMT));
 }
 
 // Exact E2M1 decision in fp32: a*b = c1 * sT with c1 = e*b exact (<= 15 bits),
@@ -82,6 +73,24 @@ static __device__ __noinline__ float qexact32_e2m1(float w, float u, float ia, f
   const bool lo_even = (lo == 0.f || lo == 1.f || lo == 2.f || lo == 4.f);
   qm = d > 0.f ? hi : (d < 0.f ? lo : (lo_even ? lo : hi));
   return copysignf(fminf(qm, 6.f), w);
+}
+
+// Exact E4M3 decision in fp32 (power-of-two a): ab = a*b is exact, h*ab too
+// (h has at most 5 significant bits), and |w| - h*ab is formed inside one fma.
+// Spacing p2/8 in the binade [p2, 2 p2) (2^-9 below 2^-6); 448 is the top.
+static __device__ __noinline__ float qexact32_e4m3(float w, float u, float ia, float ab) {
+  const float xt = u * ia;
+  const float ax = fminf(fabsf(xt), 448.f);
+  const float p2 = __uint_as_float(max(__float_as_uint(ax) & 0x7F800000u, 0x3C800000u));
+  const float magic = p2 * 1572864.f;
+  float qm = __fsub_rn(__fadd_rn(ax, magic), magic);
+  const float half = p2 * 0.0625f;
+  const float h = qm + copysignf(half, ax - qm);
+  const float lo = h - half, hi = h + half;
+  const float d = fmaf(-h, ab, fabsf(w));
+  const bool lo_even = fmodf(lo / (2.f * half), 2.f) == 0.f;
+  qm = d > 0.f ? hi : (d < 0.f ? lo : (lo_even ? lo : hi));
+  return copysignf(fminf(qm, 448.f), w);
 }
 
 // ---------------------------------------------------------------------------

@@ -103,6 +103,33 @@ __device__ __forceinline__ f2 dec_e2m1x2(uint32_t code) {  // low nibble -> low 
   return pk(f.x, f.y);
 }
 
+// E4M3 conversions of four values (pairs p, q): byte k of the word is element k
+// (the low element of p in the low byte); round to nearest even, saturating
+// at 448.  The decode is exact (every E4M3 value is an fp16 value).
+__device__ __forceinline__ uint32_t cvt_e4m3x4(f2 p, f2 q) {
+  uint32_t r;
+  asm("{\n.reg .b16 l, h;\n"
+      "cvt.rn.satfinite.e4m3x2.f32 l, %2, %1;\n"
+      "cvt.rn.satfinite.e4m3x2.f32 h, %4, %3;\n"
+      "mov.b32 %0, {l, h};\n}"
+      : "=r"(r)
+      : "f"(lo_of(p)), "f"(hi_of(p)), "f"(lo_of(q)), "f"(hi_of(q)));
+  return r;
+}
+__device__ __forceinline__ void dec_e4m3x4(uint32_t c, f2& p, f2& q) {
+  uint32_t h0, h1;
+  asm("{\n.reg .b16 l, h;\n"
+      "mov.b32 {l, h}, %2;\n"
+      "cvt.rn.f16x2.e4m3x2 %0, l;\n"
+      "cvt.rn.f16x2.e4m3x2 %1, h;\n}"
+      : "=r"(h0), "=r"(h1)
+      : "r"(c));
+  const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&h0));
+  const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h1));
+  p = pk(f0.x, f0.y);
+  q = pk(f1.x, f1.y);
+}
+
 // Stored block scale as loaded (fp16 bits or an 8-bit code), fetched a tile
 // ahead of its use and decoded only there, so the warp does not wait for the
 // load right after issuing it.
@@ -147,7 +174,7 @@ __device__ __forceinline__ f2 col_ld(const f2* tab, int i, int lane) {
 
 // Per-lane state of a column strip segment, as 4 column pairs: b, the
 // candidate factor cb = 1/b (times 1/s_T for NVFP4), fp32 column runs, and the
-// guard threshold per column (MXINT4 columns with a power-of-two b have an exact
+// guard threshold per column (MXINT4/MXINT8 columns with a power-of-two b have an exact
 // candidate and need no guard).
 struct ColState {
   const f2* tb;   // shared table of b pairs [4][32]
@@ -170,20 +197,26 @@ __device__ __forceinline__ int sig_bits(float v) {
 // fp16 W), the element's scale product P = a b = p 2^h with p odd and at most k
 // bits long, and a rounding boundary B of the grid as an odd integer over a
 // power of two: at most 4 bits on the INT4 grid (the boundaries that matter
-// after clipping are +-1/2 .. +-15/2), 3 bits on E2M1 (1/4 .. 5).  Then
-// B P = n 2^f with n odd, and if W != B P, |W - B P| >= 2^min(g, f):
-//  * g >= f: |x - B| >= |B| / n >= 1 / (2 p) on the INT4 grid (absolute), and
-//    |x - B| / |B| >= 1 / n > 2^-(3 + k) on E2M1 (relative);
+// after clipping are +-1/2 .. +-15/2; 8 bits on the INT8 grid, +-1/2 ..
+// +-255/2), 3 bits on E2M1 (1/4 .. 5), 5 bits on E4M3 (midpoints of
+// neighbours with 3 mantissa bits, 2^-10 .. 432).  Then B P = n 2^f with n
+// odd, and if W != B P, |W - B P| >= 2^min(g, f):
+//  * g >= f: |x - B| >= |B| / n >= 1 / (2 p) on the integer grids (absolute,
+//    whatever the boundary's own bits), and |x - B| / |B| >= 1 / n > 2^-(3 + k)
+//    on E2M1, > 2^-(5 + k) on E4M3 (relative);
 //  * g < f:  |x - B| >= x / 2^11, i.e. 2^-13 absolute (|B| >= 1/2) or 2^-11
 //    relative.
 // The fast paths flag an element only when x lies within 2^-14 + 2^-19 of a
-// boundary (INT4 grid, absolute; candidate error included) or within
-// 1.5 * 2^-20 of it relative (E2M1 bracket plus candidate error).  So with
-// k <= 12 (INT4 grid) or k <= 15 (E2M1) every flagged element is an exact tie
-// x == B, whose answer is the even neighbour (round half to even).
+// boundary (INT4 grid, absolute; candidate error included), within
+// 2^-14 + 4.6e-5 < 2^-13 of it (INT8 grid, |x| <= 128.5), or within
+// 1.5 * 2^-20 of it relative (E2M1 and E4M3 brackets plus candidate error).
+// So with k <= 12 (integer grids), k <= 15 (E2M1) or k <= 14 (E4M3) every
+// flagged element is an exact tie x == B, whose answer is the even neighbour
+// (round half to even).
 template <int FMT, int WDT>
 __device__ __forceinline__ bool tie_certified(int k_bits) {
   if (WDT == DT_F32 || FMT == FMT_INT4) return false;  // INT4: fp16 a and b give k up to 22
+  if (fmt_e4m3(FMT)) return k_bits <= 14;
   return fmt_e2m1(FMT) ? k_bits <= 15 : k_bits <= 12;
 }
 
@@ -193,6 +226,7 @@ __device__ __noinline__ float qexact64(float w, float a, float b, double sTd) {
   const double ab = ab_exact<FMT>(a, b, sTd);
   const float xt = (float)((double)w / ab);
   if (fmt_e2m1(FMT)) return q_e2m1<FMT>(xt, w, a, b, sTd);
+  if (fmt_e4m3(FMT)) return q_e4m3<FMT>(xt, w, a, b, sTd);
   return q_int4<FMT>(xt, w, a, b, sTd);
 }
 
@@ -259,6 +293,23 @@ __device__ __forceinline__ void req_fast(const f2 u2[4], float a, const ColState
       const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hh[i]));
       q2[i] = pk(f.x, f.y);
     }
+  } else if (fmt_e4m3(FMT)) {
+    // E4M3 codes of the bracket ends, four to a word; as for E2M1, differing
+    // codes are neighbours, and a certified tie keeps the one whose low bit
+    // (mantissa bit) is 0
+    const f2 ilo = splat(ia * (1.f - kRelGuard)), ihi = splat(ia * (1.f + kRelGuard));
+    const uint32_t tmask = cs.tie_ok ? 0xFFFFFFFFu : 0u;
+    uint32_t anyd = 0u;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t clo = cvt_e4m3x4(mul2(u2[2 * h], ilo), mul2(u2[2 * h + 1], ilo));
+      const uint32_t chi = cvt_e4m3x4(mul2(u2[2 * h], ihi), mul2(u2[2 * h + 1], ihi));
+      const uint32_t diff = clo ^ chi;
+      anyd |= diff;
+      dec_e4m3x4(clo ^ (diff & ((clo & 0x01010101u) * 0xFFu) & tmask), q2[2 * h], q2[2 * h + 1]);
+    }
+    near |= (anyd & ~tmask) != 0u;
+    tie = (anyd & tmask) != 0u;
   } else {
     const f2 ia2 = splat(ia), nia2 = splat(-ia), m2 = splat(12582912.f), nm2 = splat(-12582912.f);
     bool flagged = false;
@@ -266,11 +317,12 @@ __device__ __forceinline__ void req_fast(const f2 u2[4], float a, const ColState
     for (int i = 0; i < 4; ++i) {
       const f2 qu = add2(fma2(u2[i], ia2, m2), nm2);  // round half even
       const f2 r = fma2(u2[i], nia2, qu);             // qu - x~
-      const float t0 = FMT == FMT_MXINT4 ? cs.thr[2 * i] : 0.5f - kGuard;
-      const float t1 = FMT == FMT_MXINT4 ? cs.thr[2 * i + 1] : 0.5f - kGuard;
+      const float t0 = fmt_mxint(FMT) ? cs.thr[2 * i] : 0.5f - kGuard;
+      const float t1 = fmt_mxint(FMT) ? cs.thr[2 * i + 1] : 0.5f - kGuard;
       flagged |= fabsf(lo_of(r)) > t0;
       flagged |= fabsf(hi_of(r)) > t1;
-      q2[i] = pk(fminf(fmaxf(lo_of(qu), -8.f), 7.f), fminf(fmaxf(hi_of(qu), -8.f), 7.f));
+      q2[i] = pk(fminf(fmaxf(lo_of(qu), grid_lo(FMT)), grid_hi(FMT)),
+                 fminf(fmaxf(hi_of(qu), grid_lo(FMT)), grid_hi(FMT)));
     }
     if (flagged && cs.tie_ok) {
       // certified exact ties x~ ~ n + 1/2: the even neighbour is 2 rint(x~ / 2)
@@ -282,11 +334,11 @@ __device__ __forceinline__ void req_fast(const f2 u2[4], float a, const ColState
         const f2 r = fma2(u2[i], nia2, qu);
         const f2 h = add2(fma2(u2[i], hia2, m2), nm2);
         const f2 qe = add2(h, h);
-        const float t0 = FMT == FMT_MXINT4 ? cs.thr[2 * i] : 0.5f - kGuard;
-        const float t1 = FMT == FMT_MXINT4 ? cs.thr[2 * i + 1] : 0.5f - kGuard;
+        const float t0 = fmt_mxint(FMT) ? cs.thr[2 * i] : 0.5f - kGuard;
+        const float t1 = fmt_mxint(FMT) ? cs.thr[2 * i + 1] : 0.5f - kGuard;
         const float q0 = fabsf(lo_of(r)) > t0 ? lo_of(qe) : lo_of(qu);
         const float q1 = fabsf(hi_of(r)) > t1 ? hi_of(qe) : hi_of(qu);
-        q2[i] = pk(fminf(fmaxf(q0, -8.f), 7.f), fminf(fmaxf(q1, -8.f), 7.f));
+        q2[i] = pk(fminf(fmaxf(q0, grid_lo(FMT)), grid_hi(FMT)), fminf(fmaxf(q1, grid_lo(FMT)), grid_hi(FMT)));
       }
     } else {
       near |= flagged;
@@ -326,12 +378,23 @@ __device__ __forceinline__ void req_slow(const f2 w2[4], const f2 u2[4], float a
       if (diff & 0x0Fu) q[c] = qexact32_e2m1(w[c], u[c], ia, a * b[c], sT);
       if (diff & 0xF0u) q[c + 1] = qexact32_e2m1(w[c + 1], u[c + 1], ia, a * b[c + 1], sT);
     }
+  } else if (fmt_e4m3(FMT)) {
+    const float ilo = ia * (1.f - kRelGuard), ihi = ia * (1.f + kRelGuard);
+#pragma unroll
+    for (int c = 0; c < 8; c += 4) {
+      const uint32_t lo = cvt_e4m3x4(pk(u[c] * ilo, u[c + 1] * ilo), pk(u[c + 2] * ilo, u[c + 3] * ilo));
+      const uint32_t hi = cvt_e4m3x4(pk(u[c] * ihi, u[c + 1] * ihi), pk(u[c + 2] * ihi, u[c + 3] * ihi));
+      const uint32_t diff = lo ^ hi;
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if ((diff >> (8 * k)) & 0xFFu) q[c + k] = qexact32_e4m3(w[c + k], u[c + k], ia, a * b[c + k]);
+    }
   } else {
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
       const float qu = fmaf(u[c], ia, 12582912.f) - 12582912.f;
-      const float thr = FMT == FMT_MXINT4 ? cs.thr[c] : 0.5f - kGuard;
-      if (fabsf(fmaf(u[c], ia, -qu)) > thr) q[c] = qexact32_int4(w[c], u[c], ia, a * b[c]);
+      const float thr = fmt_mxint(FMT) ? cs.thr[c] : 0.5f - kGuard;
+      if (fabsf(fmaf(u[c], ia, -qu)) > thr) q[c] = qexact32_int<FMT>(w[c], u[c], ia, a * b[c]);
     }
   }
 #pragma unroll
@@ -451,48 +514,97 @@ __device__ __forceinline__ void row_sums64(const f2 w2[4], const f2 q2[4], const
   }
 }
 
-// The 8 codes of a lane's row packed into one word (even column in the low
-// nibble; zero is always the 0x0 nibble).
+// The 8 codes of a lane's row.  Integer grids: q + 1.5 * 2^23 holds q in the
+// low mantissa bits (two's complement).  INT8 and E4M3 grids: one byte per
+// code, column order from the low byte of .x to the high byte of .y (E4M3:
+// the bit pattern, zero as 0x00).  Other grids: packed
+// nibbles in .x (even column in the low nibble; zero is always the 0x0
+// nibble), .y = 0.
 template <int FMT>
-__device__ __forceinline__ uint32_t pack8(const f2 q2[4]) {
-  uint32_t r = 0u;
+__device__ __forceinline__ uint2 pack8(const f2 q2[4]) {
+  uint2 r = make_uint2(0u, 0u);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const float lo = __fadd_rn(lo_of(q2[i]), 0.f), hi = __fadd_rn(hi_of(q2[i]), 0.f);  // -0 becomes +0
-    uint32_t byte;
-    if (fmt_e2m1(FMT)) {
-      byte = cvt_e2m1x2(hi, lo);  // grid values convert exactly
-    } else {  // q + 1.5 * 2^23 holds the integer q in its low mantissa bits (two's complement mod 16)
-      byte = (__float_as_uint(lo + 12582912.f) & 15u) | ((__float_as_uint(hi + 12582912.f) & 15u) << 4);
+    if (fmt_e4m3(FMT)) {  // grid values convert exactly; zero is always 0x00
+      if (i & 1) {
+        const uint32_t four = cvt_e4m3x4(pk(__fadd_rn(lo_of(q2[i - 1]), 0.f), __fadd_rn(hi_of(q2[i - 1]), 0.f)),
+                                         pk(lo, hi));
+        if (i == 1) {
+          r.x = four;
+        } else {
+          r.y = four;
+        }
+      }
+    } else if (fmt_byte_codes(FMT)) {
+      const uint32_t two = (__float_as_uint(lo + 12582912.f) & 255u) | ((__float_as_uint(hi + 12582912.f) & 255u) << 8);
+      if (i < 2) {
+        r.x |= two << (16 * i);
+      } else {
+        r.y |= two << (16 * (i - 2));
+      }
+    } else {
+      uint32_t byte;
+      if (fmt_e2m1(FMT)) {
+        byte = cvt_e2m1x2(hi, lo);  // grid values convert exactly
+      } else {
+        byte = (__float_as_uint(lo + 12582912.f) & 15u) | ((__float_as_uint(hi + 12582912.f) & 15u) << 4);
+      }
+      r.x |= byte << (8 * i);
     }
-    r |= byte << (8 * i);
   }
   return r;
 }
 
-// Number of nonzero nibbles of x (codes that differ, for x = new ^ old).
-__device__ __forceinline__ uint32_t changed_nibbles(uint32_t x) {
-  x |= x >> 1;
-  x |= x >> 2;
-  return (uint32_t)__popc(x & 0x11111111u);
+// Number of codes that differ, for x = new ^ old (nonzero bytes or nibbles).
+template <int FMT>
+__device__ __forceinline__ uint32_t changed_codes(uint2 x) {
+  if (fmt_byte_codes(FMT)) {
+    x.x |= x.x >> 1;
+    x.x |= x.x >> 2;
+    x.x |= x.x >> 4;
+    x.y |= x.y >> 1;
+    x.y |= x.y >> 2;
+    x.y |= x.y >> 4;
+    return (uint32_t)(__popc(x.x & 0x01010101u) + __popc(x.y & 0x01010101u));
+  }
+  x.x |= x.x >> 1;
+  x.x |= x.x >> 2;
+  return (uint32_t)__popc(x.x & 0x11111111u);
 }
 
-// Code tracking for two rows of a lane: the packed codes replace the words at
-// cix (row x) and cix + kConsumerWarps rows (row y); with `cmp` the nibbles
-// that differ from the previous words oldx, oldy are counted into nchg.
+// The code group (8 codes) at index cix: a 32-bit word, or 8 bytes for the
+// INT8 grid.  Codes are rewritten inside the kernel: loads go through L2.
+template <int FMT>
+__device__ __forceinline__ uint2 load_codes(const void* codes, int64_t cix) {
+  if (fmt_byte_codes(FMT)) return __ldcg(reinterpret_cast<const uint2*>(codes) + cix);
+  return make_uint2(__ldcg(reinterpret_cast<const uint32_t*>(codes) + cix), 0u);
+}
+
+template <int FMT>
+__device__ __forceinline__ void store_codes(void* codes, int64_t cix, uint2 c) {
+  if (fmt_byte_codes(FMT)) {
+    reinterpret_cast<uint2*>(codes)[cix] = c;
+  } else {
+    reinterpret_cast<uint32_t*>(codes)[cix] = c.x;
+  }
+}
+
+// Code tracking for two rows of a lane: the codes replace the groups at cix
+// (row x) and cix + kConsumerWarps rows (row y); with `cmp` the codes that
+// differ from the previous groups oldx, oldy are counted into nchg.
 template <int FMT>
 __device__ __forceinline__ void track_codes(const Problem& p, const f2 qx[4], const f2 qy[4], bool actx, bool acty,
-                                            int64_t cix, uint32_t oldx, uint32_t oldy, bool cmp, unsigned& nchg) {
-  uint32_t* codes = reinterpret_cast<uint32_t*>(p.codes);
+                                            int64_t cix, uint2 oldx, uint2 oldy, bool cmp, unsigned& nchg) {
   if (actx) {
-    const uint32_t c = pack8<FMT>(qx);
-    if (cmp) nchg += changed_nibbles(c ^ oldx);
-    codes[cix] = c;
+    const uint2 c = pack8<FMT>(qx);
+    if (cmp) nchg += changed_codes<FMT>(make_uint2(c.x ^ oldx.x, c.y ^ oldx.y));
+    store_codes<FMT>(p.codes, cix, c);
   }
   if (acty) {
-    const uint32_t c = pack8<FMT>(qy);
-    if (cmp) nchg += changed_nibbles(c ^ oldy);
-    codes[cix + (int64_t)kConsumerWarps * (p.N >> 3)] = c;
+    const uint2 c = pack8<FMT>(qy);
+    if (cmp) nchg += changed_codes<FMT>(make_uint2(c.x ^ oldy.x, c.y ^ oldy.y));
+    store_codes<FMT>(p.codes, cix + (int64_t)kConsumerWarps * (p.N >> 3), c);
   }
 }
 
@@ -506,7 +618,7 @@ __device__ __forceinline__ void row_pair(const Problem& p, const f2 wx[4], float
                                          const f2 wy[4], float ay_old, int64_t bidx_y, bool has_y, bool active,
                                          bool leader, int lpb, ColState& cs, float sT, float isT, double sTd,
                                          bool scaled, f2 rscale2, unsigned* s_cnt, unsigned& tcnt, int64_t cix,
-                                         uint32_t oldx, uint32_t oldy, bool cmp, unsigned& nchg) {
+                                         uint2 oldx, uint2 oldy, bool cmp, unsigned& nchg) {
   const bool actx = active, acty = active && has_y;
   f2 ux[4], uy[4], qx[4], qy[4];
 #pragma unroll
@@ -604,8 +716,8 @@ __device__ __forceinline__ void row_pair(const Problem& p, const f2 wx[4], float
 template <int FMT>
 __device__ __forceinline__ void final_pair(const Problem& p, const f2 wx[4], float ax, const f2 wy[4], float ay,
                                            bool has_y, bool active, ColState& cs, float sT, double sTd, bool scaled,
-                                           f2 rscale2, unsigned* s_cnt, unsigned& tcnt, int64_t cix, uint32_t oldx,
-                                           uint32_t oldy, bool cmp, unsigned& nchg) {
+                                           f2 rscale2, unsigned* s_cnt, unsigned& tcnt, int64_t cix, uint2 oldx,
+                                           uint2 oldy, bool cmp, unsigned& nchg) {
   const bool actx = active, acty = active && has_y;
   f2 ux[4], uy[4], qx[4], qy[4];
 #pragma unroll
@@ -1024,8 +1136,7 @@ __global__ void __launch_bounds__(kIterThreads, 1)
   int st = 0;
   unsigned par = 0u;
   constexpr bool FIN = PASS == PASS_FINAL;
-  const uint32_t* codes_old = reinterpret_cast<const uint32_t*>(p.codes);
-  const int64_t code_step = (int64_t)kConsumerWarps * (p.N >> 3);  // code words between a warp's two rows
+  const int64_t code_step = (int64_t)kConsumerWarps * (p.N >> 3);  // code groups between a warp's two rows
   unsigned tcnt = 0u;  // lane-rows settled as certified exact ties
 
   for (int t = t_first; t <= t_last; ++t) {
@@ -1071,9 +1182,9 @@ __global__ void __launch_bounds__(kIterThreads, 1)
           cb[h] = __frcp_rn(bj[h]) * isT;
           cs.ok = cs.ok && in_range(cb[h]);
           b_bits = max(b_bits, sig_bits(bj[h]));
-          // MXINT4: a = 2^k, so a power-of-two b makes the candidate exact (for
-          // bf16/fp16 W the tie certificate covers these columns as well)
-          if (FMT == FMT_MXINT4 && WDT == DT_F32 && (__float_as_uint(bj[h]) & 0x007FFFFFu) == 0u) cs.thr[c] = 2.f;
+          // MXINT4/MXINT8: a = 2^k, so a power-of-two b makes the candidate exact
+          // (for bf16/fp16 W the tie certificate covers these columns as well)
+          if (fmt_mxint(FMT) && WDT == DT_F32 && (__float_as_uint(bj[h]) & 0x007FFFFFu) == 0u) cs.thr[c] = 2.f;
         }
         acc[(warp * 8 + c) * 32 + lane] = make_double2(0.0, 0.0);
       }
@@ -1103,11 +1214,11 @@ __global__ void __launch_bounds__(kIterThreads, 1)
       const uint32_t ra_raw = an0, rb_raw = an1;
       if (active && ra + kRowsPerTile < nrows) an0 = a_fetch<FMT>(p.a_store, aidx + a_step);
       if (active && rb + kRowsPerTile < nrows) an1 = a_fetch<FMT>(p.a_store, aidx + a_step + y_off);
-      const int64_t cix = ((r0 + ra) * p.N + col) >> 3;  // code word of row ra, this lane's 8 columns
-      uint32_t oldx = 0u, oldy = 0u;
+      const int64_t cix = ((r0 + ra) * p.N + col) >> 3;  // code group of row ra, this lane's 8 columns
+      uint2 oldx = make_uint2(0u, 0u), oldy = make_uint2(0u, 0u);
       if (PASS != PASS_ITER && cmp && active) {  // issued before the wait: the latency hides behind it
-        if (has_a) oldx = __ldcg(codes_old + cix);
-        if (has_b) oldy = __ldcg(codes_old + cix + code_step);
+        if (has_a) oldx = load_codes<FMT>(p.codes, cix);
+        if (has_b) oldy = load_codes<FMT>(p.codes, cix + code_step);
       }
       mbar_wait(&full[st], par, &p.hdr->flags);
       f2 wa[4], wb[4];

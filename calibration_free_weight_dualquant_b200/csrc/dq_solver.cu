@@ -93,7 +93,7 @@ __global__ void __launch_bounds__(kThreads) k_init(Problem p) {
     p.hdr->sT = 1.f;
     if (p.sT_out) *p.sT_out = 1.f;
   }
-  const double qmax = fmt_e2m1(FMT) ? 6.0 : 7.0;
+  const double qmax = grid_qmax(FMT);
   const int64_t nblocks = p.M * p.nb;
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   for (int64_t blk = (int64_t)blockIdx.x * kThreads + threadIdx.x; blk < nblocks; blk += stride) {
@@ -251,6 +251,8 @@ cudaError_t launch_solve(const Problem& p, int iters, int stats_ctas, cudaStream
     case FMT_INT4: return run_fmt<FMT_INT4>(p, iters, stats_ctas, st);
     case FMT_MXINT4: return run_fmt<FMT_MXINT4>(p, iters, stats_ctas, st);
     case FMT_MXFP4: return run_fmt<FMT_MXFP4>(p, iters, stats_ctas, st);
+    case FMT_MXINT8: return run_fmt<FMT_MXINT8>(p, iters, stats_ctas, st);
+    case FMT_MXFP8: return run_fmt<FMT_MXFP8>(p, iters, stats_ctas, st);
     default: return run_fmt<FMT_NVFP4>(p, iters, stats_ctas, st);
   }
 }

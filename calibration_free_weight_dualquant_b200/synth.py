@@ -28,7 +28,7 @@ class Workload:
     rows: int
     cols: int
     wdtype: str          # "f32" | "bf16"
-    fmt: str             # "int4" | "mxint4" | "nvfp4"
+    fmt: str             # "int4" | "mxint4" | "nvfp4" | "mxfp4" | "mxint8"
     group: int
     col_dtype: str       # "f16" | "bf16"
     iters: int
@@ -58,6 +58,14 @@ WORKLOADS = {
     "mxfp4_g32_downproj_4096x14336": Workload(
         "mxfp4_g32_downproj_4096x14336", 4096, 14336, "bf16", "mxfp4", 32, "bf16", 20, "student_t", 0.015, 0.005,
         20.0, 1006),
+    # the MX family's INT8 member (8-bit weights, DualQuant App. G.2) on the down_proj recipe
+    "mxint8_g32_downproj_4096x14336": Workload(
+        "mxint8_g32_downproj_4096x14336", 4096, 14336, "bf16", "mxint8", 32, "bf16", 20, "student_t", 0.015, 0.005,
+        20.0, 1007),
+    # the MX family's FP8 E4M3 member (8-bit weights, DualQuant App. G.2) on the down_proj recipe
+    "mxfp8_g32_downproj_4096x14336": Workload(
+        "mxfp8_g32_downproj_4096x14336", 4096, 14336, "bf16", "mxfp8", 32, "bf16", 20, "student_t", 0.015, 0.005,
+        20.0, 1008),
 }
 
 # Llama-3.1-8B per-layer linear shapes (rows = out features, cols = in features)

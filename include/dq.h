@@ -55,18 +55,28 @@ typedef enum {
  *            inverse scale a = s_T * e with e an FP8 E4M3 value (stored as the
  *            E4M3 byte) and one fp32 tensor scale s_T = fp32(amax|W| / 2688).
  *  DQ_MXFP4  E2M1 grid, group 32, block inverse scales 2^k stored as E8M0 bytes
- *            (the MX family's FP4 member; no tensor scale). */
-typedef enum { DQ_INT4 = 0, DQ_MXINT4 = 1, DQ_NVFP4 = 2, DQ_MXFP4 = 3 } dq_format;
+ *            (the MX family's FP4 member; no tensor scale).
+ *  DQ_MXINT8 grid [-128,127], group 32, block inverse scales 2^k stored as
+ *            E8M0 bytes (the MX family's INT8 member; the 8-bit weight format
+ *            of DualQuant App. G.2).  Absmax initialization with qmax 127.
+ *  DQ_MXFP8  FP8 E4M3 grid (3 mantissa bits, subnormals down to 2^-9, largest
+ *            value 448, ties to the even mantissa bit, larger magnitudes clip),
+ *            group 32, E8M0 block scales (the MX family's FP8 E4M3 member,
+ *            App. G.2).  Absmax initialization with qmax 448. */
+typedef enum { DQ_INT4 = 0, DQ_MXINT4 = 1, DQ_NVFP4 = 2, DQ_MXFP4 = 3, DQ_MXINT8 = 4, DQ_MXFP8 = 5 } dq_format;
 
 typedef enum { DQ_F32 = 0, DQ_BF16 = 1, DQ_F16 = 2 } dq_dtype;
 
 /* Outputs (device pointers, caller-owned).
  *  codes         uint8 [rows][cols/2]: two 4-bit codes per byte, the even
  *                column in the low nibble.  INT4/MXINT4: two's-complement
- *                nibble of q in [-8,7].  NVFP4: E2M1 nibble s|ee|m; a zero
- *                code is always 0x0.
- *  block_scales  [rows][cols/group]: fp16 (INT4), E8M0 byte (MXINT4), E4M3
- *                byte (NVFP4).
+ *                nibble of q in [-8,7].  NVFP4/MXFP4: E2M1 nibble s|ee|m; a
+ *                zero code is always 0x0.  MXINT8: int8 [rows][cols], one
+ *                two's-complement byte of q in [-128,127] per element (8-byte
+ *                aligned).  MXFP8: uint8 [rows][cols], the E4M3 bit pattern of
+ *                q per element, zero always 0x00 (8-byte aligned).
+ *  block_scales  [rows][cols/group]: fp16 (INT4), E8M0 byte (MXINT4, MXFP4,
+ *                MXINT8, MXFP8), E4M3 byte (NVFP4).
  *  tensor_scale  one float: s_T for NVFP4, 1.0 for the other formats (which
  *                accept NULL here).
  *  col_scales    [cols] inverse column scales, fp16 or bf16 (col_dtype).
@@ -91,7 +101,7 @@ size_t dq_workspace_bytes(int64_t rows, int64_t cols, int format, int group);
 
 /* Absmax round-to-nearest with column scales 1: the solver's initial iterate
  * and its comparison point (DualQuant §3 "symmetric scale max|W|/qmax", qmax 7
- * for INT4/MXINT4 and 6 for E2M1, projected onto the admissible set; an
+ * for INT4/MXINT4, 127 for MXINT8, 448 for MXFP8 and 6 for E2M1, projected onto the admissible set; an
  * all-zero block gets scale 1).  Bit-identical to dq_solve(..., iters = 0).
  * Writes codes, block_scales, tensor_scale, col_scales (all 1) and mse[0]. */
 int dq_rtn(const void* W, int w_dtype, int64_t rows, int64_t cols, int format, int group, int col_dtype,
@@ -258,7 +268,8 @@ int dq_solve_batched(const dq_matrix* mats, int count, int format, int group, in
  * then); col_scales and mse of `out` are not used.  x_dtype is DQ_BF16 or
  * DQ_F16, col_dtype the dtype of `col_scales` (DQ_BF16 or DQ_F16).  The
  * workspace (DQ_ACT_WORKSPACE_BYTES, 256-byte aligned) reports a non-finite
- * X * b through dq_sync_status. */
+ * X * b through dq_sync_status.  The 4-bit formats only: DQ_MXINT8 and
+ * DQ_MXFP8 return DQ_EUNSUPPORTED. */
 int dq_act_quant(const void* X, int x_dtype, int64_t rows, int64_t cols, const void* col_scales, int col_dtype,
                  int format, int group, const dq_outputs* out, void* workspace, size_t workspace_bytes,
                  void* stream);

@@ -10,7 +10,7 @@ def block_scale_values(fmt: str, t: torch.Tensor) -> np.ndarray:
     t = t.cpu()
     if fmt == "int4":
         return t.to(torch.float64).numpy()
-    if fmt in ("mxint4", "mxfp4"):
+    if fmt in ("mxint4", "mxfp4", "mxint8", "mxfp8"):
         return np.ldexp(1.0, t.numpy().astype(np.int64) - 127)
     return t.view(torch.float8_e4m3fn).to(torch.float64).numpy()
 

@@ -40,6 +40,8 @@ SMALL = {
     "mxint4_g32_downproj_4096x14336": (301, 608),
     "nvfp4_g16_gateup_14336x4096": (339, 528),
     "mxfp4_g32_downproj_4096x14336": (301, 608),
+    "mxint8_g32_downproj_4096x14336": (301, 608),
+    "mxfp8_g32_downproj_4096x14336": (301, 608),
 }
 
 
@@ -58,6 +60,8 @@ def test_parity_small_workload_recipe(name):
     ("int4", 64, "f16", 1000, 1344, 6),
     ("mxint4", 32, "bf16", 777, 1056, 6),
     ("nvfp4", 16, "bf16", 1203, 800, 6),
+    ("mxint8", 32, "bf16", 777, 1056, 6),
+    ("mxfp8", 32, "bf16", 777, 1056, 6),
 ])
 def test_parity_many_ctas(fmt, group, col_dtype, M, N, iters):
     wl = synth.WORKLOADS["nvfp4_g16_gateup_14336x4096"]
@@ -74,6 +78,12 @@ def test_parity_many_ctas(fmt, group, col_dtype, M, N, iters):
     ("mxint4", 32, "bf16", 2, 32, torch.float32),
     ("nvfp4", 16, "bf16", 3, 16, torch.bfloat16),
     ("nvfp4", 16, "f16", 65, 272, torch.float16),
+    ("mxint8", 32, "bf16", 2, 32, torch.float32),
+    ("mxint8", 32, "f16", 41, 288, torch.float16),
+    ("mxint8", 32, "bf16", 3, 96, torch.bfloat16),
+    ("mxfp8", 32, "bf16", 2, 32, torch.float32),
+    ("mxfp8", 32, "f16", 41, 288, torch.float16),
+    ("mxfp8", 32, "bf16", 3, 96, torch.bfloat16),
 ])
 def test_parity_edge_shapes_and_dtypes(fmt, group, col_dtype, M, N, wdtype):
     g = torch.Generator().manual_seed(M * 1000 + N)
@@ -81,10 +91,11 @@ def test_parity_edge_shapes_and_dtypes(fmt, group, col_dtype, M, N, wdtype):
     run_both(W, fmt, group, 5, col_dtype, "edge")
 
 
-FOUR = [("int4", 64, "f16"), ("mxint4", 32, "bf16"), ("nvfp4", 16, "bf16"), ("mxfp4", 32, "bf16")]
+FORMATS = [("int4", 64, "f16"), ("mxint4", 32, "bf16"), ("nvfp4", 16, "bf16"), ("mxfp4", 32, "bf16"),
+           ("mxint8", 32, "bf16"), ("mxfp8", 32, "bf16")]
 
 
-@pytest.mark.parametrize("fmt,group,col_dtype", FOUR)
+@pytest.mark.parametrize("fmt,group,col_dtype", FORMATS)
 def test_parity_zero_slices(fmt, group, col_dtype):
     g = torch.Generator().manual_seed(5)
     W = torch.randn(40, 4 * group, generator=g) * 0.02
@@ -95,7 +106,7 @@ def test_parity_zero_slices(fmt, group, col_dtype):
     run_both(torch.zeros(9, 2 * group, dtype=torch.bfloat16), fmt, group, 3, col_dtype, "all_zero")
 
 
-@pytest.mark.parametrize("fmt,group,col_dtype", FOUR)
+@pytest.mark.parametrize("fmt,group,col_dtype", FORMATS)
 def test_parity_exact_ties(fmt, group, col_dtype):
     """Weights on a coarse dyadic lattice make exact rounding ties frequent."""
     g = torch.Generator().manual_seed(9)
@@ -104,7 +115,7 @@ def test_parity_exact_ties(fmt, group, col_dtype):
     run_both(W.to(torch.bfloat16), fmt, group, 8, col_dtype, "ties")
 
 
-@pytest.mark.parametrize("fmt,group,col_dtype", FOUR)
+@pytest.mark.parametrize("fmt,group,col_dtype", FORMATS)
 @pytest.mark.parametrize("mag", [1e-33, 1e-12, 1e4, 1e30])
 def test_parity_extreme_magnitudes(fmt, group, col_dtype, mag):
     """Scales at the ends of the admissible sets (saturation, smallest values, fp64 fallback of the candidate)."""
@@ -114,7 +125,7 @@ def test_parity_extreme_magnitudes(fmt, group, col_dtype, mag):
     run_both(W.float(), fmt, group, 4, col_dtype, "mag%g" % mag)
 
 
-@pytest.mark.parametrize("fmt", ["int4", "mxint4", "nvfp4", "mxfp4"])
+@pytest.mark.parametrize("fmt", ["int4", "mxint4", "nvfp4", "mxfp4", "mxint8", "mxfp8"])
 def test_zero_iterations_is_rtn_and_deterministic(fmt):
     wl = synth.WORKLOADS["nvfp4_g16_gateup_14336x4096"]
     W = synth.make_weight(wl, 250, 1024, seed=3).cuda()
@@ -198,7 +209,8 @@ def test_full_size_qproj_int4_against_full_oracle():
 
 
 @pytest.mark.parametrize("name", ["mxint4_g32_downproj_4096x14336", "nvfp4_g16_gateup_14336x4096",
-                                  "int4_g64_256x512_f32"])
+                                  "int4_g64_256x512_f32", "mxint8_g32_downproj_4096x14336",
+                                  "mxfp8_g32_downproj_4096x14336"])
 def test_full_size_last_iteration_and_final_state(name):
     """Full-size solve: the last GPU iteration equals one oracle iteration from the GPU's previous
     iterate (every block and column scale, bit-exact); the codes equal Q(W/(a b)) of the final
@@ -232,6 +244,8 @@ def test_full_size_last_iteration_and_final_state(name):
 @pytest.mark.parametrize("fmt,group,col_dtype,name", [
     ("int4", 64, "f16", "int4_g64_qproj_4096x4096"),
     ("mxint4", 32, "bf16", "mxint4_g32_downproj_4096x14336"),
+    ("mxint8", 32, "bf16", "mxint8_g32_downproj_4096x14336"),
+    ("mxfp8", 32, "bf16", "mxfp8_g32_downproj_4096x14336"),
 ])
 def test_exact_paths_exercised_and_bit_exact(fmt, group, col_dtype, name):
     """The fp32 fast paths hand near-boundary elements, near-midpoint block scales and
@@ -240,7 +254,7 @@ def test_exact_paths_exercised_and_bit_exact(fmt, group, col_dtype, name):
     W = synth.make_weight(wl, 1024, 2048, seed=5)
     gpu, _ = run_both(W, fmt, group, 20, col_dtype, "exact_paths")
     d = binding.diagnostics(gpu["workspace"])
-    if fmt == "mxint4":  # bf16 W, 2^k a: every flagged element is a certified exact tie
+    if fmt in ("mxint4", "mxint8", "mxfp8"):  # bf16 W, 2^k a: every flagged element is a certified exact tie
         assert d["quant_tie_lane_rows"] > 0, d
     else:
         assert d["quant_exact_lane_rows"] > 0, d
@@ -293,7 +307,7 @@ def test_mxint4_exact_ties(wdtype, col_dtype):
 
 
 @pytest.mark.parametrize("mode", ["row", "col"])
-@pytest.mark.parametrize("fmt,group,col_dtype", FOUR)
+@pytest.mark.parametrize("fmt,group,col_dtype", FORMATS)
 def test_ablation_modes_parity(mode, fmt, group, col_dtype):
     """Row-only and column-only solves (DualQuant §5.3, Table 4) against the oracle's modes."""
     wl = synth.WORKLOADS["nvfp4_g16_gateup_14336x4096"]
@@ -316,3 +330,81 @@ def test_mxfp4_exact_ties():
     gpu, _ = run_both(W, "mxfp4", 32, 6, "bf16", "mxfp4_ties")
     d = binding.diagnostics(gpu["workspace"])
     assert d["quant_tie_lane_rows"] > 0, d
+
+
+@pytest.mark.parametrize("wdtype,col_dtype", [(torch.bfloat16, "bf16"), (torch.float16, "f16"),
+                                              (torch.float32, "bf16")])
+def test_mxint8_exact_ties(wdtype, col_dtype):
+    """MXINT8 on half-integer lattices: every block holds the value 127 * 2^-8, so its RTN scale is
+    exactly 2^-8 and every other W / a = m + 1/2 is an exact tie on the INT8 grid; certified on
+    the fast path for bf16/fp16 W.  For f32 W nothing is certified: with a power-of-two b the
+    candidate W * (1/b) * 2^-k is exact and its own round-half-even settles the tie."""
+    g = torch.Generator().manual_seed(15)
+    M, N = 203, 640
+    m = torch.randint(-100, 100, (M, N), generator=g).float()
+    W = (m + 0.5) * 2.0 ** -8
+    W[:, ::32] = 127.0 * 2.0 ** -8
+    gpu, _ = run_both(W.to(wdtype), "mxint8", 32, 6, col_dtype, "int8_ties")
+    d = binding.diagnostics(gpu["workspace"])
+    if wdtype != torch.float32:
+        assert d["quant_tie_lane_rows"] > 0, d
+    else:
+        assert d["quant_tie_lane_rows"] == 0, d
+
+
+def test_mxint8_grid_ends_and_clipping():
+    """Values past both ends of the INT8 grid clip to -128 and 127 (two's-complement bytes 0x80, 0x7F)."""
+    g = torch.Generator().manual_seed(16)
+    W = torch.randn(64, 256, generator=g) * 0.01
+    W[:, 0] = 0.5      # with the next column, the block scale: Proj(1/127) = 2^-7
+    W[:, 1] = -1.0     # W/a = -128, the lower end
+    W[:, 2] = 1.0      # W/a = 128 clips to 127
+    gpu, orc = run_both(W.to(torch.bfloat16), "mxint8", 32, 0, "bf16", "int8_ends")
+    codes = gpu["codes"].cpu()
+    assert codes.shape == (64, 256)
+    assert bool((codes[:, 1] == 0x80).all()) and bool((codes[:, 2] == 0x7F).all())
+
+
+def e4m3_midpoints() -> torch.Tensor:
+    """Midpoints of neighbouring nonnegative E4M3 values below 448 (from torch's float8_e4m3fn)."""
+    v = torch.arange(0, 0x7F, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64)
+    return (v[:-1] + v[1:]) / 2
+
+
+@pytest.mark.parametrize("wdtype,col_dtype", [(torch.bfloat16, "bf16"), (torch.float16, "f16"),
+                                              (torch.float32, "bf16")])
+def test_mxfp8_exact_ties(wdtype, col_dtype):
+    """MXFP8 on E4M3 midpoints: every block holds 448 * 2^-8, so its RTN scale is exactly 2^-8 and
+    every other W / a is a midpoint of two E4M3 values (an exact tie, subnormal ones included);
+    certified on the fast path for bf16/fp16 W, settled exactly for f32 W."""
+    g = torch.Generator().manual_seed(17)
+    M, N = 203, 640
+    mids = e4m3_midpoints()
+    idx = torch.randint(0, len(mids), (M, N), generator=g)
+    sign = torch.where(torch.rand(M, N, generator=g) < 0.5, -1.0, 1.0).double()
+    W = (mids[idx] * sign * 2.0 ** -8).float()
+    W[:, ::32] = 448.0 * 2.0 ** -8
+    gpu, _ = run_both(W.to(wdtype), "mxfp8", 32, 6, col_dtype, "e4m3_ties")
+    d = binding.diagnostics(gpu["workspace"])
+    if wdtype != torch.float32:
+        assert d["quant_tie_lane_rows"] > 0, d
+    else:
+        assert d["quant_tie_lane_rows"] == 0 and d["quant_exact_lane_rows"] > 0, d
+
+
+def test_mxfp8_grid_ends_and_subnormals():
+    """E4M3 saturation at +-448 (0x7E, 0xFE), the smallest subnormal 2^-9 (0x01), the midpoint 2^-10
+    (a tie that goes to zero, code 0x00) and exact zeros (0x00, never 0x80)."""
+    g = torch.Generator().manual_seed(18)
+    W = torch.randn(64, 256, generator=g) * 0.01
+    W[:, 0] = 1.75               # with the next column, the block scale: Proj(1.875 / 448) = 2^-8
+    W[:, 1] = -1.75              # -448
+    W[:, 2] = 1.875              # 480 clips to 448
+    W[:, 3] = 2.0 ** -17         # 2^-9, the smallest subnormal
+    W[:, 4] = -(2.0 ** -18)      # -2^-10: tie between 0 and -2^-9, to zero
+    W[:, 5] = 0.0
+    gpu, _ = run_both(W.to(torch.bfloat16), "mxfp8", 32, 0, "bf16", "e4m3_ends")
+    codes = gpu["codes"].cpu()
+    assert codes.shape == (64, 256)
+    for col, want in ((1, 0xFE), (2, 0x7E), (3, 0x01), (4, 0x00), (5, 0x00)):
+        assert bool((codes[:, col] == want).all()), (col, codes[:3, col].tolist())
