@@ -65,3 +65,25 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(binding, "_lib", None)
     with pytest.raises(binding.DQError):
         binding.load_library()
+
+
+def test_format_numbering_matches_header():
+    """The binding's format numbers are the header's dq_format values, and the oracle's format names
+    cover every one of them (their numbers mirror the header's by value only)."""
+    import oracle
+    text = open(os.path.join(ROOT, "include", "dq.h")).read()
+    body = re.search(r"typedef enum \{([^}]*)\} dq_format;", text).group(1)
+    header = {k: int(v) for k, v in re.findall(r"DQ_(\w+)\s*=\s*(\d+)", body)}
+    assert header == {f.name: int(f) for f in binding.Format}
+    assert set(oracle.FORMATS) == {f.name.lower() for f in binding.Format}
+
+
+def test_byte_code_formats_output_sizes():
+    """MXINT8 and MXFP8 store one byte per code; the 4-bit formats two codes per byte."""
+    for fmt in ("mxint8", "mxfp8"):
+        n = binding.output_nbytes(4096, 14336, fmt)
+        assert n["codes"] == 4096 * 14336 and n["block_scales"] == 4096 * 448 and n["tensor_scale"] == 0
+    for fmt in ("int4", "mxint4", "nvfp4", "mxfp4"):
+        assert binding.output_nbytes(64, 512, fmt)["codes"] == 64 * 256
+    out = binding.alloc_outputs(8, 64, "mxfp8", 32, "bf16", 2, "cpu")
+    assert tuple(out["codes"].shape) == (8, 64)

@@ -32,7 +32,7 @@ def _same(a: dict, b: dict):
 
 
 @pytest.mark.parametrize("fmt,group,col_dtype", [("nvfp4", 16, "bf16"), ("mxint4", 32, "bf16"), ("int4", 64, "f16"),
-                                              ("mxfp4", 32, "bf16")])
+                                              ("mxfp4", 32, "bf16"), ("mxint8", 32, "bf16"), ("mxfp8", 32, "bf16")])
 def test_batched_equals_one_by_one(fmt, group, col_dtype):
     wl = synth.WORKLOADS["nvfp4_g16_gateup_14336x4096"]
     shapes = [(300, 512), (77, 1024), (513, 256), (1024, 768)]

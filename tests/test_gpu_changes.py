@@ -32,7 +32,8 @@ def _same(a: dict, b: dict):
 
 @pytest.mark.parametrize("mode,init", [("dual", "rtn"), ("dual", "l1"), ("row", "rtn"), ("col", "l1")])
 @pytest.mark.parametrize("fmt,group,col_dtype", [("nvfp4", 16, "bf16"), ("mxint4", 32, "bf16"), ("int4", 64, "f16"),
-                                              ("mxfp4", 32, "bf16"), ("int4", 128, "bf16")])
+                                              ("mxfp4", 32, "bf16"), ("int4", 128, "bf16"),
+                                              ("mxint8", 32, "bf16"), ("mxfp8", 32, "bf16")])
 @pytest.mark.parametrize("rows,cols,dtype,iters", [(97, 768 + 128, torch.bfloat16, 6), (64, 512, torch.float32, 4),
                                                   (40, 256, torch.float16, 1)])
 def test_changes_match_oracle(mode, init, fmt, group, col_dtype, rows, cols, dtype, iters):

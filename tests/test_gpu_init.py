@@ -18,7 +18,9 @@ pytestmark = pytest.mark.gpu
 
 MSE_RTOL = 1e-4
 FORMATS = [("nvfp4", 16, "bf16"), ("mxint4", 32, "bf16"), ("int4", 64, "f16"), ("mxfp4", 32, "bf16"),
-           ("int4", 16, "bf16")]
+           ("int4", 16, "bf16"), ("mxint8", 32, "bf16"), ("mxfp8", 32, "bf16")]
+# one configuration per format
+PRIMARY = [f for f in FORMATS if f != ("int4", 16, "bf16")]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -54,7 +56,7 @@ def test_l1_init_parity(fmt, group, col_dtype, rows, cols, dtype, iters):
     assert not np.all(orc["b"] == 1.0)
 
 
-@pytest.mark.parametrize("fmt,group,col_dtype", FORMATS[:4])
+@pytest.mark.parametrize("fmt,group,col_dtype", PRIMARY)
 def test_l1_init_zero_columns_and_zero_matrix(fmt, group, col_dtype):
     W = weight(64, 512, seed=3)
     W[:, 17] = 0
@@ -81,11 +83,12 @@ def test_l1_init_extreme_magnitudes():
         compare_with_oracle(fmt, gpu, orc, MSE_RTOL, "extreme " + fmt)
 
 
-@pytest.mark.parametrize("fmt,group,col_dtype", FORMATS[:4])
+@pytest.mark.parametrize("fmt,group,col_dtype", PRIMARY)
 def test_l1_init_full_size(fmt, group, col_dtype):
     """The init at the workload's full size: every scale and code of the initial iterate bit-exact."""
     name = {"nvfp4": "nvfp4_g16_gateup_14336x4096", "mxint4": "mxint4_g32_downproj_4096x14336",
-            "int4": "int4_g64_qproj_4096x4096", "mxfp4": "mxfp4_g32_downproj_4096x14336"}[fmt]
+            "int4": "int4_g64_qproj_4096x4096", "mxfp4": "mxfp4_g32_downproj_4096x14336",
+            "mxint8": "mxint8_g32_downproj_4096x14336", "mxfp8": "mxfp8_g32_downproj_4096x14336"}[fmt]
     wl = synth.WORKLOADS[name]
     W = synth.make_weight(wl, wl.rows, wl.cols, seed=wl.seed)
     gpu = binding.dq_solve(W.cuda(), fmt, group, 0, col_dtype, init="l1")
@@ -98,7 +101,7 @@ def _given(gpu: dict) -> dict:
 
 
 @pytest.mark.parametrize("init", ["rtn", "l1"])
-@pytest.mark.parametrize("fmt,group,col_dtype", FORMATS[:4])
+@pytest.mark.parametrize("fmt,group,col_dtype", PRIMARY)
 def test_warm_start_continues_the_iteration(init, fmt, group, col_dtype):
     """T1 iterations, then a warm start of T2 more, equal T1 + T2 iterations bit for bit; the oracle
     started from the same scales agrees."""
@@ -117,7 +120,7 @@ def test_warm_start_continues_the_iteration(init, fmt, group, col_dtype):
 
 def test_warm_start_from_rtn_scales_is_rtn_init():
     W = weight(64, 512, seed=10).cuda()
-    for fmt, group, cd in FORMATS[:4]:
+    for fmt, group, cd in PRIMARY:
         r = binding.dq_solve(W, fmt, group, 3, cd)
         z = binding.dq_solve(W, fmt, group, 0, cd)
         g = binding.dq_solve(W, fmt, group, 3, cd, init="given", init_scales=_given(z))
@@ -125,13 +128,14 @@ def test_warm_start_from_rtn_scales_is_rtn_init():
             assert torch.equal(r[k], g[k]), (fmt, k)
 
 
-@pytest.mark.parametrize("fmt,group,col_dtype", FORMATS[:4])
+@pytest.mark.parametrize("fmt,group,col_dtype", PRIMARY)
 def test_warm_start_rejects_inadmissible_scales(fmt, group, col_dtype):
     """An inadmissible given scale is found by the library's own check before any iteration runs:
     DQ_EINVAL from the device status, and the outputs past the given scales are untouched."""
     W = weight(32, 256, seed=11).cuda()
     base = _given(binding.dq_solve(W, fmt, group, 0, col_dtype))
     bad_a = {"int4": [0x0000, 0x7C00, 0x8001, 0x7E00], "mxint4": [0, 254, 255], "mxfp4": [0, 254, 255],
+             "mxint8": [0, 254, 255], "mxfp8": [0, 254, 255],
              "nvfp4": [0x00, 0x7F, 0x80, 0xFF]}[fmt]
     cases = []
     for v in bad_a:
