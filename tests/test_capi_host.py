@@ -87,3 +87,33 @@ def test_byte_code_formats_output_sizes():
         assert binding.output_nbytes(64, 512, fmt)["codes"] == 64 * 256
     out = binding.alloc_outputs(8, 64, "mxfp8", 32, "bf16", 2, "cpu")
     assert tuple(out["codes"].shape) == (8, 64)
+
+
+def test_host_side_argument_checks_for_the_8bit_formats(lib_path):
+    """Rejected on the host before any device work (so no GPU is needed here): the MX 8-bit formats
+    take group 32 only, the activation quantizer writes 4-bit codes only, and the byte codes must be
+    8-byte aligned."""
+    lib = binding.load_library()
+    bufs = [ctypes.create_string_buffer(4096 + 64) for _ in range(5)]
+    base = [((ctypes.addressof(b) + 63) // 64) * 64 for b in bufs]
+    W = base[0]
+    wsbuf = ctypes.create_string_buffer(1024)
+    ws = ((ctypes.addressof(wsbuf) + 255) // 256) * 256
+
+    def outs(codes_off=0):
+        return binding._Outputs(base[1] + codes_off, base[2], base[3], base[4], base[4] + 1024)
+
+    for fmt in (int(binding.Format.MXINT8), int(binding.Format.MXFP8)):
+        for g, want in ((16, 2), (64, 2)):
+            o = outs()
+            assert lib.dq_solve(W, 1, 4, 64, fmt, g, 2, 1, ctypes.byref(o), None, 0, None) == want
+        # byte codes 4-byte aligned only: DQ_EINVAL; 8-byte aligned they pass the output checks and stop
+        # later (no device here: DQ_ECUDA; with one, the empty workspace: DQ_EWORKSPACE)
+        o = outs(codes_off=4)
+        assert lib.dq_solve(W, 1, 4, 64, fmt, 32, 2, 1, ctypes.byref(o), ws, 0, None) == 1
+        o = outs(codes_off=8)
+        assert lib.dq_solve(W, 1, 4, 64, fmt, 32, 2, 1, ctypes.byref(o), ws, 0, None) in (3, 5)
+        o = outs()
+        assert lib.dq_act_quant(W, 1, 4, 64, base[4], 1, fmt, 32, ctypes.byref(o), None, 0, None) == 2
+    o = outs()
+    assert lib.dq_solve(W, 1, 4, 64, 6, 32, 2, 1, ctypes.byref(o), None, 0, None) == 1   # no format 6
