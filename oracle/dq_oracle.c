@@ -24,7 +24,8 @@
  * (j ascending inside a block, i ascending inside a column), fp64 arithmetic,
  * no blocking or fusion.  Readings of points the pages leave open:
  *  - Q rounds to the nearest grid value, ties to the "even" neighbour (even
- *    integer for INT4; even mantissa bit for E2M1), values past the ends clip.
+ *    integer on the INT4 and INT8 grids; even mantissa bit for E2M1 and
+ *    E4M3), values past the ends clip.
  *    The decision compares W with boundary*(a*b), which is exact in fp64
  *    because a*b and boundary*(a*b) have few significant bits.
  *  - Projection onto admissible inverse scales = nearest admissible value in
