@@ -169,7 +169,11 @@ def test_quantizer_e4m3_matches_library_cast():
     for x, w in zip(xs.tolist(), want.tolist()):
         assert oracle.quant_value("mxfp8", x, 1.0) == w, (x, w)
     for x, q in {1.0625: 1.0, 1.1875: 1.25, 3 * 2.0 ** -10: 2.0 ** -8, 2.0 ** -10: 0.0, 464.0: 448.0,
-                 1e6: 448.0, -1e6: -448.0, -2.0 ** -10: 0.0}.items():
+                 1e6: 448.0, -1e6: -448.0, -2.0 ** -10: 0.0,
+                 1.9375: 2.0,                   # across a binade end: 1.875 (mantissa 7) vs 2 (mantissa 0)
+                 15 * 2.0 ** -10: 2.0 ** -6,    # largest subnormal 7 * 2^-9 vs smallest normal 2^-6
+                 432.0: 448.0,                  # 416 (mantissa 5) vs 448 (mantissa 6)
+                 -13 * 2.0 ** -10: -6 * 2.0 ** -9}.items():
         assert oracle.quant_value("mxfp8", x, 1.0) == q, x
 
 
