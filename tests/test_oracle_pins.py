@@ -95,6 +95,20 @@ def test_rtn_error_bound():
         assert np.all(np.abs(ticks) <= 0.5 + 1e-12)
 
 
+@pytest.mark.parametrize("fmt,qmax", [("mxint4", 7), ("mxfp4", 6), ("mxint8", 127), ("mxfp8", 448)])
+def test_mx_rtn_scale_straddles_the_e8m0_midpoint(fmt, qmax):
+    """Absmax RTN with power-of-two scales (RTN tutorial, 'Absmax (Symmetric) Quantization': scale
+    max|w| / qmax, 127 for INT8; projected onto E8M0, ties up): a block whose absmax / qmax lies just
+    above the midpoint 1.5 * 2^-8 gets 2^-7, just below it 2^-8.  The bands are 2^-10 relative wide,
+    narrower than the step between neighbouring qmax values, so a wrong qmax moves one of them."""
+    W = np.zeros((2, 64), np.float32)
+    W[0, 5] = 1.5 * 2.0 ** -8 * qmax * (1 + 2.0 ** -10)
+    W[1, 40] = -1.5 * 2.0 ** -8 * qmax * (1 - 2.0 ** -10)
+    W[0, 33] = W[1, 7] = 1e-3  # the other block of each row: a small absmax
+    out = oracle.rtn(W, "f32", fmt, 32, "bf16")
+    assert out["a"][0, 0] == 2.0 ** -7 and out["a"][1, 1] == 2.0 ** -8, out["a"]
+
+
 def test_storage_sizes():
     """DualQuant App. I / Table 12: 224 Llama-3.1-8B linears -> 3.49 GB codes + 0.22 GB G64 scales;
     RTN tutorial: g=128 fp16 scale overhead 3.1%."""
