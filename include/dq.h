@@ -16,7 +16,8 @@
  * Conventions shared by every entry point
  *  - All tensor pointers are DEVICE pointers unless the name says host; the
  *    caller owns every buffer.  The library allocates no memory and keeps no
- *    global state between calls; calls on different streams with different
+ *    global state between calls (dq_solve_static excepted: its scratch is one
+ *    static device array); calls on different streams with different
  *    workspaces are independent.
  *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *    stream) and is asynchronous: a DQ_OK return means the arguments were
