@@ -484,6 +484,35 @@ def test_sign_flip_nvfp4():
     np.testing.assert_array_equal(o1["q"], -o2["q"])
 
 
+@pytest.mark.parametrize("seed,wdt,mult", [(101, "f32", 1.0), (102, "bf16", 1.0), (103, "f32", 37.25),
+                                           (104, "bf16", 3.0e-5)])
+def test_nvfp4_tensor_scale_maps_amax_to_the_top_of_the_format(seed, wdt, mult):
+    """NVFP4's one fp32 per-tensor scale (summary §3, the NVFP4 configuration: E2M1 elements with
+    FP8-E4M3 block scales) is the factor that makes the largest magnitude of the two-level format,
+    E2M1's 6 times E4M3's 448, reconstruct the tensor's max |W|.  Checked on the RTN iterate from its
+    consequences, not from the formula: the block that holds max |W| gets e = 448 (the top of E4M3),
+    that element's code is +-6 (the top of E2M1), its reconstruction a q b = s_T 448 6 equals max |W|
+    to within the fp32 rounding of s_T, and no block scale leaves the E4M3 range.  A constant other
+    than 6 * 448 (448 alone, 6 alone, 7 * 448) or a power-of-two rounding of s_T fails here."""
+    Win, wdtype, Wv = tiny_matrix(24, 96, wdt, seed)
+    if mult != 1.0:
+        Wv = Wv * mult
+        if wdt == "bf16":
+            Win = bf16_bits(Wv.astype(np.float32))
+            Wv = bf16_values(Win).reshape(Wv.shape)
+        else:
+            Win = Wv.astype(np.float32)
+            Wv = Win.astype(np.float64)
+    out = oracle.solve(Win, wdtype, "nvfp4", 16, 0, "bf16", want_q=True)
+    sT, e, q = out["sT"], out["a"], out["q"]
+    i, j = np.unravel_index(np.argmax(np.abs(Wv)), Wv.shape)
+    amax = abs(float(Wv[i, j]))
+    assert e[i, j // 16] == 448.0
+    assert abs(q[i, j]) == 6.0 and np.sign(q[i, j]) == np.sign(Wv[i, j])
+    assert abs(Fraction(sT) * 448 * 6 - Fraction(amax)) <= Fraction(amax) * Fraction(1, 2 ** 24)
+    assert np.all(e <= 448.0) and np.all(e >= 2.0 ** -9)
+
+
 @pytest.mark.parametrize("fmt,G,col_dt", [("int4", 64, "f16"), ("nvfp4", 16, "bf16")])
 def test_permutation_equivariance(fmt, G, col_dt):
     """Permuting whole column groups (or rows) permutes every output the same way."""
