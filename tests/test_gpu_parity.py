@@ -208,37 +208,19 @@ def test_full_size_qproj_int4_against_full_oracle():
     run_both(W, wl.fmt, wl.group, wl.iters, wl.col_dtype, wl.name)
 
 
-@pytest.mark.parametrize("name", ["mxint4_g32_downproj_4096x14336", "nvfp4_g16_gateup_14336x4096",
-                                  "int4_g64_256x512_f32", "mxint8_g32_downproj_4096x14336",
-                                  "mxfp8_g32_downproj_4096x14336"])
-def test_full_size_last_iteration_and_final_state(name):
-    """Full-size solve: the last GPU iteration equals one oracle iteration from the GPU's previous
-    iterate (every block and column scale, bit-exact); the codes equal Q(W/(a b)) of the final
-    scales; the final MSE equals the oracle's MSE of that state; MSE is monotone."""
+@pytest.mark.parametrize("name", ["nvfp4_g16_gateup_14336x4096", "int4_g64_256x512_f32",
+                                  "mxint4_g32_downproj_4096x14336", "mxfp4_g32_downproj_4096x14336",
+                                  "mxint8_g32_downproj_4096x14336", "mxfp8_g32_downproj_4096x14336"])
+def test_full_size_whole_trajectory(name):
+    """Every full-size workload exactly as the benchmark runs it (its own shape, seed, law and
+    iteration count; the 14336x4096 NVFP4 one is the headline workload): the whole solve against
+    the oracle -- every per-iteration MSE within 1e-4, final codes, block scales, column scales and
+    s_T bit-exact (reproduction README "Core equations"; the benchmark spec's tolerances) -- and the MSE
+    never increases."""
     wl, W = full_weight(name)
-    Wd = W.cuda()
-    T = wl.iters
-    prev = binding.dq_solve(Wd, wl.fmt, wl.group, T - 1, wl.col_dtype)
-    last = binding.dq_solve(Wd, wl.fmt, wl.group, T, wl.col_dtype)
-    sT = float(last["tensor_scale"].cpu()[0]) if wl.fmt == "nvfp4" else 1.0
-    a_prev = block_scale_values(wl.fmt, prev["block_scales"])
-    b_prev = col_scale_values(prev["col_scales"])
-    Win, wdt = synth.to_oracle_input(W)
-    a_o, b_o = oracle.iterate(Win, wdt, wl.fmt, wl.group, wl.col_dtype, sT, a_prev, b_prev)
-    a_last = block_scale_values(wl.fmt, last["block_scales"])
-    b_last = col_scale_values(last["col_scales"])
-    assert np.array_equal(a_last, a_o), int((a_last != a_o).sum())
-    assert np.array_equal(b_last, b_o), int((b_last != b_o).sum())
-    # codes of the final state and its MSE
-    q = oracle.requant(Win, wdt, wl.fmt, wl.group, wl.col_dtype, sT, a_last, b_last)
-    import bruteforce as bf
-    assert np.array_equal(bf.decode_codes(wl.fmt, last["codes"].cpu().numpy()), q)
-    mse_o = oracle.mse(Win, wdt, wl.fmt, wl.group, wl.col_dtype, sT, q, a_last, b_last)
-    mse = last["mse"].cpu().numpy()
-    assert mse[-1] == pytest.approx(mse_o, rel=MSE_RTOL)
+    gpu, _ = run_both(W, wl.fmt, wl.group, wl.iters, wl.col_dtype, wl.name)
+    mse = gpu["mse"].cpu().numpy()
     assert np.all(mse[1:] <= mse[:-1] * (1 + 1e-9))
-    np.testing.assert_allclose(mse[:-1], prev["mse"].cpu().numpy()[:-1].tolist() + [mse[-2]], rtol=0)
-    assert mse[-2] == pytest.approx(float(prev["mse"][-1]), rel=1e-6)
 
 
 @pytest.mark.parametrize("fmt,group,col_dtype,name", [
