@@ -14,8 +14,6 @@
 #include "dq.h"
 #include "dq_internal.h"
 
-#include <mutex>
-
 // Scratch of dq_solve_static, shared by every call on a device.  Host code
 // must not pass this name to a kernel: on the host it denotes a stand-in
 // object, not the device array.  The device address comes from
@@ -24,24 +22,15 @@ static __device__ __align__(256) unsigned char g_static_scratch[DQ_STATIC_SCRATC
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-std::mutex g_setup_mutex;
-void* g_scratch_addr[kMaxDevices];  // device address of g_static_scratch per device, set once
-
-// Device address of the scratch array on the current device.  The first call
-// for a device looks it up (which also loads the module there) with that
-// device current; later calls reuse it.
+// Device address of the scratch array on the current device, looked up on
+// every call: a cached address would go stale if the caller tore the context
+// down (cudaDeviceReset) and the module were loaded again at another address.
+// The lookup is cheap once the module is loaded; the first one on a device
+// loads it there.
 int static_scratch_address(void** addr) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return DQ_ECUDA;
-  if (dev < 0 || dev >= kMaxDevices) return DQ_EUNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (g_scratch_addr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return DQ_ECUDA;
-    g_scratch_addr[dev] = p;
-  }
-  *addr = g_scratch_addr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return DQ_ECUDA;
+  *addr = p;
   return DQ_OK;
 }
 

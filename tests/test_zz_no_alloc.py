@@ -82,6 +82,34 @@ def test_static_matches_workspace_entry_on_consecutive_calls(lib):
         assert_same(fmt, got, ref, "call %d" % i)
 
 
+def test_static_call_leaves_free_device_memory_unchanged(lib):
+    """The call allocates nothing: the device's free memory (cudaMemGetInfo) is the same before and
+    after a solve, once the library's device code is loaded (the first call on a device loads it).
+    Every buffer the call touches is allocated beforehand; any device allocation inside the call
+    would lower the free memory by at least one 2 MiB page."""
+    wl = synth.WORKLOADS["nvfp4_g16_gateup_14336x4096"]
+    fmt, group, cd, M, N, iters, seed = CASES[0]
+    W = synth.make_weight(wl, M, N, seed=seed).cuda()
+    out = binding.alloc_outputs(M, N, binding._fmt(fmt), group, cd, iters, W.device)
+    status = torch.full((1,), -1, dtype=torch.int32, device=W.device)
+    o = binding._outputs_struct(out)
+    stream = torch.cuda.current_stream().cuda_stream
+
+    def call():
+        return lib.dq_solve_static(W.data_ptr(), binding._DTYPES[W.dtype], M, N, int(binding._fmt(fmt)), group,
+                                   iters, 1, ctypes.byref(o), status.data_ptr(), stream)
+
+    assert call() == 0  # loads the device code on this device if no call did yet
+    torch.cuda.synchronize()
+    free_before, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        assert call() == 0
+    torch.cuda.synchronize()
+    free_after, _ = torch.cuda.mem_get_info()
+    assert int(status.cpu()[0]) == 0
+    assert free_after == free_before, (free_before, free_after)
+
+
 def test_static_rejects_shape_beyond_scratch(lib):
     # one row of 2^20 columns needs about 16 MiB of scratch on a 148-SM GPU
     rows, cols, group = 1, 1 << 20, 64
