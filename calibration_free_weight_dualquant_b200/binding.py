@@ -56,7 +56,8 @@ class _Outputs(ctypes.Structure):
 
 
 class _Options(ctypes.Structure):
-    _fields_ = [("mode", ctypes.c_int), ("init", ctypes.c_int), ("code_changes", ctypes.c_void_p)]
+    _fields_ = [("mode", ctypes.c_int), ("init", ctypes.c_int), ("code_changes", ctypes.c_void_p),
+                ("full_passes", ctypes.c_int)]
 
 
 class _Matrix(ctypes.Structure):
@@ -96,8 +97,10 @@ def load_library():
     lib.dq_solve_host.argtypes = [P, I, I64, I64, I, I, I, I, ctypes.POINTER(_Outputs), P, SZ, P]
     lib.dq_solve_host.restype = I
     lib.dq_diagnostics.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint64)]
+    lib.dq_active_block_columns.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint64)]
+    lib.dq_active_block_columns.restype = I
     lib.dq_diagnostics.restype = I
-    lib.dq_wait_selftest.argtypes = [P, SZ, P]
+    lib.dq_wait_selftest.argtypes = [P, SZ, I, P]
     lib.dq_wait_selftest.restype = I
     lib.dq_solve_static.argtypes = [P, I, I64, I64, I, I, I, I, ctypes.POINTER(_Outputs), P, P]
     lib.dq_solve_static.restype = I
@@ -160,7 +163,7 @@ INITS = {"rtn": 0, "l1": 1, "given": 2}
 def dq_solve(W: torch.Tensor, fmt, group: Optional[int] = None, iters: int = 0, col_dtype: Optional[str] = None,
              out: Optional[dict] = None, workspace: Optional[torch.Tensor] = None, stream=None,
              check: bool = True, mode: str = "dual", init: str = "rtn", init_scales: Optional[dict] = None,
-             changes: bool = False) -> dict:
+             changes: bool = False, full_passes: bool = False) -> dict:
     """Enqueue dq_solve on a CUDA tensor W [rows, cols]; returns the output tensors.
 
     ``check`` waits for the stream and raises on a device-reported status
@@ -171,7 +174,8 @@ def dq_solve(W: torch.Tensor, fmt, group: Optional[int] = None, iters: int = 0, 
     "col_scales", "tensor_scale"} in storage format, e.g. a previous call's
     outputs), copied into ``out`` first, or whatever ``out`` already holds.
     ``changes`` adds out["code_changes"] (int64 [iters+1], changed codes per
-    iteration)."""
+    iteration).  ``full_passes`` makes every iteration process every
+    block-column (no skipping of block-columns at a fixed point; same outputs)."""
     lib = load_library()
     if not W.is_cuda:
         raise DQError(1, "dq_solve: W must be a CUDA tensor (use solve() for host tensors)")
@@ -183,7 +187,7 @@ def dq_solve(W: torch.Tensor, fmt, group: Optional[int] = None, iters: int = 0, 
         raise DQError(1, "dq_solve: W must be contiguous f32/bf16/f16")
     if out is None:
         out = alloc_outputs(rows, cols, f, g, cd, iters, W.device)
-    extended = init != "rtn" or changes
+    extended = init != "rtn" or changes or full_passes
     opts = None
     if extended:
         if init == "given" and init_scales is not None:
@@ -192,7 +196,8 @@ def dq_solve(W: torch.Tensor, fmt, group: Optional[int] = None, iters: int = 0, 
                     out[k].view(-1).copy_(init_scales[k].reshape(-1))
         if changes:
             out["code_changes"] = torch.empty(iters + 1, dtype=torch.int64, device=W.device)
-        opts = _Options(MODES[mode], INITS[init], out["code_changes"].data_ptr() if changes else None)
+        opts = _Options(MODES[mode], INITS[init], out["code_changes"].data_ptr() if changes else None,
+                        1 if full_passes else 0)
     if workspace is None:
         if extended:
             nbytes = lib.dq_workspace_bytes_ex(rows, cols, int(f), g, ctypes.byref(opts))
@@ -408,11 +413,12 @@ def rtn(W: torch.Tensor, fmt="nvfp4", group: Optional[int] = None, col_dtype: Op
     return solve(W, fmt, group, 0, col_dtype)
 
 
-def wait_selftest(workspace: torch.Tensor, stream=None) -> int:
+def wait_selftest(workspace: torch.Tensor, which: int = 0, stream=None) -> int:
     """Run the library's bounded-wait self-test on ``workspace`` (device, >= 512 bytes) and return the
-    device status it leaves (dq_sync_status): DQ_ECUDA (5) when the wait gave up as it should."""
+    device status it leaves (dq_sync_status): DQ_ECUDA (5) when the wait gave up as it should.
+    ``which``: 0 waits on a pending count in global memory, 1 on a shared-memory ring barrier."""
     lib = load_library()
-    st = lib.dq_wait_selftest(workspace.data_ptr(), workspace.numel(), _stream_ptr(stream))
+    st = lib.dq_wait_selftest(workspace.data_ptr(), workspace.numel(), int(which), _stream_ptr(stream))
     if st != 0:
         raise DQError(st, "dq_wait_selftest")
     return lib.dq_sync_status(workspace.data_ptr(), _stream_ptr(stream))
@@ -427,3 +433,14 @@ def diagnostics(workspace: torch.Tensor, stream=None) -> dict:
         raise DQError(st, "dq_diagnostics")
     return {"quant_exact_lane_rows": int(arr[0]), "block_exact": int(arr[1]), "col_exact": int(arr[2]),
             "quant_tie_lane_rows": int(arr[3])}
+
+
+def active_block_columns(workspace: torch.Tensor, stream=None) -> int:
+    """Block-columns the BCD iterations of the last solve on this workspace processed, summed over the
+    iterations (iters * cols/group when none reached a fixed point early)."""
+    lib = load_library()
+    out = ctypes.c_uint64(0)
+    st = lib.dq_active_block_columns(workspace.data_ptr(), _stream_ptr(stream), ctypes.byref(out))
+    if st != 0:
+        raise DQError(st, "dq_active_block_columns")
+    return int(out.value)

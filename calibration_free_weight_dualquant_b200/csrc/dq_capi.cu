@@ -3,6 +3,7 @@
 #include "dq.h"
 #include "dq_internal.h"
 
+#include <algorithm>
 #include <cstring>
 
 namespace {
@@ -13,9 +14,11 @@ constexpr size_t kAlign = 256;
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 struct Plan {
-  int TS, n_strips, P, segmax, P_final, segmax_final, nb;
+  int TSv, n_strips, P, segmax, P_final, segmax_final, nb;
   int64_t L;
-  size_t off_counters, off_amb_tick, off_sx_left, off_col_part, off_cta_part, off_amb_list, off_xpart, total;
+  size_t smem;  // dynamic shared memory of k_iter
+  size_t off_counters, off_amb_tick, off_pend, off_chg, off_col_part, off_cta_part, off_mse_seg, off_mse_bc,
+      off_amb_list, off_xpart, total;
   size_t l1_zero_bytes;  // L1 init: digit counters to zero (start of the col_part region)
   size_t off_l1_tot, off_l1_norm;
 };
@@ -28,10 +31,10 @@ int check_shape(int64_t rows, int64_t cols, int format, int group) {
   if ((format == DQ_MXINT4 || format == DQ_MXFP4 || format == DQ_MXINT8 || format == DQ_MXFP8) && group != 32)
     return DQ_EUNSUPPORTED;
   if (format == DQ_NVFP4 && group != 16) return DQ_EUNSUPPORTED;
-  // a block spans group/8 lanes of a warp: a power of two from 1 to 32
-  if (group < 8 || group > dq::kStripMax || (group & (group - 1)) != 0) return DQ_EUNSUPPORTED;
+  // a block row spans group/8 lanes of a warp: a power of two from 1 to 32
+  if (group < 8 || group > dq::kGroupMax || (group & (group - 1)) != 0) return DQ_EUNSUPPORTED;
   if (rows > ((int64_t)1 << 40) / cols) return DQ_EUNSUPPORTED;  // keeps all index products in int64 range
-  if (cols / group > INT32_MAX) return DQ_EUNSUPPORTED;
+  if (cols / group > INT32_MAX / 2) return DQ_EUNSUPPORTED;
   return DQ_OK;
 }
 
@@ -48,16 +51,14 @@ int make_plan(int64_t M, int64_t N, int group, int init, Plan* pl) {
   int st = device_sms(&sms);
   if (st != DQ_OK) return st;
   pl->nb = (int)(N / group);
-  pl->TS = (dq::kStripMax / group) * group;
-  pl->n_strips = (int)((N + pl->TS - 1) / pl->TS);
+  pl->TSv = dq::kBcPerStrip * group;
+  pl->n_strips = (pl->nb + dq::kBcPerStrip - 1) / dq::kBcPerStrip;
   pl->L = (int64_t)pl->n_strips * M;
   const int64_t byrows = pl->L / dq::kMinRowsPerCta;
   auto ctas = [&](int64_t want) { return (int)(byrows < want ? (byrows < 1 ? 1 : byrows) : want); };
-  // a CTA's contiguous range of len rows touches at most ceil(len/M) + 1 strips
-  auto segs = [&](int64_t P) { return (int)(((pl->L + P - 1) / P + M - 1) / M + 1); };
   // a grid that is a multiple of the strip count (when that keeps at least
-  // 90% of the SMs) gives every CTA rows of a single strip: no CTA pays a
-  // second column-table setup and strip end inside a pass
+  // 90% of the SMs) gives every CTA rows of a single strip in a full pass: no
+  // CTA pays a second column-table setup and strip end inside a pass
   int64_t want = (int64_t)sms * dq::kCtasPerSm;
   if (want > dq::kMaxGrid) want = dq::kMaxGrid;
   if (pl->n_strips <= want) {
@@ -65,16 +66,31 @@ int make_plan(int64_t M, int64_t N, int group, int init, Plan* pl) {
     if (10 * aligned >= 9 * want) want = aligned;
   }
   pl->P = ctas(want);
-  pl->segmax = segs(pl->P);
+  // A pass over nv <= n_strips strips splits L = nv M units over
+  // pass_ctas(P, nv, L) CTAs; a CTA's contiguous range of len units touches at
+  // most ceil(len / M) + 1 strips.  When that count is the aligned one or the
+  // grid, len <= ceil(L_full / pmin) (pmin: the fewest such CTAs over every
+  // nv); when it is capped at one CTA per kMinRowsPerCta units, len stays
+  // below 2 kMinRowsPerCta.
+  int pmin = pl->P;
+  for (int nv = 1; nv <= pl->n_strips && nv <= pl->P; ++nv)
+    pmin = std::min(pmin, dq::pass_ctas(pl->P, nv, INT64_MAX));
+  const int64_t len = std::max((pl->L + pmin - 1) / pmin, 2 * dq::kMinRowsPerCta);
+  pl->segmax = (int)((len + M - 1) / M + 1);
   pl->P_final = ctas((int64_t)sms * dq::kFinalCtasPerSm);
-  pl->segmax_final = segs(pl->P_final);
+  pl->segmax_final = pl->segmax;
+  pl->smem = (size_t)dq::iter_smem(group / 8, pl->P, pl->segmax).total;
+  if (pl->smem > (size_t)227 * 1024) return DQ_EUNSUPPORTED;  // more strips per CTA than shared memory holds
   size_t off = align_up(sizeof(dq::WsHeader));
+  // zeroed at the start of a solve: arrival counters, pending counts, change flags
   pl->off_counters = off;
   off += align_up(sizeof(unsigned) * (size_t)pl->n_strips);
   pl->off_amb_tick = off;
   off += align_up(sizeof(unsigned) * (size_t)N);
-  pl->off_sx_left = off;
-  off += align_up(sizeof(unsigned) * (size_t)pl->n_strips);
+  pl->off_pend = off;
+  off += align_up(sizeof(unsigned) * (size_t)pl->nb);
+  pl->off_chg = off;
+  off += align_up(sizeof(unsigned) * 3 * (size_t)pl->nb);
   pl->off_col_part = off;
   // the L1-init scratch overlays the column partials (the init kernels run
   // before the first iteration): per-column digits, the total's digits, norms;
@@ -85,10 +101,14 @@ int make_plan(int64_t M, int64_t N, int group, int init, Plan* pl) {
   pl->off_l1_norm = pl->off_l1_tot + tot_bytes;
   pl->l1_zero_bytes = dig_bytes + tot_bytes;
   const size_t l1_bytes = dig_bytes + tot_bytes + align_up(sizeof(double) * (size_t)N);
-  const size_t part_bytes = align_up(sizeof(double2) * (size_t)pl->P * (size_t)pl->segmax * (size_t)pl->TS);
+  const size_t part_bytes = align_up(sizeof(double2) * (size_t)pl->P * (size_t)pl->segmax * (size_t)pl->TSv);
   off += (init == DQ_INIT_L1 && l1_bytes > part_bytes) ? l1_bytes : part_bytes;
   pl->off_cta_part = off;
   off += align_up(sizeof(double) * 3 * (size_t)(pl->P > pl->P_final ? pl->P : pl->P_final));
+  pl->off_mse_seg = off;
+  off += align_up(sizeof(double) * (size_t)pl->P * (size_t)pl->segmax * dq::kBcPerStrip);
+  pl->off_mse_bc = off;
+  off += align_up(sizeof(double) * 3 * (size_t)pl->nb);
   pl->off_amb_list = off;
   off += align_up(sizeof(int) * 3 * (size_t)N);
   pl->off_xpart = off;
@@ -150,7 +170,7 @@ int solve_impl(const void* W, int w_dtype, int64_t rows, int64_t cols, int forma
   p.M = rows;
   p.N = cols;
   p.nb = pl.nb;
-  p.TS = pl.TS;
+  p.TSv = pl.TSv;
   p.n_strips = pl.n_strips;
   p.P = pl.P;
   p.segmax = pl.segmax;
@@ -159,6 +179,7 @@ int solve_impl(const void* W, int w_dtype, int64_t rows, int64_t cols, int forma
   p.L = pl.L;
   p.mode = mode;
   p.init = init;
+  p.full_passes = opt ? (opt->full_passes != 0) : 0;
   p.changes = changes;
   p.l1_dig = reinterpret_cast<unsigned long long*>(ws + pl.off_col_part);
   p.l1_tot = reinterpret_cast<unsigned long long*>(ws + pl.off_l1_tot);
@@ -174,11 +195,15 @@ int solve_impl(const void* W, int w_dtype, int64_t rows, int64_t cols, int forma
   p.cta_part = reinterpret_cast<double*>(ws + pl.off_cta_part);
   p.amb_list = reinterpret_cast<int*>(ws + pl.off_amb_list);
   p.amb_tick = reinterpret_cast<unsigned*>(ws + pl.off_amb_tick);
-  p.sx_left = reinterpret_cast<unsigned*>(ws + pl.off_sx_left);
+  p.pend = reinterpret_cast<unsigned*>(ws + pl.off_pend);
+  p.chg = reinterpret_cast<unsigned*>(ws + pl.off_chg);
+  p.mse_seg = reinterpret_cast<double*>(ws + pl.off_mse_seg);
+  p.mse_bc = reinterpret_cast<double*>(ws + pl.off_mse_bc);
   p.xpart = reinterpret_cast<double2*>(ws + pl.off_xpart);
 
-  // header and arrival counters (strips, listed columns) start at zero; the
-  // partial buffers and the column list need no init
+  // header, arrival counters (strips, listed columns), pending counts and
+  // change flags start at zero; the partial buffers and the column list need
+  // no init
   if (cudaMemsetAsync(ws, 0, pl.off_col_part, stream) != cudaSuccess) return DQ_ECUDA;
   if (init == DQ_INIT_L1 && cudaMemsetAsync(ws + pl.off_col_part, 0, pl.l1_zero_bytes, stream) != cudaSuccess)
     return DQ_ECUDA;
@@ -254,10 +279,11 @@ int dq_sync_status(const void* workspace, void* stream) {
   return (flags & dq::kFlagTimeout) ? DQ_ECUDA : DQ_OK;
 }
 
-int dq_wait_selftest(void* workspace, size_t workspace_bytes, void* stream) {
+int dq_wait_selftest(void* workspace, size_t workspace_bytes, int which, void* stream) {
   if (!workspace || !aligned(workspace, kAlign)) return DQ_EINVAL;
+  if (which != 0 && which != 1) return DQ_EINVAL;
   if (workspace_bytes < 512) return DQ_EWORKSPACE;
-  if (dq::launch_wait_selftest(workspace, static_cast<cudaStream_t>(stream)) != cudaSuccess) return DQ_ECUDA;
+  if (dq::launch_wait_selftest(workspace, which, static_cast<cudaStream_t>(stream)) != cudaSuccess) return DQ_ECUDA;
   return DQ_OK;
 }
 
@@ -270,6 +296,15 @@ int dq_diagnostics(const void* workspace, void* stream, uint64_t out[4]) {
   out[1] = h.n_block_exact;
   out[2] = h.n_col_exact;
   out[3] = h.n_quant_tie;
+  return DQ_OK;
+}
+
+int dq_active_block_columns(const void* workspace, void* stream, uint64_t* out) {
+  if (!workspace || !out) return DQ_EINVAL;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DQ_ECUDA;
+  dq::WsHeader h;
+  if (cudaMemcpy(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return DQ_ECUDA;
+  *out = h.n_active_bc;
   return DQ_OK;
 }
 

@@ -172,18 +172,64 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
   return ok != 0;
 }
 
-// Bounded wait: gives up after kSpinLimit polls (each poll may suspend the
-// thread for a while), records kFlagTimeout and returns false.
-constexpr unsigned kSpinLimit = 1u << 22;
+// Wall-clock bound of every wait in the solver's kernels (1 s): a wait that
+// runs out records kFlagTimeout in the workspace header and returns, so a lost
+// arrival ends in a status instead of a hung GPU.
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity, unsigned* flags) {
-  for (unsigned i = 0; i < kSpinLimit; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    // after a first long wait, stop at once if some wait has already given up
-    if (i == 4096 && (*reinterpret_cast<volatile unsigned*>(flags) & kFlagTimeout)) return false;
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ unsigned ld_volatile(const unsigned* a) { return *reinterpret_cast<const volatile unsigned*>(a); }
+
+// True when a bounded wait begun at t0 must give up (its time is over, or some
+// other wait already gave up); then kFlagTimeout is recorded.
+__device__ __forceinline__ bool wait_expired(unsigned* flags, unsigned long long t0) {
+  if (global_ns() - t0 > kWaitLimitNs || (ld_volatile(flags) & kFlagTimeout)) {
+    atomicOr(flags, kFlagTimeout);
+    return true;
   }
-  atomicOr(flags, kFlagTimeout);
   return false;
+}
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* a) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
+  return v;
+}
+
+// Bounded wait for the phase of `parity` of a ring barrier: polls until it
+// completes, or until kWaitLimitNs of wall time have passed or another wait has
+// given up (checked every 256 polls), then records kFlagTimeout and returns
+// false.  The first poll usually succeeds, so the timer is read only after it
+// fails.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity, unsigned* flags) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (unsigned i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 255u) == 0u && wait_expired(flags, t0)) return false;
+  }
+}
+
+// Wait for a copy this CTA issued to land before the CTA exits: bounded by
+// kWaitLimitNs alone (a copy in flight completes whatever other waits did).
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, unsigned parity) {
+  const unsigned long long t0 = global_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_ns() - t0 > kWaitLimitNs) return;
+  }
+}
+
+// Orders this thread's earlier generic-proxy accesses to shared memory (the
+// consumers' loads of a ring slot) before later async-proxy accesses (the
+// tensor copy that refills the slot once the release is observed): without it
+// a copy may overwrite a slot whose loads are not yet performed.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // Copy `bytes` (multiple of 16, both addresses 16-byte aligned) from global

@@ -10,7 +10,7 @@ namespace dq {
 
 constexpr int kThreads = 256;   // 8 warps per CTA
 constexpr int kWarps = kThreads / 32;
-constexpr int kStripMax = 256;  // columns per strip (8 per lane, 32 lanes)
+constexpr int kGroupMax = 256;  // largest block size (a block row spans at most one warp)
 constexpr int kCtasPerSm = 1;        // per-iteration pass: one 512-thread CTA per SM
 constexpr int kMaxGrid = 1024;       // CTAs of the per-iteration pass at most
 constexpr int kFinalCtasPerSm = 4;   // one-time passes
@@ -23,6 +23,83 @@ constexpr unsigned kFlagNonFinite = 1u;
 constexpr unsigned kFlagTimeout = 2u;  // a bounded pipeline wait gave up (results invalid)
 constexpr unsigned kFlagBadInit = 4u;  // a warm start was given an inadmissible scale
 constexpr unsigned kFlagAbort = kFlagNonFinite | kFlagBadInit;  // later kernels do nothing
+
+// ---------------------------------------------------------------------------
+// Geometry of the per-iteration pass k_iter (host and device).
+constexpr int kConsumerWarps = 15;
+constexpr int kConsumers = kConsumerWarps * 32;
+constexpr int kIterThreads = kConsumers + 32;
+// block-columns per strip: one per consumer warp
+constexpr int kBcPerStrip = kConsumerWarps;
+constexpr int kRun = 8;
+constexpr int kRingBytes = 96 * 1024;
+constexpr int kMaxStages = 8;
+// Tile geometry for block size G (a multiple of 8 dividing 256) and W element
+// size es: lanes per block row, row-lanes per warp, rows per tile, bytes of
+// one block-column's box and its slot in the ring (16-byte multiple, rounded
+// to 128 bytes for the tensor copy's destination), stage bytes, ring stages.
+struct TileGeo {
+  int lpb, rl, RW, box_bytes, box_stride, stage_bytes, S;
+};
+__host__ __device__ inline TileGeo tile_geo(int G, int es) {
+  TileGeo g;
+  g.lpb = G / 8;
+  g.rl = 32 / g.lpb;
+  g.RW = 2 * g.rl;
+  g.box_bytes = g.RW * G * es;
+  g.box_stride = (g.box_bytes + 127) / 128 * 128;
+  g.stage_bytes = kBcPerStrip * g.box_stride;
+  g.S = kRingBytes / g.stage_bytes < kMaxStages ? kRingBytes / g.stage_bytes : kMaxStages;
+  return g;
+}
+
+// Dynamic shared memory of k_iter (byte offsets): the tile ring; fp64 column
+// accumulators (per consumer warp: 8 columns x 32 lanes of (sum W a q,
+// sum (a q)^2)); one fp64 residual sum per consumer thread; ring barriers;
+// small ints ([0] ticket result, [1] #ambiguous, [2..5] exact-path counters,
+// [8..22] per-slot change flags, [24..38] per-slot listed columns, [40..56]
+// schedule scan); the pass schedule; the column tables (per warp: b pairs
+// [lpb][4], then 1/b pairs [lpb][4]); the first strip of each CTA's range;
+// this CTA's slice of the active list.
+struct IterSmem {
+  int acc, racc, bars, misc, sched, ctab, sfirst, act, total;
+};
+__host__ __device__ inline IterSmem iter_smem(int lpb, int P, int segmax) {
+  IterSmem s;
+  int off = kRingBytes;
+  s.acc = off;
+  off += kConsumerWarps * 8 * 32 * 16;
+  s.racc = off;
+  off += kConsumers * 8;
+  s.bars = off;
+  off += 2 * kMaxStages * 8;
+  s.misc = off;
+  off += 64 * 4;
+  s.sched = off;
+  off += 64;
+  s.ctab = off;
+  off += kConsumerWarps * 2 * 4 * lpb * 8;
+  s.sfirst = off;
+  off += (P * 4 + 15) / 16 * 16;
+  s.act = off;
+  off += (segmax * kBcPerStrip * 4 + 15) / 16 * 16;
+  s.total = off;
+  return s;
+}
+// CTAs that get units in a pass of nv strips (L = nv M units): a multiple of
+// nv (every CTA within one strip) when that keeps at least 90% of the grid,
+// else the grid; and at most one CTA per kMinRowsPerCta units, so every CTA
+// that gets units gets at least one (the strip tickets count every CTA from
+// the first to the last owner of a strip)
+__host__ __device__ inline int pass_ctas(int P, long long nv, long long L) {
+  int c = P;
+  if (nv >= 1 && nv <= P) {
+    const long long a = (long long)P / nv * nv;
+    if (10 * a >= 9LL * P) c = (int)a;
+  }
+  const long long cap = L / kMinRowsPerCta;
+  return cap < c ? (cap < 1 ? 1 : (int)cap) : c;
+}
 
 // Device workspace header (first 256 bytes of the workspace).
 struct WsHeader {
@@ -38,37 +115,43 @@ struct WsHeader {
   unsigned long long n_block_exact;  // block updates taken in fp64
   unsigned long long n_col_exact;    // column updates recomputed exactly over all rows
   unsigned long long amax_scaled;    // L1 init, NVFP4: max |W_ij| / b_j as the bits of a double
+  unsigned long long n_active_bc;    // block-columns processed, summed over the BCD passes
 };
+static_assert(sizeof(WsHeader) <= 256, "workspace header");
 
 // Everything a kernel needs, passed by value.
 struct Problem {
   const void* W;
   int wdt, fmt, G, col_dt;
   int64_t M, N;
-  int nb;        // blocks per row = N / G
-  int TS;        // strip width (columns), multiple of G and of 8, <= kStripMax
-  int n_strips;  // ceil(N / TS)
+  int nb;        // blocks per row = N / G (= block-columns)
+  int TSv;       // columns of a strip of k_iter: 15 block-columns, 15 G
+  int n_strips;  // strips of a pass over every block-column: ceil(nb / 15)
   int P;         // CTAs of the per-iteration pass
-  int segmax;    // max (CTA, strip) segments per CTA of that pass
-  int P_final;   // CTAs of the one-time passes (stats, init, final)
+  int segmax;    // max (CTA, strip) segments per CTA in any pass
+  int P_final;   // CTAs of the one-time passes (stats, init)
   int segmax_final;
-  int64_t L;     // n_strips * M (strip-major row units)
+  int64_t L;     // n_strips * M (strip-major row units of a full pass)
   void* codes;
   void* a_store;
   void* b_store;
   float* sT_out;
   double* mse;
   WsHeader* hdr;
-  unsigned* strip_counter;  // [n_strips]
-  double2* col_part;        // [P * segmax][TS] (sum W a q, sum (a q)^2)
-  double* cta_part;         // [max(P, P_final)]
+  unsigned* strip_counter;  // [n_strips] arrivals per strip (zeroed)
+  double2* col_part;        // [P * segmax][TSv] (sum W a q, sum (a q)^2)
+  double* cta_part;         // [3][max(P, P_final)] per-CTA residual totals of the final pass
+  double* mse_seg;          // [P * segmax][15] residual total per (CTA segment, block-column slot)
+  double* mse_bc;           // [3][nb] residual total per block-column, by pass mod 3
+  unsigned* chg;            // [3][nb] a scale of the block-column changed (or was listed), by pass mod 3 (zeroed)
+  unsigned* pend;           // [nb] listed columns of a block-column awaiting their exact update (zeroed)
   int* amb_list;            // [3][N] columns whose certified projection was ambiguous, by pass mod 3
   unsigned* amb_tick;       // [N] arrival counters of their row chunks (zeroed)
-  unsigned* sx_left;        // [n_strips] listed columns of a strip still awaiting their exact update (zeroed)
   double2* xpart;           // [kXPartCap] per-CTA exact partial sums of the listed columns
   int use_tmap;             // W streamed by 2-D tensor copies (else one bulk copy per row)
   int mode;                 // DQ_MODE_DUAL, DQ_MODE_ROW (b keeps its initial value) or DQ_MODE_COL
   int init;                 // DQ_INIT_RTN, DQ_INIT_L1 or DQ_INIT_GIVEN
+  int full_passes;          // every BCD pass takes every block-column (no skipping at fixed points)
   // L1 init scratch (overlays col_part, which the init kernels do not use)
   unsigned long long* l1_dig;   // [N][10] digit counters of the column magnitude sums (zeroed)
   unsigned long long* l1_tot;   // [10] digit counters of the total (zeroed)
@@ -77,8 +160,9 @@ struct Problem {
 };
 
 cudaError_t launch_solve(const Problem& p, int iters, int stats_ctas, cudaStream_t st);
-// Runs the bounded-wait self-test on `workspace` (>= 512 bytes).
-cudaError_t launch_wait_selftest(void* workspace, cudaStream_t st);
+// Runs a bounded-wait self-test on `workspace` (>= 512 bytes): `which` 0 waits
+// on a count in global memory, 1 on a shared-memory ring barrier.
+cudaError_t launch_wait_selftest(void* workspace, int which, cudaStream_t st);
 
 // Host-side validation, workspace layout and enqueue of a whole solve (the body
 // of dq_solve; `workspace` is a device address of at least the planned size).

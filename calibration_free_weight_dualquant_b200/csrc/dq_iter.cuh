@@ -1,15 +1,32 @@
 // dq_iter.cuh -- the per-iteration pass k_iter: one BCD iteration in one read
-// of W (included by dq_solver.cu).
+// of the block-columns that can still change (included by dq_solver.cu).
 //
-// CTA = 15 consumer warps + 1 producer warp (16 warps, 4 per SM sub-partition,
-// so each thread may hold 128 registers).  The producer streams the CTA's rows
-// of the current column strip into a ring of shared-memory tiles of
-// kRowsPerTile rows, guarded by full/empty mbarriers: one 2-D tensor copy (TMA)
-// per tile, or one bulk copy per row when W admits no tensor map.
-// Consumer warp w takes rows w and w + 15 of every tile; lane l takes the 8
-// consecutive columns 8l..8l+7 of the strip as 4 pairs, and the arithmetic on
-// pairs runs as packed f32x2 instructions.  Per element the consumers run the
-// fp32 fast paths and settle flagged elements exactly.  Column sums and the
+// Block-columns.  A block-column is the M x G slab of W under one column of
+// blocks.  Its block scales a_{:,g} and its column scales b_j (j in the
+// block-column) interact only with each other: the block update of a_ig reads
+// the G elements of block (i, g) and their column scales, and the column
+// update of b_j reads column j and the block scales of the blocks holding it
+// (reproduction README, "Core equations"; the NVFP4 tensor scale is fixed at
+// init).  One BCD iteration therefore maps each block-column's state to its
+// next state by itself, and a block-column whose scales all come out of an
+// iteration unchanged is at a fixed point: every later iteration repeats the
+// same sums, the same updates and the same residuals.  Such a block-column is
+// dropped from the later passes; its share of the reconstruction MSE is kept
+// from the pass that last computed it.  The results are those of the full
+// iteration, bit for bit.
+//
+// Schedule of a pass.  The active block-columns (all of them in the first pass
+// and the final pass) are taken in increasing order, 15 at a time, into
+// strips; the (strip, row) units are laid out strip-major and split into
+// equal contiguous ranges, one per CTA.  A CTA is 15 consumer warps + 1
+// producer warp (512 threads, 128 registers each).  Consumer warp w owns
+// block-column w of the strip; its lanes are (row-lane rho, octet o): lane
+// rho * (G/8) + o takes the 8 columns 8o..8o+7 of the block-column in rows rho
+// and rho + 32/(G/8) of every tile, so a tile is 2 * 32/(G/8) rows (512
+// elements per block-column).  The producer fills a shared-memory ring with
+// one 2-D tensor copy (TMA) per block-column and tile, wherever the active
+// block-columns lie; a warp's 32 lanes read 512 contiguous bytes of its slot.
+// The pair arithmetic runs as packed f32x2 instructions.  Column sums and the
 // reconstruction residuals run in fp32 for kRun rows of a lane and are then
 // added into fp64 accumulators kept in shared memory.
 #pragma once
@@ -22,19 +39,12 @@
 
 namespace dq {
 
-constexpr int kConsumerWarps = 15;
-constexpr int kConsumers = kConsumerWarps * 32;
-constexpr int kIterThreads = kConsumers + 32;
 constexpr int kConsumerTreeTop = 256;  // largest power of two below kConsumers
 static_assert(kConsumerTreeTop < kConsumers && 2 * kConsumerTreeTop >= kConsumers, "tree reduction shape");
-constexpr int kRowsPerWarp = 2;
 // kinds of k_iter pass: a BCD iteration; a BCD iteration that also tracks the
 // codes between iterates (changed-code counts); the final pass (codes of the
 // final iterate and the last MSE)
 enum : int { PASS_ITER = 0, PASS_COUNT = 1, PASS_FINAL = 2 };
-constexpr int kRowsPerTile = kConsumerWarps * kRowsPerWarp;
-constexpr int kRun = 8;
-constexpr int kRingBytes = 96 * 1024;
 // relative error bound of the fp64 column totals built from fp32 runs of kRun
 // rows (kRun roundings per run, fp64 beyond), plus the oracle's own fp64 error
 constexpr double kColErr = 2.0 * kRun * 0x1p-24 + 1e-11;
@@ -42,15 +52,15 @@ constexpr double kColErr = 2.0 * kRun * 0x1p-24 + 1e-11;
 // is within 7 * 2^-24 of W/(a b), the bracket factors add two more roundings.
 constexpr float kRelGuard = 0x1p-20f;
 
-__host__ __device__ constexpr int ring_stages(int es) { return kRingBytes / (kRowsPerTile * kStripMax * es); }
-// fp64 accumulators per consumer warp: 8 column pairs (sum W a q, sum (a q)^2) x 32 lanes + 32 residual sums
-__host__ __device__ constexpr size_t iter_acc_bytes() {
-  return (size_t)kConsumerWarps * (kStripMax * sizeof(double2) + 32 * sizeof(double));
-}
-__host__ __device__ constexpr size_t iter_smem_bytes(int es) {
-  return (size_t)kRingBytes + iter_acc_bytes() + 2 * sizeof(uint64_t) * ring_stages(es) +
-         (2 + kStripMax + 4) * sizeof(int) + 2 * 4 * 32 * sizeof(unsigned long long) + kMaxGrid * sizeof(int);
-}
+// CTA-ordered schedule of one pass, computed by every CTA from the same flags.
+struct Sched {
+  long long L;                // (strip, row) units of the pass
+  long long u_begin, u_end;   // this CTA's units
+  int nact;                   // active block-columns
+  int Pt;                     // CTAs that get units (a multiple of the strip count when that keeps 90%)
+  int v_first;                // first strip of this CTA's range
+  int ident;                  // the active list is 0 .. nb-1 (first and final pass)
+};
 
 // ---------------------------------------------------------------------------
 // Packed f32x2 arithmetic (one instruction for a pair of elements).
@@ -162,23 +172,24 @@ __device__ __forceinline__ float a_dec(uint32_t v) {
   return __half2float(__ushort_as_half((unsigned short)(h & 0xFFFFu)));
 }
 
-// Column table of the current strip in shared memory: colt[c][lane] holds
-// (b, cb) of column 8 lane + c as a float2 pair per column pair: entry
-// [(2 i) / 2][lane] = {b of pair i} and {cb of pair i}.  Loads are volatile so
-// the compiler re-reads the table at each use instead of holding 16 registers.
-__device__ __forceinline__ f2 col_ld(const f2* tab, int i, int lane) {
+// Column table of a warp's block-column in shared memory: for each octet o
+// of the block, 4 column pairs of (b) and 4 of (cb); lane (rho, o) points at
+// its octet's entries and lanes of one octet read the same word (broadcast).
+// Loads are volatile so the compiler re-reads the table at each use instead of
+// holding 16 registers.
+__device__ __forceinline__ f2 col_ld(const f2* tab, int i) {
   f2 v;
-  asm volatile("ld.shared.b64 %0, [%1];" : "=l"(v) : "r"(smem_u32(tab + i * 32 + lane)));
+  asm volatile("ld.shared.b64 %0, [%1];" : "=l"(v) : "r"(smem_u32(tab + i)));
   return v;
 }
 
-// Per-lane state of a column strip segment, as 4 column pairs: b, the
+// Per-lane state of a block-column segment, as 4 column pairs: b, the
 // candidate factor cb = 1/b (times 1/s_T for NVFP4), fp32 column runs, and the
 // guard threshold per column (MXINT4/MXINT8 columns with a power-of-two b have an exact
 // candidate and need no guard).
 struct ColState {
-  const f2* tb;   // shared table of b pairs [4][32]
-  const f2* tcb;  // shared table of cb pairs [4][32]
+  const f2* tb;   // this lane's 4 b pairs in the warp's table
+  const f2* tcb;  // this lane's 4 cb pairs
   int lane;
   f2 cn2[4], cd2[4];
   float thr[8];
@@ -361,7 +372,7 @@ __device__ __forceinline__ void req_slow(const f2 w2[4], const f2 u2[4], float a
     w[2 * i + 1] = hi_of(w2[i]);
     u[2 * i] = lo_of(u2[i]);
     u[2 * i + 1] = hi_of(u2[i]);
-    const f2 bi = col_ld(cs.tb, i, cs.lane);
+    const f2 bi = col_ld(cs.tb, i);
     b[2 * i] = lo_of(bi);
     b[2 * i + 1] = hi_of(bi);
   }
@@ -471,7 +482,7 @@ __device__ __forceinline__ void row_sums2(const f2 wx[4], const f2 qx[4], float 
   f2 nx2 = 0ull, dx2 = 0ull, ny2 = 0ull, dy2 = 0ull;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const f2 bi = col_ld(cs.tb, i, cs.lane);
+    const f2 bi = col_ld(cs.tb, i);
     const f2 px = mul2(qx[i], bi), py = mul2(qy[i], bi);
     nx2 = fma2(wx[i], px, nx2);
     dx2 = fma2(px, px, dx2);
@@ -502,7 +513,7 @@ __device__ __forceinline__ void row_sums64(const f2 w2[4], const f2 q2[4], const
   d64 = 0.0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const f2 pq = mul2(q2[i], col_ld(cs.tb, i, cs.lane));  // exact products
+    const f2 pq = mul2(q2[i], col_ld(cs.tb, i));  // exact products
     n64 = fma((double)lo_of(w2[i]), (double)lo_of(pq), n64);
     d64 = fma((double)lo_of(pq), (double)lo_of(pq), d64);
     n64 = fma((double)hi_of(w2[i]), (double)hi_of(pq), n64);
@@ -591,11 +602,12 @@ __device__ __forceinline__ void store_codes(void* codes, int64_t cix, uint2 c) {
 }
 
 // Code tracking for two rows of a lane: the codes replace the groups at cix
-// (row x) and cix + kConsumerWarps rows (row y); with `cmp` the codes that
-// differ from the previous groups oldx, oldy are counted into nchg.
+// (row x) and cix + code_step (row y); with `cmp` the codes that differ from
+// the previous groups oldx, oldy are counted into nchg.
 template <int FMT>
 __device__ __forceinline__ void track_codes(const Problem& p, const f2 qx[4], const f2 qy[4], bool actx, bool acty,
-                                            int64_t cix, uint2 oldx, uint2 oldy, bool cmp, unsigned& nchg) {
+                                            int64_t cix, int64_t code_step, uint2 oldx, uint2 oldy, bool cmp,
+                                            unsigned& nchg) {
   if (actx) {
     const uint2 c = pack8<FMT>(qx);
     if (cmp) nchg += changed_codes<FMT>(make_uint2(c.x ^ oldx.x, c.y ^ oldx.y));
@@ -604,31 +616,32 @@ __device__ __forceinline__ void track_codes(const Problem& p, const f2 qx[4], co
   if (acty) {
     const uint2 c = pack8<FMT>(qy);
     if (cmp) nchg += changed_codes<FMT>(make_uint2(c.x ^ oldy.x, c.y ^ oldy.y));
-    store_codes<FMT>(p.codes, cix + (int64_t)kConsumerWarps * (p.N >> 3), c);
+    store_codes<FMT>(p.codes, cix + code_step, c);
   }
 }
 
-// Two rows of one lane (x = row a, y = row b; y may be absent, then its data
-// are zero and nothing of it is written): requantize the incoming iterate;
-// block sums, residuals and block updates; requantize with the new block
-// scales where they changed; column sums.  Warp-collective (shuffles and
-// votes); `active` lanes hold real columns and alone write results.
+// Two rows of one lane (x = row a, y = row b; a row outside the segment holds
+// zeros and nothing of it is written): requantize the incoming iterate; block
+// sums, residuals and block updates; requantize with the new block scales
+// where they changed; column sums.  Warp-collective (shuffles and votes);
+// actx / acty say which of the lane's rows are real.  achg is raised when a
+// block scale of the lane's rows changed.
 template <int FMT, int PASS>
 __device__ __forceinline__ void row_pair(const Problem& p, const f2 wx[4], float ax_old, int64_t bidx_x,
-                                         const f2 wy[4], float ay_old, int64_t bidx_y, bool has_y, bool active,
+                                         const f2 wy[4], float ay_old, int64_t bidx_y, bool actx, bool acty,
                                          bool leader, int lpb, ColState& cs, float sT, float isT, double sTd,
                                          bool scaled, f2 rscale2, unsigned* s_cnt, unsigned& tcnt, int64_t cix,
-                                         uint2 oldx, uint2 oldy, bool cmp, unsigned& nchg) {
-  const bool actx = active, acty = active && has_y;
+                                         int64_t code_step, uint2 oldx, uint2 oldy, bool cmp, unsigned& nchg,
+                                         bool& achg) {
   f2 ux[4], uy[4], qx[4], qy[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const f2 cbi = col_ld(cs.tcb, i, cs.lane);
+    const f2 cbi = col_ld(cs.tcb, i);
     ux[i] = mul2(wx[i], cbi);
     uy[i] = mul2(wy[i], cbi);
   }
   req_pair<FMT>(wx, ux, ax_old, actx, wy, uy, ay_old, acty, cs, sT, sTd, qx, qy, s_cnt, tcnt);
-  if (PASS == PASS_COUNT) track_codes<FMT>(p, qx, qy, actx, acty, cix, oldx, oldy, cmp, nchg);
+  if (PASS == PASS_COUNT) track_codes<FMT>(p, qx, qy, actx, acty, cix, code_step, oldx, oldy, cmp, nchg);
   float nx, dx, ny, dy;
   row_sums2<FMT>(wx, qx, ax_old, wy, qy, ay_old, cs, sT, scaled, rscale2, nx, dx, ny, dy, cs.res2);
   float anx, any;
@@ -686,13 +699,14 @@ __device__ __forceinline__ void row_pair(const Problem& p, const f2 wx[4], float
   // the storage already holds the old factors; with a block scale unchanged the
   // codes are unchanged too (same a, same b), so requantize only where it changed
   const bool chx = anx != ax_old && actx, chy = any != ay_old && acty;
+  achg = achg || chx || chy;
   if (chx && leader) a_store_f<FMT>(p.a_store, bidx_x, anx);
   if (chy && leader) a_store_f<FMT>(p.a_store, bidx_y, any);
   if (__any_sync(0xffffffffu, chx || chy)) {
     // recomputed rather than kept live across the block update (registers)
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const f2 cbi = col_ld(cs.tcb, i, cs.lane);
+      const f2 cbi = col_ld(cs.tcb, i);
       ux[i] = mul2(wx[i], cbi);
       uy[i] = mul2(wy[i], cbi);
     }
@@ -710,26 +724,25 @@ __device__ __forceinline__ void row_pair(const Problem& p, const f2 wx[4], float
   }
 }
 
-// Final pass for two rows of a lane (x = row rx, y = row rx + kConsumerWarps,
-// possibly absent): codes of the final iterate, written packed, and the
-// residuals of that iterate for its MSE.
+// Final pass for two rows of a lane (x, y; a row outside the segment holds
+// zeros and is not written): codes of the final iterate, written packed, and
+// the residuals of that iterate for its MSE.
 template <int FMT>
 __device__ __forceinline__ void final_pair(const Problem& p, const f2 wx[4], float ax, const f2 wy[4], float ay,
-                                           bool has_y, bool active, ColState& cs, float sT, double sTd, bool scaled,
-                                           f2 rscale2, unsigned* s_cnt, unsigned& tcnt, int64_t cix, uint2 oldx,
-                                           uint2 oldy, bool cmp, unsigned& nchg) {
-  const bool actx = active, acty = active && has_y;
+                                           bool actx, bool acty, ColState& cs, float sT, double sTd, bool scaled,
+                                           f2 rscale2, unsigned* s_cnt, unsigned& tcnt, int64_t cix,
+                                           int64_t code_step, uint2 oldx, uint2 oldy, bool cmp, unsigned& nchg) {
   f2 ux[4], uy[4], qx[4], qy[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const f2 cbi = col_ld(cs.tcb, i, cs.lane);
+    const f2 cbi = col_ld(cs.tcb, i);
     ux[i] = mul2(wx[i], cbi);
     uy[i] = mul2(wy[i], cbi);
   }
   req_pair<FMT>(wx, ux, ax, actx, wy, uy, ay, acty, cs, sT, sTd, qx, qy, s_cnt, tcnt);
   float nx, dx, ny, dy;  // block sums: not needed here
   row_sums2<FMT>(wx, qx, ax, wy, qy, ay, cs, sT, scaled, rscale2, nx, dx, ny, dy, cs.res2);
-  track_codes<FMT>(p, qx, qy, actx, acty, cix, oldx, oldy, cmp, nchg);
+  track_codes<FMT>(p, qx, qy, actx, acty, cix, code_step, oldx, oldy, cmp, nchg);
 }
 
 // fp32 runs into the warp's fp64 accumulators (layout [warp][c][lane], then
@@ -759,37 +772,14 @@ __device__ __forceinline__ void flush_runs(ColState& cs, double2* acc, double* r
 // grid size.  The wait is bounded: it gives up after kWaitLimitNs of wall
 // time (or at once when some wait already gave up), records kFlagTimeout and
 // goes on.
-constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s
-
-__device__ __forceinline__ unsigned long long global_ns() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-// True when a bounded wait begun at t0 must give up (its time is over, or some
-// other wait already gave up); then kFlagTimeout is recorded.
-__device__ __forceinline__ bool wait_expired(unsigned* flags, unsigned long long t0) {
-  if (global_ns() - t0 > kWaitLimitNs || (*reinterpret_cast<volatile unsigned*>(flags) & kFlagTimeout)) {
-    atomicOr(flags, kFlagTimeout);
-    return true;
-  }
-  return false;
-}
-
-__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* a) {
-  unsigned v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
-  return v;
-}
-
-// MSE of a finished pass from its per-CTA residual totals `part` (P values):
-// a fixed-order tree over the CTA index, so the value does not depend on which
-// CTA sums it.  Run by the consumer threads of one CTA; `red` holds kConsumers
-// doubles.
-__device__ void mse_total(const Problem& p, const double* part, double* out, double rscale_d, double* red) {
+// MSE of a finished pass from its n partial residual totals `part` (one per
+// CTA, or one per block-column): a fixed-order tree over the index, so the
+// value does not depend on which CTA sums it.  Run by the consumer threads of
+// one CTA; `red` holds kConsumers doubles.
+__device__ void mse_total(const Problem& p, const double* part, int64_t n, double* out, double rscale_d,
+                          double* red) {
   double v = 0.0;
-  for (int64_t kk = threadIdx.x; kk < p.P; kk += kConsumers) v += __ldcg(part + kk);
+  for (int64_t kk = threadIdx.x; kk < n; kk += kConsumers) v += __ldcg(part + kk);
   red[threadIdx.x] = v;
   consumer_sync(kConsumers);
   for (int o = kConsumerTreeTop; o > 0; o >>= 1) {
@@ -800,13 +790,18 @@ __device__ void mse_total(const Problem& p, const double* part, double* out, dou
   consumer_sync(kConsumers);
 }
 
-// Per-CTA residual totals of pass t live in cta_part[(t % 3) P + k]: three
-// buffers, so the totals of pass t - 1 stay intact while pass t + 1 runs.
+// Per-CTA residual totals of the final pass t live in cta_part[(t % 3) P + k].
 __device__ __forceinline__ double* mse_part(const Problem& p, int t) { return p.cta_part + (int64_t)(t % 3) * p.P; }
 
+// Residual total of each block-column for the incoming iterate of BCD pass t:
+// mse_bc[(t % 3) nb + g].  Three buffers, so the totals of pass t - 1 stay
+// intact while pass t + 1 runs (the MSE of pass t - 1 is summed during pass t).
+__device__ __forceinline__ double* mse_bcs(const Problem& p, int t) { return p.mse_bc + (int64_t)(t % 3) * p.nb; }
+
 // Grid barrier at the end of pass t.  The first CTA to arrive has the most
-// time to spare: it sums the MSE of pass t - 1 (all of whose totals were
-// written before the barrier that ended it) while the others finish.
+// time to spare: it sums the MSE of pass t - 1 (all of whose block-column
+// totals were written before the barrier that ended it) while the others
+// finish.
 __device__ void grid_sync(const Problem& p, int t, double rscale_d, double* red, int* s_flag) {
   WsHeader* hdr = p.hdr;
   consumer_sync(kConsumers);
@@ -818,7 +813,7 @@ __device__ void grid_sync(const Problem& p, int t, double rscale_d, double* red,
     *s_flag = (ticket % gridDim.x == 0u && t >= 2) ? 1 : 0;
   }
   consumer_sync(kConsumers);
-  if (*s_flag) mse_total(p, mse_part(p, t - 1), p.mse + (t - 2), rscale_d, red);
+  if (*s_flag) mse_total(p, mse_bcs(p, t - 1), p.nb, p.mse + (t - 2), rscale_d, red);
   if (threadIdx.x == 0) {
     const unsigned long long t0 = global_ns();
     for (;;) {
@@ -859,11 +854,11 @@ __device__ void grid_sync_plain(WsHeader* hdr) {
 // one short round of loads per CTA.  A chunk's total is a fixed-order
 // reduction over the consumer threads; the last chunk of a column to arrive
 // adds the R chunk totals in chunk order (the result does not depend on the
-// schedule), writes the scale and counts the strip's p.sx_left down.  A CTA
-// reaching a strip with listed columns waits for that count to reach zero
-// (wait_strip); nobody else waits.  When the list is too long for p.xpart the
-// chunk totals go to p.col_part instead and a grid barrier follows (then no
-// strip waits).  Run by the consumer threads; `scratch` holds 2 * kConsumers
+// schedule), writes the scale and counts its block-column's p.pend down.  A
+// warp reaching a block-column with listed columns waits for that count to
+// reach zero (wait_bc); nobody else waits.  When the list is too long for
+// p.xpart the chunk totals go to p.col_part instead and a grid barrier follows
+// (then nobody waits).  Run by the consumer threads; `scratch` holds 2 * kConsumers
 // doubles.
 constexpr int kXRows = 8;
 constexpr int64_t kXMinRows = 32;  // rows of the smallest chunk
@@ -956,7 +951,7 @@ __device__ void column_settle(const Problem& p, int64_t j, const double2* part, 
   }
 }
 
-// Returns true when strips with listed columns must be waited for (wait_strip).
+// Returns true when block-columns with listed columns must be waited for (wait_bc).
 template <int FMT, int WDT>
 __device__ bool exact_listed(const Problem& p, int t, double sTd, float isT, double* scratch, int* s_flag) {
   const int lb = (t - 1) % 3;
@@ -967,7 +962,7 @@ __device__ bool exact_listed(const Problem& p, int t, double sTd, float isT, dou
   const int* list = p.amb_list + (int64_t)lb * p.N;
   const bool own = (int64_t)n <= kXPartCap;  // chunk totals in p.xpart, no barrier
   double2* part = own ? p.xpart : p.col_part;
-  const int64_t cap = own ? kXPartCap : (int64_t)p.P * p.segmax * p.TS;
+  const int64_t cap = own ? kXPartCap : (int64_t)p.P * p.segmax * p.TSv;
   const int64_t R = max((int64_t)1, min(min((p.M + kXMinRows - 1) / kXMinRows, max((int64_t)1, (int64_t)p.P / (int64_t)n)),
                                         cap / (int64_t)n));
   const int64_t chunk = (p.M + R - 1) / R;
@@ -989,9 +984,9 @@ __device__ bool exact_listed(const Problem& p, int t, double sTd, float isT, dou
         p.amb_tick[ci] = 0u;
         __threadfence();  // the scale is visible before the count drops
         if (own) {
-          atomicSub(&p.sx_left[j / p.TS], 1u);
+          atomicSub(&p.pend[j / p.G], 1u);
         } else {
-          p.sx_left[j / p.TS] = 0u;  // the barrier below orders it
+          p.pend[j / p.G] = 0u;  // the barrier below orders it
         }
       }
     }
@@ -1001,48 +996,138 @@ __device__ bool exact_listed(const Problem& p, int t, double sTd, float isT, dou
   return own;
 }
 
-// Before pass t uses the column scales of strip s: wait until the listed
-// columns of the strip are settled (bounded; gives up with kFlagTimeout).
-__device__ void wait_strip(const Problem& p, int64_t s) {
-  if (threadIdx.x == 0) {
+// Before a warp uses the column scales of block-column g: wait until its
+// listed columns are settled (lane 0 polls, bounded; gives up with
+// kFlagTimeout).  Warp-collective: the warp's later loads of the scales are
+// ordered after lane 0's acquiring load by the warp barrier.
+__device__ void wait_bc(const Problem& p, int64_t g) {
+  if ((threadIdx.x & 31) == 0) {
     const unsigned long long t0 = global_ns();
     for (;;) {
-      if (ld_acquire_gpu(&p.sx_left[s]) == 0u) break;
+      if (ld_acquire_gpu(&p.pend[g]) == 0u) break;
       if (wait_expired(&p.hdr->flags, t0)) break;
       __nanosleep(64);
     }
   }
+  __syncwarp();
 }
 
-// Passes t = t_first .. t_last over W, one read of W each, in one persistent
-// launch (cooperative: a grid barrier separates consecutive passes, so pass
-// t + 1 reads the scales that pass t wrote; the producer warp streams W on
-// across the barriers).  PASS_ITER: BCD iteration t (writes mse[t - 1], the
-// MSE of the incoming iterate).  PASS_COUNT: the same, and the incoming
-// iterate's codes replace those of the iterate before it in p.codes, the
-// changed ones counted into changes[t - 1] (t >= 2).  PASS_FINAL: the final
-// pass after T iterations, called with t_first = t_last = T + 1: the codes of
-// the final iterate, packed, and mse[T] (and changes[T] when counting, T >= 1).
-// Every pass starts with the exact update of the columns that the pass before
-// left ambiguous (exact_listed).
+
+// Named barrier of the whole CTA (consumers and producer): the schedule of a
+// pass is handed to the producer through it.
+__device__ __forceinline__ void cta_sync_all() { asm volatile("bar.sync 2, %0;" ::"r"(kIterThreads) : "memory"); }
+
+// Schedule of pass t, computed by the consumer threads of every CTA from the
+// same flags (so every CTA finds the same strips and ranges): the active
+// block-columns, this CTA's units, the first strip of every CTA's range (the
+// strip finalizers index partial sums by it) and this CTA's slice of the
+// active list.  With `ident` (the first BCD pass and the final pass) every
+// block-column is active.  Otherwise the active ones are those whose scales
+// changed in pass t - 1 (p.chg of pass t - 1, complete after the grid barrier
+// that ended it): a block-column with no change is at a fixed point, and its
+// residual total is carried into this pass's buffer.  `s_scan` holds 17 ints.
+__device__ void pass_schedule(const Problem& p, int t, bool ident, Sched* sc, int* s_act, int* s_scan, int* s_sfirst) {
+  const int nb = p.nb;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const unsigned* flags = p.chg + (int64_t)((t - 1) % 3) * nb;
+  const int per = (nb + kConsumers - 1) / kConsumers;
+  const int c0 = min(nb, tid * per), c1 = min(nb, c0 + per);
+  int nact = nb, excl = 0;
+  if (!ident) {
+    int cnt = 0;
+    for (int g = c0; g < c1; ++g) cnt += __ldcg(flags + g) != 0u;
+    int incl = cnt;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) s_scan[warp] = incl;
+    consumer_sync(kConsumers);
+    if (warp == 0) {
+      const int x = lane < kConsumerWarps ? s_scan[lane] : 0;
+      int xi = x;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, xi, o);
+        if (lane >= o) xi += y;
+      }
+      if (lane < kConsumerWarps) s_scan[lane] = xi - x;
+      if (lane == 31) s_scan[16] = xi;
+    }
+    consumer_sync(kConsumers);
+    excl = s_scan[warp] + incl - cnt;
+    nact = s_scan[16];
+  }
+  const long long nv = ((long long)nact + kBcPerStrip - 1) / kBcPerStrip;
+  const long long L = nv * p.M;
+  const int Pt = pass_ctas(p.P, nv, L);
+  const int k = blockIdx.x;
+  const long long ub = k < Pt ? range_begin(k, Pt, L) : L;
+  const long long ue = k < Pt ? range_begin(k + 1, Pt, L) : L;
+  const int v_first = (int)(ub / p.M);
+  if (!ident) {
+    const long long lo = (long long)v_first * kBcPerStrip;
+    const long long hi = lo + (long long)p.segmax * kBcPerStrip;
+    double* cur = mse_bcs(p, t);
+    const double* prev = mse_bcs(p, t - 1);
+    int idx = excl;
+    for (int g = c0; g < c1; ++g) {
+      if (__ldcg(flags + g) != 0u) {
+        if (idx >= lo && idx < hi) s_act[idx - lo] = g;
+        ++idx;
+      } else if (g % (int)gridDim.x == k) {
+        cur[g] = __ldcg(prev + g);  // at a fixed point: the same residual total
+      }
+    }
+  }
+  for (int kk = tid; kk < Pt; kk += kConsumers) s_sfirst[kk] = (int)(range_begin(kk, Pt, L) / p.M);
+  if (tid == 0) {
+    sc->L = L;
+    sc->u_begin = ub;
+    sc->u_end = ue;
+    sc->nact = nact;
+    sc->Pt = Pt;
+    sc->v_first = v_first;
+    sc->ident = ident ? 1 : 0;
+  }
+  consumer_sync(kConsumers);
+}
+
+// Passes t = t_first .. t_last, in one persistent launch (cooperative: a grid
+// barrier separates consecutive passes, so pass t + 1 reads the scales that
+// pass t wrote).  PASS_ITER: BCD iteration t over the active block-columns
+// (writes mse[t - 1], the MSE of the incoming iterate).  PASS_COUNT: the same,
+// and the incoming iterate's codes replace those of the iterate before it in
+// p.codes, the changed ones counted into changes[t - 1] (t >= 2; a
+// block-column at a fixed point keeps its codes and adds nothing).
+// PASS_FINAL: the final pass after T iterations over every block-column,
+// called with t_first = t_last = T + 1: the codes of the final iterate, packed,
+// and mse[T] (and changes[T] when counting, T >= 1).  Every pass starts with
+// the exact update of the columns that the pass before left ambiguous
+// (exact_listed).
 template <int FMT, int WDT, int PASS>
 __global__ void __launch_bounds__(kIterThreads, 1)
     k_iter(Problem p, int t_first, int t_last, const __grid_constant__ CUtensorMap wmap) {
   constexpr int ES = WDT == DT_F32 ? 4 : 2;
-  constexpr int S = ring_stages(ES);
+  constexpr bool FIN = PASS == PASS_FINAL;
+  const TileGeo geo = tile_geo(p.G, ES);
+  const IterSmem lay = iter_smem(geo.lpb, p.P, p.segmax);
+  const int S = geo.S;
   extern __shared__ __align__(128) unsigned char smem[];
   unsigned char* ring = smem;
-  double2* acc = reinterpret_cast<double2*>(smem + kRingBytes);
-  double* racc = reinterpret_cast<double*>(acc + kConsumerWarps * kStripMax);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kRingBytes + iter_acc_bytes());
-  uint64_t* empty = full + S;
-  int* s_misc = reinterpret_cast<int*>(empty + S);  // [0] ticket result, [1] #ambiguous, [2..] columns
-  unsigned* s_cnt = reinterpret_cast<unsigned*>(s_misc + 2 + kStripMax);  // exact-path counters
-  f2* ctab = reinterpret_cast<f2*>(s_cnt + 4);  // column table of the strip: b pairs, then cb pairs
-  int* s_sfirst = reinterpret_cast<int*>(ctab + 2 * 4 * 32);  // [P] first strip of each CTA's range
+  double2* acc = reinterpret_cast<double2*>(smem + lay.acc);
+  double* racc = reinterpret_cast<double*>(smem + lay.racc);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + lay.bars);
+  uint64_t* empty = full + kMaxStages;
+  int* s_misc = reinterpret_cast<int*>(smem + lay.misc);  // [0] ticket result, [1] #ambiguous
+  unsigned* s_cnt = reinterpret_cast<unsigned*>(s_misc + 2);  // [4] exact-path counters
+  int* s_chgs = s_misc + 8;    // [15] strip slot whose column scales changed or were listed
+  int* s_pend = s_misc + 24;   // [15] listed columns per strip slot
+  int* s_scan = s_misc + 40;   // [17] schedule scan
+  Sched* s_sched = reinterpret_cast<Sched*>(smem + lay.sched);
+  f2* ctab = reinterpret_cast<f2*>(smem + lay.ctab);
+  int* s_sfirst = reinterpret_cast<int*>(smem + lay.sfirst);
+  int* s_act = reinterpret_cast<int*>(smem + lay.act);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row_bytes = p.TS * ES;  // ring slot per row
-  const int stage_bytes = kRowsPerTile * row_bytes;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
@@ -1059,64 +1144,78 @@ __global__ void __launch_bounds__(kIterThreads, 1)
   griddep_wait();
   griddep_launch_dependents();
   if (p.hdr->flags & kFlagAbort) return;
-  // first strip of every CTA's range (the strip finalizers index partials by it)
-  for (int kk = threadIdx.x; kk < p.P; kk += kIterThreads) s_sfirst[kk] = (int)(range_begin(kk, p.P, p.L) / p.M);
-  __syncthreads();
-
-  const int64_t k = blockIdx.x;
-  const int64_t u_begin = range_begin(k, p.P, p.L), u_end = range_begin(k + 1, p.P, p.L);
 
   if (warp == kConsumerWarps) {
     // ---------------- producer warp ----------------
-    int st = 0;
+    // Tile n of the CTA goes to stage n % S (use n / S of that stage).  The
+    // producer stops issuing once some wait of the solve has given up, and
+    // before it returns it waits (bounded) for the copy of the last use of
+    // every stage, so no copy into this CTA's shared memory is in flight when
+    // the CTA exits.
+    int st = 0, issued = 0;
     unsigned par = 1u;
-    for (int t = t_first; t <= t_last; ++t)  // the same tiles, pass after pass
-    for (int64_t u = u_begin; u < u_end;) {
-      const int64_t s = u / p.M;
-      const int64_t r0 = u - s * p.M;
-      const int64_t r1 = min(p.M, r0 + (u_end - u));
-      const int64_t c0 = s * p.TS;
-      const int width = (int)min((int64_t)p.TS, p.N - c0);
-      const unsigned bytes = (unsigned)(width * ES);
-      const unsigned char* src = reinterpret_cast<const unsigned char*>(p.W) + ((r0 + lane) * p.N + c0) * (int64_t)ES;
-      const int64_t src_step = (int64_t)kRowsPerTile * p.N * ES;
-      if (p.use_tmap) {
-        // one tensor copy per tile: kRowsPerTile rows x TS columns (zero-filled
-        // beyond the matrix), into the same row-major slot layout
-        for (int64_t tr = r0; tr < r1; tr += kRowsPerTile) {
-          mbar_wait(&empty[st], par, &p.hdr->flags);
-          if (lane == 0) {
-            mbar_arrive_expect_tx(&full[st], (unsigned)stage_bytes);
-            tma_load_2d(ring + st * stage_bytes, &wmap, (int)c0, (int)tr, &full[st]);
+    bool stop = false;
+    for (int t = t_first; t <= t_last; ++t) {
+      cta_sync_all();  // the schedule of pass t is in shared memory
+      const long long ub = s_sched->u_begin, ue = s_sched->u_end;
+      const int nact = s_sched->nact, ident = s_sched->ident, v_first = s_sched->v_first;
+      for (long long u = ub; u < ue && !stop;) {
+        const long long v = u / p.M;
+        const long long r0 = u - v * p.M;
+        const long long r1 = min((long long)p.M, r0 + (ue - u));
+        const int i0 = (int)(v * kBcPerStrip);
+        const int nbc = min(kBcPerStrip, nact - i0);
+        const int* act = s_act - (long long)v_first * kBcPerStrip;
+        const int gl = lane < nbc ? (ident ? i0 + lane : act[i0 + lane]) : 0;
+        for (long long tr = r0; tr < r1; tr += geo.RW) {
+          if (ld_volatile(&p.hdr->flags) & kFlagTimeout) {
+            stop = true;
+            break;
           }
-          __syncwarp();
+          if (!mbar_wait(&empty[st], par, &p.hdr->flags)) {
+            stop = true;
+            break;
+          }
+          unsigned char* slot = ring + st * geo.stage_bytes;
+          if (p.use_tmap) {
+            if (lane == 0) mbar_arrive_expect_tx(&full[st], (unsigned)(nbc * geo.box_bytes));
+            __syncwarp();
+            if (lane < nbc) tma_load_2d(slot + lane * geo.box_stride, &wmap, gl * p.G, (int)tr, &full[st]);
+          } else {
+            // one bulk copy per (block-column, row) of the tile inside the segment
+            const int nr = (int)min((long long)geo.RW, r1 - tr);
+            const unsigned row_bytes = (unsigned)(p.G * ES);
+            if (lane == 0) mbar_arrive_expect_tx(&full[st], (unsigned)(nbc * nr) * row_bytes);
+            __syncwarp();
+            for (int it = lane; it < nbc * nr; it += 32) {
+              const int w = it / nr, rr = it - w * nr;
+              const long long gw = ident ? i0 + w : act[i0 + w];
+              const unsigned char* src =
+                  reinterpret_cast<const unsigned char*>(p.W) + ((tr + rr) * p.N + gw * p.G) * (long long)ES;
+              bulk_g2s(slot + w * geo.box_stride + rr * (int)row_bytes, src, row_bytes, &full[st]);
+            }
+          }
+          ++issued;
           if (++st == S) {
             st = 0;
             par ^= 1u;
           }
         }
-        u = (s + 1) * p.M;
-        continue;
+        u = (v + 1) * p.M;
       }
-      for (int64_t tr = r0; tr < r1; tr += kRowsPerTile, src += src_step) {
-        mbar_wait(&empty[st], par, &p.hdr->flags);
-        const int nr = (int)min((int64_t)kRowsPerTile, r1 - tr);
-        if (lane == 0) mbar_arrive_expect_tx(&full[st], (unsigned)nr * bytes);
-        __syncwarp();
-        if (lane < nr) bulk_g2s(ring + st * stage_bytes + lane * row_bytes, src, bytes, &full[st]);
-        if (++st == S) {
-          st = 0;
-          par ^= 1u;
-        }
-      }
-      u = (s + 1) * p.M;
     }
+    if (lane == 0) {
+      for (int s = 0; s < S && s < issued; ++s) mbar_drain(&full[s], (unsigned)(((issued - 1 - s) / S) & 1));
+    }
+    __syncwarp();
     return;
   }
 
   // ---------------- consumer warps ----------------
-  const int lpb = p.G / 8;  // lanes per block
-  const bool leader = (lane & (lpb - 1)) == 0;
+  const int lpb = geo.lpb, rl = geo.rl, RW = geo.RW;
+  const int lg = __ffs(lpb) - 1;  // lpb is a power of two
+  const int rho = lane >> lg, oct = lane & (lpb - 1);
+  const bool leader = oct == 0;
   // residuals are squared as they are when max |W| lies in [2^-8, 2^41) (no
   // square of a residual can overflow, and none that underflows matters at the
   // MSE's tolerance), otherwise after scaling by rscale = 2^-floor(log2 amax),
@@ -1132,41 +1231,52 @@ __global__ void __launch_bounds__(kIterThreads, 1)
   const float isT = FMT == FMT_NVFP4 ? __frcp_rn(sT) : 1.f;
   const bool sT_ok = FMT != FMT_NVFP4 || in_range(isT);
   const int sT_bits = sig_bits(sT);
-  const int64_t s_first = u_begin / p.M;
   int st = 0;
   unsigned par = 0u;
-  constexpr bool FIN = PASS == PASS_FINAL;
-  const int64_t code_step = (int64_t)kConsumerWarps * (p.N >> 3);  // code groups between a warp's two rows
+  const int64_t code_step = (int64_t)rl * (p.N >> 3);  // code groups between a lane's two rows
   unsigned tcnt = 0u;  // lane-rows settled as certified exact ties
+  const f2* wtab = ctab + warp * 8 * lpb;  // this warp's column table
 
   for (int t = t_first; t <= t_last; ++t) {
   const bool strip_wait = exact_listed<FMT, WDT>(p, t, sTd, isT, reinterpret_cast<double*>(acc), &s_misc[0]);
   if (FIN && blockIdx.x == 0) {
     // the MSE of the passes that no grid barrier of the iteration launch summed
     for (int tp = max(1, t - 2); tp <= t - 1; ++tp)
-      mse_total(p, mse_part(p, tp), p.mse + (tp - 1), rscale_d, reinterpret_cast<double*>(acc));
+      mse_total(p, mse_bcs(p, tp), p.nb, p.mse + (tp - 1), rscale_d, reinterpret_cast<double*>(acc));
   }
-  racc[threadIdx.x] = 0.0;
+  if (!FIN && blockIdx.x == 0) {
+    // the change flags of pass t + 1 were last read when pass t - 1 began
+    unsigned* nxt = p.chg + (int64_t)((t + 1) % 3) * p.nb;
+    for (int g = threadIdx.x; g < p.nb; g += kConsumers) nxt[g] = 0u;
+  }
+  pass_schedule(p, t, FIN || t == t_first || p.full_passes, s_sched, s_act, s_scan, s_sfirst);
+  const long long ub = s_sched->u_begin, ue = s_sched->u_end, L = s_sched->L;
+  const int nact = s_sched->nact, Pt = s_sched->Pt, v_first = s_sched->v_first;
+  const bool ident = s_sched->ident != 0;
+  if (!FIN && blockIdx.x == 0 && threadIdx.x == 0) atomicAdd(&p.hdr->n_active_bc, (unsigned long long)nact);
+  cta_sync_all();  // hand the schedule to the producer
+  const int* act = s_act - (long long)v_first * kBcPerStrip;
+  if (FIN) racc[threadIdx.x] = 0.0;
   // compare with the previous iterate's codes (kept in p.codes by the pass before)
   const bool cmp = (PASS == PASS_COUNT || (FIN && p.changes != nullptr)) && t > 1;
   unsigned nchg = 0u;
 
-  for (int64_t u = u_begin; u < u_end;) {
-    const int64_t s = u / p.M;
-    const int64_t r0 = u - s * p.M;
-    const int64_t r1 = min(p.M, r0 + (u_end - u));
-    const int64_t c0 = s * p.TS;
-    const int width = (int)min((int64_t)p.TS, p.N - c0);
-    const bool active = lane * 8 < width;
-    const int64_t col = c0 + lane * 8;
-    const int64_t blk_col = col / p.G;
+  for (long long u = ub; u < ue;) {
+    const long long v = u / p.M;
+    const long long r0 = u - v * p.M;
+    const long long r1 = min((long long)p.M, r0 + (ue - u));
+    const int i0 = (int)(v * kBcPerStrip);
+    const int nbc = min(kBcPerStrip, nact - i0);
+    const bool has = warp < nbc;  // warp-uniform: this warp owns a block-column of the strip
+    const int g = has ? (ident ? i0 + warp : act[i0 + warp]) : 0;
+    const int64_t col = (int64_t)g * p.G + 8 * oct;
 
+    consumer_sync(kConsumers);  // the previous segment's readers of acc and the tables are done
+    if (strip_wait && has) wait_bc(p, g);  // listed columns of this block-column settled first
     ColState cs;
-    cs.tb = ctab;
-    cs.tcb = ctab + 128;
+    cs.tb = wtab + oct * 4;
+    cs.tcb = wtab + 4 * lpb + oct * 4;
     cs.lane = lane;
-    if (strip_wait) wait_strip(p, s);  // listed columns of this strip settled first
-    consumer_sync(kConsumers);  // the previous segment's readers of the table are done
     cs.ok = sT_ok;
     cs.res2 = 0ull;
     int b_bits = 1;  // longest odd significand among the lane's column scales
@@ -1177,7 +1287,7 @@ __global__ void __launch_bounds__(kIterThreads, 1)
       for (int h = 0; h < 2; ++h) {
         const int c = 2 * i + h;
         cs.thr[c] = 0.5f - kGuard;
-        if (active) {
+        if (has) {
           bj[h] = b_decode_cg(p.b_store, p.col_dt, col + c);
           cb[h] = __frcp_rn(bj[h]) * isT;
           cs.ok = cs.ok && in_range(cb[h]);
@@ -1188,153 +1298,188 @@ __global__ void __launch_bounds__(kIterThreads, 1)
         }
         acc[(warp * 8 + c) * 32 + lane] = make_double2(0.0, 0.0);
       }
-      if (warp == 0) {
-        ctab[i * 32 + lane] = pk(bj[0], bj[1]);
-        ctab[128 + i * 32 + lane] = pk(cb[0], cb[1]);
+      if (rho == 0) {
+        ctab[warp * 8 * lpb + oct * 4 + i] = pk(bj[0], bj[1]);
+        ctab[warp * 8 * lpb + 4 * lpb + oct * 4 + i] = pk(cb[0], cb[1]);
       }
       cs.cn2[i] = cs.cd2[i] = 0ull;
     }
     // odd part of a b: E4M3 e has at most 4 significant bits, 2^k has 1
     cs.tie_ok = tie_certified<FMT, WDT>(FMT == FMT_NVFP4 ? sT_bits + 4 + b_bits : b_bits);
-    consumer_sync(kConsumers);  // the column table is written
+    if (!FIN) racc[threadIdx.x] = 0.0;
+    __syncwarp();  // the warp's column table is written
+    bool achg = false;
     int run = 0;
-    // block scales of this warp's rows, one tile ahead
-    const int64_t a_step = (int64_t)kRowsPerTile * p.nb;
-    int64_t aidx = (r0 + warp) * p.nb + blk_col;
-    const int64_t y_off = (int64_t)kConsumerWarps * p.nb;  // block-scale offset of the warp's second row
+    // block scales of this lane's rows, one tile ahead
+    const int64_t a_step = (int64_t)RW * p.nb;
+    int64_t aidx = (r0 + rho) * p.nb + g;
+    const int64_t y_off = (int64_t)rl * p.nb;  // block-scale offset of the lane's second row
     // rows relative to the segment start, in 32 bits (a segment has fewer than 2^31 rows)
     const int nrows = (int)(r1 - r0);
     uint32_t an0 = a_raw_one<FMT>(), an1 = a_raw_one<FMT>();
-    if (active && warp < nrows) an0 = a_fetch<FMT>(p.a_store, aidx);
-    if (active && warp + kConsumerWarps < nrows) an1 = a_fetch<FMT>(p.a_store, aidx + y_off);
+    if (has && rho < nrows) an0 = a_fetch<FMT>(p.a_store, aidx);
+    if (has && rho + rl < nrows) an1 = a_fetch<FMT>(p.a_store, aidx + y_off);
+    const unsigned char* wbase = ring + warp * geo.box_stride + (rho * p.G + 8 * oct) * ES;
+    const int y_bytes = rl * p.G * ES;
 
-    for (int tr = 0; tr < nrows; tr += kRowsPerTile, aidx += a_step) {
-      const int ra = tr + warp, rb = ra + kConsumerWarps;
-      const bool has_a = ra < nrows, has_b = rb < nrows;  // warp-uniform
+    for (int tr = 0; tr < nrows; tr += RW, aidx += a_step) {
+      const int ra = tr + rho, rb = ra + rl;
+      const bool vx = has && ra < nrows, vy = has && rb < nrows;  // per lane
       const uint32_t ra_raw = an0, rb_raw = an1;
-      if (active && ra + kRowsPerTile < nrows) an0 = a_fetch<FMT>(p.a_store, aidx + a_step);
-      if (active && rb + kRowsPerTile < nrows) an1 = a_fetch<FMT>(p.a_store, aidx + a_step + y_off);
+      if (has && ra + RW < nrows) an0 = a_fetch<FMT>(p.a_store, aidx + a_step);
+      if (has && rb + RW < nrows) an1 = a_fetch<FMT>(p.a_store, aidx + a_step + y_off);
       const int64_t cix = ((r0 + ra) * p.N + col) >> 3;  // code group of row ra, this lane's 8 columns
       uint2 oldx = make_uint2(0u, 0u), oldy = make_uint2(0u, 0u);
-      if (PASS != PASS_ITER && cmp && active) {  // issued before the wait: the latency hides behind it
-        if (has_a) oldx = load_codes<FMT>(p.codes, cix);
-        if (has_b) oldy = load_codes<FMT>(p.codes, cix + code_step);
+      if (PASS != PASS_ITER && cmp) {  // issued before the wait: the latency hides behind it
+        if (vx) oldx = load_codes<FMT>(p.codes, cix);
+        if (vy) oldy = load_codes<FMT>(p.codes, cix + code_step);
       }
       mbar_wait(&full[st], par, &p.hdr->flags);
       f2 wa[4], wb[4];
-      const unsigned char* base = ring + st * stage_bytes + lane * 8 * ES;
-      smem_row<WDT>(base + warp * row_bytes, wa);
-      smem_row<WDT>(base + (warp + kConsumerWarps) * row_bytes, wb);
+      const unsigned char* base = wbase + st * geo.stage_bytes;
+      smem_row<WDT>(base, wa);
+      smem_row<WDT>(base + y_bytes, wb);
+      // the slot's loads are performed before its release lets a copy refill it
+      fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[st]);
       if (++st == S) {
         st = 0;
         par ^= 1u;
       }
-      if (has_a) {
-        const float aa = a_dec<FMT>(ra_raw), ab = a_dec<FMT>(rb_raw);  // fetched a tile ago
-        if (!has_b) {
+      if (has) {
+        if (tr + RW > nrows) {  // warp-uniform: the segment's last tile
+          // rows outside the segment (the next CTA's, or the zero fill past
+          // the matrix) hold zeros: they add nothing and write nothing
 #pragma unroll
-          for (int i = 0; i < 4; ++i) wb[i] = 0ull;  // absent row: zeros contribute nothing
+          for (int i = 0; i < 4; ++i) {
+            if (!vx) wa[i] = 0ull;
+            if (!vy) wb[i] = 0ull;
+          }
         }
+        const float aa = a_dec<FMT>(ra_raw), ab = a_dec<FMT>(rb_raw);  // fetched a tile ago
         if (FIN) {
-          final_pair<FMT>(p, wa, aa, wb, ab, has_b, active, cs, sT, sTd, scaled, rscale2, s_cnt, tcnt, cix, oldx,
+          final_pair<FMT>(p, wa, aa, wb, ab, vx, vy, cs, sT, sTd, scaled, rscale2, s_cnt, tcnt, cix, code_step, oldx,
                           oldy, cmp, nchg);
         } else {
-          row_pair<FMT, PASS>(p, wa, aa, aidx, wb, ab, aidx + y_off, has_b, active, leader, lpb, cs,
-                              sT, isT, sTd, scaled, rscale2, s_cnt, tcnt, cix, oldx, oldy, cmp, nchg);
+          row_pair<FMT, PASS>(p, wa, aa, aidx, wb, ab, aidx + y_off, vx, vy, leader, lpb, cs, sT, isT, sTd, scaled,
+                              rscale2, s_cnt, tcnt, cix, code_step, oldx, oldy, cmp, nchg, achg);
         }
-        run += has_b ? 2 : 1;
       }
+      run += 2;
       if (run >= kRun) {
         run = 0;
-        flush_runs(cs, acc, racc, warp, lane, active);
+        flush_runs(cs, acc, racc, warp, lane, has);
       }
     }
-    flush_runs(cs, acc, racc, warp, lane, active);
+    flush_runs(cs, acc, racc, warp, lane, has);
+    const int64_t slot = (int64_t)blockIdx.x * p.segmax + (v - v_first);
+    if (!FIN) {
+      // this segment's residual total of the warp's block-column (fixed xor
+      // order over the lanes), and whether any of its block scales changed
+      double r = racc[threadIdx.x];
+      for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
+      if (has && lane == 0) p.mse_seg[slot * kBcPerStrip + warp] = r;
+      if (__any_sync(0xffffffffu, achg) && has && lane == 0) p.chg[(int64_t)(t % 3) * p.nb + g] = 1u;
+    }
     if (FIN) {  // no column update in the final pass
-      u = (s + 1) * p.M;
+      u = (v + 1) * p.M;
       continue;
     }
 
-    // CTA reduction of the column sums over the consumer warps, fixed order.
-    // Thread t sums entry (c, l) = (t / 32, t % 32), i.e. column 8 (t % 32) + t / 32.
+    // CTA totals of the column sums: column (w, o, c) of the strip, i.e. column
+    // 8 o + c of slot w's block-column, adds its row-lanes in order.
     consumer_sync(kConsumers);
-    const int64_t slot = k * p.segmax + (s - s_first);
-    if (threadIdx.x < kStripMax) {
-      const int cc = threadIdx.x >> 5, ll = threadIdx.x & 31;
-      const int colw = ll * 8 + cc;
-      if (colw < width) {
-        double2 tot = acc[cc * 32 + ll];
-        for (int wi = 1; wi < kConsumerWarps; ++wi) {
-          const double2 v = acc[(wi * 8 + cc) * 32 + ll];
-          tot.x += v.x;
-          tot.y += v.y;
-        }
-        p.col_part[slot * p.TS + colw] = tot;
+    const int width = nbc * p.G;
+    for (int vc = threadIdx.x; vc < width; vc += kConsumers) {
+      const int w = vc / p.G, rem = vc - w * p.G, oo = rem >> 3, c = rem & 7;
+      const double2* src = acc + (w * 8 + c) * 32 + oo;
+      double2 tot = src[0];
+      for (int rr = 1; rr < rl; ++rr) {
+        const double2 x = src[rr * lpb];
+        tot.x += x.x;
+        tot.y += x.y;
       }
+      p.col_part[slot * p.TSv + vc] = tot;
     }
     __threadfence();
     consumer_sync(kConsumers);
-    const int64_t k_first = cta_of(s * p.M, p.P, p.L);
-    const int64_t k_last = cta_of((s + 1) * p.M - 1, p.P, p.L);
+    const int64_t k_first = cta_of(v * p.M, Pt, L);
+    const int64_t k_last = cta_of((v + 1) * p.M - 1, Pt, L);
     if (threadIdx.x == 0) {
-      const unsigned prev = atomicAdd(&p.strip_counter[s], 1u);
+      const unsigned prev = atomicAdd(&p.strip_counter[v], 1u);
       s_misc[0] = prev == (unsigned)(k_last - k_first) ? 1 : 0;
       s_misc[1] = 0;
     }
+    if (threadIdx.x < 16) {
+      s_chgs[threadIdx.x] = 0;
+      s_pend[threadIdx.x] = 0;
+    }
     consumer_sync(kConsumers);
-    if (s_misc[0] && p.mode == DQ_MODE_ROW) {  // block scales only: b keeps its values
-      if (threadIdx.x == 0) p.strip_counter[s] = 0u;
-    } else if (s_misc[0]) {
+    if (s_misc[0]) {
+      // last CTA of the strip: column totals in CTA order, certified projection
       __threadfence();
-      // totals in CTA order, certified projection
-      double bnew = 1.0;
-      bool amb = false;
-      if (threadIdx.x < width) {
-        double2 tot = make_double2(0.0, 0.0);
-        for (int64_t kb = k_first; kb <= k_last; kb += 8) {  // 8 loads in flight, added in CTA order
-          double2 v[8];
+      if (p.mode != DQ_MODE_ROW) {  // in the row mode b keeps its values
+        for (int vc = threadIdx.x; vc < width; vc += kConsumers) {
+          double2 tot = make_double2(0.0, 0.0);
+          for (int64_t kb = k_first; kb <= k_last; kb += 8) {  // 8 loads in flight, added in CTA order
+            double2 x[8];
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const int64_t kk = kb + q;
-            v[q] = make_double2(0.0, 0.0);
-            if (kk <= k_last) v[q] = __ldcg(&p.col_part[(kk * p.segmax + (s - s_sfirst[kk])) * p.TS + threadIdx.x]);
-          }
+            for (int q = 0; q < 8; ++q) {
+              const int64_t kk = kb + q;
+              x[q] = make_double2(0.0, 0.0);
+              if (kk <= k_last) x[q] = __ldcg(&p.col_part[(kk * p.segmax + (v - s_sfirst[kk])) * p.TSv + vc]);
+            }
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            tot.x += v[q].x;
-            tot.y += v[q].y;
+            for (int q = 0; q < 8; ++q) {
+              tot.x += x[q].x;
+              tot.y += x[q].y;
+            }
           }
-        }
-        // certified only when the fp32 runs stayed well inside the normal
-        // range (no overflow; underflowed terms negligible); a zero total may
-        // be underflow and is settled exactly as well
-        const bool safe = tot.x >= 0x1p-60 && tot.x <= 0x1p100 && tot.y >= 0x1p-60 && tot.y <= 0x1p100;
-        const double v = FMT == FMT_NVFP4 ? (tot.x / tot.y) / sTd : tot.x / tot.y;
-        const double lo = safe ? b_project(v * (1.0 - kColErr), p.col_dt) : 0.0;
-        const double hi = safe ? b_project(v * (1.0 + kColErr), p.col_dt) : 1.0;
-        if (lo == hi) {
-          bnew = lo;
-        } else {
-          // ambiguous: listed for the exact update at the start of the next
-          // pass (exact_listed), which recomputes the column's sums over all
-          // rows and writes its scale (b keeps its value until then)
-          amb = true;
-          atomicAdd(&s_misc[1], 1);
-          p.amb_list[(int64_t)(t % 3) * p.N + atomicAdd(&p.hdr->amb_n[t % 3], 1u)] = (int)(c0 + threadIdx.x);
+          const int w = vc / p.G;
+          const int64_t j = (int64_t)(ident ? i0 + w : act[i0 + w]) * p.G + (vc - w * p.G);
+          // certified only when the fp32 runs stayed well inside the normal
+          // range (no overflow; underflowed terms negligible); a zero total may
+          // be underflow and is settled exactly as well
+          const bool safe = tot.x >= 0x1p-60 && tot.x <= 0x1p100 && tot.y >= 0x1p-60 && tot.y <= 0x1p100;
+          const double ratio = FMT == FMT_NVFP4 ? (tot.x / tot.y) / sTd : tot.x / tot.y;
+          const double lo = safe ? b_project(ratio * (1.0 - kColErr), p.col_dt) : 0.0;
+          const double hi = safe ? b_project(ratio * (1.0 + kColErr), p.col_dt) : 1.0;
+          if (lo == hi) {
+            if (lo != (double)b_decode_cg(p.b_store, p.col_dt, j)) {
+              b_encode(p.b_store, p.col_dt, j, lo);
+              s_chgs[w] = 1;
+            }
+          } else {
+            // ambiguous: listed for the exact update at the start of the next
+            // pass (exact_listed), which recomputes the column's sums over all
+            // rows and writes its scale (b keeps its value until then); its
+            // block-column stays active in that pass
+            atomicAdd(&s_misc[1], 1);
+            atomicAdd(&s_pend[w], 1);
+            s_chgs[w] = 1;
+            p.amb_list[(int64_t)(t % 3) * p.N + atomicAdd(&p.hdr->amb_n[t % 3], 1u)] = (int)j;
+          }
         }
       }
       consumer_sync(kConsumers);
+      if (threadIdx.x < nbc) {
+        const int w = threadIdx.x;
+        const int gw = ident ? i0 + w : act[i0 + w];
+        double m = 0.0;  // the block-column's residual total, in CTA order
+        for (int64_t kk = k_first; kk <= k_last; ++kk)
+          m += __ldcg(&p.mse_seg[(kk * p.segmax + (v - s_sfirst[kk])) * kBcPerStrip + w]);
+        mse_bcs(p, t)[gw] = m;
+        if (s_chgs[w]) p.chg[(int64_t)(t % 3) * p.nb + gw] = 1u;
+        if (s_pend[w]) p.pend[gw] = (unsigned)s_pend[w];  // the next pass waits for these
+      }
       if (threadIdx.x == 0) {
         s_cnt[2] += (unsigned)s_misc[1];
-        p.sx_left[s] = (unsigned)s_misc[1];  // listed columns the next pass must settle before using the strip
+        p.strip_counter[v] = 0u;
       }
-      if (threadIdx.x < width && !amb) b_encode(p.b_store, p.col_dt, c0 + threadIdx.x, bnew);
-      if (threadIdx.x == 0) p.strip_counter[s] = 0u;
     }
     consumer_sync(kConsumers);
-    u = (s + 1) * p.M;
+    u = (v + 1) * p.M;
   }
 
   if (PASS != PASS_ITER && cmp) {  // changed codes of this warp, one atomic per warp
@@ -1342,37 +1487,33 @@ __global__ void __launch_bounds__(kIterThreads, 1)
     if (lane == 0 && nchg) atomicAdd(&p.changes[t - 1], (unsigned long long)nchg);
   }
 
-  // MSE of the incoming iterate: per-thread residual sums, CTA tree, then the
-  // CTA-ordered total (the residual accumulators are not reused above).  The
-  // tree reuses the column accumulators: in the final pass no barrier follows
-  // the last flush into them, so wait for every consumer warp here.
-  if (FIN) consumer_sync(kConsumers);
-  double* mred = reinterpret_cast<double*>(acc);
-  mred[threadIdx.x] = racc[threadIdx.x];
-  consumer_sync(kConsumers);
-  for (int o = kConsumerTreeTop; o > 0; o >>= 1) {
-    if (threadIdx.x < o && threadIdx.x + o < kConsumers) mred[threadIdx.x] += mred[threadIdx.x + o];
+  if (FIN) {
+    // MSE of the final iterate: per-thread residual sums, CTA tree, then the
+    // CTA-ordered total by the last CTA to finish (no barrier follows)
     consumer_sync(kConsumers);
-  }
-  if (threadIdx.x == 0) {
-    mse_part(p, t)[k] = mred[0];
-    if (FIN) {  // no barrier follows the final pass: the last CTA to finish sums its MSE
+    double* mred = reinterpret_cast<double*>(acc);
+    mred[threadIdx.x] = racc[threadIdx.x];
+    consumer_sync(kConsumers);
+    for (int o = kConsumerTreeTop; o > 0; o >>= 1) {
+      if (threadIdx.x < o && threadIdx.x + o < kConsumers) mred[threadIdx.x] += mred[threadIdx.x + o];
+      consumer_sync(kConsumers);
+    }
+    if (threadIdx.x == 0) {
+      mse_part(p, t)[blockIdx.x] = mred[0];
       __threadfence();
       const unsigned prev = atomicAdd(&p.hdr->cta_counter, 1u);
       s_misc[0] = prev == (unsigned)p.P - 1u ? 1 : 0;
     }
-  }
-  if (FIN) {
     consumer_sync(kConsumers);
     if (s_misc[0]) {
       __threadfence();
-      mse_total(p, mse_part(p, t), p.mse + (t - 1), rscale_d, mred);
+      mse_total(p, mse_part(p, t), p.P, p.mse + (t - 1), rscale_d, mred);
       if (threadIdx.x == 0) p.hdr->cta_counter = 0u;
     }
   }
   // the scales of pass t (except the listed columns) are final before pass
   // t + 1 reads them
-  if (t < t_last) grid_sync(p, t, rscale_d, mred, &s_misc[0]);
+  if (t < t_last) grid_sync(p, t, rscale_d, reinterpret_cast<double*>(acc), &s_misc[0]);
   }  // passes
 
   for (int o = 16; o > 0; o >>= 1) tcnt += __shfl_xor_sync(0xffffffffu, tcnt, o);
@@ -1385,6 +1526,5 @@ __global__ void __launch_bounds__(kIterThreads, 1)
     if (s_cnt[3]) atomicAdd(&p.hdr->n_quant_tie, (unsigned long long)s_cnt[3]);
   }
 }
-
 
 }  // namespace dq

@@ -142,19 +142,20 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// 2-D tensor map of W (columns innermost) with a box of one ring tile:
-// kStripMax columns x kRowsPerTile rows.  Returns false when W cannot be
-// described (then k_iter copies one row at a time).
+// 2-D tensor map of W (columns innermost) whose box is one block-column's
+// share of a ring tile: G columns x 2 * 32/(G/8) rows.  Returns false when W
+// cannot be described (then k_iter copies one block row at a time).
 template <int WDT>
 static bool encode_w_map(const Problem& p, CUtensorMap* map) {
   constexpr int ES = WDT == DT_F32 ? 4 : 2;
   std::memset(map, 0, sizeof(*map));
-  if (p.M > INT_MAX || p.TS != kStripMax || (p.N * ES) % 16 != 0) return false;
+  if (p.M > INT_MAX || p.N > INT_MAX || (p.N * ES) % 16 != 0 || (p.G * ES) % 16 != 0) return false;
   const PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
   if (fn == nullptr) return false;
+  const TileGeo geo = tile_geo(p.G, ES);
   const cuuint64_t dims[2] = {(cuuint64_t)p.N, (cuuint64_t)p.M};
   const cuuint64_t strides[1] = {(cuuint64_t)p.N * ES};
-  const cuuint32_t box[2] = {(cuuint32_t)kStripMax, (cuuint32_t)kRowsPerTile};
+  const cuuint32_t box[2] = {(cuuint32_t)p.G, (cuuint32_t)geo.RW};
   const cuuint32_t elem_strides[2] = {1, 1};
   const CUtensorMapDataType dt = WDT == DT_F32    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
                                  : WDT == DT_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
@@ -196,8 +197,7 @@ static cudaError_t launch_coop(void (*kernel)(KArgs...), unsigned grid, unsigned
 
 template <int FMT, int WDT>
 static cudaError_t run_typed(const Problem& p, int iters, int stats_ctas, cudaStream_t st) {
-  constexpr int ES = WDT == DT_F32 ? 4 : 2;
-  const size_t smem = iter_smem_bytes(ES);
+  const size_t smem = (size_t)iter_smem(p.G / 8, p.P, p.segmax).total;
   const auto iter_kernel = p.changes ? k_iter<FMT, WDT, PASS_COUNT> : k_iter<FMT, WDT, PASS_ITER>;
   cudaError_t e = cudaFuncSetAttribute(iter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -257,27 +257,40 @@ cudaError_t launch_solve(const Problem& p, int iters, int stats_ctas, cudaStream
   }
 }
 
-// Self-test of the bounded waits: strip 0's pending count is set to 1 and
-// never released, so wait_strip gives up after its time limit and records
-// kFlagTimeout; nothing faults and the context stays usable.
-__global__ void k_wait_selftest(Problem p) {
-  if (threadIdx.x == 0) {
-    p.hdr->flags = 0u;
-    p.sx_left[0] = 1u;
-    __threadfence();
+// Self-tests of the bounded waits; nothing faults and the context stays
+// usable.  which == 0: block-column 0's pending count is set to 1 and never
+// released, so wait_bc gives up after its time limit.  which == 1: a ring
+// barrier in shared memory that nothing arrives at and no copy completes, so
+// mbar_wait gives up after its time limit.  Both record kFlagTimeout.
+__global__ void k_wait_selftest(Problem p, int which) {
+  __shared__ uint64_t bar;
+  if (which == 0) {
+    if (threadIdx.x == 0) {
+      p.hdr->flags = 0u;
+      p.pend[0] = 1u;
+      __threadfence();
+    }
+    __syncwarp();
+    wait_bc(p, 0);
+    if (threadIdx.x == 0) p.pend[0] = 0u;
+  } else {
+    if (threadIdx.x == 0) {
+      p.hdr->flags = 0u;
+      mbar_init(&bar, 1);
+      mbar_fence_init();
+    }
+    __syncwarp();
+    if (threadIdx.x == 0) mbar_wait(&bar, 0u, &p.hdr->flags);
+    __syncwarp();
   }
-  __syncthreads();
-  wait_strip(p, 0);
-  __syncthreads();
-  if (threadIdx.x == 0) p.sx_left[0] = 0u;
 }
 
-cudaError_t launch_wait_selftest(void* workspace, cudaStream_t st) {
+cudaError_t launch_wait_selftest(void* workspace, int which, cudaStream_t st) {
   Problem p;
   std::memset(&p, 0, sizeof(p));
   p.hdr = reinterpret_cast<WsHeader*>(workspace);
-  p.sx_left = reinterpret_cast<unsigned*>(static_cast<char*>(workspace) + 256);
-  k_wait_selftest<<<1, 32, 0, st>>>(p);
+  p.pend = reinterpret_cast<unsigned*>(static_cast<char*>(workspace) + 256);
+  k_wait_selftest<<<1, 32, 0, st>>>(p, which);
   return cudaGetLastError();
 }
 

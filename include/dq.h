@@ -166,6 +166,10 @@ typedef struct {
                             * App. B: the quantized matrix stabilizes; the relative change of Q is
                             * code_changes[t] / (rows*cols)).  The solver keeps the codes of the
                             * previous iterate in out->codes meanwhile. */
+  int full_passes;         /* 0 (default): a block-column (the rows x group slab under one column of
+                            * blocks) whose scales come out of an iteration unchanged is at a fixed
+                            * point of the iteration and later iterations skip it.  Nonzero: every
+                            * iteration processes every block-column.  The outputs are the same. */
 } dq_options;
 
 /* Device workspace bytes dq_solve_ex needs with these options (0 on invalid
@@ -213,18 +217,29 @@ int dq_solve_host(const void* W_host, int w_dtype, int64_t rows, int64_t cols, i
  * Counts cover the BCD iterations only (not init or the final pass). */
 int dq_diagnostics(const void* workspace, void* stream, uint64_t out[4]);
 
+/* Work done by the BCD iterations of the last solve that used `workspace`
+ * (waits for `stream`): *out = the number of block-columns (the rows x group
+ * slab under one column of blocks) processed, summed over the iterations.
+ * A block-column whose scales come out of an iteration unchanged is at a fixed
+ * point of the BCD map (its block and column updates read only its own
+ * scales), so later iterations skip it; the full count is iters * cols/group.
+ * No counterpart in the method; a work statistic. */
+int dq_active_block_columns(const void* workspace, void* stream, uint64_t* out);
+
 /* Self-test of the solver's bounded device waits (no counterpart in the
  * method; failure detection).  Every wait of the per-iteration kernel (the
- * tile pipeline, the grid barrier between BCD passes, the wait for a strip's
- * exactly updated column scales) gives up after a time limit (about 1 s),
- * records a timeout in the workspace header and lets the kernel finish, so a
- * lost arrival ends in a status instead of a hung GPU.  This call enqueues one
- * such wait on a counter that nothing releases: afterwards dq_sync_status on
- * the same workspace returns DQ_ECUDA, and the context stays usable (the next
- * dq_solve clears the header).  `workspace`: device, 256-byte aligned, at least
- * 512 bytes, overwritten.  Returns DQ_EINVAL / DQ_EWORKSPACE / DQ_ECUDA on bad
- * arguments or a failed launch. */
-int dq_wait_selftest(void* workspace, size_t workspace_bytes, void* stream);
+ * tile pipeline's ring barriers, the grid barrier between BCD passes, the wait
+ * for a block-column's exactly updated column scales) gives up after a time
+ * limit (about 1 s), records a timeout in the workspace header and lets the
+ * kernel finish, so a lost arrival ends in a status instead of a hung GPU.
+ * This call enqueues one such wait that nothing releases: which = 0 waits on a
+ * pending count in global memory, which = 1 on a shared-memory ring barrier
+ * that no copy completes.  Afterwards dq_sync_status on the same workspace
+ * returns DQ_ECUDA, and the context stays usable (the next dq_solve clears the
+ * header).  `workspace`: device, 256-byte aligned, at least 512 bytes,
+ * overwritten.  Returns DQ_EINVAL / DQ_EWORKSPACE / DQ_ECUDA on bad arguments
+ * or a failed launch. */
+int dq_wait_selftest(void* workspace, size_t workspace_bytes, int which, void* stream);
 
 /* One matrix of a batched solve: W (device, row-major rows x cols, w_dtype)
  * and its outputs (as for dq_solve, mse with iters+1 entries). */
@@ -298,9 +313,11 @@ int dq_act_quant(const void* X, int x_dtype, int64_t rows, int64_t cols, const v
  *          (device memory or mapped host memory): after the solve, a stream-
  *          ordered kernel stores DQ_OK, DQ_ENONFINITE or DQ_ECUDA there, the
  *          device-side outcome that dq_sync_status reports for dq_solve.
- * Set-up: the first call on each device, made with that device current, looks
- * up the scratch array's device address (loading the module there); make
- * that first call before any stream capture on the device.
+ * Set-up: every call looks up the scratch array's device address on the
+ * current device (cudaGetSymbolAddress; nothing is cached, so a context torn
+ * down and created again is handled).  The first call on a device also loads
+ * the library's device code there; make that first call before any stream
+ * capture on the device.
  * Sharing: all calls on one device share the same scratch, and each call
  * clears the parts that must start at zero.  Calls whose work overlaps on the
  * GPU (different streams, or several host threads, without ordering between

@@ -1,8 +1,10 @@
 """Failure detection on the GPU without a fault: every wait of the per-iteration kernel is bounded in
 time, gives up with a status the host reads, and leaves the context usable.
 
-The self-test entry point runs the kernel's strip wait on a counter that nothing releases (a flag that
-nothing sets); no GPU fault, trap or hang is involved.
+The self-test entry point runs one of the kernel's waits on something that nothing releases: a pending
+count in global memory that nothing counts down (the wait for a block-column's exactly updated column
+scales), or a shared-memory ring barrier that no copy completes and nobody arrives at (the tile
+pipeline's wait).  No copy is issued and no GPU fault, trap or hang is involved.
 """
 from __future__ import annotations
 
@@ -19,10 +21,11 @@ DQ_ECUDA = 5
 
 
 @pytest.mark.gpu
-def test_bounded_wait_gives_up_with_a_status_and_the_context_stays_usable():
+@pytest.mark.parametrize("which", [0, 1])
+def test_bounded_wait_gives_up_with_a_status_and_the_context_stays_usable(which):
     ws = torch.empty(4096, dtype=torch.uint8, device="cuda")
     t0 = time.time()
-    st = binding.wait_selftest(ws)
+    st = binding.wait_selftest(ws, which)
     elapsed = time.time() - t0
     assert st == DQ_ECUDA
     assert 0.5 < elapsed < 60.0, elapsed  # about the 1 s limit of a wait
