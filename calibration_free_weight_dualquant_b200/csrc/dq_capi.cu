@@ -17,8 +17,7 @@ struct Plan {
   int TSv, n_strips, P, segmax, P_final, segmax_final, nb;
   int64_t L;
   size_t smem;  // dynamic shared memory of k_iter
-  size_t off_counters, off_amb_tick, off_pend, off_chg, off_col_part, off_cta_part, off_mse_seg, off_mse_bc,
-      off_amb_list, off_xpart, total;
+  size_t off_counters, off_chg, off_col_part, off_cta_part, off_mse_seg, off_mse_bc, off_amb_list, total;
   size_t l1_zero_bytes;  // L1 init: digit counters to zero (start of the col_part region)
   size_t off_l1_tot, off_l1_norm;
 };
@@ -82,13 +81,9 @@ int make_plan(int64_t M, int64_t N, int group, int init, Plan* pl) {
   pl->smem = (size_t)dq::iter_smem(group / 8, pl->P, pl->segmax).total;
   if (pl->smem > (size_t)227 * 1024) return DQ_EUNSUPPORTED;  // more strips per CTA than shared memory holds
   size_t off = align_up(sizeof(dq::WsHeader));
-  // zeroed at the start of a solve: arrival counters, pending counts, change flags
+  // zeroed at the start of a solve: arrival counters, change flags
   pl->off_counters = off;
-  off += align_up(sizeof(unsigned) * (size_t)pl->n_strips);
-  pl->off_amb_tick = off;
-  off += align_up(sizeof(unsigned) * (size_t)N);
-  pl->off_pend = off;
-  off += align_up(sizeof(unsigned) * (size_t)pl->nb);
+  off += align_up(sizeof(unsigned) * 8 * (size_t)pl->n_strips);
   pl->off_chg = off;
   off += align_up(sizeof(unsigned) * 3 * (size_t)pl->nb);
   pl->off_col_part = off;
@@ -110,9 +105,7 @@ int make_plan(int64_t M, int64_t N, int group, int init, Plan* pl) {
   pl->off_mse_bc = off;
   off += align_up(sizeof(double) * 3 * (size_t)pl->nb);
   pl->off_amb_list = off;
-  off += align_up(sizeof(int) * 3 * (size_t)N);
-  pl->off_xpart = off;
-  off += align_up(sizeof(double2) * (size_t)dq::kXPartCap);
+  off += align_up(sizeof(int) * (size_t)pl->n_strips * (size_t)pl->TSv);
   pl->total = off;
   return DQ_OK;
 }
@@ -193,17 +186,13 @@ int solve_impl(const void* W, int w_dtype, int64_t rows, int64_t cols, int forma
   p.strip_counter = reinterpret_cast<unsigned*>(ws + pl.off_counters);
   p.col_part = reinterpret_cast<double2*>(ws + pl.off_col_part);
   p.cta_part = reinterpret_cast<double*>(ws + pl.off_cta_part);
-  p.amb_list = reinterpret_cast<int*>(ws + pl.off_amb_list);
-  p.amb_tick = reinterpret_cast<unsigned*>(ws + pl.off_amb_tick);
-  p.pend = reinterpret_cast<unsigned*>(ws + pl.off_pend);
   p.chg = reinterpret_cast<unsigned*>(ws + pl.off_chg);
   p.mse_seg = reinterpret_cast<double*>(ws + pl.off_mse_seg);
   p.mse_bc = reinterpret_cast<double*>(ws + pl.off_mse_bc);
-  p.xpart = reinterpret_cast<double2*>(ws + pl.off_xpart);
+  p.amb_list = reinterpret_cast<int*>(ws + pl.off_amb_list);
 
-  // header, arrival counters (strips, listed columns), pending counts and
-  // change flags start at zero; the partial buffers and the column list need
-  // no init
+  // header, strip arrival counters and change flags start at zero; the
+  // partial buffers need no init
   if (cudaMemsetAsync(ws, 0, pl.off_col_part, stream) != cudaSuccess) return DQ_ECUDA;
   if (init == DQ_INIT_L1 && cudaMemsetAsync(ws + pl.off_col_part, 0, pl.l1_zero_bytes, stream) != cudaSuccess)
     return DQ_ECUDA;

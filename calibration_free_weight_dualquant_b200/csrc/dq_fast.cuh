@@ -253,6 +253,13 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const void* map, int x, i
       : "memory");
 }
 
+// L2 prefetch of the box at (x = column, y = row) of the 2-D tensor map `map`
+// (no shared memory written, no completion to wait for).
+__device__ __forceinline__ void tma_prefetch_2d(const void* map, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(x), "r"(y)
+               : "memory");
+}
+
 // Programmatic dependent launch.  A grid launched with programmatic stream
 // serialization may start while the grid before it in the stream is still
 // running; griddep_wait() returns once every grid it depends on has completed

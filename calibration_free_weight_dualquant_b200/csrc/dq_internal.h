@@ -18,7 +18,6 @@ constexpr int64_t kMinRowsPerCta = 64;
 // 32-bit digits of an exact magnitude sum in units of 2^-149 (L1 init): one
 // value reaches bit 277, a sum of up to 2^31 values bit 308
 constexpr int kXDigits = 10;
-constexpr int64_t kXPartCap = 32768;  // entries of the exact-update partial buffer
 constexpr unsigned kFlagNonFinite = 1u;
 constexpr unsigned kFlagTimeout = 2u;  // a bounded pipeline wait gave up (results invalid)
 constexpr unsigned kFlagBadInit = 4u;  // a warm start was given an inadmissible scale
@@ -56,11 +55,10 @@ __host__ __device__ inline TileGeo tile_geo(int G, int es) {
 // Dynamic shared memory of k_iter (byte offsets): the tile ring; fp64 column
 // accumulators (per consumer warp: 8 columns x 32 lanes of (sum W a q,
 // sum (a q)^2)); one fp64 residual sum per consumer thread; ring barriers;
-// small ints ([0] ticket result, [1] #ambiguous, [2..5] exact-path counters,
-// [8..22] per-slot change flags, [24..38] per-slot listed columns, [40..56]
-// schedule scan); the pass schedule; the column tables (per warp: b pairs
-// [lpb][4], then 1/b pairs [lpb][4]); the first strip of each CTA's range;
-// this CTA's slice of the active list.
+// small ints ([0] flag, [2..5] exact-path counters, [40..56] schedule scan);
+// the pass schedule; the column tables (per warp: b pairs [lpb][4], then 1/b
+// pairs [lpb][4]); the first strip of each CTA's range; this CTA's slice of
+// the active list.
 struct IterSmem {
   int acc, racc, bars, misc, sched, ctab, sfirst, act, total;
 };
@@ -106,7 +104,6 @@ struct WsHeader {
   unsigned flags;        // kFlagNonFinite, kFlagTimeout, kFlagBadInit
   unsigned amax_bits;    // max |W| as fp32 bits
   unsigned cta_counter;  // arrival ticket for CTA-ordered totals
-  unsigned amb_n[3];     // columns listed for the exact column update, by pass mod 3
   unsigned gbar;         // arrivals at k_iter's grid-wide barrier
   float sT;              // NVFP4 tensor scale (1 otherwise)
   unsigned long long n_quant_tie;    // lane-rows with a certified exact tie settled on the fast path
@@ -138,16 +135,14 @@ struct Problem {
   float* sT_out;
   double* mse;
   WsHeader* hdr;
-  unsigned* strip_counter;  // [n_strips] arrivals per strip (zeroed)
+  unsigned* strip_counter;  // [4][2][n_strips] per strip and pass parity: arrivals, ambiguous columns,
+                            // finalizers done, exact shares done (zeroed)
+  int* amb_list;            // [n_strips][TSv] strip columns listed for the exact update
   double2* col_part;        // [P * segmax][TSv] (sum W a q, sum (a q)^2)
   double* cta_part;         // [3][max(P, P_final)] per-CTA residual totals of the final pass
   double* mse_seg;          // [P * segmax][15] residual total per (CTA segment, block-column slot)
   double* mse_bc;           // [3][nb] residual total per block-column, by pass mod 3
   unsigned* chg;            // [3][nb] a scale of the block-column changed (or was listed), by pass mod 3 (zeroed)
-  unsigned* pend;           // [nb] listed columns of a block-column awaiting their exact update (zeroed)
-  int* amb_list;            // [3][N] columns whose certified projection was ambiguous, by pass mod 3
-  unsigned* amb_tick;       // [N] arrival counters of their row chunks (zeroed)
-  double2* xpart;           // [kXPartCap] per-CTA exact partial sums of the listed columns
   int use_tmap;             // W streamed by 2-D tensor copies (else one bulk copy per row)
   int mode;                 // DQ_MODE_DUAL, DQ_MODE_ROW (b keeps its initial value) or DQ_MODE_COL
   int init;                 // DQ_INIT_RTN, DQ_INIT_L1 or DQ_INIT_GIVEN

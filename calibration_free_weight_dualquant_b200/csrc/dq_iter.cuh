@@ -844,24 +844,7 @@ __device__ void grid_sync_plain(WsHeader* hdr) {
   consumer_sync(kConsumers);
 }
 
-// Exact column update, at the start of pass t, of the columns that the strip
-// finalizers of pass t - 1 listed (their certified projection was ambiguous and
-// their scale still holds the previous value): sum W a q' and sum (a q')^2 in
-// fp64 over all rows, then b = Proj_Fb(ratio), 1 for a zero sum.
-//
-// Each listed column is cut into R row chunks and the (column, chunk) items
-// are spread over all CTAs of the grid (about one each), so the update costs
-// one short round of loads per CTA.  A chunk's total is a fixed-order
-// reduction over the consumer threads; the last chunk of a column to arrive
-// adds the R chunk totals in chunk order (the result does not depend on the
-// schedule), writes the scale and counts its block-column's p.pend down.  A
-// warp reaching a block-column with listed columns waits for that count to
-// reach zero (wait_bc); nobody else waits.  When the list is too long for
-// p.xpart the chunk totals go to p.col_part instead and a grid barrier follows
-// (then nobody waits).  Run by the consumer threads; `scratch` holds 2 * kConsumers
-// doubles.
 constexpr int kXRows = 8;
-constexpr int64_t kXMinRows = 32;  // rows of the smallest chunk
 
 // Fixed-order sum of one value per consumer thread (xor trees within the warps,
 // then the warp totals in warp order); the total is in red[0] afterwards.
@@ -887,9 +870,11 @@ __device__ __forceinline__ void consumer_sum2(double x, double y, double* red) {
   }
 }
 
-// fp64 sums of W a q and (a q)^2 of column j over rows [i_begin, i_end)
-// (every load issued before any is used); the totals go to scratch[0], [1]
-// (thread 0; the caller synchronizes before others read them).
+// Exact column sums: fp64 sums of W a q and (a q)^2 of column j over rows
+// [i_begin, i_end), with q decided exactly (every load of a round issued before
+// any is used); the totals go to scratch[0], [1] (thread 0; the caller
+// synchronizes before others read them).  Used for a column whose certified
+// projection is ambiguous.
 template <int FMT, int WDT>
 __device__ void column_rows_exact(const Problem& p, int64_t j, int64_t i_begin, int64_t i_end, double sTd, float isT,
                                   double* scratch) {
@@ -932,86 +917,187 @@ __device__ void column_rows_exact(const Problem& p, int64_t j, int64_t i_begin, 
   consumer_sum2(cn, cd, scratch);
 }
 
-// The last contributor to a listed column: adds the `cnt` chunk totals in
-// order and writes the projected scale (consumer threads; thread 0 writes).
-template <int FMT>
-__device__ void column_settle(const Problem& p, int64_t j, const double2* part, int64_t cnt, double sTd,
-                              double* scratch) {
-  double2 v = make_double2(0.0, 0.0);
-  for (int64_t k = threadIdx.x; k < cnt; k += kConsumers) {
-    const double2 c = __ldcg(part + k);
-    v.x += c.x;
-    v.y += c.y;
-  }
-  consumer_sum2(v.x, v.y, scratch);
+// Bounded wait of thread 0 until *c reaches `target` (ld.acquire; gives up
+// with kFlagTimeout after kWaitLimitNs).  The caller synchronizes the CTA
+// afterwards, which orders the other threads' later loads after the acquire.
+__device__ void wait_count(unsigned* c, unsigned target, unsigned* flags) {
   if (threadIdx.x == 0) {
-    const double tn = scratch[0], td = scratch[1];
-    const double v2 = FMT == FMT_NVFP4 ? (tn / td) / sTd : tn / td;
-    b_encode(p.b_store, p.col_dt, j, td == 0.0 ? 1.0 : b_project(v2, p.col_dt));
-  }
-}
-
-// Returns true when block-columns with listed columns must be waited for (wait_bc).
-template <int FMT, int WDT>
-__device__ bool exact_listed(const Problem& p, int t, double sTd, float isT, double* scratch, int* s_flag) {
-  const int lb = (t - 1) % 3;
-  const unsigned n = __ldcg(&p.hdr->amb_n[lb]);
-  // the list of pass t + 1 was last read in pass t - 1: empty it for its writers
-  if (blockIdx.x == 0 && threadIdx.x == 0) p.hdr->amb_n[(t + 1) % 3] = 0u;
-  if (n == 0u) return false;  // the same value in every CTA
-  const int* list = p.amb_list + (int64_t)lb * p.N;
-  const bool own = (int64_t)n <= kXPartCap;  // chunk totals in p.xpart, no barrier
-  double2* part = own ? p.xpart : p.col_part;
-  const int64_t cap = own ? kXPartCap : (int64_t)p.P * p.segmax * p.TSv;
-  const int64_t R = max((int64_t)1, min(min((p.M + kXMinRows - 1) / kXMinRows, max((int64_t)1, (int64_t)p.P / (int64_t)n)),
-                                        cap / (int64_t)n));
-  const int64_t chunk = (p.M + R - 1) / R;
-  for (int64_t it = blockIdx.x; it < (int64_t)n * R; it += gridDim.x) {
-    const int64_t ci = it / R, r = it - ci * R;
-    const int64_t j = __ldcg(list + ci);
-    column_rows_exact<FMT, WDT>(p, j, r * chunk, min(p.M, (r + 1) * chunk), sTd, isT, scratch);
-    if (threadIdx.x == 0) {
-      part[it] = make_double2(scratch[0], scratch[1]);
-      __threadfence();
-      const unsigned prev = atomicAdd(&p.amb_tick[ci], 1u);
-      *s_flag = prev == (unsigned)R - 1u ? 1 : 0;
-    }
-    consumer_sync(kConsumers);
-    if (*s_flag) {
-      __threadfence();
-      column_settle<FMT>(p, j, part + ci * R, R, sTd, scratch);
-      if (threadIdx.x == 0) {
-        p.amb_tick[ci] = 0u;
-        __threadfence();  // the scale is visible before the count drops
-        if (own) {
-          atomicSub(&p.pend[j / p.G], 1u);
-        } else {
-          p.pend[j / p.G] = 0u;  // the barrier below orders it
-        }
-      }
-    }
-    consumer_sync(kConsumers);  // the scratch and the flag are reused
-  }
-  if (!own) grid_sync_plain(p.hdr);
-  return own;
-}
-
-// Before a warp uses the column scales of block-column g: wait until its
-// listed columns are settled (lane 0 polls, bounded; gives up with
-// kFlagTimeout).  Warp-collective: the warp's later loads of the scales are
-// ordered after lane 0's acquiring load by the warp barrier.
-__device__ void wait_bc(const Problem& p, int64_t g) {
-  if ((threadIdx.x & 31) == 0) {
     const unsigned long long t0 = global_ns();
     for (;;) {
-      if (ld_acquire_gpu(&p.pend[g]) == 0u) break;
-      if (wait_expired(&p.hdr->flags, t0)) break;
+      if ((int)(ld_acquire_gpu(c) - target) >= 0) break;
+      if (wait_expired(flags, t0)) break;
       __nanosleep(64);
     }
   }
-  __syncwarp();
 }
 
+// Sum of the column partials (sum W a q, sum (a q)^2) of strip column vc over
+// the CTAs kb0 .. kb1-1 of strip v, in CTA order, 4 loads in flight.
+__device__ __forceinline__ double2 col_total(const Problem& p, int vc, int64_t v, int64_t kb0, int64_t kb1,
+                                             const int* s_sfirst) {
+  double2 tot = make_double2(0.0, 0.0);
+  for (int64_t kb = kb0; kb < kb1; kb += 4) {
+    double2 x[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int64_t kk = kb + q;
+      x[q] = make_double2(0.0, 0.0);
+      if (kk < kb1) x[q] = __ldcg(&p.col_part[(kk * p.segmax + (v - s_sfirst[kk])) * p.TSv + vc]);
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      tot.x += x[q].x;
+      tot.y += x[q].y;
+    }
+  }
+  return tot;
+}
+
+// Finalization of the strip slots w = w0, w0 + step, ... < nbc of strip v in
+// pass t, by the consumer threads of one CTA, once all K CTAs of the strip
+// (k_first ..) have written their partial sums; slots are taken in groups whose
+// loads are all issued together.  For each column: its totals from the K CTAs
+// (sp threads per column, each adding a contiguous slice in CTA order, the
+// slices then added in slice order) and the certified projection of its new
+// scale; a column whose projection is ambiguous is added to the strip's list
+// (strip column index) for the exact update that follows, and its block-column
+// counts as changed.  For each slot: its block-column's residual total (in CTA
+// order) and change flag.  `scr` is scratch shared memory of at least 2048
+// doubles; `ctab` the CTA's column tables of the strip (its last segment),
+// which hold the old scales.
+template <int FMT>
+__device__ void finalize_slots(const Problem& p, int t, int64_t v, int w0, int step, int nbc, const int* act,
+                               bool ident, int i0, int64_t k_first, int K, const int* s_sfirst, double sTd,
+                               double* scr, const f2* ctab, int* amb_list, unsigned* amb_cnt, int* s_chg) {
+  const int G = p.G;
+  const bool cols = p.mode != DQ_MODE_ROW;  // in the row mode b keeps its values
+  const int nw_all = w0 < nbc ? (nbc - w0 + step - 1) / step : 0;
+  const int grp_max = max(1, kConsumers / G);
+  for (int g0 = 0; g0 < nw_all; g0 += grp_max) {
+    const int nw = min(grp_max, nw_all - g0);
+    const int sp = max(1, min(min(K, 16), kConsumers / (G * nw)));
+    double* mpart = scr;                                                          // [nw][K]
+    double2* cpart = reinterpret_cast<double2*>(scr + ((nw * K + 1) & ~1));      // [nw][sp][G]
+    if (threadIdx.x < nw) s_chg[threadIdx.x] = 0;
+    for (int e = threadIdx.x; e < nw * K; e += kConsumers) {
+      const int iw = e / K;
+      const int w = w0 + (g0 + iw) * step;
+      const int64_t kk = k_first + (e - iw * K);
+      mpart[e] = __ldcg(&p.mse_seg[(kk * p.segmax + (v - s_sfirst[kk])) * kBcPerStrip + w]);
+    }
+    if (cols) {
+      for (int e = threadIdx.x; e < nw * sp * G; e += kConsumers) {
+        const int iw = e / (sp * G), rem = e - iw * (sp * G), part = rem / G, c = rem - part * G;
+        const int w = w0 + (g0 + iw) * step;
+        cpart[e] = col_total(p, w * G + c, v, k_first + (int64_t)part * K / sp,
+                             k_first + (int64_t)(part + 1) * K / sp, s_sfirst);
+      }
+    }
+    consumer_sync(kConsumers);
+    if (cols) {
+      for (int e = threadIdx.x; e < nw * G; e += kConsumers) {
+        const int iw = e / G, c = e - iw * G;
+        const int w = w0 + (g0 + iw) * step;
+        double2 tot = cpart[iw * sp * G + c];
+        for (int part = 1; part < sp; ++part) {
+          const double2 x = cpart[(iw * sp + part) * G + c];
+          tot.x += x.x;
+          tot.y += x.y;
+        }
+        const int64_t j = (int64_t)(ident ? i0 + w : act[i0 + w]) * G + c;
+        // certified only when the fp32 runs stayed well inside the normal range
+        // (no overflow; underflowed terms negligible); a zero total may be
+        // underflow and is settled exactly as well
+        const bool safe = tot.x >= 0x1p-60 && tot.x <= 0x1p100 && tot.y >= 0x1p-60 && tot.y <= 0x1p100;
+        const double ratio = FMT == FMT_NVFP4 ? (tot.x / tot.y) / sTd : tot.x / tot.y;
+        const double lo = safe ? b_project(ratio * (1.0 - kColErr), p.col_dt) : 0.0;
+        const double hi = safe ? b_project(ratio * (1.0 + kColErr), p.col_dt) : 1.0;
+        // the old scale: this CTA's column table of the strip (warp w, octet
+        // c / 8, pair (c % 8) / 2), loaded when its segment of the strip began
+        const f2 bp = ctab[w * 8 * (G / 8) + (c >> 3) * 4 + ((c & 7) >> 1)];
+        const double bold = (double)((c & 1) ? hi_of(bp) : lo_of(bp));
+        if (lo == hi) {
+          if (lo != bold) {
+            b_encode(p.b_store, p.col_dt, j, lo);
+            s_chg[iw] = 1;
+          }
+        } else {
+          amb_list[atomicAdd(amb_cnt, 1u)] = w * G + c;  // b keeps its value until the exact update
+          s_chg[iw] = 1;
+        }
+      }
+      consumer_sync(kConsumers);
+    }
+    for (int iw = threadIdx.x; iw < nw; iw += kConsumers) {
+      const int w = w0 + (g0 + iw) * step;
+      const int gw = ident ? i0 + w : act[i0 + w];
+      double m = 0.0;  // the block-column's residual total, in CTA order
+      for (int kq = 0; kq < K; ++kq) m += mpart[iw * K + kq];
+      mse_bcs(p, t)[gw] = m;
+      if (s_chg[iw]) p.chg[(int64_t)(t % 3) * p.nb + gw] = 1u;
+    }
+    consumer_sync(kConsumers);  // the scratch is reused
+  }
+}
+
+// Exact update of the columns of strip v listed as ambiguous (amb_list[0 ..
+// n)), shared by the nfin finalizing CTAs of the strip: finalizer q sums the
+// columns exactly (fp64, exact grid decisions) over rows [q M / nfin,
+// (q+1) M / nfin) and stores the two sums in its own partial slot `myslot` of
+// the strip (whose values every finalizer has read by now); the last of them
+// to finish adds the nfin sums of each column in finalizer order and writes
+// the projected scale.  `red` holds 3 kConsumers doubles; s_flag one int.
+template <int FMT, int WDT>
+__device__ void exact_columns(const Problem& p, int64_t v, const int* act, bool ident, int i0_strip, int q, int nfin,
+                              int64_t k_first, int64_t myslot, const int* s_sfirst, const int* amb_list, int n,
+                              unsigned* ticket, double sTd, float isT, double* red, int* s_flag, unsigned* s_cnt) {
+  const int G = p.G;
+  const int64_t lo = (int64_t)q * p.M / nfin, hi = (int64_t)(q + 1) * p.M / nfin;
+  for (int i = 0; i < n; ++i) {
+    const int vc = __ldcg(amb_list + i);
+    const int w = vc / G;
+    const int64_t j = (int64_t)(ident ? i0_strip + w : act[i0_strip + w]) * G + (vc - w * G);
+    column_rows_exact<FMT, WDT>(p, j, lo, hi, sTd, isT, red);
+    if (threadIdx.x == 0) p.col_part[myslot * p.TSv + vc] = make_double2(red[0], red[1]);
+    consumer_sync(kConsumers);  // red is reused
+  }
+  if (threadIdx.x == 0) {
+    __threadfence();
+    *s_flag = atomicAdd(ticket, 1u) == (unsigned)nfin - 1u ? 1 : 0;
+  }
+  consumer_sync(kConsumers);
+  if (*s_flag == 0) return;
+  __threadfence();
+  // every share of every listed column loaded at once (into the idle column
+  // accumulators, 2 kConsumers doubles), then each column's shares added in
+  // finalizer order
+  double2* sh = reinterpret_cast<double2*>(red) + kConsumers;
+  for (int i0 = 0; i0 < n; i0 += max(1, kConsumers / nfin)) {
+    const int nc = min(n - i0, max(1, kConsumers / nfin));
+    for (int e = threadIdx.x; e < nc * nfin; e += kConsumers) {
+      const int i = e / nfin, qq = e - i * nfin;
+      const int vc = __ldcg(amb_list + i0 + i);
+      const int64_t kk = k_first + qq;
+      sh[e] = __ldcg(&p.col_part[(kk * p.segmax + (v - s_sfirst[kk])) * p.TSv + vc]);
+    }
+    consumer_sync(kConsumers);
+    for (int i = threadIdx.x; i < nc; i += kConsumers) {
+      const int vc = __ldcg(amb_list + i0 + i);
+      const int w = vc / G;
+      const int64_t j = (int64_t)(ident ? i0_strip + w : act[i0_strip + w]) * G + (vc - w * G);
+      double tn = 0.0, td = 0.0;
+      for (int qq = 0; qq < nfin; ++qq) {
+        tn += sh[i * nfin + qq].x;
+        td += sh[i * nfin + qq].y;
+      }
+      const double r = FMT == FMT_NVFP4 ? (tn / td) / sTd : tn / td;
+      const double bnew = td == 0.0 ? 1.0 : b_project(r, p.col_dt);
+      if (bnew != (double)b_decode_cg(p.b_store, p.col_dt, j)) b_encode(p.b_store, p.col_dt, j, bnew);
+    }
+    consumer_sync(kConsumers);
+  }
+  if (threadIdx.x == 0) s_cnt[2] += (unsigned)n;
+}
 
 // Named barrier of the whole CTA (consumers and producer): the schedule of a
 // pass is handed to the producer through it.
@@ -1101,9 +1187,7 @@ __device__ void pass_schedule(const Problem& p, int t, bool ident, Sched* sc, in
 // block-column at a fixed point keeps its codes and adds nothing).
 // PASS_FINAL: the final pass after T iterations over every block-column,
 // called with t_first = t_last = T + 1: the codes of the final iterate, packed,
-// and mse[T] (and changes[T] when counting, T >= 1).  Every pass starts with
-// the exact update of the columns that the pass before left ambiguous
-// (exact_listed).
+// and mse[T] (and changes[T] when counting, T >= 1).
 template <int FMT, int WDT, int PASS>
 __global__ void __launch_bounds__(kIterThreads, 1)
     k_iter(Problem p, int t_first, int t_last, const __grid_constant__ CUtensorMap wmap) {
@@ -1120,8 +1204,6 @@ __global__ void __launch_bounds__(kIterThreads, 1)
   uint64_t* empty = full + kMaxStages;
   int* s_misc = reinterpret_cast<int*>(smem + lay.misc);  // [0] ticket result, [1] #ambiguous
   unsigned* s_cnt = reinterpret_cast<unsigned*>(s_misc + 2);  // [4] exact-path counters
-  int* s_chgs = s_misc + 8;    // [15] strip slot whose column scales changed or were listed
-  int* s_pend = s_misc + 24;   // [15] listed columns per strip slot
   int* s_scan = s_misc + 40;   // [17] schedule scan
   Sched* s_sched = reinterpret_cast<Sched*>(smem + lay.sched);
   f2* ctab = reinterpret_cast<f2*>(smem + lay.ctab);
@@ -1159,6 +1241,13 @@ __global__ void __launch_bounds__(kIterThreads, 1)
       cta_sync_all();  // the schedule of pass t is in shared memory
       const long long ub = s_sched->u_begin, ue = s_sched->u_end;
       const int nact = s_sched->nact, ident = s_sched->ident, v_first = s_sched->v_first;
+      // this lane's block-column of the first segment (read now: the list is
+      // rewritten once the consumers finish the pass)
+      int pf_gl = -1;
+      if (ub < ue) {
+        const int i0 = (int)(ub / p.M) * kBcPerStrip;
+        if (lane < min(kBcPerStrip, nact - i0)) pf_gl = ident ? i0 + lane : s_act[i0 - v_first * kBcPerStrip + lane];
+      }
       for (long long u = ub; u < ue && !stop;) {
         const long long v = u / p.M;
         const long long r0 = u - v * p.M;
@@ -1203,6 +1292,15 @@ __global__ void __launch_bounds__(kIterThreads, 1)
         }
         u = (v + 1) * p.M;
       }
+      // Late passes usually keep the active list of the pass before, and with
+      // it this CTA's range: the first tiles of that range are brought into
+      // L2 now, while the consumers finish this pass, so the next pass's first
+      // copies hit L2 (a hint only: nothing waits on it).
+      if (t < t_last && p.use_tmap && !stop && pf_gl >= 0) {
+        const long long r0 = ub - (ub / p.M) * p.M;
+        const long long r1 = min((long long)p.M, r0 + (ue - ub));
+        for (long long tr = r0, k = 0; tr < r1 && k < S; tr += geo.RW, ++k) tma_prefetch_2d(&wmap, pf_gl * p.G, (int)tr);
+      }
     }
     if (lane == 0) {
       for (int s = 0; s < S && s < issued; ++s) mbar_drain(&full[s], (unsigned)(((issued - 1 - s) / S) & 1));
@@ -1238,16 +1336,20 @@ __global__ void __launch_bounds__(kIterThreads, 1)
   const f2* wtab = ctab + warp * 8 * lpb;  // this warp's column table
 
   for (int t = t_first; t <= t_last; ++t) {
-  const bool strip_wait = exact_listed<FMT, WDT>(p, t, sTd, isT, reinterpret_cast<double*>(acc), &s_misc[0]);
   if (FIN && blockIdx.x == 0) {
     // the MSE of the passes that no grid barrier of the iteration launch summed
     for (int tp = max(1, t - 2); tp <= t - 1; ++tp)
       mse_total(p, mse_bcs(p, tp), p.nb, p.mse + (tp - 1), rscale_d, reinterpret_cast<double*>(acc));
   }
   if (!FIN && blockIdx.x == 0) {
-    // the change flags of pass t + 1 were last read when pass t - 1 began
+    // the change flags of pass t + 1 were last read when pass t - 1 began, and
+    // the strip counters of pass t + 1 were last waited on in pass t - 1
     unsigned* nxt = p.chg + (int64_t)((t + 1) % 3) * p.nb;
     for (int g = threadIdx.x; g < p.nb; g += kConsumers) nxt[g] = 0u;
+    // (four counters per strip and pass parity: arrivals, ambiguous columns,
+    // finalizers done, exact shares done)
+    for (int v = threadIdx.x; v < p.n_strips; v += kConsumers)
+      for (int c = 0; c < 4; ++c) p.strip_counter[(int64_t)(2 * c + ((t + 1) & 1)) * p.n_strips + v] = 0u;
   }
   pass_schedule(p, t, FIN || t == t_first || p.full_passes, s_sched, s_act, s_scan, s_sfirst);
   const long long ub = s_sched->u_begin, ue = s_sched->u_end, L = s_sched->L;
@@ -1272,7 +1374,6 @@ __global__ void __launch_bounds__(kIterThreads, 1)
     const int64_t col = (int64_t)g * p.G + 8 * oct;
 
     consumer_sync(kConsumers);  // the previous segment's readers of acc and the tables are done
-    if (strip_wait && has) wait_bc(p, g);  // listed columns of this block-column settled first
     ColState cs;
     cs.tb = wtab + oct * 4;
     cs.tcb = wtab + 4 * lpb + oct * 4;
@@ -1404,79 +1505,45 @@ __global__ void __launch_bounds__(kIterThreads, 1)
     }
     __threadfence();
     consumer_sync(kConsumers);
+    // The strip's K CTAs have written their partial sums once its first
+    // counter reaches K.  The nfin CTAs whose range ends in this strip (all but
+    // a last one that runs on into the next strip; a lone CTA always) then
+    // share its finalization: each waits (bounded) for the counter, finalizes
+    // its block-columns w = q, q + nfin, ... and counts itself on the second
+    // counter; once that reaches nfin the columns listed as ambiguous are
+    // settled exactly, each finalizer taking a share of the rows.  A CTA that
+    // runs on does not wait here.
     const int64_t k_first = cta_of(v * p.M, Pt, L);
     const int64_t k_last = cta_of((v + 1) * p.M - 1, Pt, L);
-    if (threadIdx.x == 0) {
-      const unsigned prev = atomicAdd(&p.strip_counter[v], 1u);
-      s_misc[0] = prev == (unsigned)(k_last - k_first) ? 1 : 0;
-      s_misc[1] = 0;
-    }
-    if (threadIdx.x < 16) {
-      s_chgs[threadIdx.x] = 0;
-      s_pend[threadIdx.x] = 0;
-    }
-    consumer_sync(kConsumers);
-    if (s_misc[0]) {
-      // last CTA of the strip: column totals in CTA order, certified projection
-      __threadfence();
-      if (p.mode != DQ_MODE_ROW) {  // in the row mode b keeps its values
-        for (int vc = threadIdx.x; vc < width; vc += kConsumers) {
-          double2 tot = make_double2(0.0, 0.0);
-          for (int64_t kb = k_first; kb <= k_last; kb += 8) {  // 8 loads in flight, added in CTA order
-            double2 x[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const int64_t kk = kb + q;
-              x[q] = make_double2(0.0, 0.0);
-              if (kk <= k_last) x[q] = __ldcg(&p.col_part[(kk * p.segmax + (v - s_sfirst[kk])) * p.TSv + vc]);
-            }
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              tot.x += x[q].x;
-              tot.y += x[q].y;
-            }
-          }
-          const int w = vc / p.G;
-          const int64_t j = (int64_t)(ident ? i0 + w : act[i0 + w]) * p.G + (vc - w * p.G);
-          // certified only when the fp32 runs stayed well inside the normal
-          // range (no overflow; underflowed terms negligible); a zero total may
-          // be underflow and is settled exactly as well
-          const bool safe = tot.x >= 0x1p-60 && tot.x <= 0x1p100 && tot.y >= 0x1p-60 && tot.y <= 0x1p100;
-          const double ratio = FMT == FMT_NVFP4 ? (tot.x / tot.y) / sTd : tot.x / tot.y;
-          const double lo = safe ? b_project(ratio * (1.0 - kColErr), p.col_dt) : 0.0;
-          const double hi = safe ? b_project(ratio * (1.0 + kColErr), p.col_dt) : 1.0;
-          if (lo == hi) {
-            if (lo != (double)b_decode_cg(p.b_store, p.col_dt, j)) {
-              b_encode(p.b_store, p.col_dt, j, lo);
-              s_chgs[w] = 1;
-            }
-          } else {
-            // ambiguous: listed for the exact update at the start of the next
-            // pass (exact_listed), which recomputes the column's sums over all
-            // rows and writes its scale (b keeps its value until then); its
-            // block-column stays active in that pass
-            atomicAdd(&s_misc[1], 1);
-            atomicAdd(&s_pend[w], 1);
-            s_chgs[w] = 1;
-            p.amb_list[(int64_t)(t % 3) * p.N + atomicAdd(&p.hdr->amb_n[t % 3], 1u)] = (int)j;
-          }
-        }
-      }
+    const int K = (int)(k_last - k_first + 1);
+    const int64_t par_off = (int64_t)(t & 1) * p.n_strips + v;
+    unsigned* cnt = p.strip_counter + par_off;
+    if (threadIdx.x == 0) atomicAdd(cnt, 1u);
+    const bool ends_here = (v + 1) * p.M >= ue;
+    const bool last_ends = range_begin(k_last + 1, Pt, L) <= (v + 1) * p.M;
+    const int nfin = (K == 1 || last_ends) ? K : K - 1;
+    const int q = (int)(blockIdx.x - k_first);
+    if ((ends_here || K == 1) && q < nfin) {
+      int* amb_list = p.amb_list + v * (int64_t)p.TSv;
+      unsigned* amb_cnt = p.strip_counter + 2 * (int64_t)p.n_strips + par_off;
+      unsigned* cnt2 = p.strip_counter + 4 * (int64_t)p.n_strips + par_off;
+      wait_count(cnt, (unsigned)K, &p.hdr->flags);
       consumer_sync(kConsumers);
-      if (threadIdx.x < nbc) {
-        const int w = threadIdx.x;
-        const int gw = ident ? i0 + w : act[i0 + w];
-        double m = 0.0;  // the block-column's residual total, in CTA order
-        for (int64_t kk = k_first; kk <= k_last; ++kk)
-          m += __ldcg(&p.mse_seg[(kk * p.segmax + (v - s_sfirst[kk])) * kBcPerStrip + w]);
-        mse_bcs(p, t)[gw] = m;
-        if (s_chgs[w]) p.chg[(int64_t)(t % 3) * p.nb + gw] = 1u;
-        if (s_pend[w]) p.pend[gw] = (unsigned)s_pend[w];  // the next pass waits for these
-      }
+      __threadfence();
+      finalize_slots<FMT>(p, t, v, q, nfin, nbc, act, ident, i0, k_first, K, s_sfirst, sTd,
+                          reinterpret_cast<double*>(acc), ctab, amb_list, amb_cnt, &s_misc[8]);
       if (threadIdx.x == 0) {
-        s_cnt[2] += (unsigned)s_misc[1];
-        p.strip_counter[v] = 0u;
+        __threadfence();
+        atomicAdd(cnt2, 1u);
       }
+      wait_count(cnt2, (unsigned)nfin, &p.hdr->flags);
+      if (threadIdx.x == 0) s_misc[1] = (int)ld_acquire_gpu(amb_cnt);
+      consumer_sync(kConsumers);
+      const int n = s_misc[1];
+      if (n > 0)
+        exact_columns<FMT, WDT>(p, v, act, ident, i0, q, nfin, k_first, slot, s_sfirst, amb_list, n,
+                                p.strip_counter + 6 * (int64_t)p.n_strips + par_off, sTd, isT,
+                                reinterpret_cast<double*>(acc), &s_misc[0], s_cnt);
     }
     consumer_sync(kConsumers);
     u = (v + 1) * p.M;

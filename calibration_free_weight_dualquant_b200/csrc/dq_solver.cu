@@ -258,21 +258,20 @@ cudaError_t launch_solve(const Problem& p, int iters, int stats_ctas, cudaStream
 }
 
 // Self-tests of the bounded waits; nothing faults and the context stays
-// usable.  which == 0: block-column 0's pending count is set to 1 and never
-// released, so wait_bc gives up after its time limit.  which == 1: a ring
-// barrier in shared memory that nothing arrives at and no copy completes, so
-// mbar_wait gives up after its time limit.  Both record kFlagTimeout.
+// usable.  which == 0: a strip counter that never reaches its target, so
+// wait_count gives up after its time limit.  which == 1: a ring barrier in
+// shared memory that nothing arrives at and no copy completes, so mbar_wait
+// gives up after its time limit.  Both record kFlagTimeout.
 __global__ void k_wait_selftest(Problem p, int which) {
   __shared__ uint64_t bar;
   if (which == 0) {
     if (threadIdx.x == 0) {
       p.hdr->flags = 0u;
-      p.pend[0] = 1u;
+      p.strip_counter[0] = 0u;
       __threadfence();
     }
     __syncwarp();
-    wait_bc(p, 0);
-    if (threadIdx.x == 0) p.pend[0] = 0u;
+    wait_count(p.strip_counter, 1u, &p.hdr->flags);
   } else {
     if (threadIdx.x == 0) {
       p.hdr->flags = 0u;
@@ -289,7 +288,7 @@ cudaError_t launch_wait_selftest(void* workspace, int which, cudaStream_t st) {
   Problem p;
   std::memset(&p, 0, sizeof(p));
   p.hdr = reinterpret_cast<WsHeader*>(workspace);
-  p.pend = reinterpret_cast<unsigned*>(static_cast<char*>(workspace) + 256);
+  p.strip_counter = reinterpret_cast<unsigned*>(static_cast<char*>(workspace) + 256);
   k_wait_selftest<<<1, 32, 0, st>>>(p, which);
   return cudaGetLastError();
 }
