@@ -72,23 +72,42 @@ def profile_traffic(workload: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 100 ms while running.
+    """SM clocks, power and clock-event (throttle) reasons sampled while the timed region runs.
 
-    Entering starts the sampler and waits (up to 5 s) for its first sample, so
-    the samples cover the timed region that follows."""
+    Samples come from NVML (nvidia-ml-py) every ~2 ms in a background thread, so even a timed
+    region of a few tens of milliseconds carries many samples; where NVML is unavailable,
+    nvidia-smi is polled every 100 ms instead.  Entering waits for the first sample."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits (nvml.h: nvmlClocksEventReason*)
+    REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40}
 
     def __init__(self, device: torch.device):
         try:
-            self.dev = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+            self.uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
         except Exception:
-            self.dev = "0"
+            self.uuid = None
         self.proc = None
+        self.stop = None
+        self.samples = []  # (sm_mhz, max_mhz, reasons set)
         self.lines = []
         self.armed = 0
+        self.source = None
+
+    def _nvml_loop(self, nvml, h):
+        mx = float(nvml.nvmlDeviceGetMaxClockInfo(h, nvml.NVML_CLOCK_SM))
+        get_reasons = getattr(nvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nvml.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self.stop.is_set():
+            try:
+                sm = float(nvml.nvmlDeviceGetClockInfo(h, nvml.NVML_CLOCK_SM))
+                bits = int(get_reasons(h))
+                self.samples.append((sm, mx, {k for k, v in self.REASON_BITS.items() if bits & v}))
+            except Exception:
+                pass
+            time.sleep(0.002)
 
     def _reader(self):
         for line in self.proc.stdout:
@@ -97,13 +116,29 @@ class ClockSampler:
 
     def __enter__(self):
         import threading
+        self.stop = threading.Event()
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.dev, "--query-gpu=" + self.FIELDS,
+            import pynvml as nvml
+            nvml.nvmlInit()
+            h = nvml.nvmlDeviceGetHandleByUUID(self.uuid) if self.uuid else nvml.nvmlDeviceGetHandleByIndex(0)
+            self.thread = threading.Thread(target=self._nvml_loop, args=(nvml, h), daemon=True)
+            self.source = "nvml, 2 ms"
+            self.thread.start()
+            t0 = time.time()
+            while not self.samples and time.time() - t0 < 5.0:
+                time.sleep(0.001)
+            self.armed = len(self.samples)
+            return self
+        except Exception:
+            self.source = None
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.uuid or "0", "--query-gpu=" + self.FIELDS,
                                           "--format=csv,noheader,nounits", "-lms", "100"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
             return self
+        self.source = "nvidia-smi, 100 ms"
         self.thread = threading.Thread(target=self._reader, daemon=True)
         self.thread.start()
         t0 = time.time()
@@ -113,6 +148,11 @@ class ClockSampler:
         return self
 
     def __exit__(self, *a):
+        if self.source and self.source.startswith("nvml"):
+            self.stop.set()
+            self.thread.join(timeout=5)
+            self.samples = self.samples[self.armed:]
+            return
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -121,24 +161,25 @@ class ClockSampler:
                 self.proc.kill()
             self.thread.join(timeout=5)
         self.lines = self.lines[self.armed:]
-
-    def summary(self) -> dict:
-        sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in self.lines:
             parts = [x.strip() for x in line.split(",")]
             if len(parts) < 9:
                 continue
             try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
+                sm, mx = float(parts[1]), float(parts[2])
             except ValueError:
                 continue
-            for nm, v in zip(names, parts[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(nm)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+            self.samples.append((sm, mx, {nm for nm, v in zip(names, parts[5:9]) if v.lower().startswith("active")}))
+
+    def summary(self) -> dict:
+        sm = [x[0] for x in self.samples]
+        reasons = set()
+        for x in self.samples:
+            reasons |= x[2]
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": self.samples[-1][1] if self.samples else None, "reasons": sorted(reasons),
+                "samples": len(sm), "source": self.source}
 
 
 def dist_setup(n_gpus: int):
@@ -413,17 +454,18 @@ def run_dq(args, wl, rank, world, local, dist):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def solve(iters, o=out):
-        binding.dq_solve(Wd, wl.fmt, wl.group, iters, wl.col_dtype, out=o, workspace=ws, stream=stream, check=False)
+    def solve(iters, o=out, full=False):
+        binding.dq_solve(Wd, wl.fmt, wl.group, iters, wl.col_dtype, out=o, workspace=ws, stream=stream, check=False,
+                         full_passes=full)
 
-    def timed(iters, steps, o=out):
+    def timed(iters, steps, o=out, full=False):
         ts = []
         for _ in range(steps):
             flush.fill_(1)
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            solve(iters, o)
+            solve(iters, o, full)
             e1.record(stream)
             e1.synchronize()
             ts.append(e0.elapsed_time(e1))
@@ -445,6 +487,7 @@ def run_dq(args, wl, rank, world, local, dist):
     barrier(dist)
     total_ms = max_over_ranks(sum(step_ms), dist)
     exact_paths = binding.diagnostics(ws, stream)
+    n_active = binding.active_block_columns(ws, stream)
 
     # steady-state iteration time of the dominant kernel (k_iter): (t(T) - t(0)) / T, median of runs
     out0 = binding.alloc_outputs(wl.rows, wl.cols, wl.fmt, wl.group, wl.col_dtype, 0, dev)
@@ -452,6 +495,12 @@ def run_dq(args, wl, rank, world, local, dist):
     tTs = step_ms
     iter_ms = (statistics.median(tTs) - statistics.median(t0s)) / T
     iter_ms = max_over_ranks(iter_ms, dist)
+    # ablation: every iteration over every block-column (no skipping of block-columns at a fixed point)
+    full_ms = None
+    if T > 0:
+        solve(T, full=True)
+        full_ms = (statistics.median(timed(T, max(3, min(args.steps, 5)), full=True)) - statistics.median(t0s)) / T
+        full_ms = max_over_ranks(full_ms, dist)
 
     e2e_line = None
     if not args.no_e2e:
@@ -473,7 +522,16 @@ def run_dq(args, wl, rank, world, local, dist):
         "ms_per_iter": iter_ms,
         "roofline": {"bound": "hbm", "kernel": "k_iter", "achieved": achieved, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
-                     "algorithmic_bytes_per_pass": alg, "passes_per_launch": T, "peak_source": peaks["source"]},
+                     "algorithmic_bytes_per_pass": alg, "passes_per_launch": T, "peak_source": peaks["source"],
+                     "note": "achieved = algorithmic bytes of one BCD iteration (W read once, block scales read "
+                             "and written, column scales) / measured time per iteration; block-columns at a "
+                             "fixed point are skipped and not read, so traffic per iteration is below that"},
+        "work": {"block_columns_processed": n_active, "block_columns_x_iters": T * (wl.cols // wl.group),
+                 "active_fraction": n_active / max(1, T * (wl.cols // wl.group))},
+        "ablation_full_passes": None if full_ms is None else {
+            "ms_per_iter": full_ms, "achieved_gbs": alg / (full_ms * 1e-3) / 1e9,
+            "frac": alg / (full_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+            "note": "same solve with dq_options.full_passes: every iteration processes every block-column"},
         "e2e": e2e_line,
         # per solve: k_stats, k_init, one k_iter for all T iterations, the final k_iter pass
         "gpu_launches": args.steps * (4 if T > 0 else 3),

@@ -22,7 +22,7 @@
 namespace dq {
 
 constexpr int kActThreads = 256;      // 8 warps; a warp covers 256 columns of a row
-constexpr int kActCtasPerSm = 4;
+constexpr int kActCtasPerSm = 2;  // 96 registers: two 256-thread CTAs per SM
 
 struct ActProblem {
   const void* X;
@@ -38,7 +38,8 @@ struct ActProblem {
 };
 
 constexpr int kActChunk = 16;  // rows of a (slab, chunk) unit: several units per resident warp
-constexpr int kActDepth = 4;   // rows whose loads are in flight ahead of the arithmetic
+constexpr int kActDepth = 4;   // rows whose loads are in flight ahead of the arithmetic (quantization pass)
+constexpr int kAmaxDepth = 16; // the same for the amax pass, whose arithmetic is short
 
 // Raw 16 bytes (8 elements) of row r at column col.
 __device__ __forceinline__ uint4 act_raw(const ActProblem& p, int64_t r, int64_t col) {
@@ -71,8 +72,8 @@ __device__ __forceinline__ void act_cols(const ActProblem& p, int64_t col, bool 
 // The (slab, chunk) units of a grid: a warp owns 256 columns of kActChunk
 // consecutive rows at a time; lane l holds columns 8l .. 8l+7.  `f(r, x)` is
 // called for every row with the lane's eight values of X' (active lanes only
-// load; inactive lanes see zeros).  Rows are loaded kActDepth ahead.
-template <int XDT, class F>
+// load; inactive lanes see zeros).  Rows are loaded DEPTH ahead.
+template <int XDT, int DEPTH, class F>
 __device__ __forceinline__ void act_rows(const ActProblem& p, F&& f) {
   const int lane = threadIdx.x & 31;
   const int64_t n_chunks = (p.M + kActChunk - 1) / kActChunk;
@@ -86,15 +87,15 @@ __device__ __forceinline__ void act_rows(const ActProblem& p, F&& f) {
     const int64_t blk = col / p.G;  // the lane's group within a row
     float bcol[8];
     act_cols(p, col, active, bcol);
-    uint4 buf[kActDepth];
+    uint4 buf[DEPTH];
 #pragma unroll
-    for (int k = 0; k < kActDepth; ++k) buf[k] = (active && rb + k < re) ? act_raw(p, rb + k, col) : make_uint4(0, 0, 0, 0);
-    for (int64_t r = rb; r < re; r += kActDepth) {
+    for (int k = 0; k < DEPTH; ++k) buf[k] = (active && rb + k < re) ? act_raw(p, rb + k, col) : make_uint4(0, 0, 0, 0);
+    for (int64_t r = rb; r < re; r += DEPTH) {
 #pragma unroll
-      for (int k = 0; k < kActDepth; ++k) {
+      for (int k = 0; k < DEPTH; ++k) {
         if (r + k >= re) break;  // warp-uniform
         const uint4 v = buf[k];
-        const int64_t rn = r + k + kActDepth;
+        const int64_t rn = r + k + DEPTH;
         if (active && rn < re) buf[k] = act_raw(p, rn, col);
         float x[8];
         act_unpack<XDT>(v, bcol, x);
@@ -106,11 +107,11 @@ __device__ __forceinline__ void act_rows(const ActProblem& p, F&& f) {
 
 // Pass 1 (NVFP4, and the non-finite check for every format): max |x b|.
 template <int XDT>
-__global__ void __launch_bounds__(kActThreads) k_act_amax(ActProblem p) {
+__global__ void __launch_bounds__(kActThreads, kActCtasPerSm) k_act_amax(ActProblem p) {
   const int lane = threadIdx.x & 31;
   float amax = 0.f;
   bool bad = false;
-  act_rows<XDT>(p, [&](int64_t, int64_t, int64_t, bool, const float x[8]) {
+  act_rows<XDT, kAmaxDepth>(p, [&](int64_t, int64_t, int64_t, bool, const float x[8]) {
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
       bad |= !isfinite(x[c]);
@@ -124,7 +125,7 @@ __global__ void __launch_bounds__(kActThreads) k_act_amax(ActProblem p) {
 
 // Pass 2: group scales and codes; a group spans G/8 lanes of a warp.
 template <int FMT, int XDT>
-__global__ void __launch_bounds__(kActThreads) k_act(ActProblem p) {
+__global__ void __launch_bounds__(kActThreads, kActCtasPerSm) k_act(ActProblem p) {
   if (p.hdr->flags & kFlagNonFinite) return;
   const int lane = threadIdx.x & 31;
   float sT = 1.f;
@@ -141,7 +142,7 @@ __global__ void __launch_bounds__(kActThreads) k_act(ActProblem p) {
   const int lpg = p.G / 8;  // lanes per group
   const bool leader = (lane & (lpg - 1)) == 0;
   bool bad = false;
-  act_rows<XDT>(p, [&](int64_t r, int64_t col, int64_t blk, bool active, const float x[8]) {
+  act_rows<XDT, kActDepth>(p, [&](int64_t r, int64_t col, int64_t blk, bool active, const float x[8]) {
     float m = 0.f;
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
@@ -258,6 +259,8 @@ extern "C" int dq_act_quant(const void* X, int x_dtype, int64_t rows, int64_t co
   p.hdr = static_cast<dq::WsHeader*>(workspace);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(workspace, 0, sizeof(dq::WsHeader), st) != cudaSuccess) return DQ_ECUDA;
+  // one resident wave: every CTA of the grid runs at once and loops over the
+  // (slab, chunk) units, so no second wave leaves SMs idle at the tail
   const int64_t units = (int64_t)p.n_slabs * ((rows + dq::kActChunk - 1) / dq::kActChunk);
   const int64_t want = (int64_t)sms * dq::kActCtasPerSm;
   const int ctas = (int)((units + 7) / 8 < want ? (units + 7) / 8 : want);  // one unit per warp at least

@@ -17,7 +17,7 @@ struct Plan {
   int TSv, n_strips, P, segmax, P_final, segmax_final, nb;
   int64_t L;
   size_t smem;  // dynamic shared memory of k_iter
-  size_t off_counters, off_chg, off_col_part, off_cta_part, off_mse_seg, off_mse_bc, off_amb_list, total;
+  size_t off_counters, off_chg, off_col_part, off_cta_part, off_mse_seg, off_mse_bc, off_amb_list, off_a_work, total;
   size_t l1_zero_bytes;  // L1 init: digit counters to zero (start of the col_part region)
   size_t off_l1_tot, off_l1_norm;
 };
@@ -45,7 +45,8 @@ int device_sms(int* sms) {
 }
 
 // Schedule and workspace layout for the current device.
-int make_plan(int64_t M, int64_t N, int group, int init, Plan* pl) {
+int make_plan(int64_t M, int64_t N, int format, int group, int init, Plan* pl) {
+  const int a_bytes = format == DQ_INT4 ? 2 : 1;  // a stored block scale
   int sms = 0;
   int st = device_sms(&sms);
   if (st != DQ_OK) return st;
@@ -106,6 +107,8 @@ int make_plan(int64_t M, int64_t N, int group, int init, Plan* pl) {
   off += align_up(sizeof(double) * 3 * (size_t)pl->nb);
   pl->off_amb_list = off;
   off += align_up(sizeof(int) * (size_t)pl->n_strips * (size_t)pl->TSv);
+  pl->off_a_work = off;
+  off += align_up((size_t)a_bytes * (size_t)pl->nb * (size_t)M);
   pl->total = off;
   return DQ_OK;
 }
@@ -148,7 +151,7 @@ int solve_impl(const void* W, int w_dtype, int64_t rows, int64_t cols, int forma
   if (st != DQ_OK) return st;
   if (!workspace || !aligned(workspace, kAlign)) return DQ_EINVAL;
   Plan pl;
-  st = make_plan(rows, cols, group, init, &pl);
+  st = make_plan(rows, cols, format, group, init, &pl);
   if (st != DQ_OK) return st;
   if (workspace_bytes < pl.total) return DQ_EWORKSPACE;
 
@@ -190,6 +193,7 @@ int solve_impl(const void* W, int w_dtype, int64_t rows, int64_t cols, int forma
   p.mse_seg = reinterpret_cast<double*>(ws + pl.off_mse_seg);
   p.mse_bc = reinterpret_cast<double*>(ws + pl.off_mse_bc);
   p.amb_list = reinterpret_cast<int*>(ws + pl.off_amb_list);
+  p.a_work = ws + pl.off_a_work;
 
   // header, strip arrival counters and change flags start at zero; the
   // partial buffers need no init
@@ -218,14 +222,14 @@ extern "C" {
 size_t dq_workspace_bytes(int64_t rows, int64_t cols, int format, int group) {
   if (check_shape(rows, cols, format, group) != DQ_OK) return 0;
   Plan pl;
-  if (make_plan(rows, cols, group, DQ_INIT_RTN, &pl) != DQ_OK) return 0;
+  if (make_plan(rows, cols, format, group, DQ_INIT_RTN, &pl) != DQ_OK) return 0;
   return pl.total;
 }
 
 size_t dq_workspace_bytes_ex(int64_t rows, int64_t cols, int format, int group, const dq_options* options) {
   if (check_shape(rows, cols, format, group) != DQ_OK) return 0;
   Plan pl;
-  if (make_plan(rows, cols, group, options ? options->init : DQ_INIT_RTN, &pl) != DQ_OK) return 0;
+  if (make_plan(rows, cols, format, group, options ? options->init : DQ_INIT_RTN, &pl) != DQ_OK) return 0;
   return pl.total;
 }
 
@@ -385,7 +389,7 @@ int dq_solve_batched(const dq_matrix* mats, int count, int format, int group, in
     if (st == DQ_OK) st = check_outputs(&m.out, format, col_dtype);
     if (st == DQ_OK) {
       Plan pl;
-      st = make_plan(m.rows, m.cols, group, DQ_INIT_RTN, &pl);
+      st = make_plan(m.rows, m.cols, format, group, DQ_INIT_RTN, &pl);
       if (st == DQ_OK && workspace_bytes < pl.total) st = DQ_EWORKSPACE;
     }
     if (st != DQ_OK) {

@@ -253,6 +253,17 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const void* map, int x, i
       : "memory");
 }
 
+// Tiled tensor copy (TMA) of the box at (x, y, z) of the 3-D tensor map `map`
+// into this CTA's shared memory, completing on `bar`; x times the element size
+// must be a multiple of 16 bytes.
+__device__ __forceinline__ void tma_load_3d(void* dst, const void* map, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+          smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // L2 prefetch of the box at (x = column, y = row) of the 2-D tensor map `map`
 // (no shared memory written, no completion to wait for).
 __device__ __forceinline__ void tma_prefetch_2d(const void* map, int x, int y) {

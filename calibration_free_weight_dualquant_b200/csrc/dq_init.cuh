@@ -200,13 +200,18 @@ __global__ void __launch_bounds__(kThreads) k_check_given(Problem p) {
     }
     p.hdr->sT = s;
   }
+  // the given block scales, checked and copied into the block-column-major
+  // working copy the iterations use
   for (int64_t k = tid; k < p.M * p.nb; k += stride) {
+    const int64_t i = k / p.nb, g = k - i * p.nb;
     if (FMT == FMT_INT4) {
-      const uint32_t h = reinterpret_cast<const unsigned short*>(p.a_store)[k];
+      const unsigned short h = reinterpret_cast<const unsigned short*>(p.a_store)[k];
       bad = bad || h == 0u || h > 0x7BFFu;
+      reinterpret_cast<unsigned short*>(p.a_work)[g * p.M + i] = h;
     } else {
-      const uint32_t v = reinterpret_cast<const uint8_t*>(p.a_store)[k];
+      const uint8_t v = reinterpret_cast<const uint8_t*>(p.a_store)[k];
       bad = bad || v == 0u || v > (fmt_pow2(FMT) ? 253u : 0x7Eu);
+      reinterpret_cast<uint8_t*>(p.a_work)[g * p.M + i] = v;
     }
   }
   for (int64_t j = tid; j < p.N; j += stride) {

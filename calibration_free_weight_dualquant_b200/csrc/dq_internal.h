@@ -130,7 +130,8 @@ struct Problem {
   int segmax_final;
   int64_t L;     // n_strips * M (strip-major row units of a full pass)
   void* codes;
-  void* a_store;
+  void* a_store;   // output block scales [M][nb] (storage format), written by the final pass
+  void* a_work;    // working block scales [nb][M] (storage format): a block-column's rows contiguous
   void* b_store;
   float* sT_out;
   double* mse;
@@ -144,6 +145,7 @@ struct Problem {
   double* mse_bc;           // [3][nb] residual total per block-column, by pass mod 3
   unsigned* chg;            // [3][nb] a scale of the block-column changed (or was listed), by pass mod 3 (zeroed)
   int use_tmap;             // W streamed by 2-D tensor copies (else one bulk copy per row)
+  int use_tmap3;            // a strip of consecutive block-columns streamed by one 3-D tensor copy per tile
   int mode;                 // DQ_MODE_DUAL, DQ_MODE_ROW (b keeps its initial value) or DQ_MODE_COL
   int init;                 // DQ_INIT_RTN, DQ_INIT_L1 or DQ_INIT_GIVEN
   int full_passes;          // every BCD pass takes every block-column (no skipping at fixed points)

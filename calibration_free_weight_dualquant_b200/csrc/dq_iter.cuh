@@ -157,6 +157,16 @@ __device__ __forceinline__ float b_decode_cg(const void* store, int col_dt, int6
   return col_dt == DT_F16 ? __half2float(__ushort_as_half(h)) : __uint_as_float((uint32_t)h << 16);
 }
 
+// Stores a block scale in its storage format from its stored bits.
+template <int FMT>
+__device__ __forceinline__ void a_put_raw(void* store, int64_t idx, uint32_t raw) {
+  if (FMT == FMT_INT4) {
+    reinterpret_cast<unsigned short*>(store)[idx] = (unsigned short)raw;
+  } else {
+    reinterpret_cast<uint8_t*>(store)[idx] = (uint8_t)raw;
+  }
+}
+
 // the stored form of the factor 1 (fp16 1.0, 2^0, E4M3 1.0)
 template <int FMT>
 __device__ __forceinline__ constexpr uint32_t a_raw_one() {
@@ -700,8 +710,8 @@ __device__ __forceinline__ void row_pair(const Problem& p, const f2 wx[4], float
   // codes are unchanged too (same a, same b), so requantize only where it changed
   const bool chx = anx != ax_old && actx, chy = any != ay_old && acty;
   achg = achg || chx || chy;
-  if (chx && leader) a_store_f<FMT>(p.a_store, bidx_x, anx);
-  if (chy && leader) a_store_f<FMT>(p.a_store, bidx_y, any);
+  if (chx && leader) a_store_f<FMT>(p.a_work, bidx_x, anx);
+  if (chy && leader) a_store_f<FMT>(p.a_work, bidx_y, any);
   if (__any_sync(0xffffffffu, chx || chy)) {
     // recomputed rather than kept live across the block update (registers)
 #pragma unroll
@@ -846,47 +856,27 @@ __device__ void grid_sync_plain(WsHeader* hdr) {
 
 constexpr int kXRows = 8;
 
-// Fixed-order sum of one value per consumer thread (xor trees within the warps,
-// then the warp totals in warp order); the total is in red[0] afterwards.
-__device__ __forceinline__ void consumer_sum2(double x, double y, double* red) {
-  for (int o = 16; o > 0; o >>= 1) {
-    x += __shfl_xor_sync(0xffffffffu, x, o);
-    y += __shfl_xor_sync(0xffffffffu, y, o);
-  }
-  const int warp = threadIdx.x >> 5;
-  if ((threadIdx.x & 31) == 0) {
-    red[2 + 2 * warp] = x;
-    red[3 + 2 * warp] = y;
-  }
-  consumer_sync(kConsumers);
-  if (threadIdx.x == 0) {
-    double sx = 0.0, sy = 0.0;
-    for (int w = 0; w < kConsumerWarps; ++w) {
-      sx += red[2 + 2 * w];
-      sy += red[3 + 2 * w];
-    }
-    red[0] = sx;
-    red[1] = sy;
-  }
-}
-
-// Exact column sums: fp64 sums of W a q and (a q)^2 of column j over rows
-// [i_begin, i_end), with q decided exactly (every load of a round issued before
-// any is used); the totals go to scratch[0], [1] (thread 0; the caller
-// synchronizes before others read them).  Used for a column whose certified
-// projection is ambiguous.
+// Exact column sums by one warp of a group of `nw` warps sharing the column:
+// fp64 sums of W a q and (a q)^2 of column j over rows i_begin + 32 wi + lane,
+// + 32 nw, ... below i_end (wi: the warp's index in the group; 8 loads in
+// flight each), with q decided exactly, added over the lanes in a fixed xor
+// tree; every lane returns the warp's totals.
 template <int FMT, int WDT>
-__device__ void column_rows_exact(const Problem& p, int64_t j, int64_t i_begin, int64_t i_end, double sTd, float isT,
-                                  double* scratch) {
+__device__ double2 column_rows_exact_warp(const Problem& p, int64_t j, int64_t i_begin, int64_t i_end, int wi, int nw,
+                                          double sTd, float isT) {
+  const int lane = threadIdx.x & 31;
+  const int64_t step = (int64_t)32 * nw;
   const unsigned short braw = __ldcg(reinterpret_cast<const unsigned short*>(p.b_store) + j);
+  const float bj = p.col_dt == DT_F16 ? __half2float(__ushort_as_half(braw)) : __uint_as_float((uint32_t)braw << 16);
+  const float cb = __frcp_rn(bj) * isT;
   const int64_t jb = j / p.G;  // block column
   double cn = 0.0, cd = 0.0;
-  for (int64_t i0 = i_begin + threadIdx.x; i0 < i_end; i0 += (int64_t)kXRows * kConsumers) {
+  for (int64_t i0 = i_begin + 32 * wi + lane; i0 < i_end; i0 += (int64_t)kXRows * step) {
     float w[kXRows];
     uint32_t araw[kXRows];
 #pragma unroll
     for (int k = 0; k < kXRows; ++k) {
-      const int64_t i = i0 + (int64_t)k * kConsumers;
+      const int64_t i = i0 + (int64_t)k * step;
       w[k] = 0.f;
       araw[k] = a_raw_one<FMT>();
       if (i < i_end) {
@@ -898,11 +888,9 @@ __device__ void column_rows_exact(const Problem& p, int64_t j, int64_t i_begin, 
         } else {
           w[k] = __half2float(__ushort_as_half(__ldg(reinterpret_cast<const unsigned short*>(p.W) + e)));
         }
-        araw[k] = a_fetch<FMT>(p.a_store, i * p.nb + jb);
+        araw[k] = a_fetch<FMT>(p.a_work, jb * p.M + i);
       }
     }
-    const float bj = p.col_dt == DT_F16 ? __half2float(__ushort_as_half(braw)) : __uint_as_float((uint32_t)braw << 16);
-    const float cb = __frcp_rn(bj) * isT;
 #pragma unroll
     for (int k = 0; k < kXRows; ++k) {  // absent rows hold w = 0, which adds nothing
       const float a = a_dec<FMT>(araw[k]);
@@ -914,7 +902,11 @@ __device__ void column_rows_exact(const Problem& p, int64_t j, int64_t i_begin, 
       cd = fma(sv, sv, cd);
     }
   }
-  consumer_sum2(cn, cd, scratch);
+  for (int o = 16; o > 0; o >>= 1) {
+    cn += __shfl_xor_sync(0xffffffffu, cn, o);
+    cd += __shfl_xor_sync(0xffffffffu, cd, o);
+  }
+  return make_double2(cn, cd);
 }
 
 // Bounded wait of thread 0 until *c reaches `target` (ld.acquire; gives up
@@ -1053,13 +1045,35 @@ __device__ void exact_columns(const Problem& p, int64_t v, const int* act, bool 
                               unsigned* ticket, double sTd, float isT, double* red, int* s_flag, unsigned* s_cnt) {
   const int G = p.G;
   const int64_t lo = (int64_t)q * p.M / nfin, hi = (int64_t)(q + 1) * p.M / nfin;
-  for (int i = 0; i < n; ++i) {
-    const int vc = __ldcg(amb_list + i);
-    const int w = vc / G;
-    const int64_t j = (int64_t)(ident ? i0_strip + w : act[i0_strip + w]) * G + (vc - w * G);
-    column_rows_exact<FMT, WDT>(p, j, lo, hi, sTd, isT, red);
-    if (threadIdx.x == 0) p.col_part[myslot * p.TSv + vc] = make_double2(red[0], red[1]);
-    consumer_sync(kConsumers);  // red is reused
+  // the 15 warps are shared evenly by the listed columns (all of them on one
+  // column when it is the only one), so each column's rows take about one
+  // round of loads; the warps' sums of a column are added in warp order
+  const int warp = threadIdx.x >> 5;
+  const int wpc = max(1, kConsumerWarps / n);     // warps per column
+  const int ncw = kConsumerWarps / wpc;           // columns handled at once
+  double2* wsum = reinterpret_cast<double2*>(red);  // [kConsumerWarps]
+  for (int i0 = 0; i0 < n; i0 += ncw) {
+    const int i = i0 + warp / wpc, wi = warp % wpc;
+    const bool mine = warp < ncw * wpc && i < n;
+    double2 s2 = make_double2(0.0, 0.0);
+    int vc = 0;
+    if (mine) {
+      vc = __ldcg(amb_list + i);
+      const int w = vc / G;
+      const int64_t j = (int64_t)(ident ? i0_strip + w : act[i0_strip + w]) * G + (vc - w * G);
+      s2 = column_rows_exact_warp<FMT, WDT>(p, j, lo, hi, wi, wpc, sTd, isT);
+    }
+    if ((threadIdx.x & 31) == 0) wsum[warp] = s2;
+    consumer_sync(kConsumers);
+    if (mine && wi == 0 && (threadIdx.x & 31) == 0) {
+      double2 tot = wsum[warp];
+      for (int k = 1; k < wpc; ++k) {
+        tot.x += wsum[warp + k].x;
+        tot.y += wsum[warp + k].y;
+      }
+      p.col_part[myslot * p.TSv + vc] = tot;
+    }
+    consumer_sync(kConsumers);  // wsum is reused
   }
   if (threadIdx.x == 0) {
     __threadfence();
@@ -1099,29 +1113,38 @@ __device__ void exact_columns(const Problem& p, int64_t v, const int* act, bool 
   if (threadIdx.x == 0) s_cnt[2] += (unsigned)n;
 }
 
+// True when a strip's nbc block-columns g_first .. g_last are consecutive and
+// W has the 3-D tensor map: then one tensor copy brings a whole tile.
+__device__ __forceinline__ bool strip_contiguous(const Problem& p, bool ident, int g_first, int g_last, int nbc) {
+  return p.use_tmap3 && (ident || g_last - g_first == nbc - 1);
+}
+
 // Named barrier of the whole CTA (consumers and producer): the schedule of a
 // pass is handed to the producer through it.
 __device__ __forceinline__ void cta_sync_all() { asm volatile("bar.sync 2, %0;" ::"r"(kIterThreads) : "memory"); }
 
 // Schedule of pass t, computed by the consumer threads of every CTA from the
 // same flags (so every CTA finds the same strips and ranges): the active
-// block-columns, this CTA's units, the first strip of every CTA's range (the
-// strip finalizers index partial sums by it) and this CTA's slice of the
-// active list.  With `ident` (the first BCD pass and the final pass) every
+// block-columns, this CTA's units and this CTA's slice of the active list.  With `ident` (the first BCD pass and the final pass) every
 // block-column is active.  Otherwise the active ones are those whose scales
 // changed in pass t - 1 (p.chg of pass t - 1, complete after the grid barrier
 // that ended it): a block-column with no change is at a fixed point, and its
 // residual total is carried into this pass's buffer.  `s_scan` holds 17 ints.
-__device__ void pass_schedule(const Problem& p, int t, bool ident, Sched* sc, int* s_act, int* s_scan, int* s_sfirst) {
+__device__ void pass_schedule(const Problem& p, int t, bool ident, Sched* sc, int* s_act, int* s_scan) {
   const int nb = p.nb;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const unsigned* flags = p.chg + (int64_t)((t - 1) % 3) * nb;
   const int per = (nb + kConsumers - 1) / kConsumers;
   const int c0 = min(nb, tid * per), c1 = min(nb, c0 + per);
   int nact = nb, excl = 0;
+  uint32_t mask = 0u;  // this thread's flags (per <= 32)
   if (!ident) {
     int cnt = 0;
-    for (int g = c0; g < c1; ++g) cnt += __ldcg(flags + g) != 0u;
+    for (int g = c0; g < c1; ++g) {
+      const bool f = __ldcg(flags + g) != 0u;
+      cnt += f;
+      if (per <= 32) mask |= (uint32_t)f << (g - c0);
+    }
     int incl = cnt;
     for (int o = 1; o < 32; o <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, incl, o);
@@ -1157,7 +1180,7 @@ __device__ void pass_schedule(const Problem& p, int t, bool ident, Sched* sc, in
     const double* prev = mse_bcs(p, t - 1);
     int idx = excl;
     for (int g = c0; g < c1; ++g) {
-      if (__ldcg(flags + g) != 0u) {
+      if (per <= 32 ? ((mask >> (g - c0)) & 1u) != 0u : __ldcg(flags + g) != 0u) {
         if (idx >= lo && idx < hi) s_act[idx - lo] = g;
         ++idx;
       } else if (g % (int)gridDim.x == k) {
@@ -1165,7 +1188,6 @@ __device__ void pass_schedule(const Problem& p, int t, bool ident, Sched* sc, in
       }
     }
   }
-  for (int kk = tid; kk < Pt; kk += kConsumers) s_sfirst[kk] = (int)(range_begin(kk, Pt, L) / p.M);
   if (tid == 0) {
     sc->L = L;
     sc->u_begin = ub;
@@ -1190,7 +1212,8 @@ __device__ void pass_schedule(const Problem& p, int t, bool ident, Sched* sc, in
 // and mse[T] (and changes[T] when counting, T >= 1).
 template <int FMT, int WDT, int PASS>
 __global__ void __launch_bounds__(kIterThreads, 1)
-    k_iter(Problem p, int t_first, int t_last, const __grid_constant__ CUtensorMap wmap) {
+    k_iter(Problem p, int t_first, int t_last, const __grid_constant__ CUtensorMap wmap,
+           const __grid_constant__ CUtensorMap wmap3) {
   constexpr int ES = WDT == DT_F32 ? 4 : 2;
   constexpr bool FIN = PASS == PASS_FINAL;
   const TileGeo geo = tile_geo(p.G, ES);
@@ -1256,6 +1279,8 @@ __global__ void __launch_bounds__(kIterThreads, 1)
         const int nbc = min(kBcPerStrip, nact - i0);
         const int* act = s_act - (long long)v_first * kBcPerStrip;
         const int gl = lane < nbc ? (ident ? i0 + lane : act[i0 + lane]) : 0;
+        const int g_first = __shfl_sync(0xffffffffu, gl, 0), g_last = __shfl_sync(0xffffffffu, gl, nbc - 1);
+        const bool wide = strip_contiguous(p, ident, g_first, g_last, nbc);
         for (long long tr = r0; tr < r1; tr += geo.RW) {
           if (ld_volatile(&p.hdr->flags) & kFlagTimeout) {
             stop = true;
@@ -1266,7 +1291,12 @@ __global__ void __launch_bounds__(kIterThreads, 1)
             break;
           }
           unsigned char* slot = ring + st * geo.stage_bytes;
-          if (p.use_tmap) {
+          if (wide) {  // the strip's block-columns are consecutive: one copy, [rows][15][G]
+            if (lane == 0) {
+              mbar_arrive_expect_tx(&full[st], (unsigned)(kBcPerStrip * geo.box_bytes));
+              tma_load_3d(slot, &wmap3, 0, g_first, (int)tr, &full[st]);
+            }
+          } else if (p.use_tmap) {  // one copy per block-column, [15][rows][G]
             if (lane == 0) mbar_arrive_expect_tx(&full[st], (unsigned)(nbc * geo.box_bytes));
             __syncwarp();
             if (lane < nbc) tma_load_2d(slot + lane * geo.box_stride, &wmap, gl * p.G, (int)tr, &full[st]);
@@ -1351,7 +1381,7 @@ __global__ void __launch_bounds__(kIterThreads, 1)
     for (int v = threadIdx.x; v < p.n_strips; v += kConsumers)
       for (int c = 0; c < 4; ++c) p.strip_counter[(int64_t)(2 * c + ((t + 1) & 1)) * p.n_strips + v] = 0u;
   }
-  pass_schedule(p, t, FIN || t == t_first || p.full_passes, s_sched, s_act, s_scan, s_sfirst);
+  pass_schedule(p, t, FIN || t == t_first || p.full_passes, s_sched, s_act, s_scan);
   const long long ub = s_sched->u_begin, ue = s_sched->u_end, L = s_sched->L;
   const int nact = s_sched->nact, Pt = s_sched->Pt, v_first = s_sched->v_first;
   const bool ident = s_sched->ident != 0;
@@ -1411,24 +1441,30 @@ __global__ void __launch_bounds__(kIterThreads, 1)
     __syncwarp();  // the warp's column table is written
     bool achg = false;
     int run = 0;
-    // block scales of this lane's rows, one tile ahead
-    const int64_t a_step = (int64_t)RW * p.nb;
-    int64_t aidx = (r0 + rho) * p.nb + g;
-    const int64_t y_off = (int64_t)rl * p.nb;  // block-scale offset of the lane's second row
+    // block scales of this lane's rows (the block-column-major working copy:
+    // a warp's rows are contiguous), one tile ahead
+    const int64_t a_step = RW;
+    int64_t aidx = (int64_t)g * p.M + r0 + rho;
+    const int64_t y_off = rl;  // block-scale offset of the lane's second row
     // rows relative to the segment start, in 32 bits (a segment has fewer than 2^31 rows)
     const int nrows = (int)(r1 - r0);
     uint32_t an0 = a_raw_one<FMT>(), an1 = a_raw_one<FMT>();
-    if (has && rho < nrows) an0 = a_fetch<FMT>(p.a_store, aidx);
-    if (has && rho + rl < nrows) an1 = a_fetch<FMT>(p.a_store, aidx + y_off);
-    const unsigned char* wbase = ring + warp * geo.box_stride + (rho * p.G + 8 * oct) * ES;
-    const int y_bytes = rl * p.G * ES;
+    if (has && rho < nrows) an0 = a_fetch<FMT>(p.a_work, aidx);
+    if (has && rho + rl < nrows) an1 = a_fetch<FMT>(p.a_work, aidx + y_off);
+    // the tile's layout: [rows][15][G] (one copy of a strip of consecutive
+    // block-columns) or [15][rows][G] (one copy per block-column)
+    const bool wide = strip_contiguous(p, ident, ident ? i0 : act[i0], ident ? i0 + nbc - 1 : act[i0 + nbc - 1], nbc);
+    const int row_stride = (wide ? kBcPerStrip : 1) * p.G * ES;
+    const int slot_stride = wide ? p.G * ES : geo.box_stride;
+    const unsigned char* wbase = ring + warp * slot_stride + rho * row_stride + 8 * oct * ES;
+    const int y_bytes = rl * row_stride;
 
     for (int tr = 0; tr < nrows; tr += RW, aidx += a_step) {
       const int ra = tr + rho, rb = ra + rl;
       const bool vx = has && ra < nrows, vy = has && rb < nrows;  // per lane
       const uint32_t ra_raw = an0, rb_raw = an1;
-      if (has && ra + RW < nrows) an0 = a_fetch<FMT>(p.a_store, aidx + a_step);
-      if (has && rb + RW < nrows) an1 = a_fetch<FMT>(p.a_store, aidx + a_step + y_off);
+      if (has && ra + RW < nrows) an0 = a_fetch<FMT>(p.a_work, aidx + a_step);
+      if (has && rb + RW < nrows) an1 = a_fetch<FMT>(p.a_work, aidx + a_step + y_off);
       const int64_t cix = ((r0 + ra) * p.N + col) >> 3;  // code group of row ra, this lane's 8 columns
       uint2 oldx = make_uint2(0u, 0u), oldy = make_uint2(0u, 0u);
       if (PASS != PASS_ITER && cmp) {  // issued before the wait: the latency hides behind it
@@ -1462,6 +1498,11 @@ __global__ void __launch_bounds__(kIterThreads, 1)
         if (FIN) {
           final_pair<FMT>(p, wa, aa, wb, ab, vx, vy, cs, sT, sTd, scaled, rscale2, s_cnt, tcnt, cix, code_step, oldx,
                           oldy, cmp, nchg);
+          // the final block scales, in the output's row-major layout
+          if (leader) {
+            if (vx) a_put_raw<FMT>(p.a_store, (r0 + ra) * p.nb + g, ra_raw);
+            if (vy) a_put_raw<FMT>(p.a_store, (r0 + rb) * p.nb + g, rb_raw);
+          }
         } else {
           row_pair<FMT, PASS>(p, wa, aa, aidx, wb, ab, aidx + y_off, vx, vy, leader, lpb, cs, sT, isT, sTd, scaled,
                               rscale2, s_cnt, tcnt, cix, code_step, oldx, oldy, cmp, nchg, achg);
@@ -1527,6 +1568,10 @@ __global__ void __launch_bounds__(kIterThreads, 1)
       int* amb_list = p.amb_list + v * (int64_t)p.TSv;
       unsigned* amb_cnt = p.strip_counter + 2 * (int64_t)p.n_strips + par_off;
       unsigned* cnt2 = p.strip_counter + 4 * (int64_t)p.n_strips + par_off;
+      // the first strip of each of the strip's CTAs (their partial slots are
+      // indexed by it)
+      for (int e = threadIdx.x; e < K; e += kConsumers)
+        s_sfirst[k_first + e] = (int)(range_begin(k_first + e, Pt, L) / p.M);
       wait_count(cnt, (unsigned)K, &p.hdr->flags);
       consumer_sync(kConsumers);
       __threadfence();

@@ -119,7 +119,7 @@ __global__ void __launch_bounds__(kThreads) k_init(Problem p) {
       m = (double)mf;
     }
     const double a = (m == 0.0) ? 1.0 : a_project<FMT>(m / qmax, sTd);
-    a_encode<FMT>(p.a_store, blk, a);
+    a_encode<FMT>(p.a_work, g * p.M + i, a);
   }
   if (!l1)
     for (int64_t j = (int64_t)blockIdx.x * kThreads + threadIdx.x; j < p.N; j += stride)
@@ -165,6 +165,32 @@ static bool encode_w_map(const Problem& p, CUtensorMap* map) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D view of W, (G columns, nb block-columns, M rows) with strides (1, G, N)
+// elements, whose box is a whole strip's share of a ring tile: G x 15 x
+// 2 * 32/(G/8).  It lands as [rows][15][G], row-major over the strip, when the
+// strip's block-columns are consecutive.  Returns false when W cannot be
+// described (then every tile takes one copy per block-column).
+template <int WDT>
+static bool encode_w_map3(const Problem& p, CUtensorMap* map) {
+  constexpr int ES = WDT == DT_F32 ? 4 : 2;
+  std::memset(map, 0, sizeof(*map));
+  if (p.M > INT_MAX || p.nb > INT_MAX || (p.N * ES) % 16 != 0 || (p.G * ES) % 16 != 0) return false;
+  const TileGeo geo = tile_geo(p.G, ES);
+  if (geo.box_stride != geo.box_bytes) return false;  // the slot layout must be dense
+  const PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)p.G, (cuuint64_t)p.nb, (cuuint64_t)p.M};
+  const cuuint64_t strides[2] = {(cuuint64_t)p.G * ES, (cuuint64_t)p.N * ES};
+  const cuuint32_t box[3] = {(cuuint32_t)p.G, (cuuint32_t)kBcPerStrip, (cuuint32_t)geo.RW};
+  const cuuint32_t elem_strides[3] = {1, 1, 1};
+  const CUtensorMapDataType dt = WDT == DT_F32    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                 : WDT == DT_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                  : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  return fn(map, dt, 3, const_cast<void*>(p.W), dims, strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Launch of k_iter: cooperative (all CTAs resident at once, for its grid
 // barrier) and with programmatic stream serialization (the grid may start while
 // the one before it in the stream finishes; the kernel waits, griddep_wait,
@@ -203,9 +229,10 @@ static cudaError_t run_typed(const Problem& p, int iters, int stats_ctas, cudaSt
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(k_iter<FMT, WDT, PASS_FINAL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  CUtensorMap wmap;
+  CUtensorMap wmap, wmap3;
   Problem pi = p;
   pi.use_tmap = encode_w_map<WDT>(p, &wmap) ? 1 : 0;
+  pi.use_tmap3 = pi.use_tmap && encode_w_map3<WDT>(p, &wmap3) ? 1 : 0;
   Problem pf = p;
   pf.P = p.P_final;
   pf.segmax = p.segmax_final;
@@ -229,10 +256,11 @@ static cudaError_t run_typed(const Problem& p, int iters, int stats_ctas, cudaSt
   }
   // all BCD iterations in one persistent launch, then the final pass
   if (iters > 0) {
-    e = launch_coop(iter_kernel, (unsigned)p.P, kIterThreads, smem, st, pi, 1, iters, wmap);
+    e = launch_coop(iter_kernel, (unsigned)p.P, kIterThreads, smem, st, pi, 1, iters, wmap, wmap3);
     if (e != cudaSuccess) return e;
   }
-  e = launch_coop(k_iter<FMT, WDT, PASS_FINAL>, (unsigned)p.P, kIterThreads, smem, st, pi, iters + 1, iters + 1, wmap);
+  e = launch_coop(k_iter<FMT, WDT, PASS_FINAL>, (unsigned)p.P, kIterThreads, smem, st, pi, iters + 1, iters + 1, wmap,
+                  wmap3);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
