@@ -63,43 +63,6 @@ struct Sched {
 };
 
 // ---------------------------------------------------------------------------
-// Packed f32x2 arithmetic (one instruction for a pair of elements).
-typedef unsigned long long f2;
-__device__ __forceinline__ f2 pk(float lo, float hi) {
-  f2 r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ float lo_of(f2 v) {
-  float a, b;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
-  (void)b;
-  return a;
-}
-__device__ __forceinline__ float hi_of(f2 v) {
-  float a, b;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
-  (void)a;
-  return b;
-}
-__device__ __forceinline__ f2 mul2(f2 a, f2 b) {
-  f2 d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
-  f2 d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-__device__ __forceinline__ f2 add2(f2 a, f2 b) {
-  f2 d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ f2 splat(float v) { return pk(v, v); }
-
-// ---------------------------------------------------------------------------
 // E2M1 conversions (round to nearest even, saturating) and decode.
 __device__ __forceinline__ uint32_t cvt_e2m1x2(float hi, float lo) {
   uint32_t r;

@@ -37,17 +37,34 @@ def run_both(X: torch.Tensor, b: torch.Tensor, fmt: str, group: int, label: str)
     return gpu, orc
 
 
-@pytest.mark.parametrize("fmt,group", [("nvfp4", 16), ("mxint4", 32), ("int4", 64), ("int4", 128), ("mxfp4", 32)])
-@pytest.mark.parametrize("tokens,cols,xdt,bdt", [
+_FMTS = [("nvfp4", 16), ("mxint4", 32), ("mxfp4", 32), ("int4", 8), ("int4", 16), ("int4", 32), ("int4", 64),
+         ("int4", 128), ("int4", 256)]
+_SHAPES = [
     (1, 256, torch.bfloat16, torch.bfloat16),
     (37, 4096, torch.bfloat16, torch.bfloat16),
     (129, 1536 + 256, torch.float16, torch.bfloat16),
     (64, 768, torch.bfloat16, torch.float16),
-])
+    (5, 1152, torch.bfloat16, torch.bfloat16),      # rows not a multiple of an item's rows; a partial slab
+    (1030, 1152, torch.float16, torch.float16),     # warp ranges that cross slab boundaries
+    (3, 1024 + 64, torch.bfloat16, torch.bfloat16),  # one lane-group past the last whole slab
+]
+
+
+@pytest.mark.parametrize("fmt,group,tokens,cols,xdt,bdt",
+                         [f + s for f in _FMTS for s in _SHAPES if s[1] % f[1] == 0])
 def test_act_parity(fmt, group, tokens, cols, xdt, bdt):
     X = synth.make_activations(tokens, cols, seed=tokens * 31 + cols).to(xdt)
     b = synth.make_col_scales(cols, seed=cols).to(bdt)
     run_both(X, b, fmt, group, "act")
+
+
+@pytest.mark.parametrize("fmt,group,tokens,cols", [("nvfp4", 16, 8192, 4096), ("mxint4", 32, 8192, 14336),
+                                                     ("int4", 64, 8192, 4096)])
+def test_act_full_size(fmt, group, tokens, cols):
+    """The prefill batches that the benchmark times (same shapes, seeds and launch), every output checked."""
+    X = synth.make_activations(tokens, cols, seed=77)
+    b = synth.make_col_scales(cols, seed=78)
+    run_both(X, b, fmt, group, "full-size act")
 
 
 @pytest.mark.parametrize("fmt", ["nvfp4", "mxint4", "int4", "mxfp4"])
