@@ -4,7 +4,8 @@
 
 A step is one full solve (RTN init, all BCD iterations, final codes and MSE) of
 the workload's synthetic matrix, already resident in HBM.  L2 is flushed
-(a 512 MB write) before every step, outside the timed events.  With N > 1
+(a 512 MB write, then a 512 MB read so that no dirty line is left to write
+back) before every step, outside the timed events.  With N > 1
 (torchrun) every rank solves its own replica of the workload (no data-path
 collective: the solver does not shard) and the value is the sum over ranks
 divided by the slowest rank's time.  Rank 0 prints one JSON line.
@@ -32,6 +33,20 @@ DEFAULT_WORKLOAD = "nvfp4_g16_gateup_14336x4096"
 METRIC = "weight-elems x BCD-iters/sec"
 UNIT = "elem*iter/s"
 L2_FLUSH_BYTES = 512 << 20
+
+
+class L2Flush:
+    """Empties L2 between timed steps: a 512 MB write (every line of L2 replaced), then a 512 MB read of a
+    second buffer, so that the dirty lines of the write are written back here, untimed, instead of during
+    the next timed step."""
+
+    def __init__(self, dev):
+        self.w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        self.r = torch.ones(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def __call__(self):
+        self.w.fill_(1)
+        self.sink = self.r.amax()
 KERNEL_SOURCES = ["calibration_free_weight_dualquant_b200/csrc/dq_solver.cu",
                   "calibration_free_weight_dualquant_b200/csrc/dq_device.cuh",
                   "calibration_free_weight_dualquant_b200/csrc/dq_fast.cuh",
@@ -282,7 +297,7 @@ def run_reference(args, wl, rank, world, dist, set_name=None):
 def config_of(wl, world) -> dict:
     return {"workload": wl.name, "rows": wl.rows, "cols": wl.cols, "format": wl.fmt, "group": wl.group,
             "iters": wl.iters, "w_dtype": wl.wdtype, "col_dtype": wl.col_dtype,
-            "l2": "flushed before each step (512 MB write, untimed)", "parallelism": "replicas x%d" % world}
+            "l2": "flushed before each step (512 MB write, then 512 MB read: no dirty line left; untimed)", "parallelism": "replicas x%d" % world}
 
 
 # beta-folded activation quantization of a prefill batch: (format, group, tokens, in-features)
@@ -298,7 +313,7 @@ def run_act(args, name, rank, world, local, dist):
     The oracle arm (--impl reference) times oracle.act_quant on a row sample."""
     fmt, g, T, K = ACT_WORKLOADS[name]
     cfg = {"workload": name, "tokens": T, "cols": K, "format": fmt, "group": g, "x_dtype": "bf16",
-           "col_dtype": "bf16", "l2": "flushed before each step (512 MB write, untimed)",
+           "col_dtype": "bf16", "l2": "flushed before each step (512 MB write, then 512 MB read: no dirty line left; untimed)",
            "parallelism": "replicas x%d" % world}
     metric, unit = "activation elems/sec", "elem/s"
     X = synth.make_activations(T, K, seed=77 + rank)
@@ -331,13 +346,13 @@ def run_act(args, name, rank, world, local, dist):
     binding.load_library()
     Xd, bd = X.to(dev), b.to(dev)
     out = binding.dq_act_quant(Xd, bd, fmt, g)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     stream = torch.cuda.current_stream(dev)
 
     def timed(steps):
         ts = []
         for _ in range(steps):
-            flush.fill_(1)
+            flush()
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(stream)
@@ -451,7 +466,7 @@ def run_dq(args, wl, rank, world, local, dist):
     T = wl.iters
     out = binding.alloc_outputs(wl.rows, wl.cols, wl.fmt, wl.group, wl.col_dtype, T, dev)
     ws = torch.empty(binding.workspace_bytes(wl.rows, wl.cols, wl.fmt, wl.group), dtype=torch.uint8, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     stream = torch.cuda.current_stream(dev)
 
     def solve(iters, o=out, full=False):
@@ -461,7 +476,7 @@ def run_dq(args, wl, rank, world, local, dist):
     def timed(iters, steps, o=out, full=False):
         ts = []
         for _ in range(steps):
-            flush.fill_(1)
+            flush()
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(stream)
@@ -472,7 +487,7 @@ def run_dq(args, wl, rank, world, local, dist):
         return ts
 
     for _ in range(args.warmup):
-        flush.fill_(1)
+        flush()
         solve(T)
     torch.cuda.synchronize()
     st = binding.load_library().dq_sync_status(ws.data_ptr(), stream.cuda_stream)
@@ -626,7 +641,7 @@ def run_e2e(args, wl, W, T, dev, stream, flush, dist, world):
     binding.solve(Wh, wl.fmt, wl.group, T, wl.col_dtype, out=host_out, device_workspace=dws)
     e2e_ms = []
     for _ in range(max(3, args.steps // 2)):
-        flush.fill_(1)
+        flush()
         torch.cuda.synchronize()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
