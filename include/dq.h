@@ -49,7 +49,11 @@ typedef enum {
 
 /* Formats (DualQuant §3; reproduction README "Local reproduction"):
  *  DQ_INT4   grid [-8,7], block inverse scales fp16, group 8, 16, 32, 64, 128
- *            or 256; column inverse scales fp16 or bf16.
+ *            or 256; column inverse scales fp16 or bf16.  Only powers of two:
+ *            a block row spans group/8 lanes of a warp, so group/8 must
+ *            divide 32; an even divisor of cols that is not a power of two
+ *            (24, 48, 96, ...) returns DQ_EUNSUPPORTED.  The pages' INT4
+ *            results and storage figures use groups of 64 and 128.
  *  DQ_MXINT4 grid [-8,7], group 32, block inverse scales 2^k with k in
  *            [-126,126] stored as E8M0 bytes (k+127).
  *  DQ_NVFP4  E2M1 grid {0,+-0.5,+-1,+-1.5,+-2,+-3,+-4,+-6}, group 16, block
@@ -285,14 +289,24 @@ int dq_solve_batched(const dq_matrix* mats, int count, int format, int group, in
  * DQ_F16, col_dtype the dtype of `col_scales` (DQ_BF16 or DQ_F16).  The
  * workspace (DQ_ACT_WORKSPACE_BYTES, 256-byte aligned) reports a non-finite
  * X * b through dq_sync_status.  The 4-bit formats only: DQ_MXINT8 and
- * DQ_MXFP8 return DQ_EUNSUPPORTED. */
+ * DQ_MXFP8 return DQ_EUNSUPPORTED.  X must be 16-byte aligned, codes 4-byte
+ * aligned (16-byte alignment lets a lane store its codes in one vector store).
+ * NVFP4 runs its amax pass and quantization pass in one cooperative launch
+ * with a grid-wide barrier whose wait is bounded (a wait that runs out is
+ * reported as DQ_ECUDA by dq_sync_status); the other formats are one pass. */
 int dq_act_quant(const void* X, int x_dtype, int64_t rows, int64_t cols, const void* col_scales, int col_dtype,
                  int format, int group, const dq_outputs* out, void* workspace, size_t workspace_bytes,
                  void* stream);
 
 /* Size of the library-owned device scratch that dq_solve_static uses: 8 MiB.
  * A shape fits when dq_workspace_bytes(rows, cols, format, group) is at most
- * this; on a 148-SM B200 that holds every shape with cols <= 196608. */
+ * this.  The workspace holds the working block scales (rows x cols/group
+ * stored values) and per-CTA column partials that grow with the group; on a
+ * 148-SM B200 the four matrix shapes of a Llama-3.1-8B layer (4096 x 4096,
+ * 1024 x 4096, 14336 x 4096, 4096 x 14336) fit in NVFP4, the MX formats and
+ * INT4 with group 32 or 64 (at most 6.1 MiB), while larger matrices (8192 x
+ * 28672 and up) and INT4 groups of 8, 16, 128 or 256 on the 14336 x 4096
+ * shape do not: those take dq_solve with a caller's workspace. */
 #define DQ_STATIC_SCRATCH_BYTES (8u << 20)
 
 /* dq_solve without a workspace argument, for callers that cannot allocate

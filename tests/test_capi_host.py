@@ -117,3 +117,22 @@ def test_host_side_argument_checks_for_the_8bit_formats(lib_path):
         assert lib.dq_act_quant(W, 1, 4, 64, base[4], 1, fmt, 32, ctypes.byref(o), None, 0, None) == 2
     o = outs()
     assert lib.dq_solve(W, 1, 4, 64, 6, 32, 2, 1, ctypes.byref(o), None, 0, None) == 1   # no format 6
+
+
+def test_int4_groups_are_powers_of_two(lib_path):
+    """INT4 takes the power-of-two groups 8 .. 256 (a block row spans group/8 lanes of a warp); an even
+    divisor of cols that is not a power of two is DQ_EUNSUPPORTED in the solver and the activation
+    quantizer, decided on the host before any device work."""
+    lib = binding.load_library()
+    bufs = [ctypes.create_string_buffer(8192 + 64) for _ in range(5)]
+    base = [((ctypes.addressof(b) + 63) // 64) * 64 for b in bufs]
+    o = binding._Outputs(base[1], base[2], base[3], base[4], base[4] + 1024)
+    for g in (24, 48, 96):
+        cols = 2 * 96  # a multiple of every group tried
+        assert lib.dq_solve(base[0], 1, 4, cols, int(binding.Format.INT4), g, 2, 2, ctypes.byref(o), None, 0,
+                            None) == 2, g
+        assert lib.dq_act_quant(base[0], 1, 4, cols, base[4], 1, int(binding.Format.INT4), g, ctypes.byref(o),
+                                None, 0, None) == 2, g
+    for g in (4, 512):
+        assert lib.dq_solve(base[0], 1, 4, 1024, int(binding.Format.INT4), g, 2, 2, ctypes.byref(o), None, 0,
+                            None) == 2, g
