@@ -94,13 +94,21 @@ __global__ void __launch_bounds__(kThreads) k_init(Problem p) {
     if (p.sT_out) *p.sT_out = 1.f;
   }
   const double qmax = grid_qmax(FMT);
-  const int64_t nblocks = p.M * p.nb;
-  const int64_t stride = (int64_t)gridDim.x * kThreads;
-  for (int64_t blk = (int64_t)blockIdx.x * kThreads + threadIdx.x; blk < nblocks; blk += stride) {
-    const int64_t i = blk / p.nb, g = blk % p.nb;
+  const float isT = FMT == FMT_NVFP4 ? __frcp_rn((float)sTd) : 1.f;
+  // A warp takes 32 consecutive rows of one block-column (lane = row): each
+  // lane reads its block's G contiguous elements (whole sectors), and the
+  // warp's 32 block scales land contiguously in the block-column-major a_work.
+  const int lane = threadIdx.x & 31;
+  const int64_t MT = (p.M + 31) / 32;
+  const int64_t ntiles = MT * p.nb;
+  const int64_t nwarps = (int64_t)gridDim.x * (kThreads / 32);
+  for (int64_t t = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); t < ntiles; t += nwarps) {
+    const int64_t g = t / MT, i = (t - g * MT) * 32 + lane;
+    if (i >= p.M) continue;
     const int64_t off = i * p.N + g * p.G;
-    double m = 0.0;
+    double a;
     if (l1) {
+      double m = 0.0;
       for (int c = 0; c < p.G; c += 8) {
         float w[8];
         load8<WDT>(p.W, off + c, w);
@@ -108,6 +116,7 @@ __global__ void __launch_bounds__(kThreads) k_init(Problem p) {
         for (int k = 0; k < 8; ++k)
           m = fmax(m, (double)fabsf(w[k]) / (double)b_decode(p.b_store, p.col_dt, g * p.G + c + k));
       }
+      a = (m == 0.0) ? 1.0 : a_project<FMT>(m / qmax, sTd);
     } else {
       float mf = 0.f;
       for (int c = 0; c < p.G; c += 8) {
@@ -116,11 +125,14 @@ __global__ void __launch_bounds__(kThreads) k_init(Problem p) {
 #pragma unroll
         for (int k = 0; k < 8; ++k) mf = fmaxf(mf, fabsf(w[k]));
       }
-      m = (double)mf;
+      // certified fp32 projection of absmax / qmax, fp64 where it is ambiguous
+      bool amb = false;
+      const float af = a_fast<FMT>(mf, (float)qmax, isT, amb);
+      a = !amb ? (double)af : (mf == 0.f ? 1.0 : a_project<FMT>((double)mf / qmax, sTd));
     }
-    const double a = (m == 0.0) ? 1.0 : a_project<FMT>(m / qmax, sTd);
     a_encode<FMT>(p.a_work, g * p.M + i, a);
   }
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
   if (!l1)
     for (int64_t j = (int64_t)blockIdx.x * kThreads + threadIdx.x; j < p.N; j += stride)
       b_encode(p.b_store, p.col_dt, j, 1.0);
