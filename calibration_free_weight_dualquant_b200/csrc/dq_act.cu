@@ -23,8 +23,8 @@ namespace dq {
 
 constexpr int kActThreads = 256;  // 8 warps
 constexpr int kActWarps = kActThreads / 32;
-// CTAs per SM of the one-pass kernels: 85 registers for E <= 16, 128 for E = 32
-__host__ __device__ constexpr int act_ctas_per_sm(int E) { return E == 32 ? 2 : 3; }
+// CTAs per SM of the one-pass kernels: 85 registers for E = 8, 128 for E = 16 and 32
+__host__ __device__ constexpr int act_ctas_per_sm(int E) { return E >= 16 ? 2 : 3; }
 constexpr int kActNvCtasPerSm = 2;  // the fused NVFP4 kernel: 128 registers
 constexpr int kActEntry = 2048;     // bytes of one ring entry of a warp (one work item)
 constexpr int kActStages = 4;       // ring entries per warp (a power of two)
