@@ -380,10 +380,10 @@ def run_act(args, name, rank, world, local, dist):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": cfg,
-            "roofline": {"bound": "hbm", "kernel": "k_act_amax+k_act" if fmt == "nvfp4" else "k_act", "achieved": achieved,
+            "roofline": {"bound": "hbm", "kernel": "k_act_nv" if fmt == "nvfp4" else "k_act", "achieved": achieved,
                          "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
                          "traffic": None, "algorithmic_bytes_per_launch": alg, "peak_source": peaks["source"],
-                         "note": "one call = quantize pass (NVFP4: amax pass + quantize pass); algorithmic bytes count one read of X"},
+                         "note": "one call = one launch (NVFP4: amax pass, grid barrier, quantization pass); algorithmic bytes count one read of X"},
             "e2e": None, "gpu_launches": (2 if fmt == "nvfp4" else 1) * args.steps, "clocks": clk.summary()}
     print(json.dumps(line), flush=True)
 

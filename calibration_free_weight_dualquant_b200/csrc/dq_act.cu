@@ -1,6 +1,6 @@
 // dq_act.cu -- the beta-folded activation quantizer: X' = X diag(b) followed by
-// the format's own row-wise absmax round-to-nearest, in one pass over X (plus
-// an amax pass for the NVFP4 tensor scale).
+// the format's own row-wise absmax round-to-nearest, in one pass over X (NVFP4:
+// an amax pass first, in the same launch, for the tensor scale).
 //
 // Method (DualQuant arXiv 2610.13767 summary, §4.4 "Inference-time procedure
 // and overhead", and the reproduction README flowchart, last two boxes): with
