@@ -47,6 +47,7 @@ _SHAPES = [
     (5, 1152, torch.bfloat16, torch.bfloat16),      # rows not a multiple of an item's rows; a partial slab
     (1030, 1152, torch.float16, torch.float16),     # warp ranges that cross slab boundaries
     (3, 1024 + 64, torch.bfloat16, torch.bfloat16),  # one lane-group past the last whole slab
+    (2, 32768, torch.bfloat16, torch.bfloat16),     # more slabs than warps: a warp changes slab between items
 ]
 
 
