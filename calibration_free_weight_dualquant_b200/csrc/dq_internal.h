@@ -30,7 +30,6 @@ constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kIterThreads = kConsumers + 32;
 // block-columns per strip: one per consumer warp
 constexpr int kBcPerStrip = kConsumerWarps;
-constexpr int kRun = 8;
 constexpr int kRingBytes = 96 * 1024;
 constexpr int kMaxStages = 8;
 // Tile geometry for block size G (a multiple of 8 dividing 256) and W element

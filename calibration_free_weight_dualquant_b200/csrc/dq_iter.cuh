@@ -27,8 +27,8 @@
 // one 2-D tensor copy (TMA) per block-column and tile, wherever the active
 // block-columns lie; a warp's 32 lanes read 512 contiguous bytes of its slot.
 // The pair arithmetic runs as packed f32x2 instructions.  Column sums and the
-// reconstruction residuals run in fp32 for kRun rows of a lane and are then
-// added into fp64 accumulators kept in shared memory.
+// reconstruction residuals run in fp32 for run_rows<FMT>() rows of a lane and
+// are then added into fp64 accumulators kept in shared memory.
 #pragma once
 
 #include <cuda.h>  // CUtensorMap
@@ -45,9 +45,17 @@ static_assert(kConsumerTreeTop < kConsumers && 2 * kConsumerTreeTop >= kConsumer
 // codes between iterates (changed-code counts); the final pass (codes of the
 // final iterate and the last MSE)
 enum : int { PASS_ITER = 0, PASS_COUNT = 1, PASS_FINAL = 2 };
-// relative error bound of the fp64 column totals built from fp32 runs of kRun
-// rows (kRun roundings per run, fp64 beyond), plus the oracle's own fp64 error
-constexpr double kColErr = 2.0 * kRun * 0x1p-24 + 1e-11;
+// rows of a lane's fp32 column-sum and residual runs before they are added
+// into fp64: shorter runs tighten the certified column projection (fewer
+// columns need the exact update) at the cost of more fp64 adds; NVFP4, whose
+// exact updates cost most, takes 4, the other formats 8 (measured)
+template <int FMT>
+constexpr int run_rows() { return FMT == FMT_NVFP4 ? 4 : 8; }
+// relative error bound of the fp64 column totals built from fp32 runs of
+// run_rows rows (that many roundings per run, fp64 beyond), plus the oracle's
+// own fp64 error
+template <int FMT>
+constexpr double col_err() { return 2.0 * run_rows<FMT>() * 0x1p-24 + 1e-11; }
 // Relative bracket of the E2M1 candidate: the fp32 candidate W*(1/b)*(1/e)*(1/s_T)
 // is within 7 * 2^-24 of W/(a b), the bracket factors add two more roundings.
 constexpr float kRelGuard = 0x1p-20f;
@@ -965,8 +973,8 @@ __device__ void finalize_slots(const Problem& p, int t, int64_t v, int w0, int s
         // underflow and is settled exactly as well
         const bool safe = tot.x >= 0x1p-60 && tot.x <= 0x1p100 && tot.y >= 0x1p-60 && tot.y <= 0x1p100;
         const double ratio = FMT == FMT_NVFP4 ? (tot.x / tot.y) / sTd : tot.x / tot.y;
-        const double lo = safe ? b_project(ratio * (1.0 - kColErr), p.col_dt) : 0.0;
-        const double hi = safe ? b_project(ratio * (1.0 + kColErr), p.col_dt) : 1.0;
+        const double lo = safe ? b_project(ratio * (1.0 - col_err<FMT>()), p.col_dt) : 0.0;
+        const double hi = safe ? b_project(ratio * (1.0 + col_err<FMT>()), p.col_dt) : 1.0;
         // the old scale: this CTA's column table of the strip (warp w, octet
         // c / 8, pair (c % 8) / 2), loaded when its segment of the strip began
         const f2 bp = ctab[w * 8 * (G / 8) + (c >> 3) * 4 + ((c & 7) >> 1)];
@@ -1472,7 +1480,7 @@ __global__ void __launch_bounds__(kIterThreads, 1)
         }
       }
       run += 2;
-      if (run >= kRun) {
+      if (run >= run_rows<FMT>()) {
         run = 0;
         flush_runs(cs, acc, racc, warp, lane, has);
       }
