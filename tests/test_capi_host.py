@@ -136,3 +136,27 @@ def test_int4_groups_are_powers_of_two(lib_path):
     for g in (4, 512):
         assert lib.dq_solve(base[0], 1, 4, 1024, int(binding.Format.INT4), g, 2, 2, ctypes.byref(o), None, 0,
                             None) == 2, g
+
+
+def test_act_quant_host_side_checks(lib_path):
+    """dq_act_quant's argument checks, decided on the host before any device work: X 16-byte aligned,
+    bf16/fp16 X and column scales, a group the format takes, codes 4-byte aligned, a workspace of
+    DQ_ACT_WORKSPACE_BYTES."""
+    lib = binding.load_library()
+    bufs = [ctypes.create_string_buffer(8192 + 64) for _ in range(5)]
+    base = [((ctypes.addressof(b) + 63) // 64) * 64 for b in bufs]
+    wsbuf = ctypes.create_string_buffer(1024)
+    ws = ((ctypes.addressof(wsbuf) + 255) // 256) * 256
+    o = binding._Outputs(base[1], base[2], base[3], base[4], base[4] + 1024)
+    I4, MX4, NV = int(binding.Format.INT4), int(binding.Format.MXINT4), int(binding.Format.NVFP4)
+    act = lib.dq_act_quant
+    assert act(base[0] + 8, 1, 4, 64, base[4], 1, I4, 64, ctypes.byref(o), ws, 256, None) == 1   # X not 16-byte aligned
+    assert act(base[0], 0, 4, 64, base[4], 1, I4, 64, ctypes.byref(o), ws, 256, None) == 2       # fp32 X
+    assert act(base[0], 1, 4, 64, base[4], 0, I4, 64, ctypes.byref(o), ws, 256, None) == 2       # fp32 column scales
+    assert act(base[0], 1, 4, 64, base[4], 1, MX4, 16, ctypes.byref(o), ws, 256, None) == 2      # MXINT4 takes 32
+    assert act(base[0], 1, 4, 64, base[4], 1, NV, 32, ctypes.byref(o), ws, 256, None) == 2       # NVFP4 takes 16
+    assert act(base[0], 1, 4, 48, base[4], 1, I4, 32, ctypes.byref(o), ws, 256, None) == 1       # cols % group
+    assert act(base[0], 1, 0, 64, base[4], 1, I4, 64, ctypes.byref(o), ws, 256, None) == 1       # no rows
+    bad = binding._Outputs(base[1] + 2, base[2], base[3], base[4], base[4] + 1024)
+    assert act(base[0], 1, 4, 64, base[4], 1, I4, 64, ctypes.byref(bad), ws, 256, None) == 1     # codes 2-byte aligned
+    assert act(base[0], 1, 4, 64, base[4], 1, I4, 64, ctypes.byref(o), ws, 128, None) == 3       # short workspace
